@@ -1,0 +1,378 @@
+// la.cu — the C ABI declared in include/la.h: argument validation on the host,
+// kernel selection, the host-buffer entry point and the device error word.
+//
+// Kernel selection for la_fwd:
+//   bf16, dk = 128           -> chunked tensor-core kernel (chunk_tc.cuh)
+//   fp32, or bf16 with dk < 128 -> per-token recurrent kernel (recurrent.cuh)
+// la_step always uses the recurrent kernel with T = 1 and the state in place.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "la.h"
+#include "device.cuh"
+#include "recurrent.cuh"
+#include "chunk_tc.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+la_status fail(la_status s, const std::string &msg) {
+    g_last_error = msg;
+    return s;
+}
+
+la_status ok() {
+    g_last_error.clear();
+    return LA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_dim(int64_t d) { return d == 32 || d == 64 || d == 128; }
+
+size_t elem_size(la_dtype t) { return t == LA_BF16 ? 2 : 4; }
+
+struct Shape {
+    int64_t B, T, H, dk, dv;
+};
+
+la_status validate_common(la_rule rule, la_dtype dtype, const Shape &s) {
+    if (rule != LA_RULE_ELU && rule != LA_RULE_GLA && rule != LA_RULE_GDN)
+        return fail(LA_ERR_INVALID_ARG, "rule must be LA_RULE_ELU, LA_RULE_GLA or LA_RULE_GDN");
+    if (dtype != LA_F32 && dtype != LA_BF16)
+        return fail(LA_ERR_INVALID_ARG, "dtype must be LA_F32 or LA_BF16");
+    if (s.B < 1 || s.H < 1 || s.T < 0)
+        return fail(LA_ERR_INVALID_ARG, "need B >= 1, H >= 1, T >= 0");
+    if (!supported_dim(s.dk) || !supported_dim(s.dv))
+        return fail(LA_ERR_UNSUPPORTED, "dk and dv must each be 32, 64 or 128");
+    // element counts stay far below 2^62 and the grid below 2^31
+    const double n = (double)s.B * (double)(s.T > 0 ? s.T : 1) * (double)s.H * 128.0;
+    if (n > 4.0e18 || (double)s.B * (double)s.H * 4.0 > 2.0e9)
+        return fail(LA_ERR_INVALID_ARG, "problem too large");
+    return LA_OK;
+}
+
+la_status validate_gates(la_rule rule, const float *g, const float *beta, const void *z0,
+                         const void *z1) {
+    if (rule == LA_RULE_ELU) {
+        if (g || beta) return fail(LA_ERR_INVALID_ARG, "ELU takes no gate: g and beta must be NULL");
+    } else {
+        if (z0 || z1) return fail(LA_ERR_INVALID_ARG, "z0/z_out (and step z) are ELU-only");
+        if (!g) return fail(LA_ERR_INVALID_ARG, rule == LA_RULE_GLA ? "GLA needs the gate g"
+                                                                    : "GDN needs alpha (g)");
+        if (rule == LA_RULE_GLA && beta) return fail(LA_ERR_INVALID_ARG, "GLA takes no beta");
+        if (rule == LA_RULE_GDN && !beta) return fail(LA_ERR_INVALID_ARG, "GDN needs beta");
+    }
+    return LA_OK;
+}
+
+la_status check_launch(const char *what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(LA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+    return ok();
+}
+
+// ---------------------------------------------------------------------------
+// Recurrent kernel dispatch (fp32 prefill, small-dk bf16 prefill, decode).
+// ---------------------------------------------------------------------------
+template <int RULE, int DK, int DV>
+la_status launch_rec_typed(const la::RecurrentParams &p, la_dtype dt, cudaStream_t st) {
+    const dim3 grid((unsigned)(p.B * p.H)), block(256);
+    if (dt == LA_BF16)
+        la::recurrent_kernel<RULE, DK, DV, __nv_bfloat16><<<grid, block, 0, st>>>(p);
+    else
+        la::recurrent_kernel<RULE, DK, DV, float><<<grid, block, 0, st>>>(p);
+    return check_launch("recurrent kernel launch");
+}
+
+template <int RULE, int DK>
+la_status launch_rec_dv(const la::RecurrentParams &p, int64_t dv, la_dtype dt, cudaStream_t st) {
+    switch (dv) {
+        case 32: return launch_rec_typed<RULE, DK, 32>(p, dt, st);
+        case 64: return launch_rec_typed<RULE, DK, 64>(p, dt, st);
+        default: return launch_rec_typed<RULE, DK, 128>(p, dt, st);
+    }
+}
+
+template <int RULE>
+la_status launch_rec_dk(const la::RecurrentParams &p, int64_t dk, int64_t dv, la_dtype dt,
+                        cudaStream_t st) {
+    switch (dk) {
+        case 32: return launch_rec_dv<RULE, 32>(p, dv, dt, st);
+        case 64: return launch_rec_dv<RULE, 64>(p, dv, dt, st);
+        default: return launch_rec_dv<RULE, 128>(p, dv, dt, st);
+    }
+}
+
+la_status launch_recurrent(la_rule rule, const la::RecurrentParams &p, int64_t dk, int64_t dv,
+                           la_dtype dt, cudaStream_t st) {
+    switch (rule) {
+        case LA_RULE_ELU: return launch_rec_dk<la::kRuleELU>(p, dk, dv, dt, st);
+        case LA_RULE_GLA: return launch_rec_dk<la::kRuleGLA>(p, dk, dv, dt, st);
+        default: return launch_rec_dk<la::kRuleGDN>(p, dk, dv, dt, st);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA descriptor encoding through the driver entry point (no -lcuda needed).
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+}  // namespace
+
+namespace la {
+// 4-D map over a [B,T,H,D] tensor (innermost first: D, H, T, B), box
+// {box_d, 1, box_t, 1}.  Rows past T read as zero.
+bool make_map_4d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int esize,
+                 int64_t B, int64_t T, int64_t H, int64_t D, int box_d, int box_t,
+                 CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)(D * esize), (cuuint64_t)(H * D * esize),
+                             (cuuint64_t)(T * H * D * esize)};
+    cuuint32_t box[4] = {(cuuint32_t)box_d, 1u, (cuuint32_t)box_t, 1u};
+    cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    CUresult r = fn(map, dtype, 4, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory (once per process
+// and device is enough; repeating it is harmless).
+cudaError_t allow_smem(const void *kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+}  // namespace la
+
+namespace {
+
+la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
+    const Shape s{a.B, a.T, a.H, a.dk, a.dv};
+    if (a.T == 0) {
+        const size_t sb = (size_t)(s.B * s.H * s.dk * s.dv) * sizeof(float);
+        const size_t zb = (size_t)(s.B * s.H * s.dk) * sizeof(float);
+        if (a.S_out && a.S_out != a.S0) {
+            cudaError_t e = a.S0 ? cudaMemcpyAsync(a.S_out, a.S0, sb, cudaMemcpyDeviceToDevice, st)
+                                 : cudaMemsetAsync(a.S_out, 0, sb, st);
+            if (e != cudaSuccess) return fail(LA_ERR_CUDA, cudaGetErrorString(e));
+        }
+        if (a.z_out && a.z_out != a.z0) {
+            cudaError_t e = a.z0 ? cudaMemcpyAsync(a.z_out, a.z0, zb, cudaMemcpyDeviceToDevice, st)
+                                 : cudaMemsetAsync(a.z_out, 0, zb, st);
+            if (e != cudaSuccess) return fail(LA_ERR_CUDA, cudaGetErrorString(e));
+        }
+        return ok();
+    }
+    if (a.dtype == LA_BF16 && a.dk == 128) {
+        la::ChunkParams p{};
+        p.B = a.B; p.T = a.T; p.H = a.H; p.dv = a.dv;
+        p.q = a.q; p.k = a.k; p.v = a.v; p.g = a.g; p.beta = a.beta;
+        p.S0 = a.S0; p.z0 = a.z0; p.S_out = a.S_out; p.z_out = a.z_out;
+        p.o = a.o; p.eps = a.eps;
+        std::string err;
+        const la_status r = (la_status)la::launch_chunk_tc((int)a.rule, p, st, &err);
+        if (r != LA_OK) return fail(r, err);
+        return check_launch("chunk kernel launch");
+    }
+    la::RecurrentParams p{};
+    p.B = a.B; p.T = a.T; p.H = a.H;
+    p.q = a.q; p.k = a.k; p.v = a.v; p.g = a.g; p.beta = a.beta;
+    p.S_in = a.S0; p.S_out = a.S_out; p.z_in = a.z0; p.z_out = a.z_out;
+    p.o = a.o; p.eps = a.eps;
+    return launch_recurrent(a.rule, p, a.dk, a.dv, a.dtype, st);
+}
+
+la_status validate_fwd(const la_fwd_args *a, bool device_ptrs) {
+    if (!a) return fail(LA_ERR_INVALID_ARG, "args is NULL");
+    if (a->struct_size < sizeof(la_fwd_args))
+        return fail(LA_ERR_INVALID_ARG, "struct_size smaller than sizeof(la_fwd_args)");
+    const Shape s{a->B, a->T, a->H, a->dk, a->dv};
+    la_status r = validate_common(a->rule, a->dtype, s);
+    if (r != LA_OK) return r;
+    r = validate_gates(a->rule, a->g, a->beta, a->z0, a->z_out);
+    if (r != LA_OK) return r;
+    if (a->T > 0 && (!a->q || !a->k || !a->v || !a->o))
+        return fail(LA_ERR_INVALID_ARG, "q, k, v and o must be non-NULL when T > 0");
+    if (!(a->eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+    if (device_ptrs) {
+        const void *ps[] = {a->q, a->k, a->v, a->g, a->beta, a->S0, a->z0, a->o, a->S_out, a->z_out};
+        for (const void *p : ps)
+            if (p && !aligned16(p)) return fail(LA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    }
+    return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+la_status la_fwd(const la_fwd_args *args, void *stream) {
+    la_status r = validate_fwd(args, true);
+    if (r != LA_OK) return r;
+    return launch_fwd(*args, static_cast<cudaStream_t>(stream));
+}
+
+la_status la_fwd_workspace_size(const la_fwd_args *args, size_t *bytes) {
+    if (!bytes) return fail(LA_ERR_INVALID_ARG, "bytes is NULL");
+    la_status r = validate_fwd(args, false);
+    if (r != LA_OK) return r;
+    *bytes = 0;
+    return ok();
+}
+
+la_status la_step(const la_step_args *a, void *stream) {
+    if (!a) return fail(LA_ERR_INVALID_ARG, "args is NULL");
+    if (a->struct_size < sizeof(la_step_args))
+        return fail(LA_ERR_INVALID_ARG, "struct_size smaller than sizeof(la_step_args)");
+    const Shape s{a->N, 1, a->H, a->dk, a->dv};
+    la_status r = validate_common(a->rule, a->dtype, s);
+    if (r != LA_OK) return r;
+    r = validate_gates(a->rule, a->g, a->beta, a->z, nullptr);
+    if (r != LA_OK) return r;
+    if (!a->q || !a->k || !a->v || !a->o || !a->S)
+        return fail(LA_ERR_INVALID_ARG, "q, k, v, o and S must be non-NULL");
+    if (a->rule == LA_RULE_ELU && !a->z) return fail(LA_ERR_INVALID_ARG, "ELU decode needs z");
+    if (!(a->eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+    const void *ps[] = {a->q, a->k, a->v, a->g, a->beta, a->S, a->z, a->o};
+    for (const void *p : ps)
+        if (p && !aligned16(p)) return fail(LA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    la::RecurrentParams p{};
+    p.B = a->N; p.T = 1; p.H = a->H;
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+    p.S_in = a->S; p.S_out = a->S; p.z_in = a->z; p.z_out = a->z;
+    p.o = a->o; p.eps = a->eps;
+    return launch_recurrent(a->rule, p, a->dk, a->dv, a->dtype, static_cast<cudaStream_t>(stream));
+}
+
+// Host-buffer path: staging layout = each tensor at a 256-byte aligned offset.
+struct StagingLayout {
+    size_t off[10];  // q k v g beta S0 z0 o S_out z_out
+    size_t bytes[10];
+    size_t total;
+};
+
+static void staging_layout(const la_fwd_args *a, StagingLayout *L) {
+    const size_t es = elem_size(a->dtype);
+    const size_t tok = (size_t)(a->B * a->T * a->H);
+    size_t gb = 0;
+    if (a->g) gb = tok * (a->rule == LA_RULE_GLA ? (size_t)a->dk : 1) * 4;
+    const size_t sb = (size_t)(a->B * a->H * a->dk * a->dv) * 4;
+    const size_t zb = (size_t)(a->B * a->H * a->dk) * 4;
+    const size_t b[10] = {tok * a->dk * es, tok * a->dk * es, tok * a->dv * es, gb,
+                          a->beta ? tok * 4 : 0, a->S0 ? sb : 0, a->z0 ? zb : 0,
+                          tok * a->dv * es, a->S_out ? sb : 0, a->z_out ? zb : 0};
+    size_t o = 0;
+    for (int i = 0; i < 10; ++i) {
+        L->off[i] = o;
+        L->bytes[i] = b[i];
+        o += (b[i] + 255) & ~(size_t)255;
+    }
+    L->total = o;
+}
+
+la_status la_fwd_host_staging_size(const la_fwd_args *args, size_t *bytes) {
+    if (!bytes) return fail(LA_ERR_INVALID_ARG, "bytes is NULL");
+    la_status r = validate_fwd(args, false);
+    if (r != LA_OK) return r;
+    StagingLayout L;
+    staging_layout(args, &L);
+    *bytes = L.total;
+    return ok();
+}
+
+la_status la_fwd_host(const la_fwd_args *h, void *staging, size_t staging_bytes, void *stream) {
+    la_status r = validate_fwd(h, false);
+    if (r != LA_OK) return r;
+    if (!staging || (reinterpret_cast<uintptr_t>(staging) & 255u))
+        return fail(LA_ERR_ALIGNMENT, "staging must be a 256-byte aligned device buffer");
+    StagingLayout L;
+    staging_layout(h, &L);
+    if (staging_bytes < L.total) return fail(LA_ERR_WORKSPACE, "staging buffer too small");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *base = static_cast<char *>(staging);
+    const void *src[7] = {h->q, h->k, h->v, h->g, h->beta, h->S0, h->z0};
+    void *dptr[10];
+    for (int i = 0; i < 10; ++i) dptr[i] = L.bytes[i] ? base + L.off[i] : nullptr;
+    for (int i = 0; i < 7; ++i) {
+        if (!L.bytes[i]) continue;
+        cudaError_t e = cudaMemcpyAsync(dptr[i], src[i], L.bytes[i], cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return fail(LA_ERR_CUDA, std::string("H2D copy: ") + cudaGetErrorString(e));
+    }
+    la_fwd_args d = *h;
+    d.q = dptr[0]; d.k = dptr[1]; d.v = dptr[2];
+    d.g = static_cast<const float *>(dptr[3]);
+    d.beta = static_cast<const float *>(dptr[4]);
+    d.S0 = static_cast<const float *>(dptr[5]);
+    d.z0 = static_cast<const float *>(dptr[6]);
+    d.o = dptr[7];
+    d.S_out = static_cast<float *>(dptr[8]);
+    d.z_out = static_cast<float *>(dptr[9]);
+    r = la_fwd(&d, stream);
+    if (r != LA_OK) return r;
+    void *dst[3] = {h->o, h->S_out, h->z_out};
+    for (int i = 0; i < 3; ++i) {
+        if (!L.bytes[7 + i] || !h->T && i == 0) continue;
+        cudaError_t e = cudaMemcpyAsync(dst[i], dptr[7 + i], L.bytes[7 + i], cudaMemcpyDeviceToHost, st);
+        if (e != cudaSuccess) return fail(LA_ERR_CUDA, std::string("D2H copy: ") + cudaGetErrorString(e));
+    }
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(LA_ERR_CUDA, std::string("sync: ") + cudaGetErrorString(e));
+    return ok();
+}
+
+la_status la_check_device(void *stream, uint32_t *flags) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(LA_ERR_CUDA, cudaGetErrorString(e));
+    uint32_t w = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&w, la::g_error_word, sizeof(w));
+    if (e == cudaSuccess && w) e = cudaMemcpyToSymbol(la::g_error_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail(LA_ERR_CUDA, cudaGetErrorString(e));
+    if (flags) *flags = w;
+    if (w & la::kErrTimeout) return fail(LA_ERR_TIMEOUT, "a bounded device wait ran out");
+    if (w & la::kErrRange)
+        return fail(LA_ERR_RANGE, "GLA cumulative gate inside a 64-token chunk fell below 1e-30");
+    return ok();
+}
+
+const char *la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+        case LA_ERR_ALIGNMENT: return "LA_ERR_ALIGNMENT";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
+        case LA_ERR_RANGE: return "LA_ERR_RANGE";
+        case LA_ERR_INTERNAL: return "LA_ERR_INTERNAL";
+        case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE";
+    }
+    return "LA_ERR_UNKNOWN";
+}
+
+const char *la_last_error_message(void) { return g_last_error.c_str(); }
+
+int la_abi_version(void) { return LA_ABI_VERSION; }
+
+}  // extern "C"

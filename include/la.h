@@ -1,0 +1,178 @@
+/*
+ * la.h — C ABI of the B200 (sm_100a) causal linear-attention library.
+ *
+ * The library computes the causal linear-attention forward that folds a
+ * sequence into a fixed dk x dv matrix state per (batch, head), for three
+ * update rules:
+ *
+ *   LA_RULE_ELU  normalized ELU+1 linear attention
+ *       S_t = S_{t-1} + phi(k_t) v_t^T,  z_t = z_{t-1} + phi(k_t),
+ *       o_t = phi(q_t)^T S_t / (phi(q_t)^T z_t + eps),  phi(x) = ELU(x) + 1
+ *       (page "Linear / RNN 路线：砍 softmax，固定 state 替代 KV", §2.1; eps in
+ *       the denominator as in page "状态空间与线性注意力", section 线性注意力)
+ *   LA_RULE_GLA  gated linear attention, per-key-dimension gate g_t in (0,1)^dk
+ *       S_t = diag(g_t) S_{t-1} + k_t v_t^T,  o_t = S_t^T q_t
+ *       (page "Linear / RNN 路线", §2.2)
+ *   LA_RULE_GDN  gated delta rule, scalar alpha_t, beta_t in (0,1)
+ *       S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,
+ *       o_t = S_t^T q_t
+ *       (page "线性注意力与 SSM：把整张关系表变成一条状态流", GDN box, written
+ *       there for the transposed dv x dk state; output read after the write as
+ *       in page "状态空间与线性注意力", section KDA recurrent reference)
+ *
+ * Entry points
+ *   la_fwd   chunked prefill over T tokens, optional initial state in, final
+ *            state out (the selective-scan contract of page "状态空间与线性注意力":
+ *            optional initial state, all outputs and the final state returned).
+ *   la_step  one decode token per sequence, state updated in place.
+ *   la_fwd_host  la_fwd on HOST buffers: copies in, runs, copies out.
+ *
+ * Conventions (all entry points)
+ *   - Layouts are dense row-major: q,k [B,T,H,dk]; v,o [B,T,H,dv]; GLA gate
+ *     [B,T,H,dk] fp32; GDN alpha,beta [B,T,H] fp32; state [B,H,dk,dv] fp32 with
+ *     rows = key dims; ELU normaliser z [B,H,dk] fp32.  Decode drops the T axis.
+ *   - Device pointers must be 16-byte aligned.  The library reads and writes
+ *     only the buffers it is given, never allocates or frees device memory,
+ *     never synchronises the stream (except la_check_device / la_fwd_host,
+ *     which say so) and never changes the current device.  The caller owns
+ *     every buffer and keeps it alive until the stream work completes.
+ *   - Each call enqueues work on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and returns immediately.  Arguments are
+ *     validated on the host before any launch; an invalid call launches nothing.
+ *   - Conditions detected on the device (a bounded wait that ran out, a GLA
+ *     chunk whose cumulative gate leaves the fp32 range) set a device-wide error
+ *     word; la_check_device() reads and clears it.
+ *   - Supported sizes: dk, dv in {32, 64, 128}; B, H >= 1; T >= 0.  T == 0
+ *     writes S_out = S0 (or zeros) and z_out = z0 (or zeros).
+ *   - There is no CPU fallback: every result comes from a CUDA kernel.
+ */
+#ifndef LA_H_
+#define LA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LA_ABI_VERSION 1
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum, size mismatch */
+    LA_ERR_UNSUPPORTED = 2,   /* dk/dv/dtype combination without a kernel */
+    LA_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned */
+    LA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    LA_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out (la_check_device) */
+    LA_ERR_RANGE = 6,         /* GLA gate product left the fp32 range in a chunk (la_check_device) */
+    LA_ERR_INTERNAL = 7,
+    LA_ERR_WORKSPACE = 8      /* workspace missing or smaller than la_fwd_workspace_size() */
+} la_status;
+
+typedef enum { LA_RULE_ELU = 0, LA_RULE_GLA = 1, LA_RULE_GDN = 2 } la_rule;
+
+/* Element type of q, k, v and o.  Gates and the state are always fp32. */
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+/*
+ * Prefill arguments.  All pointers are device pointers.
+ *   q, k   [B,T,H,dk] of `dtype`
+ *   v      [B,T,H,dv] of `dtype`
+ *   g      GLA: gate [B,T,H,dk], every entry in (0,1];  GDN: alpha [B,T,H] in (0,1];
+ *          ELU: must be NULL
+ *   beta   GDN: [B,T,H] in [0,1];  others: NULL
+ *   S0     [B,H,dk,dv] initial state, or NULL for zeros
+ *   z0     ELU: [B,H,dk] initial normaliser, or NULL for zeros; others: NULL
+ *   eps    ELU: added to the denominator after the dot product; ignored otherwise
+ *   o      [B,T,H,dv] of `dtype` (written)
+ *   S_out  [B,H,dk,dv] final state (written), or NULL; may alias S0
+ *   z_out  ELU: [B,H,dk] final normaliser, or NULL; may alias z0
+ *   workspace / workspace_bytes: device scratch of at least
+ *          la_fwd_workspace_size() bytes (may be NULL when that size is 0)
+ * q/k/v/o must not overlap S_out/z_out.
+ */
+typedef struct la_fwd_args {
+    uint32_t struct_size;     /* = sizeof(la_fwd_args) */
+    la_rule rule;
+    la_dtype dtype;
+    int64_t B, T, H, dk, dv;
+    const void *q, *k, *v;
+    const float *g;
+    const float *beta;
+    const float *S0;
+    const float *z0;
+    float eps;
+    void *o;
+    float *S_out;
+    float *z_out;
+    void *workspace;
+    size_t workspace_bytes;
+} la_fwd_args;
+
+/*
+ * Decode arguments (one token per sequence, N = batch).  Device pointers.
+ *   q, k [N,H,dk]; v, o [N,H,dv] of `dtype`
+ *   g    GLA [N,H,dk] / GDN alpha [N,H] / ELU NULL;  beta GDN [N,H] / NULL
+ *   S    [N,H,dk,dv] fp32, read and overwritten with the updated state
+ *   z    ELU [N,H,dk] fp32, read and overwritten; NULL otherwise
+ * The output is read from the state after this token's update.
+ */
+typedef struct la_step_args {
+    uint32_t struct_size;     /* = sizeof(la_step_args) */
+    la_rule rule;
+    la_dtype dtype;
+    int64_t N, H, dk, dv;
+    const void *q, *k, *v;
+    const float *g;
+    const float *beta;
+    float *S;
+    float *z;
+    float eps;
+    void *o;
+} la_step_args;
+
+/* Chunked prefill (see the struct above).  Asynchronous on `stream`. */
+la_status la_fwd(const la_fwd_args *args, void *stream);
+
+/* Bytes of device workspace la_fwd needs for these arguments (often 0). */
+la_status la_fwd_workspace_size(const la_fwd_args *args, size_t *bytes);
+
+/* One decode step with in-place state update.  Asynchronous on `stream`. */
+la_status la_step(const la_step_args *args, void *stream);
+
+/*
+ * la_fwd on HOST buffers.  `host_args` has the same fields as for la_fwd but
+ * every data pointer (q,k,v,g,beta,S0,z0 read; o,S_out,z_out written) is a
+ * host pointer (pinned memory gives asynchronous copies).  `staging` is a
+ * caller-owned device buffer of at least la_fwd_host_staging_size() bytes,
+ * 256-byte aligned, into which the inputs are copied; the kernels run on it and
+ * the outputs are copied back.  The call enqueues copies and kernels on
+ * `stream` and then synchronises that stream, so the host outputs are valid on
+ * return.  Allocates nothing.
+ */
+la_status la_fwd_host_staging_size(const la_fwd_args *host_args, size_t *bytes);
+la_status la_fwd_host(const la_fwd_args *host_args, void *staging, size_t staging_bytes,
+                      void *stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word set by
+ * earlier kernels.  Returns LA_OK, LA_ERR_TIMEOUT, LA_ERR_RANGE or LA_ERR_CUDA.
+ * `flags` (may be NULL) receives the raw word (bit 0 timeout, bit 1 range).
+ */
+la_status la_check_device(void *stream, uint32_t *flags);
+
+/* Static name of a status code. */
+const char *la_status_string(la_status s);
+
+/* Detail of the last error returned on the calling host thread ("" if none). */
+const char *la_last_error_message(void);
+
+/* LA_ABI_VERSION of the loaded library. */
+int la_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_H_ */

@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+* the library loads and exports every function ``include/la.h`` declares;
+* invalid arguments are rejected on the host with the documented status codes
+  before anything is launched (the pointers below are never dereferenced).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_attn_b200 as la
+from gated_delta_rule_attn_b200 import build as la_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    la_build.build()
+    return la.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "la.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:la_status|const char \*|int)\s*(la_\w+)\s*\(", text, re.M)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(la.EXPORTS) == names
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.la_abi_version() == 1
+    assert L.la_status_string(0) == b"LA_OK"
+    assert L.la_status_string(5) == b"LA_ERR_TIMEOUT"
+    assert L.la_status_string(99) == b"LA_ERR_UNKNOWN"
+
+
+FAKE = 0x10000  # a 16-byte aligned address that is never dereferenced
+
+
+def args(rule="gdn", dtype=1, B=1, T=8, H=2, dk=128, dv=128, **kw):
+    a = la.FwdArgs()
+    a.struct_size = ctypes.sizeof(a)
+    a.rule, a.dtype = la.RULES[rule], dtype
+    a.B, a.T, a.H, a.dk, a.dv = B, T, H, dk, dv
+    a.q = a.k = a.v = a.o = FAKE
+    if rule == "gla":
+        a.g = FAKE
+    if rule == "gdn":
+        a.g = a.beta = FAKE
+    a.eps = 1e-6
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def call(L, a):
+    return L.la_fwd(ctypes.byref(a), None), L.la_last_error_message().decode()
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dk=48), 2), (dict(dv=256), 2), (dict(dk=16), 2),
+    (dict(B=0), 1), (dict(H=0), 1), (dict(T=-1), 1),
+    (dict(rule_raw=7), 1), (dict(dtype=5), 1),
+    (dict(q=None), 1), (dict(o=None), 1),
+    (dict(q=FAKE + 8), 3), (dict(S0=FAKE + 4), 3), (dict(S_out=FAKE + 2), 3),
+    (dict(beta=None), 1), (dict(struct_size=8), 1), (dict(eps=-1.0), 1),
+])
+def test_invalid_fwd_arguments_rejected(L, kw, status):
+    rule_raw = kw.pop("rule_raw", None)
+    a = args(**kw)
+    if rule_raw is not None:
+        a.rule = rule_raw
+    r, msg = call(L, a)
+    assert r == status, msg
+    assert msg
+
+
+def test_rule_specific_gate_checks(L):
+    assert call(L, args("elu", g=FAKE))[0] == 1          # ELU takes no gate
+    assert call(L, args("gla", g=None))[0] == 1          # GLA needs g
+    assert call(L, args("gla", beta=FAKE))[0] == 1       # GLA takes no beta
+    assert call(L, args("gdn", z0=FAKE))[0] == 1         # z is ELU-only
+
+
+def test_null_args_and_workspace_query(L):
+    assert L.la_fwd(None, None) == 1
+    n = ctypes.c_size_t(123)
+    assert L.la_fwd_workspace_size(ctypes.byref(args()), ctypes.byref(n)) == 0
+    assert n.value == 0
+    assert L.la_fwd_workspace_size(ctypes.byref(args(dk=3)), ctypes.byref(n)) == 2
+
+
+def test_step_validation(L):
+    s = la.StepArgs()
+    s.struct_size = ctypes.sizeof(s)
+    s.rule, s.dtype, s.N, s.H, s.dk, s.dv = 2, 1, 4, 2, 128, 128
+    s.q = s.k = s.v = s.o = s.S = s.g = FAKE
+    assert L.la_step(ctypes.byref(s), None) == 1           # GDN needs beta
+    s.beta = FAKE + 1
+    assert L.la_step(ctypes.byref(s), None) == 3           # misaligned
+    s.rule, s.g, s.beta = 0, None, None
+    assert L.la_step(ctypes.byref(s), None) == 1           # ELU decode needs z
+    s.z, s.dk = FAKE, 100
+    assert L.la_step(ctypes.byref(s), None) == 2
+
+
+def test_host_staging_layout(L):
+    a = args("gla", B=2, T=100, H=3, dk=64, dv=32, S0=FAKE, S_out=FAKE)
+    n = ctypes.c_size_t()
+    assert L.la_fwd_host_staging_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    tok = 2 * 100 * 3
+    parts = [tok * 64 * 2, tok * 64 * 2, tok * 32 * 2, tok * 64 * 4, 0, 2 * 3 * 64 * 32 * 4, 0,
+             tok * 32 * 2, 2 * 3 * 64 * 32 * 4, 0]
+    assert n.value == sum((p + 255) // 256 * 256 for p in parts)
+    # a misaligned staging buffer is refused before any copy
+    assert L.la_fwd_host(ctypes.byref(a), ctypes.c_void_p(FAKE + 16), n.value, None) == 3
+    assert L.la_fwd_host(ctypes.byref(a), ctypes.c_void_p(FAKE), n.value - 1, None) == 8
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 1, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        la.fwd("elu", q, q, q)
