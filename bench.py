@@ -1,0 +1,491 @@
+"""Benchmark of the causal linear-attention hot path on B200.
+
+One step = one pass of every part of the path over one batch of synthetic
+input, each part a separate library call on the current stream:
+  * GLA prefill        B=2, H=16, T=8192, dk=dv=128  (gate per key dim)
+  * gated-delta prefill B=2, H=16, T=8192, dk=dv=128
+  * ELU+1 prefill      B=1, H=16, T=32768, dk=128, dv=64 (state carry-in)
+  * one GLA and one gated-delta decode step on a [256,16,128,128] fp32 state
+``value`` is the prefill throughput of the GLA + gated-delta pair at d=128,
+T=8192 (tokens = B*T, both calls), from the device time of those two calls;
+the other parts are reported per leg (decode as state GB/s).
+
+Timing: W warm-up steps, then K steps between a barrier + synchronize on both
+sides, CUDA events on the launching stream around every leg; multi-GPU runs are
+weak-scaled (every rank runs the same step on its own GPU, no collective on the
+data path) and the time is the max over ranks.  Every leg's inputs are larger
+than the 126 MB L2, so nothing stays cached between reuses.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s + % roofline (GLA/GDN d=128 T=8192); decode state GB/s"
+CHUNK = 64  # chunk length of the tensor-core kernels (for the algorithmic FLOP count)
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work (bytes each input read once / output written once; MACs of
+# the chunkwise method counting only causally needed products)
+# ---------------------------------------------------------------------------
+
+def update_macs(N: int, dk: int, dv: int) -> int:
+    """The state-update term alone: N * dk * dv multiply-adds per head (the hand
+    count of page "线性注意力与 SSM", §02: N=32768, dphi=128, dv=64 -> ~2.684e8)."""
+    return N * dk * dv
+
+
+def macs_per_token_head(rule: str, dk: int, dv: int, C: int = CHUNK) -> float:
+    P = C * (C + 1) / 2
+    if rule == "elu":
+        return (P * dk + P * (dv + 1)) / C + 2 * dk * (dv + 1)
+    base = P * (dk + dv) / C + 2 * dk * dv
+    if rule == "gla":
+        return base
+    return base + (C - 1) / 2 * dk + (C - 1) / 2 * (dk + dv) + dk * dv
+
+
+def prefill_bytes(rule: str, B: int, T: int, H: int, dk: int, dv: int, esize: int = 2,
+                  with_S0: bool = False, with_z: bool = False) -> int:
+    tok = B * T * H
+    b = tok * (2 * dk + 2 * dv) * esize              # q, k, v read; o written
+    if rule == "gla":
+        b += tok * dk * 4                            # gate
+    elif rule == "gdn":
+        b += tok * 2 * 4                             # alpha, beta
+    b += B * H * dk * dv * 4 * (2 if with_S0 else 1)  # S0 read (if given), S_out written
+    if with_z:
+        b += B * H * dk * 4 * 2
+    return b
+
+
+def decode_bytes(rule: str, N: int, H: int, dk: int, dv: int) -> int:
+    b = N * H * dk * dv * 4 * 2                     # state read + written
+    b += N * H * (2 * dk + 2 * dv) * 2               # q, k, v, o bf16
+    b += N * H * (dk * 4 if rule == "gla" else 8)    # gates
+    return b
+
+
+def prefill_flops(rule: str, B: int, T: int, H: int, dk: int, dv: int) -> float:
+    return 2.0 * macs_per_token_head(rule, dk, dv) * B * T * H
+
+
+# ---------------------------------------------------------------------------
+# Peaks, clocks, traffic records
+# ---------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_attn_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per launch from a committed ncu capture, valid only while the
+    kernel sources are unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return {}
+    if d.get("source_hash") != kernel_source_hash():
+        return {}
+    return d.get("bytes_per_launch", {})
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+               "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+               "display_clock_setting": 0x100}
+
+    def __init__(self, index: int, period: float = 0.05):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop = period, threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv:
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# Workload on the device
+# ---------------------------------------------------------------------------
+
+class Legs:
+    def __init__(self, torch, la, workloads, seed: int):
+        self.torch, self.la = torch, la
+        dev = lambda t: None if t is None else t.cuda()
+        gla = workloads.gla_prefill(B=2, H=16, T=8192, seed=seed)
+        gdn = workloads.gdn_prefill(B=2, H=16, T=8192, seed=seed)
+        elu = workloads.elu_long(seed=seed)
+        self.host = {"gla": gla, "gdn": gdn, "elu": elu}
+        self.gla = {k: dev(getattr(gla, k)) for k in ("q", "k", "v", "g")}
+        self.gdn = {k: dev(getattr(gdn, k)) for k in ("q", "k", "v", "g", "beta")}
+        self.elu = {k: dev(getattr(elu, k)) for k in ("q", "k", "v", "S0", "z0")}
+        self.S_dec = workloads.decode_state(seed=seed).cuda()
+        d_gla = workloads.decode_steps("gla", 1, seed=seed)[0]
+        d_gdn = workloads.decode_steps("gdn", 1, seed=seed)[0]
+        self.dec_gla = [x.cuda() for x in d_gla]
+        self.dec_gdn = [x.cuda() for x in d_gdn]
+        # outputs allocated once
+        e = torch.empty
+        self.o_gla = e(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
+        self.S_gla = e(2, 16, 128, 128, device="cuda")
+        self.o_gdn = e(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
+        self.S_gdn = e(2, 16, 128, 128, device="cuda")
+        self.o_elu = e(1, 32768, 16, 64, dtype=torch.bfloat16, device="cuda")
+        self.S_elu = e(1, 16, 128, 64, device="cuda")
+        self.z_elu = e(1, 16, 128, device="cuda")
+        self.o_dec = e(256, 16, 128, dtype=torch.bfloat16, device="cuda")
+        self.names = ["gla_prefill", "gdn_prefill", "elu_prefill", "gla_decode", "gdn_decode"]
+        self.launches_per_step = 5
+
+    def run(self, name):
+        la = self.la
+        if name == "gla_prefill":
+            a = self.gla
+            la.fwd("gla", a["q"], a["k"], a["v"], a["g"], o=self.o_gla, S_out=self.S_gla)
+        elif name == "gdn_prefill":
+            a = self.gdn
+            la.fwd("gdn", a["q"], a["k"], a["v"], a["g"], a["beta"], o=self.o_gdn, S_out=self.S_gdn)
+        elif name == "elu_prefill":
+            a = self.elu
+            la.fwd("elu", a["q"], a["k"], a["v"], S0=a["S0"], z0=a["z0"], eps=1e-6, o=self.o_elu,
+                   S_out=self.S_elu, z_out=self.z_elu)
+        elif name == "gla_decode":
+            q, k, v, g = self.dec_gla
+            la.step("gla", q, k, v, self.S_dec, g=g, o=self.o_dec)
+        elif name == "gdn_decode":
+            q, k, v, a_, b_ = self.dec_gdn
+            la.step("gdn", q, k, v, self.S_dec, g=a_, beta=b_, o=self.o_dec)
+
+
+def leg_work(name):
+    if name == "gla_prefill":
+        return dict(tokens=2 * 8192, bytes=prefill_bytes("gla", 2, 8192, 16, 128, 128),
+                    flops=prefill_flops("gla", 2, 8192, 16, 128, 128))
+    if name == "gdn_prefill":
+        return dict(tokens=2 * 8192, bytes=prefill_bytes("gdn", 2, 8192, 16, 128, 128),
+                    flops=prefill_flops("gdn", 2, 8192, 16, 128, 128))
+    if name == "elu_prefill":
+        return dict(tokens=32768, bytes=prefill_bytes("elu", 1, 32768, 16, 128, 64, with_S0=True,
+                                                      with_z=True),
+                    flops=prefill_flops("elu", 1, 32768, 16, 128, 64))
+    rule = name.split("_")[0]
+    return dict(tokens=256, bytes=decode_bytes(rule, 256, 16, 128, 128),
+                flops=2.0 * 2 * 128 * 128 * 256 * 16)
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import gated_delta_rule_attn_b200 as la
+    import workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    legs = Legs(torch, la, workloads, seed=rank)
+    stream = torch.cuda.current_stream()
+    # warm-up (also checks the device error word once)
+    for _ in range(max(args.warmup, 3)):
+        for n in legs.names:
+            legs.run(n)
+    torch.cuda.synchronize()
+    la.check_device()
+
+    K = args.steps
+    ev = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)] for n in legs.names}
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(K):
+            for n in legs.names:
+                ev[n][i][0].record(stream)
+                legs.run(n)
+                ev[n][i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = start.elapsed_time(end)
+    leg_ms = {n: sum(a.elapsed_time(b) for a, b in ev[n]) / K for n in legs.names}
+    la.check_device()
+
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([total_ms] + [leg_ms[n] for n in legs.names], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t[0])
+        leg_ms = {n: float(t[i + 1]) for i, n in enumerate(legs.names)}
+
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+    traffic = load_traffic()
+    legs_out = {}
+    for n in legs.names:
+        w = leg_work(n)
+        s = leg_ms[n] / 1e3
+        gbs = w["bytes"] / s / 1e9
+        legs_out[n] = {"ms": round(leg_ms[n], 4), "tokens_per_s": round(w["tokens"] / s),
+                       "alg_bytes": w["bytes"], "alg_flops": w["flops"],
+                       "gbs": round(gbs, 1), "tflops": round(w["flops"] / s / 1e12, 2),
+                       "hbm_frac": round(gbs / hbm_peak, 4)}
+    pre = ("gla_prefill", "gdn_prefill")
+    pre_ms = sum(leg_ms[n] for n in pre)
+    tokens = sum(leg_work(n)["tokens"] for n in pre)
+    value = world * tokens / (pre_ms / 1e3)
+    # roofline of the dominant kernel (longest leg)
+    dom = max(legs.names, key=lambda n: leg_ms[n])
+    w = leg_work(dom)
+    ach = w["bytes"] / (leg_ms[dom] / 1e3) / 1e9
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak,
+                "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
+                "traffic": traffic.get(dom),
+                "tensor_frac": round(w["flops"] / (leg_ms[dom] / 1e3) / 1e12 / tc_peak, 4)}
+    # roofline time = max(FLOPs at tensor peak, bytes at HBM peak) for the prefill pair
+    t_roof = sum(max(leg_work(n)["flops"] / (tc_peak * 1e12), leg_work(n)["bytes"] / (hbm_peak * 1e9))
+                 for n in pre)
+    dec_ms = leg_ms["gla_decode"] + leg_ms["gdn_decode"]
+    dec_bytes = leg_work("gla_decode")["bytes"] + leg_work("gdn_decode")["bytes"]
+
+    out = {
+        "metric": METRIC, "value": round(value), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) q/k/v and gates per the workload recipe in workloads.py; no dataset",
+        "config": {"workload": "GLA + gated-delta prefill B=2 H=16 T=8192 dk=dv=128 (value); "
+                               "ELU+1 prefill B=1 H=16 T=32768 dk=128 dv=64; GLA + gated-delta "
+                               "decode step on state [256,16,128,128] fp32",
+                   "global_batch": 2 * world, "seq_len": 8192, "chunk": CHUNK,
+                   "parallelism": f"dp{world} (independent sequences per GPU, no collective)",
+                   "l2": "inputs larger than L2 (every leg streams > 126 MB between reuses)"},
+        "prefill_roofline_frac": round(t_roof / (pre_ms / 1e3), 4),
+        "decode_state_gbs": round(dec_bytes / (dec_ms / 1e3) / 1e9, 1),
+        "legs": legs_out,
+        "roofline": roofline,
+        "gpu_launches": legs.launches_per_step * K,
+        "clocks": clk.summary(),
+    }
+
+    # end to end through the host-buffer entry point (copies inside the timed region)
+    out["e2e"] = run_e2e(torch, la, legs, min(K, args.e2e_steps), world)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(torch, la, legs, steps, world):
+    pin = lambda t: None if t is None else t.contiguous().pin_memory()
+    hg = {k: pin(getattr(legs.host["gla"], k)) for k in ("q", "k", "v", "g")}
+    hd = {k: pin(getattr(legs.host["gdn"], k)) for k in ("q", "k", "v", "g", "beta")}
+    mk = lambda: (torch.empty(2, 8192, 16, 128, dtype=torch.bfloat16).pin_memory(),
+                  torch.empty(2, 16, 128, 128).pin_memory())
+    og, Sg = mk()
+    od, Sd = mk()
+    n = max(la.host_staging_size("gla", hg["q"], hg["k"], hg["v"], hg["g"]),
+            la.host_staging_size("gdn", hd["q"], hd["k"], hd["v"], hd["g"], hd["beta"]))
+    staging = torch.empty(n, dtype=torch.uint8, device="cuda")
+    h2d = sum(t.numel() * t.element_size() for t in list(hg.values()) + list(hd.values()))
+    d2h = sum(t.numel() * t.element_size() for t in (og, Sg, od, Sd))
+
+    def step():
+        la.fwd_host("gla", hg["q"], hg["k"], hg["v"], hg["g"], o=og, S_out=Sg, staging=staging)
+        la.fwd_host("gdn", hd["q"], hd["k"], hd["v"], hd["g"], hd["beta"], o=od, S_out=Sd,
+                    staging=staging)
+
+    step()
+    s = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(s)
+    for _ in range(steps):
+        step()
+    b.record(s)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    tokens = 2 * 2 * 8192
+    return {"value": round(world * tokens / (ms / 1e3)), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms, 3), "api": "la_fwd_host (C ABI, pinned host buffers)"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+
+_ORACLE_INPUTS = []
+
+
+def _oracle_inputs():
+    if not _ORACLE_INPUTS:
+        import workloads
+        _ORACLE_INPUTS.extend([workloads.gla_prefill(B=2, H=16, T=8192),
+                               workloads.gdn_prefill(B=2, H=16, T=8192)])
+    return _ORACLE_INPUTS
+
+
+def oracle_sample(T: int, seed: int = 0):
+    """GLA + gated-delta prefill, batch 0, all 16 heads, first T tokens of the
+    d=128 T=8192 workloads; returns (seconds, full tokens processed)."""
+    import oracle
+    oracle.build.build()
+    gla, gdn = _oracle_inputs()
+    sl = lambda x: x[:1, :T].contiguous()
+    args_gla = [sl(x) for x in (gla.q, gla.k, gla.v, gla.g)]
+    args_gdn = [sl(x) for x in (gdn.q, gdn.k, gdn.v, gdn.g, gdn.beta)]
+    t0 = time.perf_counter()
+    oracle.gla_fwd(*args_gla)
+    oracle.gdn_fwd(*args_gdn)
+    dt = time.perf_counter() - t0
+    return dt, 2 * T
+
+
+def cpu_baseline(budget_s: float = 15.0):
+    import oracle
+    # size the sample so that the timed part takes about budget_s seconds
+    t_probe, tok_probe = oracle_sample(128)
+    T = int(min(8192, max(128, 128 * budget_s / max(t_probe, 1e-3))))
+    T = max(64, (T // 64) * 64)
+    dt, tokens = oracle_sample(T)
+    return {"value": round(tokens / dt, 1), "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 C oracle (OpenMP over heads): GLA + gated-delta prefill, batch 0, "
+                      f"all 16 heads, first {T} tokens of each d=128 T=8192 workload; "
+                      f"{dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    T = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_sample(T)
+    times = []
+    for _ in range(args.steps):
+        dt, tokens = oracle_sample(T)
+        times.append(dt)
+    total = sum(times)
+    value = args.steps * 2 * T / total
+    cores = oracle.num_threads()
+    sample = (f"per step: fp64 C oracle on GLA + gated-delta prefill, batch 0, 16 heads, first {T} "
+              f"tokens of each d=128 T=8192 workload ({2 * T} tokens)")
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic: seeded inputs per workloads.py; no dataset",
+           "config": {"workload": "GLA + gated-delta prefill B=2 H=16 T=8192 dk=dv=128 (sampled)",
+                      "global_batch": 2, "seq_len": 8192, "parallelism": "CPU threads"},
+           "impl": "reference",
+           "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores,
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-tokens", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -59,16 +59,19 @@ la_status validate_common(la_rule rule, la_dtype dtype, const Shape &s) {
     return LA_OK;
 }
 
+// `need` is false for an empty sequence (T == 0), whose gate tensors hold no
+// elements and may be passed as NULL.
 la_status validate_gates(la_rule rule, const float *g, const float *beta, const void *z0,
-                         const void *z1) {
+                         const void *z1, bool need) {
     if (rule == LA_RULE_ELU) {
         if (g || beta) return fail(LA_ERR_INVALID_ARG, "ELU takes no gate: g and beta must be NULL");
     } else {
         if (z0 || z1) return fail(LA_ERR_INVALID_ARG, "z0/z_out (and step z) are ELU-only");
-        if (!g) return fail(LA_ERR_INVALID_ARG, rule == LA_RULE_GLA ? "GLA needs the gate g"
-                                                                    : "GDN needs alpha (g)");
+        if (need && !g)
+            return fail(LA_ERR_INVALID_ARG, rule == LA_RULE_GLA ? "GLA needs the gate g"
+                                                                : "GDN needs alpha (g)");
         if (rule == LA_RULE_GLA && beta) return fail(LA_ERR_INVALID_ARG, "GLA takes no beta");
-        if (rule == LA_RULE_GDN && !beta) return fail(LA_ERR_INVALID_ARG, "GDN needs beta");
+        if (need && rule == LA_RULE_GDN && !beta) return fail(LA_ERR_INVALID_ARG, "GDN needs beta");
     }
     return LA_OK;
 }
@@ -211,7 +214,7 @@ la_status validate_fwd(const la_fwd_args *a, bool device_ptrs) {
     const Shape s{a->B, a->T, a->H, a->dk, a->dv};
     la_status r = validate_common(a->rule, a->dtype, s);
     if (r != LA_OK) return r;
-    r = validate_gates(a->rule, a->g, a->beta, a->z0, a->z_out);
+    r = validate_gates(a->rule, a->g, a->beta, a->z0, a->z_out, a->T > 0);
     if (r != LA_OK) return r;
     if (a->T > 0 && (!a->q || !a->k || !a->v || !a->o))
         return fail(LA_ERR_INVALID_ARG, "q, k, v and o must be non-NULL when T > 0");
@@ -249,7 +252,7 @@ la_status la_step(const la_step_args *a, void *stream) {
     const Shape s{a->N, 1, a->H, a->dk, a->dv};
     la_status r = validate_common(a->rule, a->dtype, s);
     if (r != LA_OK) return r;
-    r = validate_gates(a->rule, a->g, a->beta, a->z, nullptr);
+    r = validate_gates(a->rule, a->g, a->beta, a->z, nullptr, true);
     if (r != LA_OK) return r;
     if (!a->q || !a->k || !a->v || !a->o || !a->S)
         return fail(LA_ERR_INVALID_ARG, "q, k, v, o and S must be non-NULL");

@@ -1,0 +1,33 @@
+"""The bench's algorithmic work counts (CPU only)."""
+import math
+
+import bench
+
+
+def test_update_term_matches_pages_hand_count():
+    # page "线性注意力与 SSM", §02: N=32768, dphi=128, dv=64 -> about 2.684e8 MACs per head
+    m = bench.update_macs(32768, 128, 64)
+    assert m == 268_435_456
+    assert abs(m - 2.684e8) / 2.684e8 < 1e-3
+
+
+def test_algorithmic_bytes_of_the_workloads():
+    mb = lambda b: round(b / 1e6, 1)
+    assert mb(bench.prefill_bytes("gdn", 2, 8192, 16, 128, 128)) == 272.6
+    assert mb(bench.prefill_bytes("gla", 2, 8192, 16, 128, 128)) == 404.8
+    assert mb(bench.prefill_bytes("elu", 1, 32768, 16, 128, 64, with_S0=True, with_z=True)) == 403.7
+    assert mb(bench.decode_bytes("gla", 256, 16, 128, 128)) == 543.2
+    assert mb(bench.decode_bytes("gdn", 256, 16, 128, 128)) == 541.1
+
+
+def test_macs_per_token_head():
+    # C=64: causal pairs P = 2080; GLA = P(dk+dv)/C + 2 dk dv
+    assert bench.macs_per_token_head("gla", 128, 128) == 2080 * 256 / 64 + 2 * 128 * 128
+    assert math.isclose(bench.macs_per_token_head("gdn", 128, 128),
+                        41088 + 31.5 * 128 + 31.5 * 256 + 128 * 128)
+    assert math.isclose(bench.macs_per_token_head("elu", 128, 64), 22912.5)
+
+
+def test_reference_arm_sample_runs():
+    dt, tokens = bench.oracle_sample(16)
+    assert tokens == 32 and dt > 0
