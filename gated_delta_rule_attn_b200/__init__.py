@@ -126,9 +126,26 @@ def make_fwd_args(rule, q, k, v, g=None, beta=None, S0=None, z0=None, eps=1e-6,
     return a
 
 
+_WORKSPACES = {}
+
+
+def _workspace(device, stream_handle: int, nbytes: int):
+    """Scratch for la_fwd, cached per (device, stream): calls on one stream are
+    ordered, so they can share it."""
+    key = (device.index, stream_handle)
+    ws = _WORKSPACES.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        _WORKSPACES[key] = ws
+    return ws
+
+
 def fwd(rule: str, q, k, v, g=None, beta=None, S0=None, z0=None, eps: float = 1e-6,
-        o=None, S_out=None, z_out=None, stream=None, want_state: bool = True):
-    """Chunked prefill: returns (o, S_out, z_out-or-None). Enqueued on the current stream."""
+        o=None, S_out=None, z_out=None, stream=None, want_state: bool = True, workspace=None):
+    """Chunked prefill: returns (o, S_out, z_out-or-None). Enqueued on the current stream.
+
+    ``workspace`` (a CUDA uint8 tensor of at least ``fwd_workspace_size`` bytes)
+    is allocated and cached per stream when not given."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (S0, "S0"), (z0, "z0")):
@@ -142,7 +159,13 @@ def fwd(rule: str, q, k, v, g=None, beta=None, S0=None, z0=None, eps: float = 1e
     if rule == "elu" and z_out is None and want_state:
         z_out = torch.empty(B, H, dk, dtype=torch.float32, device=q.device)
     a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, eps, o, S_out, z_out)
-    _check(lib().la_fwd(ctypes.byref(a), _stream_handle(stream)))
+    sh = _stream_handle(stream)
+    n = ctypes.c_size_t()
+    _check(lib().la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    if n.value:
+        ws = workspace if workspace is not None else _workspace(q.device, sh.value or 0, n.value)
+        a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
+    _check(lib().la_fwd(ctypes.byref(a), sh))
     return o, S_out, z_out
 
 

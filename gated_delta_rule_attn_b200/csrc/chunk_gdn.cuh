@@ -1,0 +1,777 @@
+// chunk_gdn.cuh — gated delta rule, chunked prefill: two kernels.
+//
+// gdn_prep_kernel (fully parallel over (batch, head, chunk)): for each 64-token
+//   chunk, the state-independent triangular system of the WY / UT form:
+//     A = diag(beta) (K K^T o Gamma o strict-lower)   (K K^T on tcgen05),
+//     T = (I + A)^-1   (16x16 diagonal blocks by substitution, then two levels of
+//                       block merges on mma.sync tf32),
+//   and writes T diag(beta) and T diag(beta gamma) as bf16 operand images
+//   (128-byte swizzled, exactly as the main kernel's shared memory wants them)
+//   to the workspace: 16 KB per (batch, head, chunk).
+//
+// chunk_gdn_kernel (one CTA per (batch, head, 32-column value slab), 9 warps):
+//   warp 0      producer: TMA loads of q, k, v and a bulk copy of the chunk's
+//               T images (3 stages); alpha / beta into shared memory;
+//   warps 1-4   "local" group, one chunk ahead of the state group:
+//                 [Q;K] K^T (tcgen05, M=128) -> P = (Q K^T) o Gamma o M,
+//                 U = T diag(beta) V  and  W_k = T diag(beta gamma) K (tcgen05);
+//   warps 5-8   "state" group, the recurrence across chunks:
+//                 X1 = W_k S0, X2 = Q S0 (S0 as a bf16 operand),
+//                 W = U - X1,  dS = K^T diag(gamma_C/gamma) W,  PW = P W,
+//                 S <- gamma_C S + dS (fp32, one state row per thread),
+//                 O = diag(gamma) X2 + PW.
+// The derivation of the WY / UT form is in chunk_tc.cuh's header.
+//
+// Pairwise decays Gamma_ti = gamma_t / gamma_i (i <= t) are products of
+// gamma_t = exp2(b_t) and 1/gamma_i = exp2(-b_i) when the chunk's cumulative
+// log2-decay b_63 is >= -120 (both factors finite in fp32), otherwise
+// exp2(b_t - b_i) per element.  No factor overflows either way.
+//
+// Hand-offs use mbarriers (TMA transactions, tcgen05.commit, thread arrivals)
+// and named barriers inside a group; every wait is bounded.
+#pragma once
+
+#include "device.cuh"
+
+namespace la {
+namespace ck {
+namespace gdn {
+
+constexpr int NSTG = 3;
+constexpr int NTHREADS = 288;
+constexpr uint32_t TMEM_COLS = 512;
+// TMEM columns of the main kernel
+constexpr uint32_t C_SC = 0;     // 2 x 64, M=128 scores
+constexpr uint32_t C_U = 128;    // 2 x 32, M=64
+constexpr uint32_t C_WK = 192;   // 128,    M=64
+constexpr uint32_t C_X1 = 320;   // 32,     M=64
+constexpr uint32_t C_X2 = 352;   // 2 x 32, M=64
+constexpr uint32_t C_PW = 416;   // 2 x 32, M=64
+constexpr uint32_t C_DS = 480;   // 32,     M=128
+
+constexpr uint32_t TT_BYTES = 16384;                 // T diag(beta) | T diag(beta gamma), bf16
+
+// Main-kernel shared-memory tiles (byte offsets from a 1 KB aligned base).
+constexpr uint32_t QK_ACS = 128 * 128;               // one atom column: Q rows 0-63, K rows 64-127
+constexpr uint32_t STG_QK = 0;                       // NSTG x 2 atom columns
+constexpr uint32_t STG_QK_BYTES = 2 * QK_ACS;
+constexpr uint32_t STG_V = STG_QK + NSTG * STG_QK_BYTES;   // NSTG x [64][32] bf16, 64 B swizzle
+constexpr uint32_t STG_TT = STG_V + NSTG * 4096;           // NSTG x (T diag(beta), T diag(beta gamma))
+constexpr uint32_t TP = STG_TT + NSTG * TT_BYTES;    // 2 x P [64][64] bf16
+constexpr uint32_t TWK = TP + 2 * 8192;              // 2 x W_k [64][128] bf16 (2 atom columns)
+constexpr uint32_t TWS = TWK + 2 * 16384;            // W       [64][32] 64 B swizzle
+constexpr uint32_t TWGS = TWS + 4096;                // gamma_C/gamma W
+constexpr uint32_t TSS = TWGS + 4096;                // S       [128][32] 64 B swizzle
+constexpr uint32_t TEND = TSS + 8192;
+
+// Prep-kernel shared memory.
+constexpr int AF_LD = 68;
+constexpr int TMP_LD = 36;
+constexpr uint32_t P_K = 0;                          // 2 x K [64][128] bf16
+constexpr uint32_t P_AF = 2 * 16384;                 // A, then T, fp32 [64][AF_LD]
+constexpr uint32_t P_TMP = P_AF + 64 * AF_LD * 4;    // fp32 scratch [32][TMP_LD]
+constexpr uint32_t P_END = P_TMP + 32 * TMP_LD * 4;
+constexpr int PREP_THREADS = 128;
+
+struct GCtl {
+    uint64_t full[NSTG], empty[NSTG];
+    uint64_t sc_done[2], uw_done, lw_full[2], lw_empty[2], x1_done, ds_done;
+    uint32_t tmem_base;
+    int abort, stopL, stopS, fast;
+    float alpha[NSTG][64], beta[NSTG][64];
+    float b2[NSTG][64];            // log2 of the cumulative alpha inside the chunk
+    float gam[64], ginv[64];
+};
+
+struct PCtl {
+    uint64_t full[2], mma;
+    uint32_t tmem_base;
+    int abort, stop, fast;
+    float alpha[2][64], beta[2][64];
+    float gam[64], ginv[64], bg[64], b2[64];
+};
+
+__device__ __forceinline__ void bar_named(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// ---- mma.sync m16n8k8 tf32 (fp32 accumulate) used for the block merges ----
+__device__ __forceinline__ uint32_t tf32(float x) {
+    uint32_t u;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(u) : "f"(x));
+    return u;
+}
+// A fragment: rows r0..r0+15, cols k0..k0+7 of a row-major fp32 matrix.
+__device__ __forceinline__ void lda(uint32_t a[4], const float *M, int ld, int r0, int k0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    a[0] = tf32(M[(r0 + g) * ld + k0 + t]);
+    a[1] = tf32(M[(r0 + g + 8) * ld + k0 + t]);
+    a[2] = tf32(M[(r0 + g) * ld + k0 + t + 4]);
+    a[3] = tf32(M[(r0 + g + 8) * ld + k0 + t + 4]);
+}
+// B fragment: rows (k) k0..k0+7, cols (n) n0..n0+7 of a row-major fp32 matrix.
+__device__ __forceinline__ void ldb(uint32_t b[2], const float *M, int ld, int k0, int n0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    b[0] = tf32(M[(k0 + t) * ld + n0 + g]);
+    b[1] = tf32(M[(k0 + t + 4) * ld + n0 + g]);
+}
+__device__ __forceinline__ void mma_tf32(float c[4], const uint32_t a[4], const uint32_t b[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// Store a 16 x 16 result held as two 16x8 accumulators (scaled by s).
+__device__ __forceinline__ void stc(float *M, int ld, int r0, int c0, const float c[2][4], float s,
+                                    int lane) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int col = c0 + 8 * nt + 2 * t;
+        M[(r0 + g) * ld + col] = s * c[nt][0];
+        M[(r0 + g) * ld + col + 1] = s * c[nt][1];
+        M[(r0 + g + 8) * ld + col] = s * c[nt][2];
+        M[(r0 + g + 8) * ld + col + 1] = s * c[nt][3];
+    }
+}
+
+// Row r of a [rows][32] bf16 tile with the 64-byte swizzle (16-byte chunk c of
+// row r at chunk c ^ ((r >> 1) & 3)).
+__device__ __forceinline__ void store_row64(uint8_t *tile, int r, const float *x32) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 u;
+        u.x = pack_bf16x2(x32[8 * c + 0], x32[8 * c + 1]);
+        u.y = pack_bf16x2(x32[8 * c + 2], x32[8 * c + 3]);
+        u.z = pack_bf16x2(x32[8 * c + 4], x32[8 * c + 5]);
+        u.w = pack_bf16x2(x32[8 * c + 6], x32[8 * c + 7]);
+        *reinterpret_cast<uint4 *>(tile + r * 64 + (((c ^ (r >> 1)) & 3) << 4)) = u;
+    }
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// log2 of the cumulative product of the chunk's 64 alphas (inclusive prefix),
+// with gamma = 2^b and 1/gamma = 2^-b.  One warp, two tokens per lane.
+// Returns the fast-path flag (b_63 >= -120).
+__device__ __forceinline__ int gate_scan(const float *alpha, const float *beta, float *b2,
+                                         float *gam, float *ginv, float *bg, int lane) {
+    const float a0 = log2f(alpha[2 * lane]), a1 = log2f(alpha[2 * lane + 1]);
+    const float x1 = a0 + a1;
+    float inc = x1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += y;
+    }
+    const float e0 = inc - x1 + a0, e1 = inc;
+    if (b2) {
+        b2[2 * lane] = e0;
+        b2[2 * lane + 1] = e1;
+    }
+    const float g0 = exp2f(e0), g1 = exp2f(e1);
+    gam[2 * lane] = g0;
+    gam[2 * lane + 1] = g1;
+    ginv[2 * lane] = exp2f(-e0);
+    ginv[2 * lane + 1] = exp2f(-e1);
+    if (bg) {
+        bg[2 * lane] = beta[2 * lane] * g0;
+        bg[2 * lane + 1] = beta[2 * lane + 1] * g1;
+    }
+    const float last = __shfl_sync(0xffffffffu, e1, 31);
+    return last >= -120.f ? 1 : 0;
+}
+
+// Row t of the decayed, masked score matrix from 64 raw scores x (in place):
+//   x_i <- x_i * rowf * gamma_t / gamma_i  for i <= t (i < t if strict), else 0.
+// ncols = 32 when only the first 32 columns can be unmasked (t < 32).
+template <bool STRICT>
+__device__ __forceinline__ void decay_mask_row(float *x, int t, int ncols, float rowf, bool fast,
+                                               const float *gam, const float *ginv, const float *b2) {
+    if (fast) {
+        const float rs = rowf * gam[t];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            if (i >= ncols) { x[i] = 0.f; continue; }
+            const bool keep = STRICT ? (i < t) : (i <= t);
+            x[i] = keep ? x[i] * rs * ginv[i] : 0.f;
+        }
+    } else {
+        const float bt = b2[t];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+            if (i >= ncols) { x[i] = 0.f; continue; }
+            const bool keep = STRICT ? (i < t) : (i <= t);
+            x[i] = keep ? x[i] * rowf * exp2f(bt - b2[i]) : 0.f;
+        }
+    }
+}
+
+// T = (I + A)^-1 for a strictly lower triangular 64x64 fp32 A held in AF
+// (row stride AF_LD), in place; 128 threads (lt = 0..127) with named barriers
+// `bar` (128 threads) and `bar64` (the first 64 threads).  TMP: fp32 scratch.
+__device__ __forceinline__ void invert_unit_lower64(float *AF, float *TMP, int lt, int lane, int bar,
+                                                    int bar64) {
+    const int lw = lt >> 5;
+    // (1) 16x16 diagonal blocks by substitution, one column per thread
+    if (lt < 64) {
+        const int I = lt >> 4, jj = lt & 15;
+        const float *Ab = AF + (16 * I) * AF_LD + 16 * I;
+        float acc[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) acc[t] = (t == jj) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float ti = acc[i];
+#pragma unroll
+            for (int tt = i + 1; tt < 16; ++tt) acc[tt] = fmaf(-Ab[tt * AF_LD + i], ti, acc[tt]);
+        }
+        bar_named(bar64, 64);   // every read of the diagonal A blocks is done
+        float *Tb = AF + (16 * I) * AF_LD + 16 * I + jj;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) Tb[t * AF_LD] = acc[t];
+    }
+    bar_named(bar, 128);
+    // (2) T_10 = -D_1 A_10 D_0 and T_32 = -D_3 A_32 D_2 (two warps)
+    if (lw < 2) {
+        const int I = 2 * lw + 1, J = 2 * lw;
+        float *tw = TMP + lw * 16 * 20;
+        float y[2][4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t a[4];
+            lda(a, AF, AF_LD, 16 * I, 16 * J + 8 * ks, lane);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t bb[2];
+                ldb(bb, AF, AF_LD, 16 * J + 8 * ks, 16 * J + 8 * nt, lane);
+                mma_tf32(y[nt], a, bb);
+            }
+        }
+        stc(tw, 20, 0, 0, y, 1.f, lane);
+        __syncwarp();
+        float z[2][4] = {};
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            uint32_t a[4];
+            lda(a, AF, AF_LD, 16 * I, 16 * I + 8 * ks, lane);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t bb[2];
+                ldb(bb, tw, 20, 8 * ks, 8 * nt, lane);
+                mma_tf32(z[nt], a, bb);
+            }
+        }
+        stc(AF, AF_LD, 16 * I, 16 * J, z, -1.f, lane);
+    }
+    bar_named(bar, 128);
+    // (3) bottom-left 32x32: Z = -Y' (A_[23][01] X'), X' = T[0:32,0:32], Y' = T[32:64,32:64]
+    const int mt = lw >> 1, nh = lw & 1;
+    float m[2][4] = {};
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        if (nh == 1 && ks < 2) continue;   // X'[k][16..31] = 0 for k < 16
+        uint32_t a[4];
+        lda(a, AF, AF_LD, 32 + 16 * mt, 8 * ks, lane);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t bb[2];
+            ldb(bb, AF, AF_LD, 8 * ks, 16 * nh + 8 * nt, lane);
+            mma_tf32(m[nt], a, bb);
+        }
+    }
+    stc(TMP, TMP_LD, 16 * mt, 16 * nh, m, 1.f, lane);
+    bar_named(bar, 128);
+    float z[2][4] = {};
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        if (ks >= 2 * (mt + 1)) continue;   // Y'[16mt+r][k] = 0 for k >= 16(mt+1)
+        uint32_t a[4];
+        lda(a, AF, AF_LD, 32 + 16 * mt, 32 + 8 * ks, lane);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t bb[2];
+            ldb(bb, TMP, TMP_LD, 8 * ks, 16 * nh + 8 * nt, lane);
+            mma_tf32(z[nt], a, bb);
+        }
+    }
+    bar_named(bar, 128);   // all reads of A_[23][01] are done before it is overwritten
+    stc(AF, AF_LD, 32 + 16 * mt, 16 * nh, z, -1.f, lane);
+    bar_named(bar, 128);
+}
+
+}  // namespace gdn
+
+struct GdnPrepParams {
+    int64_t B, T, H;
+    int nchunks;
+    const float *alpha, *beta;
+    uint8_t *ws;   // [B*H*nchunks][TT_BYTES]
+};
+
+// One CTA handles (batch, head, chunk) items in a grid-stride loop; the K tile
+// of the next item is loaded while the current one is processed.
+__global__ void __launch_bounds__(gdn::PREP_THREADS)
+gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p) {
+    using namespace gdn;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    PCtl *ctl = reinterpret_cast<PCtl *>(smem_raw);
+    uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(PCtl) + (smem_u32(smem_raw) & 1023u)) -
+                     (smem_u32(smem_raw) & 1023u);
+    const uint32_t tb = smem_u32(tiles);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t items = p.B * p.H * (int64_t)p.nchunks;
+    float *AF = reinterpret_cast<float *>(tiles + P_AF);
+    float *TMP = reinterpret_cast<float *>(tiles + P_TMP);
+
+    if (tid == 0) {
+        mbar_init(&ctl->full[0], 32);
+        mbar_init(&ctl->full[1], 32);
+        mbar_init(&ctl->mma, 1);
+        ctl->abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&mapk);
+    }
+    if (warp == 0) {
+        tmem_alloc(&ctl->tmem_base, 64);
+        tc_fence_before_sync();
+    }
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+    const uint32_t tq = tmem + ((uint32_t)(32 * warp) << 16);
+
+    // warp 0: TMA of the K tile + this chunk's alpha / beta into buffer `buf`
+    auto issue = [&](int64_t w, int buf) {
+        const int64_t bh = w / p.nchunks;
+        const int c = (int)(w % p.nchunks);
+        const int64_t b = bh / p.H, h = bh % p.H;
+        const int t0 = c * C;
+        if (lane == 0) {
+            mbar_expect_tx(&ctl->full[buf], 2u * C * 128u);
+            for (int a = 0; a < KA; ++a)
+                tma_load_4d(tiles + P_K + buf * 16384 + a * (C * 128), &mapk, &ctl->full[buf], 64 * a,
+                            (int)h, t0, (int)b);
+        }
+        for (int i = lane; i < C; i += 32) {
+            const int64_t tt = (int64_t)t0 + i;
+            float al = 1.f, be = 0.f;
+            if (tt < p.T) {
+                const int64_t idx = (b * p.T + tt) * p.H + h;
+                al = p.alpha[idx];
+                be = p.beta[idx];
+            }
+            ctl->alpha[buf][i] = al;
+            ctl->beta[buf][i] = be;
+        }
+        mbar_arrive(&ctl->full[buf]);
+    };
+
+    constexpr uint32_t ID_KK = idesc_bf16(64, 64, false, false);
+    int it = 0;
+    if (warp == 0 && (int64_t)blockIdx.x < items) issue(blockIdx.x, 0);
+    for (int64_t w = blockIdx.x; w < items; w += gridDim.x, ++it) {
+        const int buf = it & 1;
+        if (tid == 0) ctl->stop = ctl->abort;   // one thread decides, everyone reads after the barrier
+        bar_named(1, 128);
+        if (ctl->stop) break;
+        if (warp == 0 && w + gridDim.x < items) issue(w + gridDim.x, buf ^ 1);
+        if (!mbar_wait(&ctl->full[buf], (uint32_t)(it >> 1) & 1u)) ctl->abort = 1;
+        if (warp == 0)
+            ctl->fast = gate_scan(ctl->alpha[buf], ctl->beta[buf], ctl->b2, ctl->gam, ctl->ginv, ctl->bg,
+                                  lane);
+        if (tid == 32) {
+            tc_fence_after_sync();
+            const uint32_t kb = tb + P_K + buf * 16384;
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                umma_bf16(tmem, desc_k(kb, C * 128, kk), desc_k(kb, C * 128, kk), ID_KK, kk > 0);
+            umma_commit(&ctl->mma);
+        }
+        bar_named(1, 128);
+        if (!mbar_wait(&ctl->mma, (uint32_t)it & 1u)) ctl->abort = 1;
+        tc_fence_after_sync();
+        {   // A = diag(beta) (K K^T o Gamma o strict-lower); rows t = 16*warp + lane (lane < 16)
+            const int t = 16 * warp + lane;
+            const int ncols = (warp < 2) ? 32 : 64;
+            float x[64];
+            tmem_ld32(tq, *reinterpret_cast<float(*)[32]>(x));
+            if (warp >= 2) tmem_ld32(tq + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+            tmem_wait_ld();
+            if (lane < 16) {
+                decay_mask_row<true>(x, t, ncols, ctl->beta[buf][t], ctl->fast != 0, ctl->gam, ctl->ginv,
+                                     ctl->b2);
+                float *arow = AF + t * AF_LD;
+#pragma unroll
+                for (int i = 0; i < 64; i += 4)
+                    *reinterpret_cast<float4 *>(arow + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+            }
+        }
+        tc_fence_before_sync();
+        bar_named(1, 128);
+        invert_unit_lower64(AF, TMP, tid, lane, 1, 2);
+        {   // T diag(beta) and T diag(beta gamma) -> workspace, 128-byte swizzled [64][64] bf16 images
+            const int t = tid >> 1, hh = tid & 1;
+            const float *Trow = AF + t * AF_LD + 32 * hh;
+            const float *be = ctl->beta[buf] + 32 * hh, *bgp = ctl->bg + 32 * hh;
+            uint8_t *dst = p.ws + w * (int64_t)TT_BYTES;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint4 u1, u2;
+                uint32_t *p1 = &u1.x, *p2 = &u2.x;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 8 * cc + 2 * e;
+                    const float t0v = Trow[j], t1v = Trow[j + 1];
+                    p1[e] = pack_bf16x2(t0v * be[j], t1v * be[j + 1]);
+                    p2[e] = pack_bf16x2(t0v * bgp[j], t1v * bgp[j + 1]);
+                }
+                const int chunk = 4 * hh + cc;
+                const uint32_t off = (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4);
+                *reinterpret_cast<uint4 *>(dst + off) = u1;
+                *reinterpret_cast<uint4 *>(dst + 8192 + off) = u2;
+            }
+        }
+        bar_named(1, 128);   // AF, gates and the K buffer are reused by the next items
+    }
+    // let a prefetched copy land before the CTA exits
+    if (warp == 0 && lane == 0) {
+        const int64_t wn = (int64_t)blockIdx.x + (int64_t)it * gridDim.x;
+        if (wn < items) (void)mbar_wait(&ctl->full[it & 1], (uint32_t)(it >> 1) & 1u);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+__global__ void __launch_bounds__(gdn::NTHREADS, 1)
+chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const uint8_t *ws) {
+    using namespace gdn;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    GCtl *ctl = reinterpret_cast<GCtl *>(smem_raw);
+    uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(GCtl) + (smem_u32(smem_raw) & 1023u)) -
+                     (smem_u32(smem_raw) & 1023u);
+    const uint32_t tb = smem_u32(tiles);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3;
+    const int nslab = (int)(p.dv / DVT);
+    const int dvt = (int)(blockIdx.x % nslab);
+    const int64_t bh = blockIdx.x / nslab;
+    const int64_t b = bh / p.H, h = bh % p.H;
+    const int nchunks = (int)((p.T + C - 1) / C);
+
+    if (tid == 0) {
+        for (int s = 0; s < NSTG; ++s) {
+            mbar_init(&ctl->full[s], 32);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->sc_done[i], 1);
+            mbar_init(&ctl->lw_full[i], 128);
+            mbar_init(&ctl->lw_empty[i], 1);
+        }
+        mbar_init(&ctl->uw_done, 1);
+        mbar_init(&ctl->x1_done, 1);
+        mbar_init(&ctl->ds_done, 1);
+        ctl->abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&maps.q);
+        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(&maps.v);
+    }
+    if (warp == 0) {
+        tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+        tc_fence_before_sync();
+    }
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+    const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16);   // this warp's TMEM lanes
+
+    constexpr uint32_t ID_SC = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t ID_U = idesc_bf16(64, DVT, false, true);
+    constexpr uint32_t ID_WK = idesc_bf16(64, DK, false, true);
+    constexpr uint32_t ID_X = idesc_bf16(64, DVT, false, true);
+    constexpr uint32_t ID_DS = idesc_bf16(128, DVT, true, true);
+
+    auto stage_qk = [&](int c) { return tb + STG_QK + (uint32_t)(c % NSTG) * STG_QK_BYTES; };
+    auto stage_v = [&](int c) { return tb + STG_V + (uint32_t)(c % NSTG) * 4096u; };
+    auto stage_tt = [&](int c) { return tb + STG_TT + (uint32_t)(c % NSTG) * TT_BYTES; };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        int issued = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NSTG;
+            if (c >= NSTG) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&ctl->empty[s], (uint32_t)((c / NSTG) - 1) & 1u);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok && lane == 0) ctl->abort = 1;
+            }
+            int stop = (lane == 0) ? ctl->abort : 0;
+            stop = __shfl_sync(0xffffffffu, stop, 0);
+            if (stop) break;
+            const int t0 = c * C;
+            if (lane == 0) {
+                mbar_expect_tx(&ctl->full[s], 2u * KA * C * 128u + C * DVT * 2u + TT_BYTES);
+                uint8_t *qk = tiles + STG_QK + s * STG_QK_BYTES;
+#pragma unroll
+                for (int a = 0; a < KA; ++a) {
+                    tma_load_4d(qk + a * QK_ACS, &maps.q, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
+                    tma_load_4d(qk + a * QK_ACS + 64 * 128, &maps.k, &ctl->full[s], 64 * a, (int)h, t0,
+                                (int)b);
+                }
+                tma_load_4d(tiles + STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, t0,
+                            (int)b);
+                bulk_load(tiles + STG_TT + s * TT_BYTES, ws + (bh * nchunks + c) * (int64_t)TT_BYTES,
+                          TT_BYTES, &ctl->full[s]);
+            }
+#pragma unroll
+            for (int i = lane; i < C; i += 32) {
+                const int64_t tt = (int64_t)t0 + i;
+                float al = 1.f, be = 0.f;
+                if (tt < p.T) {
+                    const int64_t idx = (b * p.T + tt) * p.H + h;
+                    al = p.g[idx];
+                    be = p.beta[idx];
+                }
+                ctl->alpha[s][i] = al;
+                ctl->beta[s][i] = be;
+            }
+            mbar_arrive(&ctl->full[s]);
+            issued = c + 1;
+        }
+        // let copies still in flight land before the CTA can exit
+        if (lane == 0)
+            for (int c = (issued > NSTG ? issued - NSTG : 0); c < issued; ++c)
+                (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
+    } else if (warp < 5) {
+        // ------------------------------------------------------------------ local group
+        const int lt = tid - 32, lw = warp - 1;
+        const bool leader = (lt == 0);
+        auto issue_scores = [&](int c) {
+            const uint32_t qk = stage_qk(c), kb = qk + 64 * 128;
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                umma_bf16(tmem + C_SC + 64u * (c & 1), desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk),
+                          ID_SC, kk > 0);
+            umma_commit(&ctl->sc_done[c & 1]);
+        };
+        if (leader && nchunks > 0) {
+            if (!mbar_wait(&ctl->full[0], 0)) ctl->abort = 1;
+            tc_fence_after_sync();
+            issue_scores(0);
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NSTG, pb = c & 1;
+            if (leader) ctl->stopL = ctl->abort;
+            bar_named(1, 128);
+            if (ctl->stopL) break;
+            if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
+            if (c >= 2 && !mbar_wait(&ctl->lw_empty[pb], (uint32_t)((c - 2) >> 1) & 1u)) ctl->abort = 1;
+            if (lw == 0)
+                ctl->fast = gate_scan(ctl->alpha[s], nullptr, ctl->b2[s], ctl->gam, ctl->ginv, nullptr, lane);
+            bar_named(1, 128);
+
+            // ---- scores -> P (bf16): TMEM lanes 0..63 hold Q K^T (quadrants 0 and 1)
+            if (!mbar_wait(&ctl->sc_done[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
+            tc_fence_after_sync();
+            if (quad < 2) {
+                const int t = 32 * quad + lane;
+                const int ncols = quad == 0 ? 32 : 64;
+                float x[64];
+                tmem_ld32(tq + C_SC + 64u * pb, *reinterpret_cast<float(*)[32]>(x));
+                if (quad == 1) tmem_ld32(tq + C_SC + 64u * pb + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                tmem_wait_ld();
+                decay_mask_row<false>(x, t, ncols, 1.f, ctl->fast != 0, ctl->gam, ctl->ginv, ctl->b2[s]);
+                store_row_bf16(tiles + TP + pb * 8192, t, x);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            bar_named(1, 128);
+
+            // ---- U = T diag(beta) V ; W_k = T diag(beta gamma) K ; then the next chunk's scores
+            if (leader) {
+                tc_fence_after_sync();
+                const uint32_t kb = stage_qk(c) + 64 * 128, vb = stage_v(c), tt = stage_tt(c);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + C_U + 32u * pb, desc_k(tt, C * 128, kk), desc_mn64(vb, kk), ID_U,
+                              kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + C_WK, desc_k(tt + 8192, C * 128, kk), desc_mn128(kb, QK_ACS, kk),
+                              ID_WK, kk > 0);
+                umma_commit(&ctl->uw_done);
+                if (c + 1 < nchunks) {
+                    if (!mbar_wait(&ctl->full[(c + 1) % NSTG], (uint32_t)((c + 1) / NSTG) & 1u))
+                        ctl->abort = 1;
+                    tc_fence_after_sync();
+                    issue_scores(c + 1);
+                }
+            }
+            if (!mbar_wait(&ctl->uw_done, (uint32_t)c & 1u)) ctl->abort = 1;
+            tc_fence_after_sync();
+            {
+                const int t = 16 * quad + lane;
+                float x[64];
+                uint8_t *wk = tiles + TWK + pb * 16384;
+                tmem_ld32(tq + C_WK, *reinterpret_cast<float(*)[32]>(x));
+                tmem_ld32(tq + C_WK + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                tmem_wait_ld();
+                if (lane < 16) store_row_bf16(wk, t, x);
+                tmem_ld32(tq + C_WK + 64, *reinterpret_cast<float(*)[32]>(x));
+                tmem_ld32(tq + C_WK + 96, *reinterpret_cast<float(*)[32]>(x + 32));
+                tmem_wait_ld();
+                if (lane < 16) store_row_bf16(wk + C * 128, t, x);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(&ctl->lw_full[pb]);
+        }
+    } else {
+        // ------------------------------------------------------------------ state group
+        const int st = tid - 160;
+        const bool leader = (st == 0);
+        const int d = 32 * quad + lane;        // state row (M=128 accumulators)
+        const int tr = 16 * quad + lane;       // chunk row (M=64 accumulators, lane < 16)
+        float S[DVT];
+        {
+            const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVT) : nullptr;
+#pragma unroll
+            for (int j = 0; j < DVT; j += 4) {
+                float4 x = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
+                S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+            }
+            store_row64(tiles + TSS, d, S);
+        }
+        fence_proxy_async_smem();
+        bar_named(2, 128);
+        auto issue_x = [&](int c) {
+            const uint32_t qk = stage_qk(c), wk = tb + TWK + (uint32_t)(c & 1) * 16384u, ss = tb + TSS;
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                umma_bf16(tmem + C_X1, desc_k(wk, C * 128, kk), desc_mn64(ss, kk), ID_X, kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                umma_bf16(tmem + C_X2 + 32u * (c & 1), desc_k(qk, QK_ACS, kk), desc_mn64(ss, kk), ID_X,
+                          kk > 0);
+            umma_commit(&ctl->x1_done);
+        };
+        if (leader && nchunks > 0) {
+            if (!mbar_wait(&ctl->lw_full[0], 0)) ctl->abort = 1;
+            tc_fence_after_sync();
+            issue_x(0);
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NSTG, pb = c & 1;
+            const int t0 = c * C;
+            const int nvalid = (int)min((int64_t)C, p.T - t0);
+            if (leader) ctl->stopS = ctl->abort;
+            bar_named(2, 128);
+            if (ctl->stopS) break;
+            if (!mbar_wait(&ctl->lw_full[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
+            if (!mbar_wait(&ctl->x1_done, (uint32_t)c & 1u)) ctl->abort = 1;
+            tc_fence_after_sync();
+            float gam_t = 0.f, gC;
+            {
+                float x1[DVT], u[DVT];
+                tmem_ld32(tq + C_X1, x1);
+                tmem_ld32(tq + C_U + 32u * pb, u);
+                tmem_wait_ld();
+                const float *b2 = ctl->b2[s];
+                gC = exp2f(b2[C - 1]);
+                if (lane < 16) {
+                    const float bt = b2[tr];
+                    gam_t = exp2f(bt);
+                    const float gct = exp2f(b2[C - 1] - bt);
+                    float w[DVT], wg[DVT];
+#pragma unroll
+                    for (int j = 0; j < DVT; ++j) {
+                        w[j] = u[j] - x1[j];
+                        wg[j] = w[j] * gct;
+                    }
+                    store_row64(tiles + TWS, tr, w);
+                    store_row64(tiles + TWGS, tr, wg);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            bar_named(2, 128);
+            if (leader) {
+                tc_fence_after_sync();
+                const uint32_t kb = stage_qk(c) + 64 * 128;
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + C_DS, desc_mn128(kb, QK_ACS, kk), desc_mn64(tb + TWGS, kk), ID_DS,
+                              kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + C_PW + 32u * pb, desc_k(tb + TP + pb * 8192u, C * 128, kk),
+                              desc_mn64(tb + TWS, kk), ID_X, kk > 0);
+                umma_commit(&ctl->ds_done);
+                umma_commit(&ctl->lw_empty[pb]);
+                umma_commit(&ctl->empty[s]);
+            }
+            if (!mbar_wait(&ctl->ds_done, (uint32_t)c & 1u)) ctl->abort = 1;
+            tc_fence_after_sync();
+            {
+                float ds[DVT];
+                tmem_ld32(tq + C_DS, ds);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < DVT; ++j) S[j] = fmaf(gC, S[j], ds[j]);
+                store_row64(tiles + TSS, d, S);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            bar_named(2, 128);
+            if (leader && c + 1 < nchunks) {
+                if (!mbar_wait(&ctl->lw_full[(c + 1) & 1], (uint32_t)((c + 1) >> 1) & 1u)) ctl->abort = 1;
+                tc_fence_after_sync();
+                issue_x(c + 1);
+            }
+            {
+                float x2[DVT], pw[DVT];
+                tmem_ld32(tq + C_X2 + 32u * pb, x2);
+                tmem_ld32(tq + C_PW + 32u * pb, pw);
+                tmem_wait_ld();
+                if (lane < 16 && tr < nvalid) {
+#pragma unroll
+                    for (int j = 0; j < DVT; ++j) x2[j] = fmaf(gam_t, x2[j], pw[j]);
+                    store_out_row(p.o, p, b, h, t0 + tr, dvt, x2);
+                }
+            }
+            tc_fence_before_sync();
+        }
+        if (!ctl->abort && p.S_out) {
+            float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVT);
+#pragma unroll
+            for (int j = 0; j < DVT; j += 4)
+                *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace ck
+}  // namespace la

@@ -45,6 +45,7 @@
 // stops issuing work, waits for its copies in flight and frees its TMEM.
 #pragma once
 
+#include <algorithm>
 #include <string>
 
 #include "device.cuh"
@@ -428,347 +429,32 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
     if (warp == 0) tmem_dealloc(tmem, TM_COLS);
 }
 
-// ---------------------------------------------------------------------------
-// Gated delta rule
-// ---------------------------------------------------------------------------
-struct LayoutGDN {
-    // staged: QK = KA atom columns of 128 rows (Q rows 0..63, K rows 64..127), V
-    static constexpr uint32_t QK_ACS = 128 * 128;
-    static constexpr uint32_t QK = 0;
-    static constexpr uint32_t V = QK + 2 * KA * QK_ACS;
-    static constexpr uint32_t TB = V + 2 * 4096;         // T diag(beta)        [64][64]
-    static constexpr uint32_t TBG = TB + C * 128;        // T diag(beta gamma)  [64][64]
-    static constexpr uint32_t WK = TBG + C * 128;        // W_k                 [64][DK]
-    static constexpr uint32_t ST = WK + tile_bytes(C);   // S^T                 [32][DK]
-    static constexpr uint32_t ST_ACS = DVT * 128;
-    static constexpr uint32_t P = ST + tile_bytes(DVT);  // P                   [64][64]
-    static constexpr uint32_t WT = P + C * 128;          // W^T                 [32][64]
-    static constexpr uint32_t WGT = WT + DVT * 128;      // (gamma_C/gamma W)^T [32][64]
-    static constexpr uint32_t A = WGT + DVT * 128;       // A fp32 [64][68]
-    static constexpr int A_LD = 68;
-    static constexpr uint32_t END = A + C * A_LD * 4;
-};
-
-__global__ void __launch_bounds__(NT, 1)
-chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
-    using L = LayoutGDN;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    Ctl *ctl = reinterpret_cast<Ctl *>(smem_raw);
-    uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(Ctl) + (smem_u32(smem_raw) & 1023u)) -
-                     (smem_u32(smem_raw) & 1023u);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nslab = (int)(p.dv / DVT);
-    const int dvt = (int)(blockIdx.x % nslab);
-    const int64_t bh = blockIdx.x / nslab;
-    const int64_t b = bh / p.H, h = bh % p.H;
-    const int nchunks = (int)((p.T + C - 1) / C);
-
-    if (tid == 0) {
-        mbar_init(&ctl->tma_bar[0], 1);
-        mbar_init(&ctl->tma_bar[1], 1);
-        mbar_init(&ctl->mma_bar, 1);
-        ctl->abort = 0;
-        fence_barrier_init();
-        tma_prefetch_desc(&maps.q);
-        tma_prefetch_desc(&maps.k);
-        tma_prefetch_desc(&maps.v);
-    }
-    if (warp == 0) {
-        tmem_alloc(&ctl->tmem_base, TM_COLS);
-        tc_fence_before_sync();
-    }
-    // gates of chunk 0
-    auto load_gates = [&](int t0, float &al, float &be) {
-        const int t = tid & 63;
-        const int64_t tt = t0 + t;
-        if (tt < p.T) {
-            const int64_t idx = (b * p.T + tt) * p.H + h;
-            al = p.g[idx];
-            be = p.beta[idx];
-        } else {
-            al = 1.f;
-            be = 0.f;
-        }
-    };
-    float nal = 1.f, nbe = 0.f;
-    if (nchunks > 0) load_gates(0, nal, nbe);
-    if (tid < 64) {
-        ctl->alpha[tid] = nal;
-        ctl->beta[tid] = nbe;
-    }
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem = ctl->tmem_base;
-    const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);
-
-    float S[DVT];
-    {
-        const float *src = p.S0 ? p.S0 + ((bh * DK + tid) * p.dv + dvt * DVT) : nullptr;
-#pragma unroll
-        for (int j = 0; j < DVT; j += 4) {
-            float4 x = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
-            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-        }
-    }
-    uint8_t *St = tiles + L::ST;
-    auto write_state_copy = [&]() {
-        const int a = tid >> 6, d = tid & 63;
-#pragma unroll
-        for (int j = 0; j < DVT; ++j) *elem(St + a * L::ST_ACS, j, d) = __float2bfloat16_rn(S[j]);
-    };
-    write_state_copy();
-
-    if (tid == 0 && nchunks > 0)
-        issue_loads(maps, ctl, 0, tiles + L::QK, tiles + L::QK + 64 * 128, L::QK_ACS, L::QK_ACS,
-                    tiles + L::V, nullptr, b, h, 0, dvt, false);
-
-    uint32_t mma_phase = 0;
-    constexpr uint32_t ID_QKK = idesc_bf16(128, 64, false, false);
-    constexpr uint32_t ID_U = idesc_bf16(64, DVT, false, true);
-    constexpr uint32_t ID_WK = idesc_bf16(64, DK, false, true);
-    constexpr uint32_t ID_X = idesc_bf16(64, DVT, false, false);
-    constexpr uint32_t ID_D = idesc_bf16(128, DVT, true, false);
-    // TMEM columns
-    constexpr uint32_t C_QKK = 0, C_X1 = 0, C_X2 = 32, C_U = 64, C_WK = 96, C_PW = 96, C_D = 128;
-    float *As = reinterpret_cast<float *>(tiles + L::A);
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int st = c & 1;
-        const int t0 = c * C;
-        const int nvalid = (int)min((int64_t)C, p.T - t0);
-        uint8_t *QKs = tiles + L::QK + st * (KA * L::QK_ACS);
-        uint8_t *Vs = tiles + L::V + st * 4096;
-        const uint32_t qkb = smem_u32(QKs), kb = qkb + 64 * 128, vb = smem_u32(Vs);
-
-        if (tid == 0 && c + 1 < nchunks && !ctl->abort) {
-            const int s2 = st ^ 1;
-            uint8_t *q2 = tiles + L::QK + s2 * (KA * L::QK_ACS);
-            issue_loads(maps, ctl, s2, q2, q2 + 64 * 128, L::QK_ACS, L::QK_ACS,
-                        tiles + L::V + s2 * 4096, nullptr, b, h, t0 + C, dvt, false);
-        }
-        if (c + 1 < nchunks) load_gates(t0 + C, nal, nbe);   // in flight during this chunk
-        if (!mbar_wait(&ctl->tma_bar[st], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
-
-        // ---- MMA a: [Q;K] K^T -> lanes 0..63 = Q K^T, lanes 64..127 = K K^T
-        if (tid == 0 && !ctl->abort) {
-            tc_fence_after_sync();
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem + C_QKK, desc_k(qkb, L::QK_ACS, kk), desc_k(kb, L::QK_ACS, kk), ID_QKK,
-                          kk > 0);
-            umma_commit(&ctl->mma_bar);
-        }
-        // log2 cumulative alpha (warp 0, two tokens per lane)
-        if (warp == 0) {
-            const float a0 = log2f(ctl->alpha[2 * lane]), a1 = log2f(ctl->alpha[2 * lane + 1]);
-            const float x1 = a0 + a1;
-            float inc = x1;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, inc, off);
-                if (lane >= off) inc += y;
-            }
-            const float ex = inc - x1;
-            ctl->b2[2 * lane] = ex + a0;
-            ctl->b2[2 * lane + 1] = ex + x1;
-        }
-        __syncthreads();
-        if (ctl->abort) break;
-        if (!mbar_wait(&ctl->mma_bar, mma_phase)) ctl->abort = 1;
-        mma_phase ^= 1u;
-        tc_fence_after_sync();
-        {
-            float x[64];
-            tmem_ld32(tw + C_QKK, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(tw + C_QKK + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-            tmem_wait_ld();
-            if (warp < 2) {  // row t of Q K^T -> P
-                const int t = tid;
-                const float bt = ctl->b2[t];
-#pragma unroll
-                for (int i = 0; i < 64; ++i) x[i] = (i <= t) ? x[i] * exp2f(bt - ctl->b2[i]) : 0.f;
-                store_row_bf16(tiles + L::P, t, x);
-            } else {         // row t of K K^T -> A (strictly lower, scaled by beta_t)
-                const int t = tid - 64;
-                const float bt = ctl->b2[t], be = ctl->beta[t];
-                float *arow = As + t * L::A_LD;
-#pragma unroll
-                for (int i = 0; i < 64; i += 4) {
-                    float4 v4;
-                    v4.x = (i + 0 < t) ? be * x[i + 0] * exp2f(bt - ctl->b2[i + 0]) : 0.f;
-                    v4.y = (i + 1 < t) ? be * x[i + 1] * exp2f(bt - ctl->b2[i + 1]) : 0.f;
-                    v4.z = (i + 2 < t) ? be * x[i + 2] * exp2f(bt - ctl->b2[i + 2]) : 0.f;
-                    v4.w = (i + 3 < t) ? be * x[i + 3] * exp2f(bt - ctl->b2[i + 3]) : 0.f;
-                    *reinterpret_cast<float4 *>(arow + i) = v4;
-                }
-            }
-        }
-        tc_fence_before_sync();
-        __syncthreads();
-
-        // ---- T = (I + A)^-1 by forward substitution, one column per thread (64 threads)
-        if (tid < 64) {
-            const int j = tid;
-            float col[64];
-#pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                float acc = 0.f;
-                const float *arow = As + t * L::A_LD;
-#pragma unroll
-                for (int i = 0; i < t; ++i) acc = fmaf(arow[i], col[i], acc);
-                col[t] = ((t == j) ? 1.f : 0.f) - acc;
-            }
-            const float bj = ctl->beta[j];
-            const float bgj = bj * exp2f(ctl->b2[j]);
-            uint8_t *tb = tiles + L::TB, *tbg = tiles + L::TBG;
-#pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                *elem(tb, t, j) = __float2bfloat16_rn(col[t] * bj);
-                *elem(tbg, t, j) = __float2bfloat16_rn(col[t] * bgj);
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-
-        // ---- MMA b/c: U = T diag(beta) V ; W_k = T diag(beta gamma) K
-        if (tid == 0) {
-            tc_fence_after_sync();
-            const uint32_t tb = smem_u32(tiles + L::TB), tbg = smem_u32(tiles + L::TBG);
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(tmem + C_U, desc_k(tb, C * 128, kk), desc_mn64(vb, kk), ID_U, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(tmem + C_WK, desc_k(tbg, C * 128, kk), desc_mn128(kb, L::QK_ACS, kk), ID_WK,
-                          kk > 0);
-            umma_commit(&ctl->mma_bar);
-        }
-        if (!mbar_wait(&ctl->mma_bar, mma_phase)) ctl->abort = 1;
-        mma_phase ^= 1u;
-        tc_fence_after_sync();
-        float u[DVT];
-        {
-            tmem_ld32(tw + C_U, u);
-            float x[64];
-            tmem_ld32(tw + C_WK, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(tw + C_WK + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-            tmem_wait_ld();
-            const int t = 16 * warp + lane;
-            if (lane < 16) store_row_bf16(tiles + L::WK, t, x);
-            tmem_ld32(tw + C_WK + 64, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(tw + C_WK + 96, *reinterpret_cast<float(*)[32]>(x + 32));
-            tmem_wait_ld();
-            if (lane < 16) store_row_bf16(tiles + L::WK + C * 128, t, x);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-
-        // ---- MMA d/e: X1 = W_k S0 ; X2 = Q S0
-        if (tid == 0) {
-            tc_fence_after_sync();
-            const uint32_t wkb = smem_u32(tiles + L::WK), stb = smem_u32(St);
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem + C_X1, desc_k(wkb, C * 128, kk), desc_k(stb, L::ST_ACS, kk), ID_X,
-                          kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem + C_X2, desc_k(qkb, L::QK_ACS, kk), desc_k(stb, L::ST_ACS, kk), ID_X,
-                          kk > 0);
-            umma_commit(&ctl->mma_bar);
-        }
-        if (!mbar_wait(&ctl->mma_bar, mma_phase)) ctl->abort = 1;
-        mma_phase ^= 1u;
-        tc_fence_after_sync();
-        float oi[DVT];
-        {
-            float x1[DVT];
-            tmem_ld32(tw + C_X1, x1);
-            tmem_ld32(tw + C_X2, oi);
-            tmem_wait_ld();
-            const int t = 16 * warp + lane;
-            if (lane < 16) {
-                const float bt = ctl->b2[t];
-                const float gt = exp2f(bt), gct = exp2f(ctl->b2[C - 1] - bt);
-                uint8_t *wt = tiles + L::WT, *wgt = tiles + L::WGT;
-#pragma unroll
-                for (int j = 0; j < DVT; ++j) {
-                    const float w = u[j] - x1[j];
-                    *elem(wt, j, t) = __float2bfloat16_rn(w);
-                    *elem(wgt, j, t) = __float2bfloat16_rn(w * gct);
-                    oi[j] *= gt;
-                }
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-
-        // ---- MMA f/g: PW = P W ; dS = K^T (gamma_C/gamma W)
-        if (tid == 0) {
-            tc_fence_after_sync();
-            const uint32_t pb = smem_u32(tiles + L::P), wtb = smem_u32(tiles + L::WT),
-                           wgtb = smem_u32(tiles + L::WGT);
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(tmem + C_PW, desc_k(pb, C * 128, kk), desc_k(wtb, DVT * 128, kk), ID_X,
-                          kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(tmem + C_D, desc_mn128(kb, L::QK_ACS, kk), desc_k(wgtb, DVT * 128, kk), ID_D,
-                          kk > 0);
-            umma_commit(&ctl->mma_bar);
-        }
-        if (!mbar_wait(&ctl->mma_bar, mma_phase)) ctl->abort = 1;
-        mma_phase ^= 1u;
-        tc_fence_after_sync();
-        {
-            float pw[DVT], dS[DVT];
-            tmem_ld32(tw + C_PW, pw);
-            tmem_ld32(tw + C_D, dS);
-            tmem_wait_ld();
-            const int t = 16 * warp + lane;
-            if (lane < 16 && t < nvalid) {
-#pragma unroll
-                for (int j = 0; j < DVT; ++j) oi[j] += pw[j];
-                store_out_row(p.o, p, b, h, t0 + t, dvt, oi);
-            }
-            const float gC = exp2f(ctl->b2[C - 1]);
-#pragma unroll
-            for (int j = 0; j < DVT; ++j) S[j] = fmaf(gC, S[j], dS[j]);
-            write_state_copy();
-        }
-        __syncthreads();   // everyone is done with this chunk's gates
-        if (tid < 64) {
-            ctl->alpha[tid] = nal;
-            ctl->beta[tid] = nbe;
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-        if (ctl->abort) break;
-    }
-
-    if (ctl->abort) {
-        if (tid == 0)
-            for (int s = 0; s < 2; ++s) (void)mbar_try_wait(&ctl->tma_bar[s], 0);
-    } else if (p.S_out) {
-        float *dst = p.S_out + ((bh * DK + tid) * p.dv + dvt * DVT);
-#pragma unroll
-        for (int j = 0; j < DVT; j += 4)
-            *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-    }
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, TM_COLS);
-}
-
 }  // namespace ck
+}  // namespace la
+
+#include "chunk_gdn.cuh"
+
+namespace la {
 
 // Host launcher.  Returns an la_status value (0 = ok).
-inline int launch_chunk_tc(int rule, const ChunkParams &p, cudaStream_t st, std::string *err) {
+// Device workspace the chunked path needs: the gated delta rule keeps the
+// per-chunk T diag(beta) | T diag(beta gamma) operand images (16 KB per
+// (batch, head, chunk)); the other rules need none.
+inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H) {
+    if (rule != kRuleGDN || T <= 0) return 0;
+    return (size_t)(B * H * ((T + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;
+}
+
+inline int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    return n;
+}
+
+inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_bytes, cudaStream_t st,
+                           std::string *err) {
     using namespace ck;
     if (p.dv % DVT != 0) {
         *err = "chunk kernel needs dv % 32 == 0";
@@ -793,9 +479,25 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, cudaStream_t st, std:
     const int ctl = (int)((sizeof(Ctl) + 1023) / 1024 * 1024) + 1024;
     cudaError_t e;
     if (rule == kRuleGDN) {
-        const int smem = ctl + (int)LayoutGDN::END;
-        e = allow_smem((const void *)chunk_gdn_kernel, smem);
-        if (e == cudaSuccess) chunk_gdn_kernel<<<grid, NT, smem, st>>>(m, p);
+        const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H);
+        if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
+            *err = "the gated delta rule needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
+            return 8;
+        }
+        GdnPrepParams pp{};
+        pp.B = p.B; pp.T = p.T; pp.H = p.H;
+        pp.nchunks = (int)((p.T + C - 1) / C);
+        pp.alpha = p.g; pp.beta = p.beta;
+        pp.ws = static_cast<uint8_t *>(ws);
+        const int64_t items = p.B * p.H * (int64_t)pp.nchunks;
+        const int psmem = (int)((sizeof(gdn::PCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::P_END;
+        const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * 4);
+        e = allow_smem((const void *)gdn_prep_kernel, psmem);
+        if (e == cudaSuccess) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.k, pp);
+        const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::TEND;
+        if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel, smem);
+        if (e == cudaSuccess)
+            chunk_gdn_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, p, static_cast<const uint8_t *>(ws));
     } else if (rule == kRuleGLA) {
         const int smem = ctl + (int)LayoutGE<kRuleGLA>::END;
         e = allow_smem((const void *)chunk_ge_kernel<kRuleGLA>, smem);

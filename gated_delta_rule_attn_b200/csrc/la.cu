@@ -171,6 +171,8 @@ cudaError_t allow_smem(const void *kernel, int bytes) {
 
 namespace {
 
+bool uses_chunk_kernels(const la_fwd_args &a) { return a.dtype == LA_BF16 && a.dk == 128 && a.T > 0; }
+
 la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
     const Shape s{a.B, a.T, a.H, a.dk, a.dv};
     if (a.T == 0) {
@@ -188,14 +190,15 @@ la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
         }
         return ok();
     }
-    if (a.dtype == LA_BF16 && a.dk == 128) {
+    if (uses_chunk_kernels(a)) {
         la::ChunkParams p{};
         p.B = a.B; p.T = a.T; p.H = a.H; p.dv = a.dv;
         p.q = a.q; p.k = a.k; p.v = a.v; p.g = a.g; p.beta = a.beta;
         p.S0 = a.S0; p.z0 = a.z0; p.S_out = a.S_out; p.z_out = a.z_out;
         p.o = a.o; p.eps = a.eps;
         std::string err;
-        const la_status r = (la_status)la::launch_chunk_tc((int)a.rule, p, st, &err);
+        const la_status r =
+            (la_status)la::launch_chunk_tc((int)a.rule, p, a.workspace, a.workspace_bytes, st, &err);
         if (r != LA_OK) return fail(r, err);
         return check_launch("chunk kernel launch");
     }
@@ -234,6 +237,12 @@ extern "C" {
 la_status la_fwd(const la_fwd_args *args, void *stream) {
     la_status r = validate_fwd(args, true);
     if (r != LA_OK) return r;
+    if (uses_chunk_kernels(*args)) {
+        const size_t need = la::chunk_workspace_bytes((int)args->rule, args->B, args->T, args->H);
+        if (need && (!args->workspace || args->workspace_bytes < need || !aligned16(args->workspace)))
+            return fail(LA_ERR_WORKSPACE,
+                        "workspace missing, misaligned or smaller than la_fwd_workspace_size()");
+    }
     return launch_fwd(*args, static_cast<cudaStream_t>(stream));
 }
 
@@ -241,7 +250,9 @@ la_status la_fwd_workspace_size(const la_fwd_args *args, size_t *bytes) {
     if (!bytes) return fail(LA_ERR_INVALID_ARG, "bytes is NULL");
     la_status r = validate_fwd(args, false);
     if (r != LA_OK) return r;
-    *bytes = 0;
+    *bytes = uses_chunk_kernels(*args)
+                 ? la::chunk_workspace_bytes((int)args->rule, args->B, args->T, args->H)
+                 : 0;
     return ok();
 }
 
@@ -271,8 +282,8 @@ la_status la_step(const la_step_args *a, void *stream) {
 
 // Host-buffer path: staging layout = each tensor at a 256-byte aligned offset.
 struct StagingLayout {
-    size_t off[10];  // q k v g beta S0 z0 o S_out z_out
-    size_t bytes[10];
+    size_t off[11];  // q k v g beta S0 z0 o S_out z_out workspace
+    size_t bytes[11];
     size_t total;
 };
 
@@ -283,11 +294,14 @@ static void staging_layout(const la_fwd_args *a, StagingLayout *L) {
     if (a->g) gb = tok * (a->rule == LA_RULE_GLA ? (size_t)a->dk : 1) * 4;
     const size_t sb = (size_t)(a->B * a->H * a->dk * a->dv) * 4;
     const size_t zb = (size_t)(a->B * a->H * a->dk) * 4;
-    const size_t b[10] = {tok * a->dk * es, tok * a->dk * es, tok * a->dv * es, gb,
+    const size_t wb = uses_chunk_kernels(*a)
+                          ? la::chunk_workspace_bytes((int)a->rule, a->B, a->T, a->H)
+                          : 0;
+    const size_t b[11] = {tok * a->dk * es, tok * a->dk * es, tok * a->dv * es, gb,
                           a->beta ? tok * 4 : 0, a->S0 ? sb : 0, a->z0 ? zb : 0,
-                          tok * a->dv * es, a->S_out ? sb : 0, a->z_out ? zb : 0};
+                          tok * a->dv * es, a->S_out ? sb : 0, a->z_out ? zb : 0, wb};
     size_t o = 0;
-    for (int i = 0; i < 10; ++i) {
+    for (int i = 0; i < 11; ++i) {
         L->off[i] = o;
         L->bytes[i] = b[i];
         o += (b[i] + 255) & ~(size_t)255;
@@ -316,8 +330,8 @@ la_status la_fwd_host(const la_fwd_args *h, void *staging, size_t staging_bytes,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *base = static_cast<char *>(staging);
     const void *src[7] = {h->q, h->k, h->v, h->g, h->beta, h->S0, h->z0};
-    void *dptr[10];
-    for (int i = 0; i < 10; ++i) dptr[i] = L.bytes[i] ? base + L.off[i] : nullptr;
+    void *dptr[11];
+    for (int i = 0; i < 11; ++i) dptr[i] = L.bytes[i] ? base + L.off[i] : nullptr;
     for (int i = 0; i < 7; ++i) {
         if (!L.bytes[i]) continue;
         cudaError_t e = cudaMemcpyAsync(dptr[i], src[i], L.bytes[i], cudaMemcpyHostToDevice, st);
@@ -332,6 +346,8 @@ la_status la_fwd_host(const la_fwd_args *h, void *staging, size_t staging_bytes,
     d.o = dptr[7];
     d.S_out = static_cast<float *>(dptr[8]);
     d.z_out = static_cast<float *>(dptr[9]);
+    d.workspace = dptr[10];
+    d.workspace_bytes = L.bytes[10];
     r = la_fwd(&d, stream);
     if (r != LA_OK) return r;
     void *dst[3] = {h->o, h->S_out, h->z_out};

@@ -89,7 +89,13 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *   S_out  [B,H,dk,dv] final state (written), or NULL; may alias S0
  *   z_out  ELU: [B,H,dk] final normaliser, or NULL; may alias z0
  *   workspace / workspace_bytes: device scratch of at least
- *          la_fwd_workspace_size() bytes (may be NULL when that size is 0)
+ *          la_fwd_workspace_size() bytes, 16-byte aligned (may be NULL when that
+ *          size is 0).  The gated delta rule on the tensor-core path (bf16,
+ *          dk = 128) needs 16 KB per (batch, head, 64-token chunk): the chunk's
+ *          T diag(beta) and T diag(beta gamma) operands, written by a first
+ *          kernel and read by the second within the same call.  Calls that share
+ *          one workspace must be ordered (same stream), otherwise they race.
+ *          A missing or short workspace returns LA_ERR_WORKSPACE before any launch.
  * q/k/v/o must not overlap S_out/z_out.
  */
 typedef struct la_fwd_args {
@@ -147,7 +153,8 @@ la_status la_step(const la_step_args *args, void *stream);
  * host pointer (pinned memory gives asynchronous copies).  `staging` is a
  * caller-owned device buffer of at least la_fwd_host_staging_size() bytes,
  * 256-byte aligned, into which the inputs are copied; the kernels run on it and
- * the outputs are copied back.  The call enqueues copies and kernels on
+ * the outputs are copied back; the staging also holds la_fwd's workspace.  The
+ * call enqueues copies and kernels on
  * `stream` and then synchronises that stream, so the host outputs are valid on
  * return.  Allocates nothing.
  */

@@ -93,8 +93,12 @@ def test_rule_specific_gate_checks(L):
 def test_null_args_and_workspace_query(L):
     assert L.la_fwd(None, None) == 1
     n = ctypes.c_size_t(123)
-    assert L.la_fwd_workspace_size(ctypes.byref(args()), ctypes.byref(n)) == 0
-    assert n.value == 0
+    # gated delta rule, bf16, dk=128: 16 KB of T operand images per (batch, head, 64-token chunk)
+    assert L.la_fwd_workspace_size(ctypes.byref(args(T=130)), ctypes.byref(n)) == 0
+    assert n.value == 1 * 2 * 3 * 16384
+    for a in (args("gla"), args("elu"), args(dtype=0), args(dk=64), args(T=0)):
+        assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+        assert n.value == 0
     assert L.la_fwd_workspace_size(ctypes.byref(args(dk=3)), ctypes.byref(n)) == 2
 
 
@@ -110,6 +114,12 @@ def test_step_validation(L):
     assert L.la_step(ctypes.byref(s), None) == 1           # ELU decode needs z
     s.z, s.dk = FAKE, 100
     assert L.la_step(ctypes.byref(s), None) == 2
+
+
+def test_missing_workspace_rejected_before_launch(L):
+    # the workspace check happens on the host, before anything is launched
+    assert call(L, args(T=64))[0] == 8
+    assert call(L, args(T=64, workspace=FAKE, workspace_bytes=100))[0] == 8
 
 
 def test_host_staging_layout(L):
