@@ -41,13 +41,13 @@ constexpr int NSTG = 3;
 constexpr int NTHREADS = 288;
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns of the main kernel
-constexpr uint32_t C_SC = 0;     // 2 x 64, M=128 scores
-constexpr uint32_t C_U = 128;    // 2 x 32, M=64
-constexpr uint32_t C_WK = 192;   // 128,    M=64
-constexpr uint32_t C_X1 = 320;   // 32,     M=64
-constexpr uint32_t C_X2 = 352;   // 2 x 32, M=64
-constexpr uint32_t C_PW = 416;   // 2 x 32, M=64
-constexpr uint32_t C_DS = 480;   // 32,     M=128
+constexpr uint32_t C_SC = 0;     // 64,     M=128 scores [Q;K] K^T
+constexpr uint32_t C_U = 64;     // 2 x 32, M=64
+constexpr uint32_t C_WK = 128;   // 128,    M=64
+constexpr uint32_t C_X1 = 256;   // 32,     M=64
+constexpr uint32_t C_X2 = 288;   // 2 x 32, M=64
+constexpr uint32_t C_PW = 352;   // 2 x 32, M=64
+constexpr uint32_t C_DS = 416;   // 32,     M=128
 
 constexpr uint32_t TT_BYTES = 16384;                 // T diag(beta) | T diag(beta gamma), bf16
 
@@ -75,12 +75,13 @@ constexpr int PREP_THREADS = 128;
 
 struct GCtl {
     uint64_t full[NSTG], empty[NSTG];
-    uint64_t sc_done[2], uw_done, lw_full[2], lw_empty[2], x1_done, ds_done;
+    uint64_t l_done, lw_full[2], lw_empty[2], x1_done, ds_done;
     uint32_t tmem_base;
-    int abort, stopL, stopS, fast;
-    float alpha[NSTG][64], beta[NSTG][64];
-    float b2[NSTG][64];            // log2 of the cumulative alpha inside the chunk
-    float gam[64], ginv[64];
+    int abort, stopL, stopS;
+    int fast[NSTG];
+    // per stage: b = log2 of the inclusive cumulative alpha, gamma = 2^b,
+    // 1/gamma and gamma_C/gamma (written by the producer)
+    float b2[NSTG][64], gam[NSTG][64], ginv[NSTG][64], gct[NSTG][64];
 };
 
 struct PCtl {
@@ -171,9 +172,10 @@ __device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint
 // log2 of the cumulative product of the chunk's 64 alphas (inclusive prefix),
 // with gamma = 2^b and 1/gamma = 2^-b.  One warp, two tokens per lane.
 // Returns the fast-path flag (b_63 >= -120).
-__device__ __forceinline__ int gate_scan(const float *alpha, const float *beta, float *b2,
+// `al` holds this lane's two alphas (tokens 2*lane and 2*lane+1).
+__device__ __forceinline__ int gate_scan(const float *al, const float *beta, float *b2,
                                          float *gam, float *ginv, float *bg, int lane) {
-    const float a0 = log2f(alpha[2 * lane]), a1 = log2f(alpha[2 * lane + 1]);
+    const float a0 = log2f(al[0]), a1 = log2f(al[1]);
     const float x1 = a0 + a1;
     float inc = x1;
 #pragma unroll
@@ -395,8 +397,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         if (warp == 0 && w + gridDim.x < items) issue(w + gridDim.x, buf ^ 1);
         if (!mbar_wait(&ctl->full[buf], (uint32_t)(it >> 1) & 1u)) ctl->abort = 1;
         if (warp == 0)
-            ctl->fast = gate_scan(ctl->alpha[buf], ctl->beta[buf], ctl->b2, ctl->gam, ctl->ginv, ctl->bg,
-                                  lane);
+            ctl->fast = gate_scan(&ctl->alpha[buf][2 * lane], ctl->beta[buf], ctl->b2, ctl->gam, ctl->ginv,
+                                  ctl->bg, lane);
         if (tid == 32) {
             tc_fence_after_sync();
             const uint32_t kb = tb + P_K + buf * 16384;
@@ -483,11 +485,10 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             mbar_init(&ctl->empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&ctl->sc_done[i], 1);
             mbar_init(&ctl->lw_full[i], 128);
             mbar_init(&ctl->lw_empty[i], 1);
         }
-        mbar_init(&ctl->uw_done, 1);
+        mbar_init(&ctl->l_done, 1);
         mbar_init(&ctl->x1_done, 1);
         mbar_init(&ctl->ds_done, 1);
         ctl->abort = 0;
@@ -544,18 +545,20 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 bulk_load(tiles + STG_TT + s * TT_BYTES, ws + (bh * nchunks + c) * (int64_t)TT_BYTES,
                           TT_BYTES, &ctl->full[s]);
             }
+            // the chunk's decay factors: b = log2 of the inclusive cumulative alpha,
+            // gamma = 2^b, 1/gamma, gamma_C/gamma = 2^(b_63 - b)
+            float al[2];
 #pragma unroll
-            for (int i = lane; i < C; i += 32) {
-                const int64_t tt = (int64_t)t0 + i;
-                float al = 1.f, be = 0.f;
-                if (tt < p.T) {
-                    const int64_t idx = (b * p.T + tt) * p.H + h;
-                    al = p.g[idx];
-                    be = p.beta[idx];
-                }
-                ctl->alpha[s][i] = al;
-                ctl->beta[s][i] = be;
+            for (int e = 0; e < 2; ++e) {
+                const int64_t tt = (int64_t)t0 + 2 * lane + e;
+                al[e] = (tt < p.T) ? p.g[(b * p.T + tt) * p.H + h] : 1.f;
             }
+            const int fast = gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
+            const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
+            __syncwarp();
+            ctl->gct[s][2 * lane] = exp2f(blast - ctl->b2[s][2 * lane]);
+            ctl->gct[s][2 * lane + 1] = exp2f(blast - ctl->b2[s][2 * lane + 1]);
+            if (lane == 0) ctl->fast[s] = fast;
             mbar_arrive(&ctl->full[s]);
             issued = c + 1;
         }
@@ -565,21 +568,8 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
     } else if (warp < 5) {
         // ------------------------------------------------------------------ local group
-        const int lt = tid - 32, lw = warp - 1;
+        const int lt = tid - 32;
         const bool leader = (lt == 0);
-        auto issue_scores = [&](int c) {
-            const uint32_t qk = stage_qk(c), kb = qk + 64 * 128;
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem + C_SC + 64u * (c & 1), desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk),
-                          ID_SC, kk > 0);
-            umma_commit(&ctl->sc_done[c & 1]);
-        };
-        if (leader && nchunks > 0) {
-            if (!mbar_wait(&ctl->full[0], 0)) ctl->abort = 1;
-            tc_fence_after_sync();
-            issue_scores(0);
-        }
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTG, pb = c & 1;
             if (leader) ctl->stopL = ctl->abort;
@@ -587,61 +577,48 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             if (ctl->stopL) break;
             if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
             if (c >= 2 && !mbar_wait(&ctl->lw_empty[pb], (uint32_t)((c - 2) >> 1) & 1u)) ctl->abort = 1;
-            if (lw == 0)
-                ctl->fast = gate_scan(ctl->alpha[s], nullptr, ctl->b2[s], ctl->gam, ctl->ginv, nullptr, lane);
-            bar_named(1, 128);
 
-            // ---- scores -> P (bf16): TMEM lanes 0..63 hold Q K^T (quadrants 0 and 1)
-            if (!mbar_wait(&ctl->sc_done[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
+            // ---- [Q;K] K^T ; U = T diag(beta) V ; W_k = T diag(beta gamma) K
+            if (leader) {
+                tc_fence_after_sync();
+                const uint32_t qk = stage_qk(c), kb = qk + 64 * 128, vb = stage_v(c), tt = stage_tt(c);
+                // three independent accumulations, interleaved so that consecutive
+                // instructions never wait on the same accumulator
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    umma_bf16(tmem + C_SC, desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk), ID_SC, kk > 0);
+                    if (kk < C / 16) {
+                        umma_bf16(tmem + C_WK, desc_k(tt + 8192, C * 128, kk), desc_mn128(kb, QK_ACS, kk),
+                                  ID_WK, kk > 0);
+                        umma_bf16(tmem + C_U + 32u * pb, desc_k(tt, C * 128, kk), desc_mn64(vb, kk), ID_U,
+                                  kk > 0);
+                    }
+                }
+                umma_commit(&ctl->l_done);
+            }
+            if (!mbar_wait(&ctl->l_done, (uint32_t)c & 1u)) ctl->abort = 1;
             tc_fence_after_sync();
+
+            // ---- P = (Q K^T) o Gamma o M: TMEM lanes 0..63 (quadrants 0 and 1), one row per thread
             if (quad < 2) {
                 const int t = 32 * quad + lane;
                 const int ncols = quad == 0 ? 32 : 64;
                 float x[64];
-                tmem_ld32(tq + C_SC + 64u * pb, *reinterpret_cast<float(*)[32]>(x));
-                if (quad == 1) tmem_ld32(tq + C_SC + 64u * pb + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                tmem_ld32(tq + C_SC, *reinterpret_cast<float(*)[32]>(x));
+                if (quad == 1) tmem_ld32(tq + C_SC + 32, *reinterpret_cast<float(*)[32]>(x + 32));
                 tmem_wait_ld();
-                decay_mask_row<false>(x, t, ncols, 1.f, ctl->fast != 0, ctl->gam, ctl->ginv, ctl->b2[s]);
+                decay_mask_row<false>(x, t, ncols, 1.f, ctl->fast[s] != 0, ctl->gam[s], ctl->ginv[s],
+                                      ctl->b2[s]);
                 store_row_bf16(tiles + TP + pb * 8192, t, x);
             }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            bar_named(1, 128);
-
-            // ---- U = T diag(beta) V ; W_k = T diag(beta gamma) K ; then the next chunk's scores
-            if (leader) {
-                tc_fence_after_sync();
-                const uint32_t kb = stage_qk(c) + 64 * 128, vb = stage_v(c), tt = stage_tt(c);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + C_U + 32u * pb, desc_k(tt, C * 128, kk), desc_mn64(vb, kk), ID_U,
-                              kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + C_WK, desc_k(tt + 8192, C * 128, kk), desc_mn128(kb, QK_ACS, kk),
-                              ID_WK, kk > 0);
-                umma_commit(&ctl->uw_done);
-                if (c + 1 < nchunks) {
-                    if (!mbar_wait(&ctl->full[(c + 1) % NSTG], (uint32_t)((c + 1) / NSTG) & 1u))
-                        ctl->abort = 1;
-                    tc_fence_after_sync();
-                    issue_scores(c + 1);
-                }
-            }
-            if (!mbar_wait(&ctl->uw_done, (uint32_t)c & 1u)) ctl->abort = 1;
-            tc_fence_after_sync();
+            // ---- W_k -> bf16: row t = 16*quad + (lane & 15); lanes 0-15 columns 0-63, 16-31 columns 64-127
             {
-                const int t = 16 * quad + lane;
+                const int t = 16 * quad + (lane & 15), hf = lane >> 4;
                 float x[64];
-                uint8_t *wk = tiles + TWK + pb * 16384;
-                tmem_ld32(tq + C_WK, *reinterpret_cast<float(*)[32]>(x));
-                tmem_ld32(tq + C_WK + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+                tmem_ld16x2_32<64>(tq + C_WK, *reinterpret_cast<float(*)[32]>(x));
+                tmem_ld16x2_32<64>(tq + C_WK + 32, *reinterpret_cast<float(*)[32]>(x + 32));
                 tmem_wait_ld();
-                if (lane < 16) store_row_bf16(wk, t, x);
-                tmem_ld32(tq + C_WK + 64, *reinterpret_cast<float(*)[32]>(x));
-                tmem_ld32(tq + C_WK + 96, *reinterpret_cast<float(*)[32]>(x + 32));
-                tmem_wait_ld();
-                if (lane < 16) store_row_bf16(wk + C * 128, t, x);
+                store_row_bf16(tiles + TWK + pb * 16384 + hf * 8192, t, x);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -651,8 +628,9 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         // ------------------------------------------------------------------ state group
         const int st = tid - 160;
         const bool leader = (st == 0);
-        const int d = 32 * quad + lane;        // state row (M=128 accumulators)
-        const int tr = 16 * quad + lane;       // chunk row (M=64 accumulators, lane < 16)
+        const int d = 32 * quad + lane;               // state row (M=128 accumulators)
+        const int tr = 16 * quad + (lane & 15);       // chunk row (M=64 accumulators)
+        const int hf = lane >> 4;                     // which 16 of the 32 columns
         float S[DVT];
         {
             const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVT) : nullptr;
@@ -668,13 +646,25 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         auto issue_x = [&](int c) {
             const uint32_t qk = stage_qk(c), wk = tb + TWK + (uint32_t)(c & 1) * 16384u, ss = tb + TSS;
 #pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
+            for (int kk = 0; kk < DK / 16; ++kk) {   // X1 and X2 interleaved (independent)
                 umma_bf16(tmem + C_X1, desc_k(wk, C * 128, kk), desc_mn64(ss, kk), ID_X, kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
                 umma_bf16(tmem + C_X2 + 32u * (c & 1), desc_k(qk, QK_ACS, kk), desc_mn64(ss, kk), ID_X,
                           kk > 0);
+            }
             umma_commit(&ctl->x1_done);
+        };
+        // half row (16 columns, 2 chunks of 16 B) of a [rows][32] bf16 tile, 64-byte swizzle
+        auto store_half64 = [&](uint32_t tile_off, int r, const float *x16) {
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c = 2 * hf + cc;
+                uint4 u;
+                u.x = pack_bf16x2(x16[8 * cc + 0], x16[8 * cc + 1]);
+                u.y = pack_bf16x2(x16[8 * cc + 2], x16[8 * cc + 3]);
+                u.z = pack_bf16x2(x16[8 * cc + 4], x16[8 * cc + 5]);
+                u.w = pack_bf16x2(x16[8 * cc + 6], x16[8 * cc + 7]);
+                *reinterpret_cast<uint4 *>(tiles + tile_off + r * 64 + (((c ^ (r >> 1)) & 3) << 4)) = u;
+            }
         };
         if (leader && nchunks > 0) {
             if (!mbar_wait(&ctl->lw_full[0], 0)) ctl->abort = 1;
@@ -691,27 +681,20 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             if (!mbar_wait(&ctl->lw_full[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
             if (!mbar_wait(&ctl->x1_done, (uint32_t)c & 1u)) ctl->abort = 1;
             tc_fence_after_sync();
-            float gam_t = 0.f, gC;
-            {
-                float x1[DVT], u[DVT];
-                tmem_ld32(tq + C_X1, x1);
-                tmem_ld32(tq + C_U + 32u * pb, u);
+            const float gam_t = ctl->gam[s][tr], gC = ctl->gam[s][C - 1];
+            {   // W = U - X1 and (gamma_C / gamma) W, rows tr, columns 16*hf..
+                float x1[16], u[16], w[16], wg[16];
+                tmem_ld16x2_16<16>(tq + C_X1, x1);
+                tmem_ld16x2_16<16>(tq + C_U + 32u * pb, u);
                 tmem_wait_ld();
-                const float *b2 = ctl->b2[s];
-                gC = exp2f(b2[C - 1]);
-                if (lane < 16) {
-                    const float bt = b2[tr];
-                    gam_t = exp2f(bt);
-                    const float gct = exp2f(b2[C - 1] - bt);
-                    float w[DVT], wg[DVT];
+                const float gct = ctl->gct[s][tr];
 #pragma unroll
-                    for (int j = 0; j < DVT; ++j) {
-                        w[j] = u[j] - x1[j];
-                        wg[j] = w[j] * gct;
-                    }
-                    store_row64(tiles + TWS, tr, w);
-                    store_row64(tiles + TWGS, tr, wg);
+                for (int j = 0; j < 16; ++j) {
+                    w[j] = u[j] - x1[j];
+                    wg[j] = w[j] * gct;
                 }
+                store_half64(TWS, tr, w);
+                store_half64(TWGS, tr, wg);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -720,13 +703,12 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 tc_fence_after_sync();
                 const uint32_t kb = stage_qk(c) + 64 * 128;
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
+                for (int kk = 0; kk < C / 16; ++kk) {   // dS and PW interleaved (independent)
                     umma_bf16(tmem + C_DS, desc_mn128(kb, QK_ACS, kk), desc_mn64(tb + TWGS, kk), ID_DS,
                               kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
                     umma_bf16(tmem + C_PW + 32u * pb, desc_k(tb + TP + pb * 8192u, C * 128, kk),
                               desc_mn64(tb + TWS, kk), ID_X, kk > 0);
+                }
                 umma_commit(&ctl->ds_done);
                 umma_commit(&ctl->lw_empty[pb]);
                 umma_commit(&ctl->empty[s]);
@@ -749,15 +731,25 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 tc_fence_after_sync();
                 issue_x(c + 1);
             }
-            {
-                float x2[DVT], pw[DVT];
-                tmem_ld32(tq + C_X2 + 32u * pb, x2);
-                tmem_ld32(tq + C_PW + 32u * pb, pw);
+            {   // O = diag(gamma) X2 + P W, rows tr, columns 16*hf..
+                float x2[16], pw[16];
+                tmem_ld16x2_16<16>(tq + C_X2 + 32u * pb, x2);
+                tmem_ld16x2_16<16>(tq + C_PW + 32u * pb, pw);
                 tmem_wait_ld();
-                if (lane < 16 && tr < nvalid) {
+                if (tr < nvalid) {
 #pragma unroll
-                    for (int j = 0; j < DVT; ++j) x2[j] = fmaf(gam_t, x2[j], pw[j]);
-                    store_out_row(p.o, p, b, h, t0 + tr, dvt, x2);
+                    for (int j = 0; j < 16; ++j) x2[j] = fmaf(gam_t, x2[j], pw[j]);
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
+                                         ((b * p.T + t0 + tr) * p.H + h) * p.dv + dvt * DVT + 16 * hf;
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint4 u;
+                        u.x = pack_bf16x2(x2[8 * cc + 0], x2[8 * cc + 1]);
+                        u.y = pack_bf16x2(x2[8 * cc + 2], x2[8 * cc + 3]);
+                        u.z = pack_bf16x2(x2[8 * cc + 4], x2[8 * cc + 5]);
+                        u.w = pack_bf16x2(x2[8 * cc + 6], x2[8 * cc + 7]);
+                        reinterpret_cast<uint4 *>(dst)[cc] = u;
+                    }
                 }
             }
             tc_fence_before_sync();

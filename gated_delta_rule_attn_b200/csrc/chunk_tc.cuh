@@ -77,21 +77,31 @@ constexpr int KA = DK / 64;   // 64-wide atom columns along dk
 constexpr uint32_t TM_COLS = 256;
 
 // --- descriptors --------------------------------------------------------------
+// A descriptor is built once per operand (k-step 0) and advanced per k-step by
+// adding the byte offset >> 4 to its start-address field (the tiles live below
+// 256 KB, so the 14-bit field never carries).
+__device__ __forceinline__ uint64_t dk0(uint32_t base) { return smem_desc(base, 16u, 1024u, kSwizzle128); }
+__device__ __forceinline__ uint64_t dmn128_0(uint32_t base, uint32_t lbo) {
+    return smem_desc(base, lbo, 1024u, kSwizzle128);
+}
+__device__ __forceinline__ uint64_t dmn64_0(uint32_t base) { return smem_desc(base, 4096u, 512u, kSwizzle64); }
 // K-major, 128-byte swizzle: rows of 64 elements, `acs` bytes between atom
 // columns, k-step kk covers K elements [16kk, 16kk+16).
+__device__ __forceinline__ uint64_t kstep_k(uint64_t d0, uint32_t acs, int kk) {
+    return d0 + (uint64_t)(((uint32_t)(kk >> 2) * acs + (uint32_t)(kk & 3) * 32u) >> 4);
+}
+// MN-major, 128-byte swizzle: K runs down 128-byte rows, 16 rows per k-step.
+__device__ __forceinline__ uint64_t kstep_mn128(uint64_t d0, int kk) { return d0 + (uint64_t)(kk * 128); }
+// MN-major, 64-byte swizzle (32 MN elements per 64-byte row), 16 rows per k-step.
+__device__ __forceinline__ uint64_t kstep_mn64(uint64_t d0, int kk) { return d0 + (uint64_t)(kk * 64); }
+
 __device__ __forceinline__ uint64_t desc_k(uint32_t base, uint32_t acs, int kk) {
-    const uint32_t a = base + (uint32_t)(kk >> 2) * acs + (uint32_t)(kk & 3) * 32u;
-    return smem_desc(a, 16u, 1024u, kSwizzle128);
+    return kstep_k(dk0(base), acs, kk);
 }
-// MN-major, 128-byte swizzle: K runs down the rows (128 B each), MN along the
-// row; 64-wide MN blocks are `lbo` bytes apart.
 __device__ __forceinline__ uint64_t desc_mn128(uint32_t base, uint32_t lbo, int kk) {
-    return smem_desc(base + (uint32_t)kk * 2048u, lbo, 1024u, kSwizzle128);
+    return kstep_mn128(dmn128_0(base, lbo), kk);
 }
-// MN-major, 64-byte swizzle (32 MN elements per 64-byte row).
-__device__ __forceinline__ uint64_t desc_mn64(uint32_t base, int kk) {
-    return smem_desc(base + (uint32_t)kk * 1024u, 4096u, 512u, kSwizzle64);
-}
+__device__ __forceinline__ uint64_t desc_mn64(uint32_t base, int kk) { return kstep_mn64(dmn64_0(base), kk); }
 
 __device__ __forceinline__ void store_row_bf16(uint8_t *tile, int r, const float *x64) {
     // row r of a [rows][64] SW128 tile from 64 floats (16-byte stores)
