@@ -92,9 +92,6 @@ struct PCtl {
     float gam[64], ginv[64], bg[64], b2[64];
 };
 
-__device__ __forceinline__ void bar_named(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 // ---- mma.sync m16n8k8 tf32 (fp32 accumulate) used for the block merges ----
 __device__ __forceinline__ uint32_t tf32(float x) {
@@ -155,9 +152,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
                  "r"(bytes)
                  : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 

@@ -140,309 +140,24 @@ struct Maps {
     CUtensorMap q, k, v, g;
 };
 
-// Shared bookkeeping at the start of dynamic shared memory.
-struct Ctl {
-    uint64_t tma_bar[2];
-    uint64_t mma_bar;
-    uint32_t tmem_base;
-    int abort;
-    float gC[DK];       // GLA: gamma at chunk end per key dim; ELU: z0 staging
-    float b2[C];        // GDN: log2 cumulative alpha
-    float alpha[C], beta[C];
-};
-
 __device__ __forceinline__ uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 
 // Bytes of a [rows] x DK tile as KA atom columns.
 constexpr uint32_t tile_bytes(int rows) { return (uint32_t)rows * 128u * KA; }
 
-// ---------------------------------------------------------------------------
-// Common prologue / epilogue helpers
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void issue_loads(const Maps &m, Ctl *ctl, int stage, uint8_t *qdst,
-                                            uint8_t *kdst, uint32_t q_acs, uint32_t k_acs,
-                                            uint8_t *vdst, uint8_t *gdst, int64_t b, int64_t h,
-                                            int t0, int dvt, bool has_g) {
-    const uint32_t bytes = 2u * KA * C * 128u + C * DVT * 2u + (has_g ? C * DK * 4u : 0u);
-    mbar_arrive_expect_tx(&ctl->tma_bar[stage], bytes);
-#pragma unroll
-    for (int a = 0; a < KA; ++a) {
-        tma_load_4d(qdst + a * q_acs, &m.q, &ctl->tma_bar[stage], 64 * a, (int)h, t0, (int)b);
-        tma_load_4d(kdst + a * k_acs, &m.k, &ctl->tma_bar[stage], 64 * a, (int)h, t0, (int)b);
-    }
-    tma_load_4d(vdst, &m.v, &ctl->tma_bar[stage], dvt * DVT, (int)h, t0, (int)b);
-    if (has_g) tma_load_4d(gdst, &m.g, &ctl->tma_bar[stage], 0, (int)h, t0, (int)b);
+__device__ __forceinline__ void bar_named(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
-// ---------------------------------------------------------------------------
-// GLA and ELU+1 share one kernel body (RULE selects the feature map / gates).
-// ---------------------------------------------------------------------------
-template <int RULE>
-struct LayoutGE {
-    // staged: Q, K (KA x 64 rows), V (64 x 64 B), G (GLA: 64 x DK fp32)
-    static constexpr uint32_t Q = 0;
-    static constexpr uint32_t K = Q + 2 * tile_bytes(C);
-    static constexpr uint32_t V = K + 2 * tile_bytes(C);
-    static constexpr uint32_t G = V + 2 * 4096;
-    static constexpr uint32_t GSZ = (RULE == kRuleGLA) ? C * DK * 4 : 0;
-    // Kx: [K~ or phiK (64 rows); S^T (32 rows); ELU: z^T + 7 zero rows]
-    static constexpr int KX_ROWS = (RULE == kRuleELU) ? 104 : 96;
-    static constexpr uint32_t KX = G + 2 * GSZ;
-    static constexpr uint32_t KX_ACS = KX_ROWS * 128;
-    static constexpr uint32_t P = KX + tile_bytes(KX_ROWS);
-    static constexpr uint32_t END = P + C * 128;
-    static constexpr int N1 = KX_ROWS;   // N of the score/inter MMA
-};
-
-template <int RULE>
-__global__ void __launch_bounds__(NT, 1)
-chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
-    using L = LayoutGE<RULE>;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // control block first, tiles from the next 1 KB boundary
-    Ctl *ctl = reinterpret_cast<Ctl *>(smem_raw);
-    uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(Ctl) + (smem_u32(smem_raw) & 1023u)) -
-                     (smem_u32(smem_raw) & 1023u);
-    const uint32_t tiles_s = smem_u32(tiles);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nslab = (int)(p.dv / DVT);
-    const int dvt = (int)(blockIdx.x % nslab);
-    const int64_t bh = blockIdx.x / nslab;
-    const int64_t b = bh / p.H, h = bh % p.H;
-    const int nchunks = (int)((p.T + C - 1) / C);
-
-    if (tid == 0) {
-        mbar_init(&ctl->tma_bar[0], 1);
-        mbar_init(&ctl->tma_bar[1], 1);
-        mbar_init(&ctl->mma_bar, 1);
-        ctl->abort = 0;
-        fence_barrier_init();
-        tma_prefetch_desc(&maps.q);
-        tma_prefetch_desc(&maps.k);
-        tma_prefetch_desc(&maps.v);
-        if (RULE == kRuleGLA) tma_prefetch_desc(&maps.g);
-    }
-    if (warp == 0) {
-        tmem_alloc(&ctl->tmem_base, TM_COLS);
-        tc_fence_before_sync();
-    }
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem = ctl->tmem_base;
-    const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's lane quadrant
-
-    // State slab: thread d owns row d (DVT fp32 values).
-    float S[DVT];
-    {
-        const float *src = p.S0 ? p.S0 + ((bh * DK + tid) * p.dv + dvt * DVT) : nullptr;
-#pragma unroll
-        for (int j = 0; j < DVT; j += 4) {
-            float4 x = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
-            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-        }
-    }
-    float z = 0.f;  // ELU: normaliser z_d for d = tid
-    if (RULE == kRuleELU && p.z0) z = p.z0[bh * DK + tid];
-
-    uint8_t *Kx = tiles + L::KX;
-    uint8_t *Ps = tiles + L::P;
-    // bf16 copy of S^T (and z^T for ELU) into Kx rows 64.. ; zero rows 97..103
-    auto write_state_copy = [&]() {
-        const int a = tid >> 6, d = tid & 63;
-#pragma unroll
-        for (int j = 0; j < DVT; ++j) *elem(Kx + a * L::KX_ACS, 64 + j, d) = __float2bfloat16_rn(S[j]);
-        if (RULE == kRuleELU) *elem(Kx + a * L::KX_ACS, 96, d) = __float2bfloat16_rn(z);
-    };
-    if (RULE == kRuleELU) {
-        const int a = tid >> 6, d = tid & 63;
-#pragma unroll
-        for (int r = 97; r < 104; ++r) *elem(Kx + a * L::KX_ACS, r, d) = __float2bfloat16_rn(0.f);
-    }
-    write_state_copy();
-
-    if (tid == 0 && nchunks > 0)
-        issue_loads(maps, ctl, 0, tiles + L::Q, tiles + L::K, C * 128, C * 128, tiles + L::V,
-                    tiles + L::G, b, h, 0, dvt, RULE == kRuleGLA);
-
-    uint32_t mma_phase = 0;
-    constexpr uint32_t ID_SCORE = idesc_bf16(64, L::N1, false, false);
-    constexpr uint32_t ID_UPD = idesc_bf16(128, DVT, true, true);
-    constexpr uint32_t ID_PV = idesc_bf16(64, DVT, false, true);
-    constexpr uint32_t COL_P = 0, COL_O = 64, COL_D = 128;  // TMEM columns
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int st = c & 1;
-        const int t0 = c * C;
-        const int nvalid = (int)min((int64_t)C, p.T - t0);
-        uint8_t *Qs = tiles + L::Q + st * tile_bytes(C);
-        uint8_t *Ks = tiles + L::K + st * tile_bytes(C);
-        uint8_t *Vs = tiles + L::V + st * 4096;
-        float *Gs = reinterpret_cast<float *>(tiles + L::G + st * L::GSZ);
-
-        // prefetch the next chunk into the other stage (its previous user, chunk c-1, is done)
-        if (tid == 0 && c + 1 < nchunks && !ctl->abort) {
-            const int s2 = st ^ 1;
-            issue_loads(maps, ctl, s2, tiles + L::Q + s2 * tile_bytes(C),
-                        tiles + L::K + s2 * tile_bytes(C), C * 128, C * 128,
-                        tiles + L::V + s2 * 4096, tiles + L::G + s2 * L::GSZ, b, h, t0 + C, dvt,
-                        RULE == kRuleGLA);
-        }
-        if (!mbar_wait(&ctl->tma_bar[st], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
-
-        // ---- feature map / gates on CUDA cores: thread tid owns key dim d = tid
-        {
-            const int d = tid, a = d >> 6, dc = d & 63;
-            uint8_t *qa = Qs + a * (C * 128), *ka = Ks + a * (C * 128), *kxa = Kx + a * L::KX_ACS;
-            if constexpr (RULE == kRuleGLA) {
-                float gam = 1.f;
-                for (int t = 0; t < C; ++t) {
-                    const float gt = (t < nvalid) ? Gs[t * DK + d] : 1.f;
-                    gam *= gt;
-                    Gs[t * DK + d] = gam;
-                }
-                const float gC = gam;
-                if (!(gC >= 1e-30f)) raise_error(kErrRange);
-                for (int t = 0; t < C; ++t) {
-                    const float gm = Gs[t * DK + d];
-                    const float inv = 1.f / gm;
-                    __nv_bfloat16 *qe = elem(qa, t, dc), *ke = elem(ka, t, dc);
-                    const float qv = __bfloat162float(*qe), kv = __bfloat162float(*ke);
-                    *qe = __float2bfloat16_rn(qv * gm);                 // Qt (in place)
-                    *elem(kxa, t, dc) = __float2bfloat16_rn(kv * inv);   // Kt
-                    *ke = __float2bfloat16_rn(kv * (inv * gC));          // Kh (in place)
-                }
-                ctl->gC[d] = gC;
-            } else {  // ELU+1
-                float zs = 0.f;
-                for (int t = 0; t < C; ++t) {
-                    __nv_bfloat16 *qe = elem(qa, t, dc);
-                    const float pq = elu_feature(__bfloat162float(*qe));
-                    const float pk = (t < nvalid) ? elu_feature(__bfloat162float(*elem(ka, t, dc))) : 0.f;
-                    *qe = __float2bfloat16_rn(pq);
-                    const __nv_bfloat16 pkb = __float2bfloat16_rn(pk);
-                    *elem(kxa, t, dc) = pkb;
-                    zs += pk;
-                }
-                ctl->gC[d] = zs;   // chunk sum of phi(k) for dim d
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-        if (ctl->abort) break;
-
-        // ---- MMA 1: [P | O_inter (| den_inter)] = Q' [K' ; S^T (; z^T)]^T ; MMA 2: dS = K''^T V
-        if (tid == 0) {
-            tc_fence_after_sync();
-            const uint32_t qb = smem_u32(Qs), kxb = smem_u32(Kx);
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem + COL_P, desc_k(qb, C * 128, kk), desc_k(kxb, L::KX_ACS, kk), ID_SCORE,
-                          kk > 0);
-            // update operand: GLA uses Kh (in place in Ks); ELU uses phiK (Kx rows 0..63)
-            const uint32_t ub = (RULE == kRuleGLA) ? smem_u32(Ks) : kxb;
-            const uint32_t ulbo = (RULE == kRuleGLA) ? (uint32_t)(C * 128) : L::KX_ACS;
-            const uint32_t vb = smem_u32(Vs);
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(tmem + COL_D, desc_mn128(ub, ulbo, kk), desc_mn64(vb, kk), ID_UPD, kk > 0);
-            umma_commit(&ctl->mma_bar);
-        }
-        if (!mbar_wait(&ctl->mma_bar, mma_phase)) ctl->abort = 1;
-        mma_phase ^= 1u;
-        tc_fence_after_sync();
-
-        // ---- P (rows 16w+lane for lane < 16), masked -> bf16; den (ELU); state update
-        float den = 0.f;
-        {
-            float x[64];
-            tmem_ld32(tw + COL_P, *reinterpret_cast<float(*)[32]>(x));
-            tmem_ld32(tw + COL_P + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-            float dI[16];
-            if (RULE == kRuleELU) tmem_ld16(tw + 96, dI);   // col 96 = phiQ z0
-            float dS[DVT];
-            tmem_ld32(tw + COL_D, *reinterpret_cast<float(*)[32]>(dS));
-            tmem_wait_ld();
-            const int t = 16 * warp + lane;
-            if (lane < 16) {
-                float rs = 0.f;
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    x[i] = (i <= t) ? x[i] : 0.f;
-                    rs += x[i];
-                }
-                store_row_bf16(Ps, t, x);
-                if (RULE == kRuleELU) den = dI[0] + rs + p.eps;
-            }
-            // S <- diag(gamma_C) S + dS (GLA) / S + dS (ELU); thread tid owns row tid
-            const float gC = ctl->gC[tid];
-            if (RULE == kRuleGLA) {
-#pragma unroll
-                for (int j = 0; j < DVT; ++j) S[j] = fmaf(gC, S[j], dS[j]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < DVT; ++j) S[j] += dS[j];
-                z += gC;
-            }
-            write_state_copy();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncthreads();
-
-        // ---- MMA 3: O += P V
-        if (tid == 0) {
-            tc_fence_after_sync();
-            const uint32_t pb = smem_u32(Ps), vb = smem_u32(Vs);
-#pragma unroll
-            for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(tmem + COL_O, desc_k(pb, C * 128, kk), desc_mn64(vb, kk), ID_PV, 1u);
-            umma_commit(&ctl->mma_bar);
-        }
-        if (!mbar_wait(&ctl->mma_bar, mma_phase)) ctl->abort = 1;
-        mma_phase ^= 1u;
-        tc_fence_after_sync();
-        {
-            float x[DVT];
-            tmem_ld32(tw + COL_O, x);
-            tmem_wait_ld();
-            const int t = 16 * warp + lane;
-            if (lane < 16 && t < nvalid) {
-                if (RULE == kRuleELU) {
-                    const float inv = 1.f / den;
-#pragma unroll
-                    for (int j = 0; j < DVT; ++j) x[j] *= inv;
-                }
-                store_out_row(p.o, p, b, h, t0 + t, dvt, x);
-            }
-        }
-        tc_fence_before_sync();
-        __syncthreads();
-        if (ctl->abort) break;
-    }
-
-    if (ctl->abort) {
-        // let any copy still in flight land before the shared memory is released
-        if (tid == 0)
-            for (int s = 0; s < 2; ++s) (void)mbar_try_wait(&ctl->tma_bar[s], 0);
-    } else {
-        if (p.S_out) {
-            float *dst = p.S_out + ((bh * DK + tid) * p.dv + dvt * DVT);
-#pragma unroll
-            for (int j = 0; j < DVT; j += 4)
-                *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-        }
-        if (RULE == kRuleELU && p.z_out && dvt == 0) p.z_out[bh * DK + tid] = z;
-    }
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, TM_COLS);
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 }  // namespace ck
 }  // namespace la
 
 #include "chunk_gdn.cuh"
+#include "chunk_ge.cuh"
 
 namespace la {
 
@@ -486,7 +201,6 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         return 4;
     }
     const unsigned grid = (unsigned)(p.B * p.H * (p.dv / DVT));
-    const int ctl = (int)((sizeof(Ctl) + 1023) / 1024 * 1024) + 1024;
     cudaError_t e;
     if (rule == kRuleGDN) {
         const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H);
@@ -509,13 +223,13 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         if (e == cudaSuccess)
             chunk_gdn_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, p, static_cast<const uint8_t *>(ws));
     } else if (rule == kRuleGLA) {
-        const int smem = ctl + (int)LayoutGE<kRuleGLA>::END;
+        const int smem = (int)((sizeof(GECtl) + 1023) / 1024 * 1024) + 1024 + (int)GE<kRuleGLA>::END;
         e = allow_smem((const void *)chunk_ge_kernel<kRuleGLA>, smem);
-        if (e == cudaSuccess) chunk_ge_kernel<kRuleGLA><<<grid, NT, smem, st>>>(m, p);
+        if (e == cudaSuccess) chunk_ge_kernel<kRuleGLA><<<grid, GE<kRuleGLA>::NTHREADS, smem, st>>>(m, p);
     } else {
-        const int smem = ctl + (int)LayoutGE<kRuleELU>::END;
+        const int smem = (int)((sizeof(GECtl) + 1023) / 1024 * 1024) + 1024 + (int)GE<kRuleELU>::END;
         e = allow_smem((const void *)chunk_ge_kernel<kRuleELU>, smem);
-        if (e == cudaSuccess) chunk_ge_kernel<kRuleELU><<<grid, NT, smem, st>>>(m, p);
+        if (e == cudaSuccess) chunk_ge_kernel<kRuleELU><<<grid, GE<kRuleELU>::NTHREADS, smem, st>>>(m, p);
     }
     if (e != cudaSuccess) {
         *err = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);

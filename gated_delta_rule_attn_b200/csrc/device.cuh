@@ -40,14 +40,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+// One potentially blocking test: the hardware suspends the calling thread until
+// the phase completes or about `kSuspendNs` nanoseconds pass, so waiting warps
+// do not spin on the issue slots and shared-memory pipe that working warps use.
+constexpr uint32_t kSuspendNs = 1000000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
@@ -265,5 +269,45 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 
 // phi(x) = ELU(x) + 1 (ELU alpha = 1): x + 1 for x > 0, e^x otherwise.
 __device__ __forceinline__ float elu_feature(float x) { return x > 0.f ? x + 1.f : __expf(x); }
+
+// ---------------------------------------------------------------------------
+// FMA-pipe replacements for the two transcendental operations of the chunk
+// kernels' per-element work (the special-function unit is far narrower than
+// the FMA pipe and becomes the bottleneck of those loops).
+// ---------------------------------------------------------------------------
+// 1/x for normal positive x: Newton-Raphson iteration y <- y (2 - x y) from an
+// exponent-negating integer seed bits(y0) = K - bits(x).  K = 0x7EF311C0
+// minimises the seed's worst relative error over a binade (5.1%); two steps
+// leave at most 6.6e-6.
+__device__ __forceinline__ float rcp_nr(float x) {
+    float y = __int_as_float(0x7EF311C0 - __float_as_int(x));
+    y = y * fmaf(-x, y, 2.f);
+    y = y * fmaf(-x, y, 2.f);
+    return y;
+}
+
+// 2^t for t <= 0: t = n + f with n = round(t), |f| <= 1/2; 2^f = e^(f ln 2) by
+// its Taylor polynomial of degree 5 (relative error 3.3e-6 on |f| <= 1/2), then
+// scaled by 2^n through the exponent field.  Rounding uses the 1.5 * 2^23 add /
+// subtract trick, so everything stays on the FMA and integer pipes (no
+// conversion instructions).  Returns 0 below 2^-126.
+__device__ __forceinline__ float exp2_neg(float t) {
+    t = fmaxf(t, -127.f);
+    const float r = t + 12582912.f;                         // 1.5 * 2^23: round to integer
+    const int e = __float_as_int(r) - 0x4B400000;           // that integer
+    const float f = t - (r - 12582912.f);
+    float p = 1.3333558146428443e-3f;           // (ln 2)^5 / 5!
+    p = fmaf(p, f, 9.618129107628477e-3f);       // (ln 2)^4 / 4!
+    p = fmaf(p, f, 5.550410866482158e-2f);       // (ln 2)^3 / 3!
+    p = fmaf(p, f, 2.402265069591007e-1f);       // (ln 2)^2 / 2!
+    p = fmaf(p, f, 6.931471805599453e-1f);       // ln 2
+    p = fmaf(p, f, 1.f);
+    return e < -126 ? 0.f : __int_as_float(__float_as_int(p) + (e << 23));
+}
+
+// phi(x) = ELU(x) + 1 with e^x = 2^(x log2 e) evaluated on the FMA pipe.
+__device__ __forceinline__ float elu_feature_fma(float x) {
+    return x > 0.f ? x + 1.f : exp2_neg(fminf(x, 0.f) * 1.4426950408889634f);
+}
 
 }  // namespace la
