@@ -26,7 +26,7 @@ STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_E
 # Symbols include/la.h declares (checked by the CPU test suite).
 EXPORTS = ("la_fwd", "la_fwd_workspace_size", "la_step", "la_fwd_host_staging_size",
            "la_fwd_host", "la_check_device", "la_status_string", "la_last_error_message",
-           "la_abi_version")
+           "la_abi_version", "la_fwd_noalloc")
 
 
 class LAError(RuntimeError):
@@ -73,11 +73,12 @@ def lib():
         L.la_fwd_host_staging_size.argtypes = [ctypes.POINTER(FwdArgs), ctypes.POINTER(ctypes.c_size_t)]
         L.la_fwd_host.argtypes = [ctypes.POINTER(FwdArgs), P, ctypes.c_size_t, P]
         L.la_check_device.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+        L.la_fwd_noalloc.argtypes = [ctypes.POINTER(FwdArgs), P]
         L.la_status_string.argtypes = [ctypes.c_int]
         L.la_status_string.restype = ctypes.c_char_p
         L.la_last_error_message.restype = ctypes.c_char_p
         for f in (L.la_fwd, L.la_fwd_workspace_size, L.la_step, L.la_fwd_host_staging_size,
-                  L.la_fwd_host, L.la_check_device):
+                  L.la_fwd_host, L.la_check_device, L.la_fwd_noalloc):
             f.restype = ctypes.c_int
         L.la_abi_version.restype = ctypes.c_int
         _lib = L

@@ -281,7 +281,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         if (leader)
             for (int c = 0; c < NSTG && c < nchunks; ++c) load_chunk(c);
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c % NSTG, kb = c & 1;
+            const int kb = c & 1;
             const int t0 = c * C;
             const int nvalid = (int)min((int64_t)C, p.T - t0);
             if (leader) ctl->stopS = ctl->abort;

@@ -246,6 +246,57 @@ la_status la_fwd(const la_fwd_args *args, void *stream) {
     return launch_fwd(*args, static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------------------
+// la_fwd_noalloc: the workspace is this library's own fixed device array.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+constexpr int kMaxDevices = 256;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once
+// per device; the host-side symbol itself is not a device address).
+la_status noalloc_scratch(void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(LA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(LA_ERR_UNSUPPORTED, "device ordinal out of range");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(LA_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LA_OK;
+}
+}  // namespace
+
+la_status la_fwd_noalloc(const la_fwd_args *args, void *stream) {
+    la_status r = validate_fwd(args, true);
+    if (r != LA_OK) return r;
+    la_fwd_args a = *args;
+    a.workspace = nullptr;
+    a.workspace_bytes = 0;
+    const size_t need =
+        uses_chunk_kernels(a) ? la::chunk_workspace_bytes((int)a.rule, a.B, a.T, a.H) : 0;
+    if (need > LA_NOALLOC_SCRATCH_BYTES)
+        return fail(LA_ERR_WORKSPACE, "problem needs " + std::to_string(need) +
+                                          " bytes of scratch; la_fwd_noalloc has " +
+                                          std::to_string((size_t)LA_NOALLOC_SCRATCH_BYTES) +
+                                          " (use la_fwd with a caller workspace)");
+    if (need) {
+        r = noalloc_scratch(&a.workspace);
+        if (r != LA_OK) return r;
+        a.workspace_bytes = LA_NOALLOC_SCRATCH_BYTES;
+    }
+    return launch_fwd(a, static_cast<cudaStream_t>(stream));
+}
+
 la_status la_fwd_workspace_size(const la_fwd_args *args, size_t *bytes) {
     if (!bytes) return fail(LA_ERR_INVALID_ARG, "bytes is NULL");
     la_status r = validate_fwd(args, false);

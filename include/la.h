@@ -163,6 +163,39 @@ la_status la_fwd_host(const la_fwd_args *host_args, void *staging, size_t stagin
                       void *stream);
 
 /*
+ * la_fwd_noalloc — la_fwd for callers that cannot allocate device memory.
+ *
+ * No counterpart in the pages: this is an interface for integrators.  Some
+ * callers of this library cannot call cudaMalloc (or any allocating routine):
+ * code that runs under a host framework which owns all device memory, plugins
+ * and embedded runtimes with a fixed memory budget, or a latency-critical path
+ * that must not take the allocator's locks or trigger a synchronising
+ * allocation.  They cannot provide la_fwd's `workspace` (the gated delta rule's
+ * tensor-core path needs one).  This entry point takes the same arguments as
+ * la_fwd but ignores args->workspace / workspace_bytes and uses a scratch array
+ * that is part of the library itself: a file-scope `__device__` array of
+ * LA_NOALLOC_SCRATCH_BYTES (16 MiB), 256-byte aligned.  Every GPU on which the
+ * library is loaded holds that array until the process exits.
+ *
+ *   - The problem's scratch need (la_fwd_workspace_size) must be at most
+ *     LA_NOALLOC_SCRATCH_BYTES, otherwise LA_ERR_WORKSPACE is returned before
+ *     anything is launched.  For the gated delta rule that is 1024
+ *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 4096.
+ *   - The first call on a device looks up the array's device address there
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.  Later calls on the device reuse the address.
+ *   - All calls share the one array and it keeps the last call's contents; the
+ *     kernels write every scratch byte they read within the same call, so no
+ *     clearing is needed.  Calls that overlap on the GPU (different streams
+ *     without ordering, or several host threads) race on the array: serialise
+ *     them.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Otherwise identical to la_fwd (validation, status codes, asynchrony).
+ */
+#define LA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+la_status la_fwd_noalloc(const la_fwd_args *args, void *stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word set by
  * earlier kernels.  Returns LA_OK, LA_ERR_TIMEOUT, LA_ERR_RANGE or LA_ERR_CUDA.
  * `flags` (may be NULL) receives the raw word (bit 0 timeout, bit 1 range).
