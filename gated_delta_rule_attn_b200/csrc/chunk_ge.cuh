@@ -1,21 +1,35 @@
-// chunk_ge.cuh — GLA and normalized ELU+1 chunked prefill, warp-specialised.
+// chunk_ge.cuh — GLA and normalized ELU+1 chunked prefill, warp-specialised and
+// software-pipelined across chunks.
 //
-// One CTA per (batch, head, 32-column value slab), 12 warps:
-//   warps 0-7   "prep" group, one chunk ahead: the feature map / gate scaling of
-//               q and k on CUDA cores (8 key dims x 4 tokens per thread, 16-byte
-//               accesses).  GLA: gamma_t = prod_{s<=t} g_s per key dim (local
-//               products over 4 tokens, then an exclusive product over the 16
-//               token groups),
-//               Qt = Q o gamma (in place), Kt = K / gamma (operand tile Kx),
-//               Kh = Kt o gamma_C (in place), gamma_C per dim.  ELU+1:
-//               phi(Q) in place, phi(K) into Kx, the chunk's sum of phi(k) per dim;
-//   warps 8-11  "state" group: issues the TMA loads of q, k, v (and the GLA
-//               gate) into a ring of stages and the MMAs of its chunk, and owns
-//               the fp32 state (one key-dim row per thread):
-//                 MMA1  [P | O_inter (| den_inter)] = Q' [K' ; S^T (; z^T)]^T,
-//                 MMA2  dS = K''^T V,
-//                 P masked -> bf16, S <- diag(gamma_C) S + dS (ELU: S + dS, z += sum phi(k)),
-//                 MMA3  O += P V,  O -> global (ELU: / (phi(q).z0 + rowsum(P) + eps)).
+// One CTA per (batch, head, 32-column value slab), 17 warps:
+//   warps 0-7    prep: the feature map / gate scaling of q and k on CUDA cores.
+//                Thread (pr, qt) owns key dims 2pr, 2pr+1 of tokens 16qt..16qt+15
+//                (a warp covers a full 128-byte row per access, conflict-free).
+//                GLA: gamma_t = prod_{s<=t} g_s per key dim (local products, then
+//                the product of the earlier token quarters), Qt = Q o gamma,
+//                Kt = K / gamma (both in place), gamma_C.  ELU+1: phi(Q), phi(K)
+//                in place and the chunk's sum of phi(k).  The GLA gate tiles come
+//                through a two-slot TMA ring of their own (prefetched into L2 two
+//                chunks ahead); the ELU exponential runs on the FMA pipe.
+//   warps 8-11   group A: the score epilogue (causal mask of P, bf16 P tile for
+//                MMA3; ELU row sums of P) and the output epilogue; its thread 0
+//                issues the TMA loads of q, k, v into a ring of stages.
+//   warps 12-15  group B: owns the fp32 state slab (one key-dim row per thread),
+//                applies each chunk's dS and writes the bf16 copy of the state
+//                that the next chunk's MMA1 reads.
+//   warp 16      issues every MMA (lane 0), in dependency order.
+// A stage holds Q and a K tile whose rows 64.. carry the bf16 S^T (and ELU z^T)
+// of the state entering the chunk, so [K' ; S^T (; z^T)] is one operand; it is
+// refilled as soon as MMA1 and MMA2 of its chunk are done.  V has a ring of its
+// own (its last reader, MMA3, comes later).
+// Per chunk c the tensor core computes
+//   MMA2(c)  dS = K'^T V                                   -> DS[c%2]
+//   MMA1(c)  [P | O_inter (| den_inter)] = Q' [K' ; S^T (; z^T)]^T -> ACC[c%3]
+//   MMA3(c)  O += P V                                      -> ACC[c%3] (O columns)
+// and the state update is S <- diag(gamma_C) (S + dS) (ELU: S + dS, z += sum phi(k)).
+// MMA2 runs two chunks ahead (it does not need the state), MMA1(c+1) starts as
+// soon as the state copy of chunk c exists, and MMA3(c) once the P tile of c is
+// written; TMEM accumulators are triple-buffered, DS and the P tile doubled.
 // Method and notation: see the header of chunk_tc.cuh.
 #pragma once
 
@@ -27,36 +41,53 @@ namespace ck {
 template <int RULE>
 struct GE {
     static constexpr bool kGLA = (RULE == kRuleGLA);
-    static constexpr int NSTG = kGLA ? 2 : 3;
-    static constexpr int NTHREADS = 384;
-    static constexpr uint32_t TMEM_COLS = 256;
-    static constexpr uint32_t C_ACC = 0;     // MMA1: P (0-63), O (64-95), ELU den (96)
-    static constexpr uint32_t C_DS = 128;    // MMA2: dS, M=128
-    static constexpr int KX_ROWS = kGLA ? 96 : 104;   // K' (0-63), S^T (64-95), ELU z^T (96), zeros
-    static constexpr uint32_t KX_ACS = KX_ROWS * 128;
-    static constexpr uint32_t KX_BYTES = KX_ACS * KA;
+    static constexpr int NSTG = kGLA ? 3 : 4;
+    static constexpr int NTHREADS = 544;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t C_ACC = 0;     // ACC[j] at 128 j: P (0-63), O (64-95), ELU den (96)
+    static constexpr uint32_t C_DS = 384;    // DS[b] at 384 + 32 b (M=128)
+    static constexpr int KR = kGLA ? 96 : 104;   // K tile rows: K' (0-63), S^T (64-95), ELU z^T (96), zeros
+    static constexpr uint32_t K_ACS = KR * 128;                // bytes per atom column of the K tile
     static constexpr uint32_t Q_BYTES = C * 128 * KA;           // [atom col][64 rows]
-    static constexpr uint32_t G_BYTES = kGLA ? C * DK * 4 : 0;  // fp32 [64][128]
-    static constexpr uint32_t STG_BYTES = 2 * Q_BYTES + 4096 + G_BYTES;
+    static constexpr uint32_t K_BYTES = K_ACS * KA;
+    static constexpr uint32_t V_BYTES = C * DVT * 2;            // 64-byte swizzled [64][32]
+    static constexpr uint32_t STG_BYTES = Q_BYTES + K_BYTES;
+    static constexpr int NV = 4;                                // V ring slots
+    static constexpr uint32_t G_BYTES = C * DK * 4;             // GLA gate tile, fp32 [64][128]
     // tiles
     static constexpr uint32_t STG = 0;
-    static constexpr uint32_t KX = STG + NSTG * STG_BYTES;
-    static constexpr uint32_t PS = KX + 2 * KX_BYTES;
-    static constexpr uint32_t END = PS + C * 128;
-    static constexpr int N1 = KX_ROWS;
+    static constexpr uint32_t VR = STG + NSTG * STG_BYTES;      // V ring
+    static constexpr uint32_t GT = VR + NV * V_BYTES;           // GLA: two gate slots
+    static constexpr uint32_t PS = GT + (kGLA ? 2 * G_BYTES : 0);
+    static constexpr uint32_t END = PS + 2 * C * 128;
+    static constexpr int N1 = KR;
 };
 
 struct GECtl {
-    uint64_t full[3];
-    uint64_t pfull[2], pempty[2], m1_done, m3_done;
+    uint64_t full[4];                // TMA of a stage's q and k landed
+    uint64_t vfull[4];               // TMA of a V slot landed
+    uint64_t pfull[4];               // the stage's chunk prepared (8 prep warps)
+    uint64_t gfull[2];               // GLA gate slot landed
+    uint64_t mP[3];                  // MMA1 of the chunk (and everything issued before it) done
+    uint64_t m3[3];                  // MMA3 of the chunk done
+    uint64_t oA[3];                  // output epilogue of the chunk done (128)
+    uint64_t mD[2];                  // MMA2 of the chunk done
+    uint64_t pA[2];                  // P tile written (128)
+    uint64_t sB[2];                  // state copy written (128)
+    uint64_t s0;                     // initial state copy written (128)
+    uint64_t drain;
     uint32_t tmem_base;
-    int abort, stopP, stopS;
-    alignas(16) float gC[2][128];    // GLA: gamma at chunk end per key dim; ELU: chunk sum of phi(k)
-    alignas(16) float tot[16][128];  // prep: per token-group products (GLA) / sums of phi(k) (ELU)
+    int abort, stopP;
+    alignas(16) float gC[4][128];    // GLA: gamma at chunk end per key dim; ELU: chunk sum of phi(k)
+    alignas(16) float2 tot[4][64];   // prep: per-quarter gate products (GLA) / sums of phi(k) (ELU)
 };
 
+__device__ __forceinline__ bool aborted(const GECtl *ctl) {
+    return __any_sync(0xffffffffu, *reinterpret_cast<const volatile int *>(&ctl->abort) != 0);
+}
+
 template <int RULE>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(544, 1)
 chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
     using L = GE<RULE>;
     constexpr bool kGLA = L::kGLA;
@@ -78,13 +109,24 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
     auto stg = [&](int c) { return tiles + L::STG + (uint32_t)(c % NSTG) * L::STG_BYTES; };
 
     if (tid == 0) {
-        for (int s = 0; s < NSTG; ++s) mbar_init(&ctl->full[s], 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&ctl->pfull[i], 256);
-            mbar_init(&ctl->pempty[i], 1);
+        for (int s = 0; s < L::NV; ++s) mbar_init(&ctl->vfull[s], 1);
+        for (int s = 0; s < NSTG; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->pfull[s], 8);
         }
-        mbar_init(&ctl->m1_done, 1);
-        mbar_init(&ctl->m3_done, 1);
+        for (int i = 0; i < 3; ++i) {
+            mbar_init(&ctl->mP[i], 1);
+            mbar_init(&ctl->m3[i], 1);
+            mbar_init(&ctl->oA[i], 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->mD[i], 1);
+            mbar_init(&ctl->gfull[i], 1);
+            mbar_init(&ctl->pA[i], 128);
+            mbar_init(&ctl->sB[i], 128);
+        }
+        mbar_init(&ctl->s0, 128);
+        mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_barrier_init();
         tma_prefetch_desc(&maps.q);
@@ -101,220 +143,170 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16);
 
-    // TMA of chunk c into its stage (issued by the state group's leader)
-    auto load_chunk = [&](int c) {
-        const int s = c % NSTG;
-        uint8_t *st = stg(c);
-        const int t0 = c * C;
-        mbar_arrive_expect_tx(&ctl->full[s], 2u * L::Q_BYTES + C * DVT * 2u + L::G_BYTES);
-#pragma unroll
-        for (int a = 0; a < KA; ++a) {
-            tma_load_4d(st + a * (C * 128), &maps.q, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
-            tma_load_4d(st + L::Q_BYTES + a * (C * 128), &maps.k, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
-        }
-        tma_load_4d(st + 2 * L::Q_BYTES, &maps.v, &ctl->full[s], dvt * DVT, (int)h, t0, (int)b);
-        if (kGLA) tma_load_4d(st + 2 * L::Q_BYTES + 4096, &maps.g, &ctl->full[s], 0, (int)h, t0, (int)b);
-    };
-
     if (warp < 8) {
-        // ------------------------------------------------------------------ prep group
+        // ------------------------------------------------------------------ prep
+        // Thread (pr, qt) owns key dims 2pr, 2pr+1 of tokens 16qt..16qt+15.  One
+        // warp covers 32 consecutive pairs (a full 128-byte row of one atom
+        // column) of one token per access, so its 4- and 8-byte shared-memory
+        // accesses are free of bank conflicts.  All loads of a chunk are issued
+        // before its first store.
         const int lt = tid;
         const bool leader = (lt == 0);
-        const int j = lt & 15, tg = lt >> 4;           // dims 8j..8j+7, tokens 4tg..4tg+3
-        const int a = j >> 3, cj = j & 7;              // atom column, 16-byte chunk in the row
+        const int pr = lt & 63, qt = lt >> 6;
+        const int a = pr >> 5;                                   // atom column
+        const uint32_t cpos = (uint32_t)((pr & 31) >> 2), cin = (uint32_t)(pr & 3) << 2;
+        // GLA gate tile of chunk c into slot c & 1 (issued by prep thread 0 once
+        // every prep thread is done with the slot's previous chunk)
+        auto gate_load = [&](int c) {
+            uint64_t *bar = &ctl->gfull[c & 1];
+            mbar_arrive_expect_tx(bar, L::G_BYTES);
+            tma_load_4d(tiles + L::GT + (uint32_t)(c & 1) * L::G_BYTES, &maps.g, bar, 0, (int)h, c * C, (int)b);
+        };
+        if (kGLA && leader)
+            for (int c = 0; c < 2 && c < nchunks; ++c) gate_load(c);
         for (int c = 0; c < nchunks; ++c) {
-            const int s = c % NSTG, kb = c & 1;
+            const int s = c % NSTG;
             const int nvalid = (int)min((int64_t)C, p.T - (int64_t)c * C);
             if (leader) ctl->stopP = ctl->abort;
             bar_named(1, 256);
             if (ctl->stopP) break;
+            if (kGLA && leader && c >= 1 && c + 1 < nchunks) {
+                fence_proxy_async_smem();
+                gate_load(c + 1);
+            }
+            if (kGLA && !mbar_wait(&ctl->gfull[c & 1], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
             if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
-            if (c >= 2 && !mbar_wait(&ctl->pempty[kb], (uint32_t)((c - 2) >> 1) & 1u)) ctl->abort = 1;
             uint8_t *st = stg(c);
-            uint8_t *qa = st + a * (C * 128), *ka = st + L::Q_BYTES + a * (C * 128);
-            uint8_t *kxa = tiles + L::KX + kb * L::KX_BYTES + a * L::KX_ACS;
+            uint8_t *qa = st + a * (C * 128), *ka = st + L::Q_BYTES + a * L::K_ACS;
+            auto off = [&](int i) {
+                const uint32_t t = (uint32_t)(16 * qt + i);
+                return t * 128u + (((cpos ^ t) & 7u) << 4) + cin;
+            };
             if constexpr (kGLA) {
-                const float *G = reinterpret_cast<const float *>(st + 2 * L::Q_BYTES + 4096);
-                float gam[4][8];   // [token][dim], products from the start of this thread's 4 tokens
-                float run[8];
+                // gamma_t = prod_{s<=t} g_s inside the chunk: local products over
+                // this thread's 16 tokens, then the product of the earlier quarters.
+                const uint8_t *G = tiles + L::GT + (uint32_t)(c & 1) * L::G_BYTES;   // fp32 [64][128]
+                float2 gv[16];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) run[e] = 1.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = 4 * tg + i;
-                    float gv[8];
-                    const float4 g0 = *reinterpret_cast<const float4 *>(G + t * DK + 8 * j);
-                    const float4 g1 = *reinterpret_cast<const float4 *>(G + t * DK + 8 * j + 4);
-                    gv[0] = g0.x; gv[1] = g0.y; gv[2] = g0.z; gv[3] = g0.w;
-                    gv[4] = g1.x; gv[5] = g1.y; gv[6] = g1.z; gv[7] = g1.w;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        run[e] *= (t < nvalid) ? gv[e] : 1.f;
-                        gam[i][e] = run[e];
-                    }
+                for (int i = 0; i < 16; ++i) {
+                    const int t = 16 * qt + i;
+                    gv[i] = *reinterpret_cast<const float2 *>(G + t * 512 + pr * 8);
+                    if (t >= nvalid) gv[i] = make_float2(1.f, 1.f);
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ctl->tot[tg][8 * j + e] = run[e];
+                for (int i = 1; i < 16; ++i) gv[i] = __fmul2_rn(gv[i - 1], gv[i]);
+                ctl->tot[qt][pr] = gv[15];
                 bar_named(1, 256);
-                if (lt < DK) {   // exclusive product over the 16 token groups, one key dim per thread
-                    float acc = 1.f;
-#pragma unroll
-                    for (int g2 = 0; g2 < 16; ++g2) {
-                        const float tv = ctl->tot[g2][lt];
-                        ctl->tot[g2][lt] = acc;
-                        acc *= tv;
-                    }
-                    ctl->gC[kb][lt] = acc;
-                    if (!(acc >= 1e-30f)) raise_error(kErrRange);
+                float2 pre = make_float2(1.f, 1.f);
+                for (int q2 = 0; q2 < qt; ++q2) pre = __fmul2_rn(pre, ctl->tot[q2][pr]);
+                if (qt == 3) {
+                    const float2 gc = __fmul2_rn(pre, gv[15]);
+                    *reinterpret_cast<float2 *>(&ctl->gC[c & 3][2 * pr]) = gc;
+                    if (!(fminf(gc.x, gc.y) >= 1e-30f)) raise_error(kErrRange);
                 }
-                bar_named(1, 256);
-                float pre[8], gC[8];
-                {
-                    const float4 p0 = *reinterpret_cast<const float4 *>(&ctl->tot[tg][8 * j]);
-                    const float4 p1 = *reinterpret_cast<const float4 *>(&ctl->tot[tg][8 * j + 4]);
-                    const float4 c0 = *reinterpret_cast<const float4 *>(&ctl->gC[kb][8 * j]);
-                    const float4 c1 = *reinterpret_cast<const float4 *>(&ctl->gC[kb][8 * j + 4]);
-                    pre[0] = p0.x; pre[1] = p0.y; pre[2] = p0.z; pre[3] = p0.w;
-                    pre[4] = p1.x; pre[5] = p1.y; pre[6] = p1.z; pre[7] = p1.w;
-                    gC[0] = c0.x; gC[1] = c0.y; gC[2] = c0.z; gC[3] = c0.w;
-                    gC[4] = c1.x; gC[5] = c1.y; gC[6] = c1.z; gC[7] = c1.w;
-                }
+                // Qt = Q o gamma, Kt = K / gamma (both in place), 8 tokens at a time
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = 4 * tg + i;
-                    const uint32_t off = (uint32_t)t * 128u + (uint32_t)(((cj ^ t) & 7) << 4);
-                    const uint4 qv = *reinterpret_cast<const uint4 *>(qa + off);
-                    const uint4 kv = *reinterpret_cast<const uint4 *>(ka + off);
-                    const uint32_t *qw = &qv.x, *kw = &kv.x;
-                    uint4 q2, kt, kh;
-                    uint32_t *q2w = &q2.x, *ktw = &kt.x, *khw = &kh.x;
+                for (int h8 = 0; h8 < 16; h8 += 8) {
+                    uint32_t qv[8], kv[8];
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const float2 qf = unpack_bf16x2(qw[e2]), kf = unpack_bf16x2(kw[e2]);
-                        const float ga = pre[2 * e2] * gam[i][2 * e2], gb = pre[2 * e2 + 1] * gam[i][2 * e2 + 1];
-                        const float ia = rcp_nr(ga), ib = rcp_nr(gb);
-                        q2w[e2] = pack_bf16x2(qf.x * ga, qf.y * gb);
-                        ktw[e2] = pack_bf16x2(kf.x * ia, kf.y * ib);
-                        khw[e2] = pack_bf16x2(kf.x * (ia * gC[2 * e2]), kf.y * (ib * gC[2 * e2 + 1]));
+                    for (int i = 0; i < 8; ++i) {
+                        qv[i] = *reinterpret_cast<const uint32_t *>(qa + off(h8 + i));
+                        kv[i] = *reinterpret_cast<const uint32_t *>(ka + off(h8 + i));
                     }
-                    *reinterpret_cast<uint4 *>(qa + off) = q2;
-                    *reinterpret_cast<uint4 *>(kxa + off) = kt;
-                    *reinterpret_cast<uint4 *>(ka + off) = kh;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float2 gm = __fmul2_rn(pre, gv[h8 + i]);
+                        const float2 ig = make_float2(rcp_approx(gm.x), rcp_approx(gm.y));
+                        const float2 qs = __fmul2_rn(unpack_bf16x2(qv[i]), gm);
+                        const float2 ks = __fmul2_rn(unpack_bf16x2(kv[i]), ig);
+                        *reinterpret_cast<uint32_t *>(qa + off(h8 + i)) = pack_bf16x2(qs.x, qs.y);
+                        *reinterpret_cast<uint32_t *>(ka + off(h8 + i)) = pack_bf16x2(ks.x, ks.y);
+                    }
                 }
             } else {
-                float zs[8];
+                // phi(Q), phi(K) in place (phi(k) = 0 past T), chunk sum of phi(k)
+                uint32_t qv[16], kv[16];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) zs[e] = 0.f;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = 4 * tg + i;
-                    const uint32_t off = (uint32_t)t * 128u + (uint32_t)(((cj ^ t) & 7) << 4);
-                    const uint4 qv = *reinterpret_cast<const uint4 *>(qa + off);
-                    const uint4 kv = *reinterpret_cast<const uint4 *>(ka + off);
-                    const uint32_t *qw = &qv.x, *kw = &kv.x;
-                    uint4 pq, pk;
-                    uint32_t *pqw = &pq.x, *pkw = &pk.x;
-                    const bool valid = t < nvalid;
-#pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const float2 qf = unpack_bf16x2(qw[e2]), kf = unpack_bf16x2(kw[e2]);
-                        const float k0 = valid ? elu_feature(kf.x) : 0.f, k1 = valid ? elu_feature(kf.y) : 0.f;
-                        pqw[e2] = pack_bf16x2(elu_feature(qf.x), elu_feature(qf.y));
-                        pkw[e2] = pack_bf16x2(k0, k1);
-                        zs[2 * e2] += k0;
-                        zs[2 * e2 + 1] += k1;
-                    }
-                    *reinterpret_cast<uint4 *>(qa + off) = pq;
-                    *reinterpret_cast<uint4 *>(kxa + off) = pk;
+                for (int i = 0; i < 16; ++i) {
+                    qv[i] = *reinterpret_cast<const uint32_t *>(qa + off(i));
+                    kv[i] = *reinterpret_cast<const uint32_t *>(ka + off(i));
                 }
+                float2 zs = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) ctl->tot[tg][8 * j + e] = zs[e];
+                for (int i = 0; i < 16; ++i) {
+                    const float2 qf = unpack_bf16x2(qv[i]), kf = unpack_bf16x2(kv[i]);
+                    float2 fk = elu_feature2(kf);
+                    if (16 * qt + i >= nvalid) fk = make_float2(0.f, 0.f);
+                    const float2 fq = elu_feature2(qf);
+                    *reinterpret_cast<uint32_t *>(qa + off(i)) = pack_bf16x2(fq.x, fq.y);
+                    *reinterpret_cast<uint32_t *>(ka + off(i)) = pack_bf16x2(fk.x, fk.y);
+                    zs = __fadd2_rn(zs, fk);
+                }
+                ctl->tot[qt][pr] = zs;
                 bar_named(1, 256);
-                if (lt < DK) {   // chunk sum of phi(k) per key dim over the 16 token groups
-                    float zsum = 0.f;
-#pragma unroll
-                    for (int g2 = 0; g2 < 16; ++g2) zsum += ctl->tot[g2][lt];
-                    ctl->gC[kb][lt] = zsum;
+                if (qt == 0) {
+                    float2 z = __fadd2_rn(ctl->tot[0][pr], ctl->tot[1][pr]);
+                    z = __fadd2_rn(z, __fadd2_rn(ctl->tot[2][pr], ctl->tot[3][pr]));
+                    *reinterpret_cast<float2 *>(&ctl->gC[c & 3][2 * pr]) = z;
                 }
             }
             fence_proxy_async_smem();
-            mbar_arrive(&ctl->pfull[kb]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->pfull[s]);
         }
-    } else {
-        // ------------------------------------------------------------------ state group
-        const int st = tid - 256;
-        const bool leader = (st == 0);
-        const int d = 32 * quad + lane;             // state row (key dim)
-        const int tr = 16 * quad + (lane & 15);     // chunk row of M=64 accumulators
+    } else if (warp < 12) {
+        // ------------------------------------------------------------------ group A
+        const bool a0 = (tid == 256);
+        const int tr = 16 * quad + (lane & 15);     // chunk row of the M=64 accumulators
         const int hf = lane >> 4;
-        constexpr uint32_t ID1 = idesc_bf16(64, L::N1, false, false);
-        constexpr uint32_t ID2 = idesc_bf16(128, DVT, true, true);
-        constexpr uint32_t ID3 = idesc_bf16(64, DVT, false, true);
-        float S[DVT];
-        float z = 0.f;
-        {
-            const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVT) : nullptr;
-#pragma unroll
-            for (int jj = 0; jj < DVT; jj += 4) {
-                float4 x = src ? *reinterpret_cast<const float4 *>(src + jj) : make_float4(0, 0, 0, 0);
-                S[jj] = x.x; S[jj + 1] = x.y; S[jj + 2] = x.z; S[jj + 3] = x.w;
-            }
-            if (!kGLA && p.z0) z = p.z0[bh * DK + d];
-        }
-        // bf16 copy of S^T (and z^T) into rows 64.. of Kx buffer kb; ELU: zero rows 97..103
-        auto write_state = [&](int kb) {
-            uint8_t *kxa = tiles + L::KX + kb * L::KX_BYTES + (d >> 6) * L::KX_ACS;
-            const int dc = d & 63;
-#pragma unroll
-            for (int jj = 0; jj < DVT; ++jj) *elem(kxa, 64 + jj, dc) = __float2bfloat16_rn(S[jj]);
-            if (!kGLA) *elem(kxa, 96, dc) = __float2bfloat16_rn(z);
-        };
-        if (!kGLA) {
-            for (int kb = 0; kb < 2; ++kb) {
-                uint8_t *kxa = tiles + L::KX + kb * L::KX_BYTES + (d >> 6) * L::KX_ACS;
-#pragma unroll
-                for (int r = 97; r < 104; ++r) *elem(kxa, r, d & 63) = __float2bfloat16_rn(0.f);
-            }
-        }
-        write_state(0);
-        fence_proxy_async_smem();
-        if (leader)
-            for (int c = 0; c < NSTG && c < nchunks; ++c) load_chunk(c);
-        for (int c = 0; c < nchunks; ++c) {
-            const int kb = c & 1;
+        int issued = -1, issued_v = -1;             // last chunks whose TMA thread a0 issued
+        // TMA of q and k for chunk c
+        auto load_chunk = [&](int c) {
+            const int s = c % NSTG;
+            uint8_t *st = stg(c);
             const int t0 = c * C;
-            const int nvalid = (int)min((int64_t)C, p.T - t0);
-            if (leader) ctl->stopS = ctl->abort;
-            bar_named(2, 128);
-            if (ctl->stopS) break;
-            if (!mbar_wait(&ctl->pfull[kb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
-            uint8_t *sg = stg(c);
-            const uint32_t qb = smem_u32(sg), kxb = tb + L::KX + kb * L::KX_BYTES;
-            const uint32_t vb = qb + 2 * L::Q_BYTES;
-            if (leader) {
-                tc_fence_after_sync();
-                const uint64_t dq = dk0(qb), dkx = dk0(kxb);
-                const uint64_t du = kGLA ? dmn128_0(qb + L::Q_BYTES, C * 128) : dmn128_0(kxb, L::KX_ACS);
-                const uint64_t dv = dmn64_0(vb);
+            mbar_arrive_expect_tx(&ctl->full[s], 2u * L::Q_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    umma_bf16(tmem + L::C_ACC, kstep_k(dq, C * 128, kk), kstep_k(dkx, L::KX_ACS, kk), ID1,
-                              kk > 0);
-                    if (kk < C / 16)
-                        umma_bf16(tmem + L::C_DS, kstep_mn128(du, kk), kstep_mn64(dv, kk), ID2, kk > 0);
-                }
-                umma_commit(&ctl->m1_done);
+            for (int a = 0; a < KA; ++a) {
+                tma_load_4d(st + a * (C * 128), &maps.q, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
+                tma_load_4d(st + L::Q_BYTES + a * L::K_ACS, &maps.k, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
             }
-            if (!mbar_wait(&ctl->m1_done, (uint32_t)c & 1u)) ctl->abort = 1;
+            // the gate tile of chunk c+2 is loaded about one chunk period from
+            // now: start bringing it into L2
+            if (kGLA && dvt == 0 && c + 2 < nchunks) tma_prefetch_l2_4d(&maps.g, 0, (int)h, t0 + 2 * C, (int)b);
+            issued = c;
+        };
+        // TMA of this CTA's V slab for chunk c
+        auto load_v = [&](int c) {
+            const int j = c % L::NV;
+            mbar_arrive_expect_tx(&ctl->vfull[j], L::V_BYTES);
+            tma_load_4d(tiles + L::VR + (uint32_t)j * L::V_BYTES, &maps.v, &ctl->vfull[j], dvt * DVT, (int)h, c * C,
+                        (int)b);
+            issued_v = c;
+        };
+        if (a0) {
+            for (int c = 0; c < NSTG && c < nchunks; ++c) load_chunk(c);
+            for (int c = 0; c < L::NV && c < nchunks; ++c) load_v(c);
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const int bb = c & 1, j3 = c % 3;
+            const uint32_t acc = L::C_ACC + 128u * (uint32_t)j3;
+            const int64_t t0 = (int64_t)c * C;
+            const int nvalid = (int)min((int64_t)C, p.T - t0);
+            if (aborted(ctl)) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->mP[j3], (uint32_t)(c / 3) & 1u))) {
+                ctl->abort = 1;
+                break;
+            }
+            // MMA1(c) and MMA2(c) were the last readers of the stage's q and k
+            if (a0 && !ctl->abort && c + NSTG < nchunks) load_chunk(c + NSTG);
             tc_fence_after_sync();
             float den = 0.f;
-            {   // P row tr, columns 32*hf..: causal mask -> bf16 tile; ELU row sums
+            {   // P row tr, columns 32*hf..: causal mask -> bf16 tile PS[bb]; ELU row sums
                 float x[32];
-                tmem_ld16x2_32<32>(tq + L::C_ACC, x);
+                tmem_ld16x2_32<32>(tq + acc, x);
                 float dI[16];
-                if (!kGLA) tmem_ld16(tq + L::C_ACC + 96, dI);
-                float ds[DVT];
-                tmem_ld32(tq + L::C_DS, ds);
+                if (!kGLA) tmem_ld16(tq + acc + 96, dI);
                 tmem_wait_ld();
                 float rs = 0.f;
 #pragma unroll
@@ -322,6 +314,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                     x[i] = (32 * hf + i <= tr) ? x[i] : 0.f;
                     rs += x[i];
                 }
+                uint8_t *ps = tiles + L::PS + bb * (C * 128);
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
                     uint4 u;
@@ -330,43 +323,25 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                     u.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
                     u.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
                     const int chunk = 4 * hf + cc;
-                    *reinterpret_cast<uint4 *>(tiles + L::PS + tr * 128 + (((chunk ^ tr) & 7) << 4)) = u;
+                    *reinterpret_cast<uint4 *>(ps + tr * 128 + (((chunk ^ tr) & 7) << 4)) = u;
                 }
                 if (!kGLA) {
                     rs += __shfl_xor_sync(0xffffffffu, rs, 16);
                     const float dz = __shfl_sync(0xffffffffu, dI[0], lane & 15);
                     den = dz + rs + p.eps;
                 }
-                // state update (row d), then its bf16 copy for the next chunk
-                const float g = ctl->gC[kb][d];
-                if (kGLA) {
-#pragma unroll
-                    for (int jj = 0; jj < DVT; ++jj) S[jj] = fmaf(g, S[jj], ds[jj]);
-                } else {
-#pragma unroll
-                    for (int jj = 0; jj < DVT; ++jj) S[jj] += ds[jj];
-                    z += g;
-                }
-                if (c + 1 < nchunks) write_state(kb ^ 1);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
-            bar_named(2, 128);
-            if (leader) {
-                tc_fence_after_sync();
-                const uint64_t dp = dk0(tb + L::PS), dv = dmn64_0(vb);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + L::C_ACC + 64, kstep_k(dp, C * 128, kk), kstep_mn64(dv, kk), ID3, 1u);
-                umma_commit(&ctl->m3_done);
-                umma_commit(&ctl->pempty[kb]);
+            mbar_arrive(&ctl->pA[bb]);
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->m3[j3], (uint32_t)(c / 3) & 1u))) {
+                ctl->abort = 1;
+                break;
             }
-            if (!mbar_wait(&ctl->m3_done, (uint32_t)c & 1u)) ctl->abort = 1;
-            if (leader && c + NSTG < nchunks && !ctl->abort) load_chunk(c + NSTG);   // its stage is free now
             tc_fence_after_sync();
             {
                 float o[16];
-                tmem_ld16x2_16<16>(tq + L::C_ACC + 64, o);
+                tmem_ld16x2_16<16>(tq + acc + 64, o);
                 tmem_wait_ld();
                 if (tr < nvalid) {
                     if (!kGLA) {
@@ -388,6 +363,84 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                 }
             }
             tc_fence_before_sync();
+            mbar_arrive(&ctl->oA[j3]);
+            // MMA3(c) was the last reader of the chunk's V slot: refill it
+            if (a0 && !ctl->abort && c + L::NV < nchunks) load_v(c + L::NV);
+        }
+        if (a0 && ctl->abort) {   // let copies still in flight land before the CTA exits
+            for (int c = (issued - NSTG + 1 > 0 ? issued - NSTG + 1 : 0); c <= issued; ++c)
+                (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
+            for (int c = (issued_v - L::NV + 1 > 0 ? issued_v - L::NV + 1 : 0); c <= issued_v; ++c)
+                (void)mbar_wait(&ctl->vfull[c % L::NV], (uint32_t)(c / L::NV) & 1u);
+        }
+    } else if (warp < 16) {
+        // ------------------------------------------------------------------ group B
+        const int d = 32 * quad + lane;             // state row (key dim)
+        float S[DVT];
+        float z = 0.f;
+        {
+            const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVT) : nullptr;
+#pragma unroll
+            for (int jj = 0; jj < DVT; jj += 4) {
+                float4 x = src ? *reinterpret_cast<const float4 *>(src + jj) : make_float4(0, 0, 0, 0);
+                S[jj] = x.x; S[jj + 1] = x.y; S[jj + 2] = x.z; S[jj + 3] = x.w;
+            }
+            if (!kGLA && p.z0) z = p.z0[bh * DK + d];
+        }
+        // bf16 copy of S^T (and z^T) into rows 64.. of the K tile of stage s
+        auto write_state = [&](int s) {
+            uint8_t *ka = tiles + L::STG + (uint32_t)s * L::STG_BYTES + L::Q_BYTES + (d >> 6) * L::K_ACS;
+            const int dc = d & 63;
+#pragma unroll
+            for (int jj = 0; jj < DVT; ++jj) *elem(ka, 64 + jj, dc) = __float2bfloat16_rn(S[jj]);
+            if (!kGLA) *elem(ka, 96, dc) = __float2bfloat16_rn(z);
+        };
+        if (!kGLA) {   // rows 97..103 of every stage's K tile stay zero
+            for (int s = 0; s < NSTG; ++s) {
+                uint8_t *ka = tiles + L::STG + (uint32_t)s * L::STG_BYTES + L::Q_BYTES + (d >> 6) * L::K_ACS;
+#pragma unroll
+                for (int r = 97; r < 104; ++r) *elem(ka, r, d & 63) = __float2bfloat16_rn(0.f);
+            }
+        }
+        write_state(0);
+        fence_proxy_async_smem();
+        mbar_arrive(&ctl->s0);
+        bool ok = nchunks == 0 || __all_sync(0xffffffffu, mbar_wait(&ctl->pfull[0], 0u));
+        if (!ok) ctl->abort = 1;
+        for (int c = 0; c < nchunks && ok; ++c) {
+            const int bb = c & 1;
+            if (aborted(ctl)) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->mD[bb], (uint32_t)(c >> 1) & 1u))) {
+                ctl->abort = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            {
+                float ds[DVT];
+                tmem_ld32(tq + L::C_DS + 32u * (uint32_t)bb, ds);
+                tmem_wait_ld();
+                const float g = ctl->gC[c & 3][d];
+                if (kGLA) {
+#pragma unroll
+                    for (int jj = 0; jj < DVT; ++jj) S[jj] = g * (S[jj] + ds[jj]);
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < DVT; ++jj) S[jj] += ds[jj];
+                    z += g;
+                }
+            }
+            if (c + 1 < nchunks) {
+                write_state((c + 1) % NSTG);
+                // the prep of c+1 is complete (its gamma_C / sum of phi(k) is readable)
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->pfull[(c + 1) % NSTG],
+                                                               (uint32_t)((c + 1) / NSTG) & 1u))) {
+                    ctl->abort = 1;
+                    break;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(&ctl->sB[bb]);
         }
         if (!ctl->abort) {
             if (p.S_out) {
@@ -398,10 +451,83 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             }
             if (!kGLA && p.z_out && dvt == 0) p.z_out[bh * DK + d] = z;
         }
-    }
-    if (tid == 256 && ctl->abort) {   // let copies still in flight land before exit
-        for (int s = 0; s < NSTG; ++s) (void)mbar_try_wait(&ctl->full[s], 0);
-        for (int s = 0; s < NSTG; ++s) (void)mbar_try_wait(&ctl->full[s], 1);
+    } else if (lane == 0) {
+        // ------------------------------------------------------------------ MMA issue
+        constexpr uint32_t ID1 = idesc_bf16(64, L::N1, false, false);
+        constexpr uint32_t ID2 = idesc_bf16(128, DVT, true, true);
+        constexpr uint32_t ID3 = idesc_bf16(64, DVT, false, true);
+        // MMA1(c): [P | O_inter (| den)] = Q'(c) [K'(c) ; S^T (; z^T)]^T, K = dk
+        auto issue_mma1 = [&](int c) {
+            const uint32_t qb = smem_u32(stg(c)), kb = qb + L::Q_BYTES;
+            const uint64_t dq = dk0(qb), dkx = dk0(kb);
+            const uint32_t acc = tmem + L::C_ACC + 128u * (uint32_t)(c % 3);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                umma_bf16(acc, kstep_k(dq, C * 128, kk), kstep_k(dkx, L::K_ACS, kk), ID1, kk > 0);
+            umma_commit(&ctl->mP[c % 3]);
+        };
+        // MMA2(c): dS = K'(c)^T V(c), K = tokens
+        auto issue_mma2 = [&](int c) {
+            const uint32_t kb = smem_u32(stg(c)) + L::Q_BYTES, vb = tb + L::VR + (uint32_t)(c % L::NV) * L::V_BYTES;
+            const uint64_t du = dmn128_0(kb, L::K_ACS), dv = dmn64_0(vb);
+            const uint32_t ds = tmem + L::C_DS + 32u * (uint32_t)(c & 1);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_bf16(ds, kstep_mn128(du, kk), kstep_mn64(dv, kk), ID2, kk > 0);
+            umma_commit(&ctl->mD[c & 1]);
+        };
+        // MMA3(c): O += P(c) V(c)
+        auto issue_mma3 = [&](int c) {
+            const uint32_t vb = tb + L::VR + (uint32_t)(c % L::NV) * L::V_BYTES;
+            const uint64_t dp = dk0(tb + L::PS + (uint32_t)(c & 1) * (C * 128)), dv = dmn64_0(vb);
+            const uint32_t acc = tmem + L::C_ACC + 128u * (uint32_t)(c % 3) + 64u;
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_bf16(acc, kstep_k(dp, C * 128, kk), kstep_mn64(dv, kk), ID3, 1u);
+            umma_commit(&ctl->m3[c % 3]);
+        };
+        auto ready = [&](bool w) {
+            if (!w) ctl->abort = 1;
+            fence_proxy_async_smem();
+            tc_fence_after_sync();
+            return w;
+        };
+        // MMA2(c) needs the chunk prepared and its V slot landed
+        auto mma2_ready = [&](int c) {
+            return ready(mbar_wait(&ctl->pfull[c % NSTG], (uint32_t)(c / NSTG) & 1u) &&
+                         mbar_wait(&ctl->vfull[c % L::NV], (uint32_t)(c / L::NV) & 1u));
+        };
+        bool ok = true;
+        if (nchunks > 0) {
+            ok = mma2_ready(0);
+            if (ok) issue_mma2(0);
+            ok = ok && ready(mbar_wait(&ctl->s0, 0u));
+            if (ok) issue_mma1(0);
+            if (ok && nchunks > 1) {
+                ok = mma2_ready(1);
+                if (ok) issue_mma2(1);
+            }
+        }
+        for (int c = 0; c < nchunks && ok; ++c) {
+            if (*reinterpret_cast<volatile int *>(&ctl->abort)) break;
+            if (c + 1 < nchunks) {
+                // the state copy of chunk c is written (and DS[c&1] read); ACC[(c+1)%3]
+                // was released by the output epilogue of chunk c-2
+                ok = mbar_wait(&ctl->sB[c & 1], (uint32_t)(c >> 1) & 1u);
+                if (ok && c >= 2) ok = mbar_wait(&ctl->oA[(c + 1) % 3], (uint32_t)((c - 2) / 3) & 1u);
+                if (!ready(ok)) break;
+                issue_mma1(c + 1);
+            }
+            if (!ready(mbar_wait(&ctl->pA[c & 1], (uint32_t)(c >> 1) & 1u))) break;
+            issue_mma3(c);
+            if (c + 2 < nchunks) {
+                if (!mma2_ready(c + 2)) break;
+                issue_mma2(c + 2);
+            }
+        }
+        // every MMA issued so far has finished before TMEM is released
+        umma_commit(&ctl->drain);
+        (void)mbar_wait(&ctl->drain, 0u);
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);

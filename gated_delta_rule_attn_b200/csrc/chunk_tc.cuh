@@ -17,8 +17,8 @@
 //     P = (phiQ phiK^T) o M,   O = phiQ S0 + P V,   den = phiQ z0 + P 1 + eps
 //     S <- S0 + phiK^T V,  z <- z0 + phiK^T 1
 //   GLA (§2.2): gamma_t = prod_{s<=t} g_s (per key dim, reference = chunk start)
-//     Qt = Q o gamma,  Kt = K / gamma,  Kh = Kt o gamma_C
-//     P = (Qt Kt^T) o M,  O = Qt S0 + P V,  S <- diag(gamma_C) S0 + Kh^T V
+//     Qt = Q o gamma,  Kt = K / gamma
+//     P = (Qt Kt^T) o M,  O = Qt S0 + P V,  S <- diag(gamma_C) (S0 + Kt^T V)
 //   Gated delta rule (page "线性注意力与 SSM", GDN box): gamma_t = prod alpha,
 //     Gamma_ti = gamma_t / gamma_i (computed as exp2 of log2 differences <= 0),
 //     A = diag(beta) (K K^T o Gamma o strict-lower), T = (I + A)^-1,
@@ -178,6 +178,18 @@ inline int sm_count() {
     return n;
 }
 
+// GLA / ELU: one CTA per (batch, head, 32-column value slab).
+template <int RULE>
+cudaError_t launch_ge(const ck::Maps &m, const ChunkParams &p, cudaStream_t st) {
+    using L = ck::GE<RULE>;
+    const int smem = (int)((sizeof(ck::GECtl) + 1023) / 1024 * 1024) + 1024 + (int)L::END;
+    cudaError_t e = allow_smem((const void *)ck::chunk_ge_kernel<RULE>, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(p.B * p.H * (p.dv / ck::DVT));
+    ck::chunk_ge_kernel<RULE><<<grid, L::NTHREADS, smem, st>>>(m, p);
+    return cudaGetLastError();
+}
+
 inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_bytes, cudaStream_t st,
                            std::string *err) {
     using namespace ck;
@@ -223,16 +235,12 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         if (e == cudaSuccess)
             chunk_gdn_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, p, static_cast<const uint8_t *>(ws));
     } else if (rule == kRuleGLA) {
-        const int smem = (int)((sizeof(GECtl) + 1023) / 1024 * 1024) + 1024 + (int)GE<kRuleGLA>::END;
-        e = allow_smem((const void *)chunk_ge_kernel<kRuleGLA>, smem);
-        if (e == cudaSuccess) chunk_ge_kernel<kRuleGLA><<<grid, GE<kRuleGLA>::NTHREADS, smem, st>>>(m, p);
+        e = launch_ge<kRuleGLA>(m, p, st);
     } else {
-        const int smem = (int)((sizeof(GECtl) + 1023) / 1024 * 1024) + 1024 + (int)GE<kRuleELU>::END;
-        e = allow_smem((const void *)chunk_ge_kernel<kRuleELU>, smem);
-        if (e == cudaSuccess) chunk_ge_kernel<kRuleELU><<<grid, GE<kRuleELU>::NTHREADS, smem, st>>>(m, p);
+        e = launch_ge<kRuleELU>(m, p, st);
     }
     if (e != cudaSuccess) {
-        *err = std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e);
+        *err = std::string("chunk kernel launch: ") + cudaGetErrorString(e);
         return 4;
     }
     return 0;

@@ -91,6 +91,14 @@ __device__ __forceinline__ void tma_load_4d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// L2 prefetch of one 4-D tile (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -270,44 +278,44 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 // phi(x) = ELU(x) + 1 (ELU alpha = 1): x + 1 for x > 0, e^x otherwise.
 __device__ __forceinline__ float elu_feature(float x) { return x > 0.f ? x + 1.f : __expf(x); }
 
-// ---------------------------------------------------------------------------
-// FMA-pipe replacements for the two transcendental operations of the chunk
-// kernels' per-element work (the special-function unit is far narrower than
-// the FMA pipe and becomes the bottleneck of those loops).
-// ---------------------------------------------------------------------------
-// 1/x for normal positive x: Newton-Raphson iteration y <- y (2 - x y) from an
-// exponent-negating integer seed bits(y0) = K - bits(x).  K = 0x7EF311C0
-// minimises the seed's worst relative error over a binade (5.1%); two steps
-// leave at most 6.6e-6.
-__device__ __forceinline__ float rcp_nr(float x) {
-    float y = __int_as_float(0x7EF311C0 - __float_as_int(x));
-    y = y * fmaf(-x, y, 2.f);
-    y = y * fmaf(-x, y, 2.f);
+// 1/x from the special-function unit's approximate reciprocal (relative error
+// about 1 ulp), for normal x; one instruction.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 
-// 2^t for t <= 0: t = n + f with n = round(t), |f| <= 1/2; 2^f = e^(f ln 2) by
-// its Taylor polynomial of degree 5 (relative error 3.3e-6 on |f| <= 1/2), then
-// scaled by 2^n through the exponent field.  Rounding uses the 1.5 * 2^23 add /
-// subtract trick, so everything stays on the FMA and integer pipes (no
-// conversion instructions).  Returns 0 below 2^-126.
-__device__ __forceinline__ float exp2_neg(float t) {
-    t = fmaxf(t, -127.f);
-    const float r = t + 12582912.f;                         // 1.5 * 2^23: round to integer
-    const int e = __float_as_int(r) - 0x4B400000;           // that integer
-    const float f = t - (r - 12582912.f);
-    float p = 1.3333558146428443e-3f;           // (ln 2)^5 / 5!
-    p = fmaf(p, f, 9.618129107628477e-3f);       // (ln 2)^4 / 4!
-    p = fmaf(p, f, 5.550410866482158e-2f);       // (ln 2)^3 / 3!
-    p = fmaf(p, f, 2.402265069591007e-1f);       // (ln 2)^2 / 2!
-    p = fmaf(p, f, 6.931471805599453e-1f);       // ln 2
-    p = fmaf(p, f, 1.f);
-    return e < -126 ? 0.f : __int_as_float(__float_as_int(p) + (e << 23));
+// ---------------------------------------------------------------------------
+// FMA-pipe exponential for the ELU feature map of the chunk kernels: there the
+// special-function unit delivers only a few results per clock per SM and
+// bounds the per-element loop.  Two lanes at a time (packed fp32 instructions).
+// ---------------------------------------------------------------------------
+// 2^t for t <= 0: t = n + f with n = round(t) (the 1.5 * 2^23 add/subtract
+// trick), |f| <= 1/2, 2^f from the degree-4 Taylor polynomial of e^(f ln 2)
+// (relative error at most 4.2e-5 on |f| <= 1/2), then 2^n added to the exponent
+// field.  t is clamped at -125 so the result stays a normal number (below
+// that the true value is under 3e-38).
+__device__ __forceinline__ float2 exp2_neg2(float2 t) {
+    t = make_float2(fmaxf(t.x, -125.f), fmaxf(t.y, -125.f));
+    const float2 magic = make_float2(12582912.f, 12582912.f);
+    const float2 r = __fadd2_rn(t, magic);
+    const float2 n = __fadd2_rn(r, make_float2(-12582912.f, -12582912.f));
+    const float2 f = __fadd2_rn(t, make_float2(-n.x, -n.y));
+    float2 q = make_float2(9.618129107628477e-3f, 9.618129107628477e-3f);   // (ln 2)^4 / 4!
+    q = __ffma2_rn(q, f, make_float2(5.550410866482158e-2f, 5.550410866482158e-2f));   // (ln 2)^3 / 3!
+    q = __ffma2_rn(q, f, make_float2(2.402265069591007e-1f, 2.402265069591007e-1f));   // (ln 2)^2 / 2!
+    q = __ffma2_rn(q, f, make_float2(6.931471805599453e-1f, 6.931471805599453e-1f));   // ln 2
+    q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
+    return make_float2(__int_as_float(__float_as_int(q.x) + ((__float_as_int(r.x) - 0x4B400000) << 23)),
+                       __int_as_float(__float_as_int(q.y) + ((__float_as_int(r.y) - 0x4B400000) << 23)));
 }
 
-// phi(x) = ELU(x) + 1 with e^x = 2^(x log2 e) evaluated on the FMA pipe.
-__device__ __forceinline__ float elu_feature_fma(float x) {
-    return x > 0.f ? x + 1.f : exp2_neg(fminf(x, 0.f) * 1.4426950408889634f);
+// phi(x) = ELU(x) + 1 for two lanes, the exponential on the FMA pipe.
+__device__ __forceinline__ float2 elu_feature2(float2 x) {
+    const float2 e = exp2_neg2(make_float2(fminf(x.x, 0.f) * 1.4426950408889634f, fminf(x.y, 0.f) * 1.4426950408889634f));
+    return make_float2(x.x > 0.f ? x.x + 1.f : e.x, x.y > 0.f ? x.y + 1.f : e.y);
 }
+
 
 }  // namespace la
