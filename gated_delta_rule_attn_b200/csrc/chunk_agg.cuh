@@ -1,0 +1,203 @@
+// chunk_agg.cuh — sequence-parallel prefill of normalized ELU+1, first pass.
+//
+// The ELU+1 state after token t is a plain sum over the tokens up to t
+// (page "Linear / RNN 路线", §2.1: S_t = S_{t-1} + phi(k_t) v_t^T, z_t = z_{t-1} +
+// phi(k_t)), so a sequence cut into segments can be processed by independent
+// CTAs once each segment j knows S0 + the contributions of segments < j.  This
+// kernel computes those contributions: for every (batch, head) and every
+// segment but the last, dS = sum_t phi(k_t) v_t^T (dk x dv) and dz = sum_t
+// phi(k_t), each segment split into `nparts` chunk ranges handled by separate
+// CTAs (partial sums; the main pass adds them up).
+//
+// 9 warps per CTA:
+//   warps 0-7  phi(K) in place (FMA-pipe exponential; zero past T) and the
+//              running sums of phi(k) per key dim;
+//   warp 8     TMA loads of k and v into a ring of stages and, lane 0, the MMAs
+//              dS += phi(K)^T V, accumulated in TMEM over the whole range.
+// Afterwards warps 0-3 copy the accumulator (one key-dim row per thread) out.
+#pragma once
+
+#include "device.cuh"
+
+namespace la {
+
+struct AggParams {
+    int64_t B, T, H, dv;
+    float *agg;     // [B*H][nseg-1][nparts] blocks of DK*dv (dS, row-major) + DK (dz) floats
+    int nseg, nparts, seg_chunks;
+};
+
+namespace ck {
+
+template <int DV>
+struct AG {
+    static constexpr int NSTG = 4;
+    static constexpr uint32_t K_BYTES = C * 128 * KA;   // phi(K), [atom col][64 rows], 128-byte swizzle
+    static constexpr uint32_t V_BYTES = C * DV * 2;     // DV/32 slabs of [64][32], 64-byte swizzle
+    static constexpr uint32_t STG_BYTES = K_BYTES + V_BYTES;
+    static constexpr uint32_t END = NSTG * STG_BYTES;
+    static constexpr uint32_t TMEM_COLS = DV;           // 32, 64 or 128
+};
+
+struct AGCtl {
+    uint64_t full[4], pfull[4], mdone[4], done;
+    uint32_t tmem_base;
+    int abort, stop;
+    alignas(16) float2 tot[4][64];
+};
+
+template <int DV>
+__global__ void __launch_bounds__(288, 1)
+chunk_agg_kernel(const __grid_constant__ Maps maps, const AggParams p) {
+    using L = AG<DV>;
+    constexpr int NSTG = L::NSTG;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    AGCtl *ctl = reinterpret_cast<AGCtl *>(smem_raw);
+    uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(AGCtl) + (smem_u32(smem_raw) & 1023u)) -
+                     (smem_u32(smem_raw) & 1023u);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int part = (int)(blockIdx.x % p.nparts);
+    const int rest = (int)(blockIdx.x / p.nparts);
+    const int seg = rest % (p.nseg - 1);
+    const int64_t bh = rest / (p.nseg - 1);
+    const int64_t b = bh / p.H, h = bh % p.H;
+    const int cseg = seg * p.seg_chunks;   // segments before the last are full
+    const int cbeg = cseg + (int)((int64_t)p.seg_chunks * part / p.nparts);
+    const int cend = cseg + (int)((int64_t)p.seg_chunks * (part + 1) / p.nparts);
+    const int n = cend - cbeg;
+    float *out = p.agg + ((bh * (p.nseg - 1) + seg) * p.nparts + part) * (int64_t)(DK * DV + DK);
+
+    auto stg = [&](int c) { return tiles + (uint32_t)(c % NSTG) * L::STG_BYTES; };
+
+    if (tid == 0) {
+        for (int s = 0; s < NSTG; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->pfull[s], 8);
+            mbar_init(&ctl->mdone[s], 1);
+        }
+        mbar_init(&ctl->done, 1);
+        ctl->abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(&maps.v);
+    }
+    if (warp == 0) {
+        tmem_alloc(&ctl->tmem_base, L::TMEM_COLS);
+        tc_fence_before_sync();
+    }
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp < 8) {
+        // phi(K) in place; thread (pr, qt) owns key dims 2pr, 2pr+1 of tokens
+        // 16qt..16qt+15 (a warp covers a full 128-byte row per access)
+        const bool leader = (tid == 0);
+        const int pr = tid & 63, qt = tid >> 6;
+        const int a = pr >> 5;
+        const uint32_t cpos = (uint32_t)((pr & 31) >> 2), cin = (uint32_t)(pr & 3) << 2;
+        float2 zacc = make_float2(0.f, 0.f);
+        for (int c = 0; c < n; ++c) {
+            const int s = c % NSTG;
+            const int nvalid = (int)min((int64_t)C, p.T - (int64_t)(cbeg + c) * C);
+            if (leader) ctl->stop = ctl->abort;
+            bar_named(1, 256);
+            if (ctl->stop) break;
+            if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
+            uint8_t *ka = stg(c) + a * (C * 128);
+            auto off = [&](int i) {
+                const uint32_t t = (uint32_t)(16 * qt + i);
+                return t * 128u + (((cpos ^ t) & 7u) << 4) + cin;
+            };
+            uint32_t kv[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) kv[i] = *reinterpret_cast<const uint32_t *>(ka + off(i));
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float2 fk = elu_feature2(unpack_bf16x2(kv[i]));
+                if (16 * qt + i >= nvalid) fk = make_float2(0.f, 0.f);
+                *reinterpret_cast<uint32_t *>(ka + off(i)) = pack_bf16x2(fk.x, fk.y);
+                zacc = __fadd2_rn(zacc, fk);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->pfull[s]);
+        }
+        ctl->tot[qt][pr] = zacc;
+        bar_named(1, 256);
+        if (qt == 0 && !ctl->abort) {
+            const float2 z = __fadd2_rn(__fadd2_rn(ctl->tot[0][pr], ctl->tot[1][pr]),
+                                        __fadd2_rn(ctl->tot[2][pr], ctl->tot[3][pr]));
+            *reinterpret_cast<float2 *>(out + DK * DV + 2 * pr) = z;
+        }
+    } else if (lane == 0) {
+        // TMA producer and MMA issuer
+        constexpr uint32_t ID = idesc_bf16(128, DV, true, true);
+        int issued = -1;
+        auto load = [&](int c) {
+            const int s = c % NSTG;
+            uint8_t *st = stg(c);
+            const int t0 = (cbeg + c) * C;
+            mbar_arrive_expect_tx(&ctl->full[s], L::STG_BYTES);
+#pragma unroll
+            for (int a = 0; a < KA; ++a)
+                tma_load_4d(st + a * (C * 128), &maps.k, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
+#pragma unroll
+            for (int j = 0; j < DV / DVT; ++j)
+                tma_load_4d(st + L::K_BYTES + j * (C * DVT * 2), &maps.v, &ctl->full[s], j * DVT, (int)h, t0, (int)b);
+            issued = c;
+        };
+        for (int c = 0; c < NSTG && c < n; ++c) load(c);
+        for (int c = 0; c < n; ++c) {
+            const int s = c % NSTG;
+            if (!mbar_wait(&ctl->pfull[s], (uint32_t)(c / NSTG) & 1u)) {
+                ctl->abort = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t kb = smem_u32(stg(c)), vb = kb + L::K_BYTES;
+            const uint64_t du = dmn128_0(kb, C * 128), dv = dmn64_0(vb);
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_bf16(tmem, kstep_mn128(du, kk), kstep_mn64(dv, kk), ID, (c > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&ctl->mdone[s]);
+            // the stage of chunk c-1 is free once its MMA is done: refill it
+            if (c >= 1 && c - 1 + NSTG < n) {
+                if (!mbar_wait(&ctl->mdone[(c - 1) % NSTG], (uint32_t)((c - 1) / NSTG) & 1u)) {
+                    ctl->abort = 1;
+                    break;
+                }
+                load(c - 1 + NSTG);
+            }
+        }
+        umma_commit(&ctl->done);
+        if (ctl->abort)   // let copies still in flight land before the CTA exits
+            for (int c = (issued - NSTG + 1 > 0 ? issued - NSTG + 1 : 0); c <= issued; ++c)
+                (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
+    }
+    if (warp < 4) {   // dS rows out: thread d = key dim
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->done, 0u));
+        tc_fence_after_sync();
+        const int d = 32 * warp + lane;
+        const uint32_t tq = tmem + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+        for (int j = 0; j < DV / 32; ++j) {
+            float x[32];
+            tmem_ld32(tq + 32u * (uint32_t)j, x);
+            tmem_wait_ld();
+            if (ok && !ctl->abort) {
+                float *dst = out + (int64_t)d * DV + 32 * j;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(dst + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+            }
+        }
+        tc_fence_before_sync();
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
+}
+
+}  // namespace ck
+}  // namespace la

@@ -102,9 +102,12 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
     const int quad = warp & 3;
     const int nslab = (int)(p.dv / DVT);
     const int dvt = (int)(blockIdx.x % nslab);
-    const int64_t bh = blockIdx.x / nslab;
+    const int seg = (int)((blockIdx.x / nslab) % p.nseg);
+    const int64_t bh = blockIdx.x / nslab / p.nseg;
     const int64_t b = bh / p.H, h = bh % p.H;
-    const int nchunks = (int)((p.T + C - 1) / C);
+    // this CTA's chunks: [cbase, cbase + nchunks) of the sequence
+    const int cbase = seg * p.seg_chunks;
+    const int nchunks = (int)min((int64_t)p.seg_chunks, (p.T + C - 1) / C - cbase);
 
     auto stg = [&](int c) { return tiles + L::STG + (uint32_t)(c % NSTG) * L::STG_BYTES; };
 
@@ -160,13 +163,14 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         auto gate_load = [&](int c) {
             uint64_t *bar = &ctl->gfull[c & 1];
             mbar_arrive_expect_tx(bar, L::G_BYTES);
-            tma_load_4d(tiles + L::GT + (uint32_t)(c & 1) * L::G_BYTES, &maps.g, bar, 0, (int)h, c * C, (int)b);
+            tma_load_4d(tiles + L::GT + (uint32_t)(c & 1) * L::G_BYTES, &maps.g, bar, 0, (int)h, (cbase + c) * C,
+                        (int)b);
         };
         if (kGLA && leader)
             for (int c = 0; c < 2 && c < nchunks; ++c) gate_load(c);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTG;
-            const int nvalid = (int)min((int64_t)C, p.T - (int64_t)c * C);
+            const int nvalid = (int)min((int64_t)C, p.T - (int64_t)(cbase + c) * C);
             if (leader) ctl->stopP = ctl->abort;
             bar_named(1, 256);
             if (ctl->stopP) break;
@@ -264,7 +268,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         auto load_chunk = [&](int c) {
             const int s = c % NSTG;
             uint8_t *st = stg(c);
-            const int t0 = c * C;
+            const int t0 = (cbase + c) * C;
             mbar_arrive_expect_tx(&ctl->full[s], 2u * L::Q_BYTES);
 #pragma unroll
             for (int a = 0; a < KA; ++a) {
@@ -280,8 +284,8 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         auto load_v = [&](int c) {
             const int j = c % L::NV;
             mbar_arrive_expect_tx(&ctl->vfull[j], L::V_BYTES);
-            tma_load_4d(tiles + L::VR + (uint32_t)j * L::V_BYTES, &maps.v, &ctl->vfull[j], dvt * DVT, (int)h, c * C,
-                        (int)b);
+            tma_load_4d(tiles + L::VR + (uint32_t)j * L::V_BYTES, &maps.v, &ctl->vfull[j], dvt * DVT, (int)h,
+                        (cbase + c) * C, (int)b);
             issued_v = c;
         };
         if (a0) {
@@ -291,7 +295,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         for (int c = 0; c < nchunks; ++c) {
             const int bb = c & 1, j3 = c % 3;
             const uint32_t acc = L::C_ACC + 128u * (uint32_t)j3;
-            const int64_t t0 = (int64_t)c * C;
+            const int64_t t0 = (int64_t)(cbase + c) * C;
             const int nvalid = (int)min((int64_t)C, p.T - t0);
             if (aborted(ctl)) break;
             if (!__all_sync(0xffffffffu, mbar_wait(&ctl->mP[j3], (uint32_t)(c / 3) & 1u))) {
@@ -386,6 +390,18 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                 S[jj] = x.x; S[jj + 1] = x.y; S[jj + 2] = x.z; S[jj + 3] = x.w;
             }
             if (!kGLA && p.z0) z = p.z0[bh * DK + d];
+            // sequence-parallel ELU+1: add the contributions of the earlier segments
+            const int64_t blk = (int64_t)DK * p.dv + DK;
+            for (int i = 0; i < seg * p.nparts; ++i) {
+                const float *a = p.agg + (bh * (p.nseg - 1) * p.nparts + i) * blk;
+                const float *row = a + (int64_t)d * p.dv + dvt * DVT;
+#pragma unroll
+                for (int jj = 0; jj < DVT; jj += 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(row + jj);
+                    S[jj] += x.x; S[jj + 1] += x.y; S[jj + 2] += x.z; S[jj + 3] += x.w;
+                }
+                z += a[DK * p.dv + d];
+            }
         }
         // bf16 copy of S^T (and z^T) into rows 64.. of the K tile of stage s
         auto write_state = [&](int s) {
@@ -442,7 +458,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             tc_fence_before_sync();
             mbar_arrive(&ctl->sB[bb]);
         }
-        if (!ctl->abort) {
+        if (!ctl->abort && seg == p.nseg - 1) {
             if (p.S_out) {
                 float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVT);
 #pragma unroll

@@ -65,6 +65,10 @@ struct ChunkParams {
     float *S_out, *z_out;
     void *o;
     float eps;
+    // sequence-parallel ELU+1 (nseg > 1): segment j of every (batch, head)
+    // starts from S0 plus the partial sums in `agg` of segments < j
+    int nseg = 1, nparts = 1, seg_chunks = 0;
+    const float *agg = nullptr;
 };
 
 namespace ck {
@@ -158,24 +162,53 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 
 #include "chunk_gdn.cuh"
 #include "chunk_ge.cuh"
+#include "chunk_agg.cuh"
 
 namespace la {
 
 // Host launcher.  Returns an la_status value (0 = ok).
-// Device workspace the chunked path needs: the gated delta rule keeps the
-// per-chunk T diag(beta) | T diag(beta gamma) operand images (16 KB per
-// (batch, head, chunk)); the other rules need none.
-inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H) {
-    if (rule != kRuleGDN || T <= 0) return 0;
-    return (size_t)(B * H * ((T + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;
-}
-
 inline int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
         n = 148;
     return n;
+}
+
+// Sequence parallelism for ELU+1: when the (batch, head, value slab) CTAs fill
+// only a fraction of the SMs, every sequence is cut into `nseg` segments of
+// `seg_chunks` chunks that run side by side; a first pass reduces the state
+// contributions of each segment but the last, in `nparts` pieces per segment.
+struct SegPlan {
+    int nseg = 1, nparts = 1, seg_chunks = 0;
+};
+
+inline SegPlan seg_plan(int rule, int64_t B, int64_t T, int64_t H, int64_t dv) {
+    SegPlan sp;
+    const int64_t nch = (T + ck::C - 1) / ck::C;
+    sp.seg_chunks = (int)nch;
+    if (rule != kRuleELU || nch < 16 || dv % ck::DVT != 0) return sp;
+    const int64_t sms = sm_count(), ctas = B * H * (dv / ck::DVT);
+    const int64_t nseg = std::min<int64_t>(sms / ctas, nch / 8);
+    if (nseg < 2) return sp;
+    sp.seg_chunks = (int)((nch + nseg - 1) / nseg);
+    sp.nseg = (int)((nch + sp.seg_chunks - 1) / sp.seg_chunks);   // no empty segment
+    if (sp.nseg < 2) return SegPlan{1, 1, (int)nch};
+    const int64_t units = B * H * (sp.nseg - 1);
+    sp.nparts = (int)std::max<int64_t>(1, std::min<int64_t>(sms / units, sp.seg_chunks / 4));
+    return sp;
+}
+
+// Device workspace the chunked path needs: the gated delta rule keeps the
+// per-chunk T diag(beta) | T diag(beta gamma) operand images (16 KB per
+// (batch, head, chunk)); sequence-parallel ELU+1 the partial state sums of its
+// first pass; GLA needs none.
+inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv) {
+    if (T <= 0) return 0;
+    if (rule == kRuleGDN) return (size_t)(B * H * ((T + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;
+    const SegPlan sp = seg_plan(rule, B, T, H, dv);
+    if (sp.nseg < 2) return 0;
+    return (size_t)(B * H * (sp.nseg - 1) * sp.nparts) * (size_t)(ck::DK * dv + ck::DK) * sizeof(float);
 }
 
 // GLA / ELU: one CTA per (batch, head, 32-column value slab).
@@ -185,8 +218,20 @@ cudaError_t launch_ge(const ck::Maps &m, const ChunkParams &p, cudaStream_t st) 
     const int smem = (int)((sizeof(ck::GECtl) + 1023) / 1024 * 1024) + 1024 + (int)L::END;
     cudaError_t e = allow_smem((const void *)ck::chunk_ge_kernel<RULE>, smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)(p.B * p.H * (p.dv / ck::DVT));
+    const unsigned grid = (unsigned)(p.B * p.H * (p.dv / ck::DVT) * p.nseg);
     ck::chunk_ge_kernel<RULE><<<grid, L::NTHREADS, smem, st>>>(m, p);
+    return cudaGetLastError();
+}
+
+// First pass of sequence-parallel ELU+1.
+template <int DV>
+cudaError_t launch_agg(const ck::Maps &m, const AggParams &a, cudaStream_t st) {
+    using L = ck::AG<DV>;
+    const int smem = (int)((sizeof(ck::AGCtl) + 1023) / 1024 * 1024) + 1024 + (int)L::END;
+    cudaError_t e = allow_smem((const void *)ck::chunk_agg_kernel<DV>, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(a.B * a.H * (a.nseg - 1) * a.nparts);
+    ck::chunk_agg_kernel<DV><<<grid, 288, smem, st>>>(m, a);
     return cudaGetLastError();
 }
 
@@ -215,7 +260,7 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
     const unsigned grid = (unsigned)(p.B * p.H * (p.dv / DVT));
     cudaError_t e;
     if (rule == kRuleGDN) {
-        const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H);
+        const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv);
         if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
             *err = "the gated delta rule needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
             return 8;
@@ -234,10 +279,28 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel, smem);
         if (e == cudaSuccess)
             chunk_gdn_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, p, static_cast<const uint8_t *>(ws));
-    } else if (rule == kRuleGLA) {
-        e = launch_ge<kRuleGLA>(m, p, st);
     } else {
-        e = launch_ge<kRuleELU>(m, p, st);
+        const SegPlan sp = seg_plan(rule, p.B, p.T, p.H, p.dv);
+        ChunkParams q = p;
+        if (sp.nseg > 1) {
+            const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv);
+            if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
+                *err = "sequence-parallel ELU+1 needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
+                return 8;
+            }
+            AggParams a{};
+            a.B = p.B; a.T = p.T; a.H = p.H; a.dv = p.dv;
+            a.agg = static_cast<float *>(ws);
+            a.nseg = sp.nseg; a.nparts = sp.nparts; a.seg_chunks = sp.seg_chunks;
+            e = p.dv == 32 ? launch_agg<32>(m, a, st) : p.dv == 64 ? launch_agg<64>(m, a, st) : launch_agg<128>(m, a, st);
+            if (e != cudaSuccess) {
+                *err = std::string("chunk kernel launch: ") + cudaGetErrorString(e);
+                return 4;
+            }
+            q.agg = a.agg;
+        }
+        q.nseg = sp.nseg; q.nparts = sp.nparts; q.seg_chunks = sp.seg_chunks;
+        e = rule == kRuleGLA ? launch_ge<kRuleGLA>(m, q, st) : launch_ge<kRuleELU>(m, q, st);
     }
     if (e != cudaSuccess) {
         *err = std::string("chunk kernel launch: ") + cudaGetErrorString(e);

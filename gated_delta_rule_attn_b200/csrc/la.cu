@@ -238,7 +238,7 @@ la_status la_fwd(const la_fwd_args *args, void *stream) {
     la_status r = validate_fwd(args, true);
     if (r != LA_OK) return r;
     if (uses_chunk_kernels(*args)) {
-        const size_t need = la::chunk_workspace_bytes((int)args->rule, args->B, args->T, args->H);
+        const size_t need = la::chunk_workspace_bytes((int)args->rule, args->B, args->T, args->H, args->dv);
         if (need && (!args->workspace || args->workspace_bytes < need || !aligned16(args->workspace)))
             return fail(LA_ERR_WORKSPACE,
                         "workspace missing, misaligned or smaller than la_fwd_workspace_size()");
@@ -283,7 +283,7 @@ la_status la_fwd_noalloc(const la_fwd_args *args, void *stream) {
     a.workspace = nullptr;
     a.workspace_bytes = 0;
     const size_t need =
-        uses_chunk_kernels(a) ? la::chunk_workspace_bytes((int)a.rule, a.B, a.T, a.H) : 0;
+        uses_chunk_kernels(a) ? la::chunk_workspace_bytes((int)a.rule, a.B, a.T, a.H, a.dv) : 0;
     if (need > LA_NOALLOC_SCRATCH_BYTES)
         return fail(LA_ERR_WORKSPACE, "problem needs " + std::to_string(need) +
                                           " bytes of scratch; la_fwd_noalloc has " +
@@ -302,7 +302,7 @@ la_status la_fwd_workspace_size(const la_fwd_args *args, size_t *bytes) {
     la_status r = validate_fwd(args, false);
     if (r != LA_OK) return r;
     *bytes = uses_chunk_kernels(*args)
-                 ? la::chunk_workspace_bytes((int)args->rule, args->B, args->T, args->H)
+                 ? la::chunk_workspace_bytes((int)args->rule, args->B, args->T, args->H, args->dv)
                  : 0;
     return ok();
 }
@@ -346,7 +346,7 @@ static void staging_layout(const la_fwd_args *a, StagingLayout *L) {
     const size_t sb = (size_t)(a->B * a->H * a->dk * a->dv) * 4;
     const size_t zb = (size_t)(a->B * a->H * a->dk) * 4;
     const size_t wb = uses_chunk_kernels(*a)
-                          ? la::chunk_workspace_bytes((int)a->rule, a->B, a->T, a->H)
+                          ? la::chunk_workspace_bytes((int)a->rule, a->B, a->T, a->H, a->dv)
                           : 0;
     const size_t b[11] = {tok * a->dk * es, tok * a->dk * es, tok * a->dv * es, gb,
                           a->beta ? tok * 4 : 0, a->S0 ? sb : 0, a->z0 ? zb : 0,

@@ -149,6 +149,15 @@ def test_single_sequence_long_chain(la, rule):
     check(p, *run_gpu(la, p), TOL_BF16)
 
 
+@pytest.mark.parametrize("B,H,T,dv", [(1, 2, 1500, 64), (1, 1, 4096 + 33, 32), (2, 1, 3000, 128)])
+def test_elu_sequence_parallel(la, B, H, T, dv):
+    """Few heads and long sequences: the ELU+1 path cuts every sequence into
+    segments that run side by side, each starting from S0 plus the state
+    contributions of the earlier segments (summed by a first pass)."""
+    p = workloads.make_problem("elu", B, T, H, 128, dv, seed=T + dv, init_state="abs")
+    check(p, *run_gpu(la, p), TOL_BF16)
+
+
 @pytest.mark.parametrize("rule", ["elu", "gla", "gdn"])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_zero_length(la, rule, dtype):
