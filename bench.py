@@ -203,7 +203,10 @@ class Legs:
         self.z_elu = e(1, 16, 128, device="cuda")
         self.o_dec = e(256, 16, 128, dtype=torch.bfloat16, device="cuda")
         self.names = ["gla_prefill", "gdn_prefill", "elu_prefill", "gla_decode", "gdn_decode"]
-        self.launches_per_step = 5
+        # kernels per step: GLA 1; gated delta rule 2 (T operand images, then the
+        # main pass); ELU+1 at this shape 2 (segment sums, then the segment-parallel
+        # main pass); each decode step 1
+        self.launches_per_step = 7
 
     def run(self, name):
         la = self.la
@@ -406,34 +409,43 @@ def _oracle_inputs():
     return _ORACLE_INPUTS
 
 
-def oracle_sample(T: int, seed: int = 0):
-    """GLA + gated-delta prefill, batch 0, all 16 heads, first T tokens of the
-    d=128 T=8192 workloads; returns (seconds, full tokens processed)."""
+def oracle_sample(T: int, batches: int = 1, repeats: int = 1):
+    """GLA + gated-delta prefill, the first `batches` batches (all 16 heads) and
+    first T tokens of the d=128 T=8192 workloads, `repeats` times; returns
+    (seconds, tokens processed)."""
     import oracle
     oracle.build.build()
     gla, gdn = _oracle_inputs()
-    sl = lambda x: x[:1, :T].contiguous()
+    sl = lambda x: x[:batches, :T].contiguous()
     args_gla = [sl(x) for x in (gla.q, gla.k, gla.v, gla.g)]
     args_gdn = [sl(x) for x in (gdn.q, gdn.k, gdn.v, gdn.g, gdn.beta)]
     t0 = time.perf_counter()
-    oracle.gla_fwd(*args_gla)
-    oracle.gdn_fwd(*args_gdn)
+    for _ in range(repeats):
+        oracle.gla_fwd(*args_gla)
+        oracle.gdn_fwd(*args_gdn)
     dt = time.perf_counter() - t0
-    return dt, 2 * T
+    return dt, 2 * T * batches * repeats
 
 
 def cpu_baseline(budget_s: float = 15.0):
     import oracle
-    # size the sample so that the timed part takes about budget_s seconds
+    # size the sample so that the timed part takes about budget_s seconds: a
+    # prefix of batch 0, or the whole workload (both batches) repeated
     t_probe, tok_probe = oracle_sample(128)
-    T = int(min(8192, max(128, 128 * budget_s / max(t_probe, 1e-3))))
-    T = max(64, (T // 64) * 64)
-    dt, tokens = oracle_sample(T)
+    want = tok_probe / max(t_probe, 1e-3) * budget_s
+    if want <= 2 * 8192:
+        T, B, R = max(64, int(want / 2) // 64 * 64), 1, 1
+    else:
+        T = 8192
+        B = 2 if want >= 2 * 2 * 8192 else 1
+        R = max(1, min(64, round(want / (2 * T * B))))
+    dt, tokens = oracle_sample(T, B, R)
+    what = (f"first {T} tokens of batch 0" if B == 1 and R == 1 else
+            f"all {B} batch(es), all 8192 tokens, {R} time(s)")
     return {"value": round(tokens / dt, 1), "unit": "tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"fp64 C oracle (OpenMP over heads): GLA + gated-delta prefill, batch 0, "
-                      f"all 16 heads, first {T} tokens of each d=128 T=8192 workload; "
-                      f"{dt:.1f} s"}
+            "sample": f"fp64 C oracle (OpenMP over heads): GLA + gated-delta prefill of the d=128 "
+                      f"T=8192 workloads, 16 heads, {what}; {dt:.1f} s"}
 
 
 def run_reference(args):

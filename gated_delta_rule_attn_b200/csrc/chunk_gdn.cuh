@@ -16,10 +16,11 @@
 //                 [Q;K] K^T (tcgen05, M=128) -> P = (Q K^T) o Gamma o M,
 //                 U = T diag(beta) V  and  W_k = T diag(beta gamma) K (tcgen05);
 //   warps 5-8   "state" group, the recurrence across chunks:
-//                 X1 = W_k S0, X2 = Q S0 (S0 as a bf16 operand),
-//                 W = U - X1,  dS = K^T diag(gamma_C/gamma) W,  PW = P W,
-//                 S <- gamma_C S + dS (fp32, one state row per thread),
-//                 O = diag(gamma) X2 + PW.
+//                 X1 = W_k S0 (S0 as a bf16 operand), W = U - X1,
+//                 dS = K^T diag(gamma_C/gamma) W,
+//                 S <- gamma_C S + dS (fp32, one state row per thread);
+//               off that chain, issued after dS and run during the state
+//               update: X2 = Q S0, PW = P W, then O = diag(gamma) X2 + PW.
 // The derivation of the WY / UT form is in chunk_tc.cuh's header.
 //
 // Pairwise decays Gamma_ti = gamma_t / gamma_i (i <= t) are products of
@@ -56,13 +57,13 @@ constexpr uint32_t QK_ACS = 128 * 128;               // one atom column: Q rows 
 constexpr uint32_t STG_QK = 0;                       // NSTG x 2 atom columns
 constexpr uint32_t STG_QK_BYTES = 2 * QK_ACS;
 constexpr uint32_t STG_V = STG_QK + NSTG * STG_QK_BYTES;   // NSTG x [64][32] bf16, 64 B swizzle
-constexpr uint32_t STG_TT = STG_V + NSTG * 4096;           // NSTG x (T diag(beta), T diag(beta gamma))
-constexpr uint32_t TP = STG_TT + NSTG * TT_BYTES;    // 2 x P [64][64] bf16
+constexpr uint32_t STG_TT = STG_V + NSTG * 4096;           // 2 x (T diag(beta), T diag(beta gamma))
+constexpr uint32_t TP = STG_TT + 2 * TT_BYTES;       // 2 x P [64][64] bf16
 constexpr uint32_t TWK = TP + 2 * 8192;              // 2 x W_k [64][128] bf16 (2 atom columns)
 constexpr uint32_t TWS = TWK + 2 * 16384;            // W       [64][32] 64 B swizzle
 constexpr uint32_t TWGS = TWS + 4096;                // gamma_C/gamma W
-constexpr uint32_t TSS = TWGS + 4096;                // S       [128][32] 64 B swizzle
-constexpr uint32_t TEND = TSS + 8192;
+constexpr uint32_t TSS = TWGS + 4096;                // 2 x S   [128][32] 64 B swizzle
+constexpr uint32_t TEND = TSS + 2 * 8192;
 
 // Prep-kernel shared memory.
 constexpr int AF_LD = 68;
@@ -75,7 +76,8 @@ constexpr int PREP_THREADS = 128;
 
 struct GCtl {
     uint64_t full[NSTG], empty[NSTG];
-    uint64_t l_done, lw_full[2], lw_empty[2], x1_done, ds_done;
+    uint64_t l_done, lw_full[2], lw_empty[2], x1_done, ds_done, o_done;
+    uint64_t ttfree[2];              // the local group's MMAs of a T-image slot are done
     uint32_t tmem_base;
     int abort, stopL, stopS;
     int fast[NSTG];
@@ -481,10 +483,12 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ctl->lw_full[i], 128);
             mbar_init(&ctl->lw_empty[i], 1);
+            mbar_init(&ctl->ttfree[i], 1);
         }
         mbar_init(&ctl->l_done, 1);
         mbar_init(&ctl->x1_done, 1);
         mbar_init(&ctl->ds_done, 1);
+        mbar_init(&ctl->o_done, 1);
         ctl->abort = 0;
         fence_barrier_init();
         tma_prefetch_desc(&maps.q);
@@ -508,16 +512,19 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
 
     auto stage_qk = [&](int c) { return tb + STG_QK + (uint32_t)(c % NSTG) * STG_QK_BYTES; };
     auto stage_v = [&](int c) { return tb + STG_V + (uint32_t)(c % NSTG) * 4096u; };
-    auto stage_tt = [&](int c) { return tb + STG_TT + (uint32_t)(c % NSTG) * TT_BYTES; };
+    auto stage_tt = [&](int c) { return tb + STG_TT + (uint32_t)(c & 1) * TT_BYTES; };
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
         int issued = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTG;
-            if (c >= NSTG) {
+            if (c >= 2) {   // stage and T-image slot released by their last readers
                 int ok = 1;
-                if (lane == 0) ok = mbar_wait(&ctl->empty[s], (uint32_t)((c / NSTG) - 1) & 1u);
+                if (lane == 0) {
+                    if (c >= NSTG) ok = mbar_wait(&ctl->empty[s], (uint32_t)((c / NSTG) - 1) & 1u);
+                    ok = mbar_wait(&ctl->ttfree[c & 1], (uint32_t)((c - 2) >> 1) & 1u) && ok;
+                }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok && lane == 0) ctl->abort = 1;
             }
@@ -536,7 +543,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 }
                 tma_load_4d(tiles + STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, t0,
                             (int)b);
-                bulk_load(tiles + STG_TT + s * TT_BYTES, ws + (bh * nchunks + c) * (int64_t)TT_BYTES,
+                bulk_load(tiles + STG_TT + (c & 1) * TT_BYTES, ws + (bh * nchunks + c) * (int64_t)TT_BYTES,
                           TT_BYTES, &ctl->full[s]);
             }
             // the chunk's decay factors: b = log2 of the inclusive cumulative alpha,
@@ -589,6 +596,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                     }
                 }
                 umma_commit(&ctl->l_done);
+                umma_commit(&ctl->ttfree[c & 1]);
             }
             if (!mbar_wait(&ctl->l_done, (uint32_t)c & 1u)) ctl->abort = 1;
             tc_fence_after_sync();
@@ -637,14 +645,13 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         }
         fence_proxy_async_smem();
         bar_named(2, 128);
-        auto issue_x = [&](int c) {
-            const uint32_t qk = stage_qk(c), wk = tb + TWK + (uint32_t)(c & 1) * 16384u, ss = tb + TSS;
+        // the bf16 copy of the state entering chunk c sits in buffer c & 1
+        auto ss_of = [&](int c) { return tb + TSS + (uint32_t)(c & 1) * 8192u; };
+        auto issue_x1 = [&](int c) {
+            const uint32_t wk = tb + TWK + (uint32_t)(c & 1) * 16384u, ss = ss_of(c);
 #pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk) {   // X1 and X2 interleaved (independent)
+            for (int kk = 0; kk < DK / 16; ++kk)
                 umma_bf16(tmem + C_X1, desc_k(wk, C * 128, kk), desc_mn64(ss, kk), ID_X, kk > 0);
-                umma_bf16(tmem + C_X2 + 32u * (c & 1), desc_k(qk, QK_ACS, kk), desc_mn64(ss, kk), ID_X,
-                          kk > 0);
-            }
             umma_commit(&ctl->x1_done);
         };
         // half row (16 columns, 2 chunks of 16 B) of a [rows][32] bf16 tile, 64-byte swizzle
@@ -663,7 +670,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         if (leader && nchunks > 0) {
             if (!mbar_wait(&ctl->lw_full[0], 0)) ctl->abort = 1;
             tc_fence_after_sync();
-            issue_x(0);
+            issue_x1(0);
         }
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTG, pb = c & 1;
@@ -695,15 +702,20 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             bar_named(2, 128);
             if (leader) {
                 tc_fence_after_sync();
-                const uint32_t kb = stage_qk(c) + 64 * 128;
+                const uint32_t qk = stage_qk(c), kb = qk + 64 * 128, ss = ss_of(c);
+                // dS first (the recurrence waits for it), then the output-only X2 and PW
 #pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk) {   // dS and PW interleaved (independent)
-                    umma_bf16(tmem + C_DS, desc_mn128(kb, QK_ACS, kk), desc_mn64(tb + TWGS, kk), ID_DS,
-                              kk > 0);
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + C_DS, desc_mn128(kb, QK_ACS, kk), desc_mn64(tb + TWGS, kk), ID_DS, kk > 0);
+                umma_commit(&ctl->ds_done);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    umma_bf16(tmem + C_X2 + 32u * pb, desc_k(qk, QK_ACS, kk), desc_mn64(ss, kk), ID_X, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
                     umma_bf16(tmem + C_PW + 32u * pb, desc_k(tb + TP + pb * 8192u, C * 128, kk),
                               desc_mn64(tb + TWS, kk), ID_X, kk > 0);
-                }
-                umma_commit(&ctl->ds_done);
+                umma_commit(&ctl->o_done);
                 umma_commit(&ctl->lw_empty[pb]);
                 umma_commit(&ctl->empty[s]);
             }
@@ -715,7 +727,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < DVT; ++j) S[j] = fmaf(gC, S[j], ds[j]);
-                store_row64(tiles + TSS, d, S);
+                store_row64(tiles + TSS + (uint32_t)((c + 1) & 1) * 8192u, d, S);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -723,8 +735,10 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             if (leader && c + 1 < nchunks) {
                 if (!mbar_wait(&ctl->lw_full[(c + 1) & 1], (uint32_t)((c + 1) >> 1) & 1u)) ctl->abort = 1;
                 tc_fence_after_sync();
-                issue_x(c + 1);
+                issue_x1(c + 1);
             }
+            if (!mbar_wait(&ctl->o_done, (uint32_t)c & 1u)) ctl->abort = 1;
+            tc_fence_after_sync();
             {   // O = diag(gamma) X2 + P W, rows tr, columns 16*hf..
                 float x2[16], pw[16];
                 tmem_ld16x2_16<16>(tq + C_X2 + 32u * pb, x2);
