@@ -5,22 +5,23 @@
 //     A = diag(beta) (K K^T o Gamma o strict-lower)   (K K^T on tcgen05),
 //     T = (I + A)^-1   (16x16 diagonal blocks by substitution, then two levels of
 //                       block merges on mma.sync tf32),
-//   and writes T diag(beta) and T diag(beta gamma) as bf16 operand images
-//   (128-byte swizzled, exactly as the main kernel's shared memory wants them)
-//   to the workspace: 16 KB per (batch, head, chunk).
+//   and writes T as a bf16 operand image (128-byte swizzled, exactly as the main
+//   kernel's shared memory wants it) to the workspace: 8 KB per (batch, head,
+//   chunk).
 //
 // chunk_gdn_kernel (one CTA per (batch, head, 32-column value slab), 9 warps):
 //   warp 0      producer: TMA loads of q, k, v and a bulk copy of the chunk's
-//               T images (3 stages); alpha / beta into shared memory;
-//   warps 1-4   "local" group, one chunk ahead of the state group:
-//                 [Q;K] K^T (tcgen05, M=128) -> P = (Q K^T) o Gamma o M,
-//                 U = T diag(beta) V  and  W_k = T diag(beta gamma) K (tcgen05);
-//   warps 5-8   "state" group, the recurrence across chunks:
-//                 X1 = W_k S0 (S0 as a bf16 operand), W = U - X1,
+//               T image (3 stages); the chunk's decay factors and betas;
+//   warps 1-4   "score" group: P = (Q K^T) o Gamma o M  (tcgen05, M=64) ->
+//               bf16 tile [P ; 0] for chunk c, then, one chunk behind the state
+//               group, PW = [P ; 0] W and O = diag(gamma) X2 + PW for chunk c-1;
+//   warps 5-8   "state" group, the recurrence across chunks.  With
+//               W = U - W_k S0 = T diag(beta) (V - diag(gamma) K S0):
+//                 [X2 ; KS] = [Q ; K] S0        (one M=128 MMA chain, S0 bf16),
+//                 R = diag(beta) (V - diag(gamma) KS)   (bf16),
+//                 W = T R,
 //                 dS = K^T diag(gamma_C/gamma) W,
-//                 S <- gamma_C S + dS (fp32, one state row per thread);
-//               off that chain, issued after dS and run during the state
-//               update: X2 = Q S0, PW = P W, then O = diag(gamma) X2 + PW.
+//                 S <- gamma_C S + dS (fp32, one state row per thread).
 // The derivation of the WY / UT form is in chunk_tc.cuh's header.
 //
 // Pairwise decays Gamma_ti = gamma_t / gamma_i (i <= t) are products of
@@ -42,26 +43,24 @@ constexpr int NSTG = 3;
 constexpr int NTHREADS = 288;
 constexpr uint32_t TMEM_COLS = 512;
 // TMEM columns of the main kernel
-constexpr uint32_t C_SC = 0;     // 64,     M=128 scores [Q;K] K^T
-constexpr uint32_t C_U = 64;     // 2 x 32, M=64
-constexpr uint32_t C_WK = 128;   // 128,    M=64
-constexpr uint32_t C_X1 = 256;   // 32,     M=64
-constexpr uint32_t C_X2 = 288;   // 2 x 32, M=64
-constexpr uint32_t C_PW = 352;   // 2 x 32, M=64
-constexpr uint32_t C_DS = 416;   // 32,     M=128
+constexpr uint32_t C_SC = 0;     // 2 x 64, M=64  scores Q K^T
+constexpr uint32_t C_XK = 128;   // 2 x 32, M=128 [Q ; K] S0
+constexpr uint32_t C_W = 192;    // 32,     M=64  W = T R
+constexpr uint32_t C_DS = 224;   // 32,     M=128 dS
+constexpr uint32_t C_PW = 256;   // 2 x 32, M=128 [P ; 0] W (rows 0-63)
 
-constexpr uint32_t TT_BYTES = 16384;                 // T diag(beta) | T diag(beta gamma), bf16
+constexpr uint32_t TT_BYTES = 8192;                  // T, bf16 [64][64]
 
 // Main-kernel shared-memory tiles (byte offsets from a 1 KB aligned base).
 constexpr uint32_t QK_ACS = 128 * 128;               // one atom column: Q rows 0-63, K rows 64-127
 constexpr uint32_t STG_QK = 0;                       // NSTG x 2 atom columns
 constexpr uint32_t STG_QK_BYTES = 2 * QK_ACS;
 constexpr uint32_t STG_V = STG_QK + NSTG * STG_QK_BYTES;   // NSTG x [64][32] bf16, 64 B swizzle
-constexpr uint32_t STG_TT = STG_V + NSTG * 4096;           // 2 x (T diag(beta), T diag(beta gamma))
-constexpr uint32_t TP = STG_TT + 2 * TT_BYTES;       // 2 x P [64][64] bf16
-constexpr uint32_t TWK = TP + 2 * 8192;              // 2 x W_k [64][128] bf16 (2 atom columns)
-constexpr uint32_t TWS = TWK + 2 * 16384;            // W       [64][32] 64 B swizzle
-constexpr uint32_t TWGS = TWS + 4096;                // gamma_C/gamma W
+constexpr uint32_t STG_TT = STG_V + NSTG * 4096;           // NSTG x T
+constexpr uint32_t TP = STG_TT + NSTG * TT_BYTES;    // 2 x [P ; 0] [128][64] bf16 (rows 64-127 zero)
+constexpr uint32_t TR = TP + 2 * 16384;              // R       [64][32] 64 B swizzle
+constexpr uint32_t TWS = TR + 4096;                  // 2 x W
+constexpr uint32_t TWGS = TWS + 2 * 4096;            // gamma_C/gamma W
 constexpr uint32_t TSS = TWGS + 4096;                // 2 x S   [128][32] 64 B swizzle
 constexpr uint32_t TEND = TSS + 2 * 8192;
 
@@ -76,14 +75,13 @@ constexpr int PREP_THREADS = 128;
 
 struct GCtl {
     uint64_t full[NSTG], empty[NSTG];
-    uint64_t l_done, lw_full[2], lw_empty[2], x1_done, ds_done, o_done;
-    uint64_t ttfree[2];              // the local group's MMAs of a T-image slot are done
+    uint64_t l_done[2], wready[2], pw_done[2], oA[2], xk_done, w_done, ds_done, drain;
     uint32_t tmem_base;
-    int abort, stopL, stopS;
+    int abort, stopS, stopL[2];
     int fast[NSTG];
     // per stage: b = log2 of the inclusive cumulative alpha, gamma = 2^b,
-    // 1/gamma and gamma_C/gamma (written by the producer)
-    float b2[NSTG][64], gam[NSTG][64], ginv[NSTG][64], gct[NSTG][64];
+    // 1/gamma, gamma_C/gamma and beta (written by the producer)
+    float b2[NSTG][64], gam[NSTG][64], ginv[NSTG][64], gct[NSTG][64], bet[NSTG][64];
 };
 
 struct PCtl {
@@ -91,7 +89,7 @@ struct PCtl {
     uint32_t tmem_base;
     int abort, stop, fast;
     float alpha[2][64], beta[2][64];
-    float gam[64], ginv[64], bg[64], b2[64];
+    float gam[64], ginv[64], b2[64];
 };
 
 
@@ -394,7 +392,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         if (!mbar_wait(&ctl->full[buf], (uint32_t)(it >> 1) & 1u)) ctl->abort = 1;
         if (warp == 0)
             ctl->fast = gate_scan(&ctl->alpha[buf][2 * lane], ctl->beta[buf], ctl->b2, ctl->gam, ctl->ginv,
-                                  ctl->bg, lane);
+                                  nullptr, lane);
         if (tid == 32) {
             tc_fence_after_sync();
             const uint32_t kb = tb + P_K + buf * 16384;
@@ -425,26 +423,18 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         tc_fence_before_sync();
         bar_named(1, 128);
         invert_unit_lower64(AF, TMP, tid, lane, 1, 2);
-        {   // T diag(beta) and T diag(beta gamma) -> workspace, 128-byte swizzled [64][64] bf16 images
+        {   // T -> workspace, a 128-byte swizzled [64][64] bf16 image
             const int t = tid >> 1, hh = tid & 1;
             const float *Trow = AF + t * AF_LD + 32 * hh;
-            const float *be = ctl->beta[buf] + 32 * hh, *bgp = ctl->bg + 32 * hh;
             uint8_t *dst = p.ws + w * (int64_t)TT_BYTES;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-                uint4 u1, u2;
-                uint32_t *p1 = &u1.x, *p2 = &u2.x;
+                uint4 u;
+                uint32_t *pu = &u.x;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = 8 * cc + 2 * e;
-                    const float t0v = Trow[j], t1v = Trow[j + 1];
-                    p1[e] = pack_bf16x2(t0v * be[j], t1v * be[j + 1]);
-                    p2[e] = pack_bf16x2(t0v * bgp[j], t1v * bgp[j + 1]);
-                }
+                for (int e = 0; e < 4; ++e) pu[e] = pack_bf16x2(Trow[8 * cc + 2 * e], Trow[8 * cc + 2 * e + 1]);
                 const int chunk = 4 * hh + cc;
-                const uint32_t off = (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4);
-                *reinterpret_cast<uint4 *>(dst + off) = u1;
-                *reinterpret_cast<uint4 *>(dst + 8192 + off) = u2;
+                *reinterpret_cast<uint4 *>(dst + (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4)) = u;
             }
         }
         bar_named(1, 128);   // AF, gates and the K buffer are reused by the next items
@@ -456,6 +446,22 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+
+// Row t's 32 columns col0.. of the decayed, causally masked score matrix, in
+// place: x_i <- x_i * gamma_t / gamma_i for i <= t, 0 above the diagonal.
+__device__ __forceinline__ void decay_mask32(float *x, int t, int col0, bool fast, const float *gam,
+                                             const float *ginv, const float *b2) {
+    if (fast) {
+        const float gt = gam[t];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = (col0 + j <= t) ? x[j] * gt * ginv[col0 + j] : 0.f;
+    } else {
+        const float bt = b2[t];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = (col0 + j <= t) ? x[j] * exp2f(bt - b2[col0 + j]) : 0.f;
+    }
 }
 
 __global__ void __launch_bounds__(gdn::NTHREADS, 1)
@@ -478,17 +484,18 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
     if (tid == 0) {
         for (int s = 0; s < NSTG; ++s) {
             mbar_init(&ctl->full[s], 32);
-            mbar_init(&ctl->empty[s], 1);
+            mbar_init(&ctl->empty[s], 2);   // the state group's and the score group's MMAs
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&ctl->lw_full[i], 128);
-            mbar_init(&ctl->lw_empty[i], 1);
-            mbar_init(&ctl->ttfree[i], 1);
+            mbar_init(&ctl->l_done[i], 1);
+            mbar_init(&ctl->wready[i], 128);
+            mbar_init(&ctl->pw_done[i], 1);
+            mbar_init(&ctl->oA[i], 128);
         }
-        mbar_init(&ctl->l_done, 1);
-        mbar_init(&ctl->x1_done, 1);
+        mbar_init(&ctl->xk_done, 1);
+        mbar_init(&ctl->w_done, 1);
         mbar_init(&ctl->ds_done, 1);
-        mbar_init(&ctl->o_done, 1);
+        mbar_init(&ctl->drain, 2);   // one commit from each MMA-issuing thread
         ctl->abort = 0;
         fence_barrier_init();
         tma_prefetch_desc(&maps.q);
@@ -499,32 +506,34 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         tmem_alloc(&ctl->tmem_base, TMEM_COLS);
         tc_fence_before_sync();
     }
+    // rows 64-127 of both [P ; 0] tiles stay zero
+    for (int i = tid; i < 2 * 8192 / 16; i += NTHREADS) {
+        const int tile = i / 512, off = (i % 512) * 16;
+        *reinterpret_cast<uint4 *>(tiles + TP + tile * 16384 + 8192 + off) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16);   // this warp's TMEM lanes
 
-    constexpr uint32_t ID_SC = idesc_bf16(128, 64, false, false);
-    constexpr uint32_t ID_U = idesc_bf16(64, DVT, false, true);
-    constexpr uint32_t ID_WK = idesc_bf16(64, DK, false, true);
-    constexpr uint32_t ID_X = idesc_bf16(64, DVT, false, true);
+    constexpr uint32_t ID_SC = idesc_bf16(64, 64, false, false);
+    constexpr uint32_t ID_XK = idesc_bf16(128, DVT, false, true);
+    constexpr uint32_t ID_W = idesc_bf16(64, DVT, false, true);
     constexpr uint32_t ID_DS = idesc_bf16(128, DVT, true, true);
 
     auto stage_qk = [&](int c) { return tb + STG_QK + (uint32_t)(c % NSTG) * STG_QK_BYTES; };
-    auto stage_v = [&](int c) { return tb + STG_V + (uint32_t)(c % NSTG) * 4096u; };
-    auto stage_tt = [&](int c) { return tb + STG_TT + (uint32_t)(c & 1) * TT_BYTES; };
+    auto stage_v = [&](int c) { return tiles + STG_V + (uint32_t)(c % NSTG) * 4096u; };
+    auto stage_tt = [&](int c) { return tb + STG_TT + (uint32_t)(c % NSTG) * TT_BYTES; };
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
         int issued = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTG;
-            if (c >= 2) {   // stage and T-image slot released by their last readers
+            if (c >= NSTG) {   // the stage's last readers are done
                 int ok = 1;
-                if (lane == 0) {
-                    if (c >= NSTG) ok = mbar_wait(&ctl->empty[s], (uint32_t)((c / NSTG) - 1) & 1u);
-                    ok = mbar_wait(&ctl->ttfree[c & 1], (uint32_t)((c - 2) >> 1) & 1u) && ok;
-                }
+                if (lane == 0) ok = mbar_wait(&ctl->empty[s], (uint32_t)((c / NSTG) - 1) & 1u);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok && lane == 0) ctl->abort = 1;
             }
@@ -543,16 +552,18 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 }
                 tma_load_4d(tiles + STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, t0,
                             (int)b);
-                bulk_load(tiles + STG_TT + (c & 1) * TT_BYTES, ws + (bh * nchunks + c) * (int64_t)TT_BYTES,
+                bulk_load(tiles + STG_TT + s * TT_BYTES, ws + (bh * nchunks + c) * (int64_t)TT_BYTES,
                           TT_BYTES, &ctl->full[s]);
             }
             // the chunk's decay factors: b = log2 of the inclusive cumulative alpha,
-            // gamma = 2^b, 1/gamma, gamma_C/gamma = 2^(b_63 - b)
+            // gamma = 2^b, 1/gamma, gamma_C/gamma = 2^(b_63 - b); beta (0 past T)
             float al[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int64_t tt = (int64_t)t0 + 2 * lane + e;
-                al[e] = (tt < p.T) ? p.g[(b * p.T + tt) * p.H + h] : 1.f;
+                const bool in = tt < p.T;
+                al[e] = in ? p.g[(b * p.T + tt) * p.H + h] : 1.f;
+                ctl->bet[s][2 * lane + e] = in ? p.beta[(b * p.T + tt) * p.H + h] : 0.f;
             }
             const int fast = gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
             const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
@@ -568,71 +579,110 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             for (int c = (issued > NSTG ? issued - NSTG : 0); c < issued; ++c)
                 (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
     } else if (warp < 5) {
-        // ------------------------------------------------------------------ local group
+        // ------------------------------------------------------------------ score group
         const int lt = tid - 32;
         const bool leader = (lt == 0);
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % NSTG, pb = c & 1;
-            if (leader) ctl->stopL = ctl->abort;
+        const int t = 16 * quad + (lane & 15), hf = lane >> 4;   // M=64 row, column half
+        const int ro = 32 * quad + lane;                          // M=128 row: output rows 0-63 in quads 0, 1
+        // PW = [P ; 0] W and O = diag(gamma) X2 + PW of chunk j, X2 = rows 0-63 of [X2 ; KS]
+        // (a failed wait sets the abort flag; every thread still takes every barrier)
+        auto finish = [&](int j) {
+            const int sj = j % NSTG, jb = j & 1;
+            const int64_t tj = (int64_t)j * C;
+            const int nvalid = (int)min((int64_t)C, p.T - tj);
+            if (!mbar_wait(&ctl->wready[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
+            const float gam_o = ctl->gam[sj][ro & 63];   // read before the stage can be refilled
             bar_named(1, 128);
-            if (ctl->stopL) break;
-            if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
-            if (c >= 2 && !mbar_wait(&ctl->lw_empty[pb], (uint32_t)((c - 2) >> 1) & 1u)) ctl->abort = 1;
-
-            // ---- [Q;K] K^T ; U = T diag(beta) V ; W_k = T diag(beta gamma) K
             if (leader) {
                 tc_fence_after_sync();
-                const uint32_t qk = stage_qk(c), kb = qk + 64 * 128, vb = stage_v(c), tt = stage_tt(c);
-                // three independent accumulations, interleaved so that consecutive
-                // instructions never wait on the same accumulator
+                const uint32_t ps = tb + TP + (uint32_t)jb * 16384u, wsb = tb + TWS + (uint32_t)jb * 4096u;
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    umma_bf16(tmem + C_SC, desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk), ID_SC, kk > 0);
-                    if (kk < C / 16) {
-                        umma_bf16(tmem + C_WK, desc_k(tt + 8192, C * 128, kk), desc_mn128(kb, QK_ACS, kk),
-                                  ID_WK, kk > 0);
-                        umma_bf16(tmem + C_U + 32u * pb, desc_k(tt, C * 128, kk), desc_mn64(vb, kk), ID_U,
-                                  kk > 0);
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + C_PW + 32u * jb, desc_k(ps, 16384, kk), desc_mn64(wsb, kk), ID_XK, kk > 0);
+                umma_commit(&ctl->pw_done[jb]);
+                umma_commit(&ctl->empty[sj]);
+            }
+            if (!mbar_wait(&ctl->pw_done[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
+            tc_fence_after_sync();
+            if (quad < 2) {
+                float x2[32], pw[32];
+                tmem_ld32(tq + C_XK + 32u * jb, x2);
+                tmem_ld32(tq + C_PW + 32u * jb, pw);
+                tmem_wait_ld();
+                if (ro < nvalid) {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
+                                         ((b * p.T + tj + ro) * p.H + h) * p.dv + dvt * DVT;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        uint4 u;
+                        u.x = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 0], pw[8 * cc + 0]),
+                                          fmaf(gam_o, x2[8 * cc + 1], pw[8 * cc + 1]));
+                        u.y = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 2], pw[8 * cc + 2]),
+                                          fmaf(gam_o, x2[8 * cc + 3], pw[8 * cc + 3]));
+                        u.z = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 4], pw[8 * cc + 4]),
+                                          fmaf(gam_o, x2[8 * cc + 5], pw[8 * cc + 5]));
+                        u.w = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 6], pw[8 * cc + 6]),
+                                          fmaf(gam_o, x2[8 * cc + 7], pw[8 * cc + 7]));
+                        reinterpret_cast<uint4 *>(dst)[cc] = u;
                     }
                 }
-                umma_commit(&ctl->l_done);
-                umma_commit(&ctl->ttfree[c & 1]);
             }
-            if (!mbar_wait(&ctl->l_done, (uint32_t)c & 1u)) ctl->abort = 1;
+            tc_fence_before_sync();
+            mbar_arrive(&ctl->oA[jb]);
+        };
+        // iteration c: P of chunk c (c < nchunks), then PW and O of chunk c-1.
+        // The stop flag alternates between two words so that the leader's write
+        // for iteration c+1 cannot reach a thread still reading iteration c's.
+        for (int c = 0; c <= nchunks; ++c) {
+            const int s = c % NSTG, pb = c & 1;
+            if (leader) ctl->stopL[pb] = ctl->abort;
+            bar_named(1, 128);
+            if (ctl->stopL[pb]) break;
+            if (c == nchunks) {
+                if (c >= 1) finish(c - 1);
+                break;
+            }
+            // (the P tile and score accumulator of chunk c-2 were freed by finish(c-2))
+            if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
+            if (leader) {
+                tc_fence_after_sync();
+                const uint32_t qk = stage_qk(c), kb = qk + 64 * 128;
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk)
+                    umma_bf16(tmem + C_SC + 64u * pb, desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk), ID_SC, kk > 0);
+                umma_commit(&ctl->l_done[pb]);
+            }
+            if (!mbar_wait(&ctl->l_done[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
             tc_fence_after_sync();
-
-            // ---- P = (Q K^T) o Gamma o M: TMEM lanes 0..63 (quadrants 0 and 1), one row per thread
-            if (quad < 2) {
-                const int t = 32 * quad + lane;
-                const int ncols = quad == 0 ? 32 : 64;
-                float x[64];
-                tmem_ld32(tq + C_SC, *reinterpret_cast<float(*)[32]>(x));
-                if (quad == 1) tmem_ld32(tq + C_SC + 32, *reinterpret_cast<float(*)[32]>(x + 32));
+            {   // P row t, columns 32hf..32hf+31 -> bf16 rows 0-63 of [P ; 0]
+                float x[32];
+                tmem_ld16x2_32<32>(tq + C_SC + 64u * pb, x);
                 tmem_wait_ld();
-                decay_mask_row<false>(x, t, ncols, 1.f, ctl->fast[s] != 0, ctl->gam[s], ctl->ginv[s],
-                                      ctl->b2[s]);
-                store_row_bf16(tiles + TP + pb * 8192, t, x);
-            }
-            // ---- W_k -> bf16: row t = 16*quad + (lane & 15); lanes 0-15 columns 0-63, 16-31 columns 64-127
-            {
-                const int t = 16 * quad + (lane & 15), hf = lane >> 4;
-                float x[64];
-                tmem_ld16x2_32<64>(tq + C_WK, *reinterpret_cast<float(*)[32]>(x));
-                tmem_ld16x2_32<64>(tq + C_WK + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-                tmem_wait_ld();
-                store_row_bf16(tiles + TWK + pb * 16384 + hf * 8192, t, x);
+                decay_mask32(x, t, 32 * hf, ctl->fast[s] != 0, ctl->gam[s], ctl->ginv[s], ctl->b2[s]);
+                uint8_t *ps = tiles + TP + pb * 16384;
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint4 u;
+                    u.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
+                    u.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
+                    u.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
+                    u.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
+                    const int chunk = 4 * hf + cc;
+                    *reinterpret_cast<uint4 *>(ps + t * 128 + (((chunk ^ t) & 7) << 4)) = u;
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
-            mbar_arrive(&ctl->lw_full[pb]);
+            if (c >= 1) finish(c - 1);
         }
+        if (leader) umma_commit(&ctl->drain);
     } else {
         // ------------------------------------------------------------------ state group
         const int st = tid - 160;
         const bool leader = (st == 0);
-        const int d = 32 * quad + lane;               // state row (M=128 accumulators)
-        const int tr = 16 * quad + (lane & 15);       // chunk row (M=64 accumulators)
-        const int hf = lane >> 4;                     // which 16 of the 32 columns
+        const int d = 32 * quad + lane;               // row of the M=128 accumulators (state row)
+        const int tr = 16 * quad + (lane & 15);       // row of the M=64 accumulator W
+        const int hf = lane >> 4;                     // which 16 of W's 32 columns
         float S[DVT];
         {
             const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVT) : nullptr;
@@ -647,12 +697,13 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         bar_named(2, 128);
         // the bf16 copy of the state entering chunk c sits in buffer c & 1
         auto ss_of = [&](int c) { return tb + TSS + (uint32_t)(c & 1) * 8192u; };
-        auto issue_x1 = [&](int c) {
-            const uint32_t wk = tb + TWK + (uint32_t)(c & 1) * 16384u, ss = ss_of(c);
+        // [X2 ; KS] = [Q ; K] S0, K = dk
+        auto issue_xk = [&](int c) {
+            const uint32_t qk = stage_qk(c), ss = ss_of(c);
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem + C_X1, desc_k(wk, C * 128, kk), desc_mn64(ss, kk), ID_X, kk > 0);
-            umma_commit(&ctl->x1_done);
+                umma_bf16(tmem + C_XK + 32u * (c & 1), desc_k(qk, QK_ACS, kk), desc_mn64(ss, kk), ID_XK, kk > 0);
+            umma_commit(&ctl->xk_done);
         };
         // half row (16 columns, 2 chunks of 16 B) of a [rows][32] bf16 tile, 64-byte swizzle
         auto store_half64 = [&](uint32_t tile_off, int r, const float *x16) {
@@ -668,60 +719,85 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             }
         };
         if (leader && nchunks > 0) {
-            if (!mbar_wait(&ctl->lw_full[0], 0)) ctl->abort = 1;
+            if (!mbar_wait(&ctl->full[0], 0u)) ctl->abort = 1;
             tc_fence_after_sync();
-            issue_x1(0);
+            issue_xk(0);
         }
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTG, pb = c & 1;
-            const int t0 = c * C;
-            const int nvalid = (int)min((int64_t)C, p.T - t0);
             if (leader) ctl->stopS = ctl->abort;
             bar_named(2, 128);
             if (ctl->stopS) break;
-            if (!mbar_wait(&ctl->lw_full[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
-            if (!mbar_wait(&ctl->x1_done, (uint32_t)c & 1u)) ctl->abort = 1;
+            // the stage landed (V, T and the decay factors are read directly)
+            bool ok = mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u);
+            ok = mbar_wait(&ctl->xk_done, (uint32_t)c & 1u) && ok;
+            if (!ok) ctl->abort = 1;
             tc_fence_after_sync();
-            const float gam_t = ctl->gam[s][tr], gC = ctl->gam[s][C - 1];
-            {   // W = U - X1 and (gamma_C / gamma) W, rows tr, columns 16*hf..
-                float x1[16], u[16], w[16], wg[16];
-                tmem_ld16x2_16<16>(tq + C_X1, x1);
-                tmem_ld16x2_16<16>(tq + C_U + 32u * pb, u);
+            const float gC = ctl->gam[s][C - 1];
+            const float gct_r = ctl->gct[s][tr];
+            if (quad >= 2) {   // R = diag(beta) (V - diag(gamma) KS): rows 64..127 of [X2 ; KS]
+                const int t = d - 64;
+                float ks[32];
+                tmem_ld32(tq + C_XK + 32u * pb, ks);
                 tmem_wait_ld();
-                const float gct = ctl->gct[s][tr];
+                const uint8_t *vt = stage_v(c);
+                const float be = ctl->bet[s][t], ga = ctl->gam[s][t];
+                float r[32];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    w[j] = u[j] - x1[j];
-                    wg[j] = w[j] * gct;
+                for (int cc = 0; cc < 4; ++cc) {
+                    const uint4 u = *reinterpret_cast<const uint4 *>(vt + t * 64 + (((cc ^ (t >> 1)) & 3) << 4));
+                    const uint32_t *w = &u.x;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 v2 = unpack_bf16x2(w[e]);
+                        const int j = 8 * cc + 2 * e;
+                        r[j] = be * fmaf(-ga, ks[j], v2.x);
+                        r[j + 1] = be * fmaf(-ga, ks[j + 1], v2.y);
+                    }
                 }
-                store_half64(TWS, tr, w);
-                store_half64(TWGS, tr, wg);
+                store_row64(tiles + TR, t, r);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             bar_named(2, 128);
-            if (leader) {
+            if (leader) {   // W = T R, K = tokens
                 tc_fence_after_sync();
-                const uint32_t qk = stage_qk(c), kb = qk + 64 * 128, ss = ss_of(c);
-                // dS first (the recurrence waits for it), then the output-only X2 and PW
+                const uint32_t tt = stage_tt(c);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + C_W, desc_k(tt, C * 128, kk), desc_mn64(tb + TR, kk), ID_W, kk > 0);
+                umma_commit(&ctl->w_done);
+            }
+            ok = mbar_wait(&ctl->w_done, (uint32_t)c & 1u);
+            // the W tile of chunk c-2 was read by PW(c-2)
+            if (c >= 2) ok = mbar_wait(&ctl->pw_done[pb], (uint32_t)((c - 2) >> 1) & 1u) && ok;
+            if (!ok) ctl->abort = 1;
+            tc_fence_after_sync();
+            {   // W and (gamma_C / gamma) W -> bf16, rows tr, columns 16 hf..
+                float w[16], wg[16];
+                tmem_ld16x2_16<16>(tq + C_W, w);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) wg[j] = w[j] * gct_r;
+                store_half64(TWS + (uint32_t)pb * 4096u, tr, w);
+                store_half64(TWGS, tr, wg);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(&ctl->wready[pb]);   // the score group may issue PW(c)
+            bar_named(2, 128);
+            if (leader) {   // dS = K^T diag(gamma_C / gamma) W, K = tokens
+                tc_fence_after_sync();
+                const uint32_t kb = stage_qk(c) + 64 * 128;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     umma_bf16(tmem + C_DS, desc_mn128(kb, QK_ACS, kk), desc_mn64(tb + TWGS, kk), ID_DS, kk > 0);
                 umma_commit(&ctl->ds_done);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16(tmem + C_X2 + 32u * pb, desc_k(qk, QK_ACS, kk), desc_mn64(ss, kk), ID_X, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + C_PW + 32u * pb, desc_k(tb + TP + pb * 8192u, C * 128, kk),
-                              desc_mn64(tb + TWS, kk), ID_X, kk > 0);
-                umma_commit(&ctl->o_done);
-                umma_commit(&ctl->lw_empty[pb]);
                 umma_commit(&ctl->empty[s]);
             }
             if (!mbar_wait(&ctl->ds_done, (uint32_t)c & 1u)) ctl->abort = 1;
             tc_fence_after_sync();
-            {
+            {   // S <- gamma_C S + dS, then its bf16 copy for chunk c+1
                 float ds[DVT];
                 tmem_ld32(tq + C_DS, ds);
                 tmem_wait_ld();
@@ -733,34 +809,18 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             tc_fence_before_sync();
             bar_named(2, 128);
             if (leader && c + 1 < nchunks) {
-                if (!mbar_wait(&ctl->lw_full[(c + 1) & 1], (uint32_t)((c + 1) >> 1) & 1u)) ctl->abort = 1;
+                // the stage of c+1 landed, and the output epilogue of c-1 is done with
+                // the [X2 ; KS] accumulator that [Q ; K] S of c+1 overwrites
+                bool w1 = mbar_wait(&ctl->full[(c + 1) % NSTG], (uint32_t)((c + 1) / NSTG) & 1u);
+                if (c >= 1) w1 = mbar_wait(&ctl->oA[(c + 1) & 1], (uint32_t)((c - 1) >> 1) & 1u) && w1;
+                if (!w1) ctl->abort = 1;
                 tc_fence_after_sync();
-                issue_x1(c + 1);
+                issue_xk(c + 1);
             }
-            if (!mbar_wait(&ctl->o_done, (uint32_t)c & 1u)) ctl->abort = 1;
-            tc_fence_after_sync();
-            {   // O = diag(gamma) X2 + P W, rows tr, columns 16*hf..
-                float x2[16], pw[16];
-                tmem_ld16x2_16<16>(tq + C_X2 + 32u * pb, x2);
-                tmem_ld16x2_16<16>(tq + C_PW + 32u * pb, pw);
-                tmem_wait_ld();
-                if (tr < nvalid) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) x2[j] = fmaf(gam_t, x2[j], pw[j]);
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
-                                         ((b * p.T + t0 + tr) * p.H + h) * p.dv + dvt * DVT + 16 * hf;
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        uint4 u;
-                        u.x = pack_bf16x2(x2[8 * cc + 0], x2[8 * cc + 1]);
-                        u.y = pack_bf16x2(x2[8 * cc + 2], x2[8 * cc + 3]);
-                        u.z = pack_bf16x2(x2[8 * cc + 4], x2[8 * cc + 5]);
-                        u.w = pack_bf16x2(x2[8 * cc + 6], x2[8 * cc + 7]);
-                        reinterpret_cast<uint4 *>(dst)[cc] = u;
-                    }
-                }
-            }
-            tc_fence_before_sync();
+        }
+        if (leader) {   // every MMA issued by either group has finished before TMEM is released
+            umma_commit(&ctl->drain);
+            (void)mbar_wait(&ctl->drain, 0u);
         }
         if (!ctl->abort && p.S_out) {
             float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVT);

@@ -200,9 +200,9 @@ inline SegPlan seg_plan(int rule, int64_t B, int64_t T, int64_t H, int64_t dv) {
 }
 
 // Device workspace the chunked path needs: the gated delta rule keeps the
-// per-chunk T diag(beta) | T diag(beta gamma) operand images (16 KB per
-// (batch, head, chunk)); sequence-parallel ELU+1 the partial state sums of its
-// first pass; GLA needs none.
+// per-chunk T = (I + A)^-1 operand images (8 KB per (batch, head, chunk));
+// sequence-parallel ELU+1 the partial state sums of its first pass; GLA needs
+// none.
 inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv) {
     if (T <= 0) return 0;
     if (rule == kRuleGDN) return (size_t)(B * H * ((T + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;

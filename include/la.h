@@ -91,9 +91,11 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *   workspace / workspace_bytes: device scratch of at least
  *          la_fwd_workspace_size() bytes, 16-byte aligned (may be NULL when that
  *          size is 0).  The gated delta rule on the tensor-core path (bf16,
- *          dk = 128) needs 16 KB per (batch, head, 64-token chunk): the chunk's
- *          T diag(beta) and T diag(beta gamma) operands, written by a first
- *          kernel and read by the second within the same call.  Calls that share
+ *          dk = 128) needs 8 KB per (batch, head, 64-token chunk): the chunk's
+ *          T = (I + A)^-1 operand, written by a first kernel and read by the
+ *          second within the same call.  ELU+1 over few heads and long sequences
+ *          runs segment-parallel and keeps per-segment partial state sums there
+ *          (dk*dv + dk floats per piece).  Calls that share
  *          one workspace must be ordered (same stream), otherwise they race.
  *          A missing or short workspace returns LA_ERR_WORKSPACE before any launch.
  * q/k/v/o must not overlap S_out/z_out.
@@ -179,8 +181,8 @@ la_status la_fwd_host(const la_fwd_args *host_args, void *staging, size_t stagin
  *
  *   - The problem's scratch need (la_fwd_workspace_size) must be at most
  *     LA_NOALLOC_SCRATCH_BYTES, otherwise LA_ERR_WORKSPACE is returned before
- *     anything is launched.  For the gated delta rule that is 1024
- *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 4096.
+ *     anything is launched.  For the gated delta rule that is 2048
+ *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 8192.
  *   - The first call on a device looks up the array's device address there
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.  Later calls on the device reuse the address.
