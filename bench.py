@@ -176,37 +176,45 @@ class ClockSampler:
 # Workload on the device
 # ---------------------------------------------------------------------------
 
+LEG_NAMES = ["gla_prefill", "gdn_prefill", "elu_prefill", "gla_decode", "gdn_decode"]
+# kernels per call: GLA 1; gated delta rule 2 (T operand images, then the main
+# pass); ELU+1 at this shape 2 (segment sums, then the segment-parallel main
+# pass); each decode step 1
+LEG_LAUNCHES = {"gla_prefill": 1, "gdn_prefill": 2, "elu_prefill": 2, "gla_decode": 1, "gdn_decode": 1}
+
+
 class Legs:
-    def __init__(self, torch, la, workloads, seed: int):
+    """Device inputs and preallocated outputs of the legs in `names` (all by default)."""
+
+    def __init__(self, torch, la, workloads, seed: int, names=None):
         self.torch, self.la = torch, la
+        self.names = list(names or LEG_NAMES)
+        want = set(self.names)
         dev = lambda t: None if t is None else t.cuda()
-        gla = workloads.gla_prefill(B=2, H=16, T=8192, seed=seed)
-        gdn = workloads.gdn_prefill(B=2, H=16, T=8192, seed=seed)
-        elu = workloads.elu_long(seed=seed)
-        self.host = {"gla": gla, "gdn": gdn, "elu": elu}
-        self.gla = {k: dev(getattr(gla, k)) for k in ("q", "k", "v", "g")}
-        self.gdn = {k: dev(getattr(gdn, k)) for k in ("q", "k", "v", "g", "beta")}
-        self.elu = {k: dev(getattr(elu, k)) for k in ("q", "k", "v", "S0", "z0")}
-        self.S_dec = workloads.decode_state(seed=seed).cuda()
-        d_gla = workloads.decode_steps("gla", 1, seed=seed)[0]
-        d_gdn = workloads.decode_steps("gdn", 1, seed=seed)[0]
-        self.dec_gla = [x.cuda() for x in d_gla]
-        self.dec_gdn = [x.cuda() for x in d_gdn]
-        # outputs allocated once
         e = torch.empty
-        self.o_gla = e(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
-        self.S_gla = e(2, 16, 128, 128, device="cuda")
-        self.o_gdn = e(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
-        self.S_gdn = e(2, 16, 128, 128, device="cuda")
-        self.o_elu = e(1, 32768, 16, 64, dtype=torch.bfloat16, device="cuda")
-        self.S_elu = e(1, 16, 128, 64, device="cuda")
-        self.z_elu = e(1, 16, 128, device="cuda")
-        self.o_dec = e(256, 16, 128, dtype=torch.bfloat16, device="cuda")
-        self.names = ["gla_prefill", "gdn_prefill", "elu_prefill", "gla_decode", "gdn_decode"]
-        # kernels per step: GLA 1; gated delta rule 2 (T operand images, then the
-        # main pass); ELU+1 at this shape 2 (segment sums, then the segment-parallel
-        # main pass); each decode step 1
-        self.launches_per_step = 7
+        self.host = {}
+        if "gla_prefill" in want:
+            gla = self.host["gla"] = workloads.gla_prefill(B=2, H=16, T=8192, seed=seed)
+            self.gla = {k: dev(getattr(gla, k)) for k in ("q", "k", "v", "g")}
+            self.o_gla = e(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
+            self.S_gla = e(2, 16, 128, 128, device="cuda")
+        if "gdn_prefill" in want:
+            gdn = self.host["gdn"] = workloads.gdn_prefill(B=2, H=16, T=8192, seed=seed)
+            self.gdn = {k: dev(getattr(gdn, k)) for k in ("q", "k", "v", "g", "beta")}
+            self.o_gdn = e(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
+            self.S_gdn = e(2, 16, 128, 128, device="cuda")
+        if "elu_prefill" in want:
+            elu = self.host["elu"] = workloads.elu_long(seed=seed)
+            self.elu = {k: dev(getattr(elu, k)) for k in ("q", "k", "v", "S0", "z0")}
+            self.o_elu = e(1, 32768, 16, 64, dtype=torch.bfloat16, device="cuda")
+            self.S_elu = e(1, 16, 128, 64, device="cuda")
+            self.z_elu = e(1, 16, 128, device="cuda")
+        if want & {"gla_decode", "gdn_decode"}:
+            self.S_dec = workloads.decode_state(seed=seed).cuda()
+            self.dec_gla = [x.cuda() for x in workloads.decode_steps("gla", 1, seed=seed)[0]]
+            self.dec_gdn = [x.cuda() for x in workloads.decode_steps("gdn", 1, seed=seed)[0]]
+            self.o_dec = e(256, 16, 128, dtype=torch.bfloat16, device="cuda")
+        self.launches_per_step = sum(LEG_LAUNCHES[n] for n in self.names)
 
     def run(self, name):
         la = self.la
@@ -242,6 +250,24 @@ def leg_work(name):
     rule = name.split("_")[0]
     return dict(tokens=256, bytes=decode_bytes(rule, 256, 16, 128, 128),
                 flops=2.0 * 2 * 128 * 128 * 256 * 16)
+
+
+def run_profile_leg(args):
+    """One leg only, `--reps` times with no timing: a small, fixed launch
+    sequence for ncu captures (3 warm-up calls, then the reps)."""
+    import torch
+
+    import gated_delta_rule_attn_b200 as la
+    import workloads
+
+    torch.cuda.set_device(0)
+    legs = Legs(torch, la, workloads, seed=0, names=[args.profile_leg])
+    for _ in range(3 + args.reps):
+        legs.run(args.profile_leg)
+    torch.cuda.synchronize()
+    la.check_device()
+    print(json.dumps({"profile_leg": args.profile_leg, "calls": 3 + args.reps,
+                      "launches": (3 + args.reps) * LEG_LAUNCHES[args.profile_leg]}), flush=True)
 
 
 def run_gpu(args):
@@ -490,10 +516,15 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-leg", choices=LEG_NAMES, default=None,
+                    help="run one leg 3 + --reps times without timing (for ncu captures)")
+    ap.add_argument("--reps", type=int, default=1)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile_leg:
+        run_profile_leg(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)
