@@ -286,35 +286,23 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
-// ---------------------------------------------------------------------------
-// FMA-pipe exponential for the ELU feature map of the chunk kernels: there the
-// special-function unit delivers only a few results per clock per SM and
-// bounds the per-element loop.  Two lanes at a time (packed fp32 instructions).
-// ---------------------------------------------------------------------------
-// 2^t for t <= 0: t = n + f with n = round(t) (the 1.5 * 2^23 add/subtract
-// trick), |f| <= 1/2, 2^f from the degree-4 Taylor polynomial of e^(f ln 2)
-// (relative error at most 4.2e-5 on |f| <= 1/2), then 2^n added to the exponent
-// field.  t is clamped at -125 so the result stays a normal number (below
-// that the true value is under 3e-38).
-__device__ __forceinline__ float2 exp2_neg2(float2 t) {
-    t = make_float2(fmaxf(t.x, -125.f), fmaxf(t.y, -125.f));
-    const float2 magic = make_float2(12582912.f, 12582912.f);
-    const float2 r = __fadd2_rn(t, magic);
-    const float2 n = __fadd2_rn(r, make_float2(-12582912.f, -12582912.f));
-    const float2 f = __fadd2_rn(t, make_float2(-n.x, -n.y));
-    float2 q = make_float2(9.618129107628477e-3f, 9.618129107628477e-3f);   // (ln 2)^4 / 4!
-    q = __ffma2_rn(q, f, make_float2(5.550410866482158e-2f, 5.550410866482158e-2f));   // (ln 2)^3 / 3!
-    q = __ffma2_rn(q, f, make_float2(2.402265069591007e-1f, 2.402265069591007e-1f));   // (ln 2)^2 / 2!
-    q = __ffma2_rn(q, f, make_float2(6.931471805599453e-1f, 6.931471805599453e-1f));   // ln 2
-    q = __ffma2_rn(q, f, make_float2(1.f, 1.f));
-    return make_float2(__int_as_float(__float_as_int(q.x) + ((__float_as_int(r.x) - 0x4B400000) << 23)),
-                       __int_as_float(__float_as_int(q.y) + ((__float_as_int(r.y) - 0x4B400000) << 23)));
+// 2^x on the special-function unit (approximate, flush-to-zero; relative
+// error about 1e-6 on the range the feature map uses).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-// phi(x) = ELU(x) + 1 for two lanes, the exponential on the FMA pipe.
+// phi(x) = ELU(x) + 1 for two lanes, written as max(x, 0) + exp(min(x, 0)):
+// x + 1 for x > 0 and e^x otherwise, with no select.  Measured on B200 this
+// form runs at about 15 elements per clock per SM (the special-function unit's
+// rate) against about 10 for a range-reduced polynomial on the FMA pipe, and
+// leaves the FMA and integer pipes to the surrounding work.
 __device__ __forceinline__ float2 elu_feature2(float2 x) {
-    const float2 e = exp2_neg2(make_float2(fminf(x.x, 0.f) * 1.4426950408889634f, fminf(x.y, 0.f) * 1.4426950408889634f));
-    return make_float2(x.x > 0.f ? x.x + 1.f : e.x, x.y > 0.f ? x.y + 1.f : e.y);
+    const float2 t = __fmul2_rn(make_float2(fminf(x.x, 0.f), fminf(x.y, 0.f)),
+                                make_float2(1.4426950408889634f, 1.4426950408889634f));
+    return make_float2(fmaxf(x.x, 0.f) + ex2_approx(t.x), fmaxf(x.y, 0.f) + ex2_approx(t.y));
 }
 
 
