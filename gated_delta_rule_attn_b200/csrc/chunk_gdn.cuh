@@ -67,8 +67,8 @@ constexpr uint32_t TEND = TSS + 2 * 8192;
 // Prep-kernel shared memory.
 constexpr int AF_LD = 68;
 constexpr int TMP_LD = 36;
-constexpr uint32_t P_K = 0;                          // 2 x K [64][128] bf16
-constexpr uint32_t P_AF = 2 * 16384;                 // A, then T, fp32 [64][AF_LD]
+constexpr uint32_t P_K = 0;                          // K [64][128] bf16
+constexpr uint32_t P_AF = 16384;                     // A, then T, fp32 [64][AF_LD]
 constexpr uint32_t P_TMP = P_AF + 64 * AF_LD * 4;    // fp32 scratch [32][TMP_LD]
 constexpr uint32_t P_END = P_TMP + 32 * TMP_LD * 4;
 constexpr int PREP_THREADS = 128;
@@ -85,10 +85,10 @@ struct GCtl {
 };
 
 struct PCtl {
-    uint64_t full[2], mma;
+    uint64_t full, mma;
     uint32_t tmem_base;
     int abort, stop, fast;
-    float alpha[2][64], beta[2][64];
+    float alpha[64], beta[64];
     float gam[64], ginv[64], b2[64];
 };
 
@@ -193,6 +193,21 @@ __device__ __forceinline__ int gate_scan(const float *al, const float *beta, flo
     }
     const float last = __shfl_sync(0xffffffffu, e1, 31);
     return last >= -120.f ? 1 : 0;
+}
+
+// Row t's 32 columns col0.. of A = diag(beta) (K K^T o Gamma o strict-lower), in
+// place: x_i <- x_i * rowf * gamma_t / gamma_i for i < t, 0 on and above the diagonal.
+__device__ __forceinline__ void decay_mask32_strict(float *x, int t, int col0, float rowf, bool fast,
+                                                    const float *gam, const float *ginv, const float *b2) {
+    if (fast) {
+        const float rs = rowf * gam[t];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = (col0 + j < t) ? x[j] * rs * ginv[col0 + j] : 0.f;
+    } else {
+        const float bt = b2[t];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = (col0 + j < t) ? x[j] * rowf * exp2f(bt - b2[col0 + j]) : 0.f;
+    }
 }
 
 // Row t of the decayed, masked score matrix from 64 raw scores x (in place):
@@ -322,9 +337,12 @@ struct GdnPrepParams {
     uint8_t *ws;   // [B*H*nchunks][TT_BYTES]
 };
 
-// One CTA handles (batch, head, chunk) items in a grid-stride loop; the K tile
-// of the next item is loaded while the current one is processed.
-__global__ void __launch_bounds__(gdn::PREP_THREADS)
+// One CTA handles (batch, head, chunk) items in a grid-stride loop.  The next
+// item's K tile is loaded (TMA) as soon as this item's K K^T MMA has read the
+// buffer, and its alpha and beta are fetched into registers at the same point,
+// so neither load is waited for.  The grid is sized to the CTAs that are
+// resident at once.
+__global__ void __launch_bounds__(gdn::PREP_THREADS, 4)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p) {
     using namespace gdn;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -338,8 +356,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
     float *TMP = reinterpret_cast<float *>(tiles + P_TMP);
 
     if (tid == 0) {
-        mbar_init(&ctl->full[0], 32);
-        mbar_init(&ctl->full[1], 32);
+        mbar_init(&ctl->full, 1);
         mbar_init(&ctl->mma, 1);
         ctl->abort = 0;
         fence_barrier_init();
@@ -354,48 +371,56 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tq = tmem + ((uint32_t)(32 * warp) << 16);
 
-    // warp 0: TMA of the K tile + this chunk's alpha / beta into buffer `buf`
-    auto issue = [&](int64_t w, int buf) {
+    // warp 0, lane 0: TMA of item w's K tile
+    auto load_k = [&](int64_t w) {
         const int64_t bh = w / p.nchunks;
         const int c = (int)(w % p.nchunks);
         const int64_t b = bh / p.H, h = bh % p.H;
-        const int t0 = c * C;
-        if (lane == 0) {
-            mbar_expect_tx(&ctl->full[buf], 2u * C * 128u);
-            for (int a = 0; a < KA; ++a)
-                tma_load_4d(tiles + P_K + buf * 16384 + a * (C * 128), &mapk, &ctl->full[buf], 64 * a,
-                            (int)h, t0, (int)b);
+        mbar_arrive_expect_tx(&ctl->full, 2u * C * 128u);
+        for (int a = 0; a < KA; ++a)
+            tma_load_4d(tiles + P_K + a * (C * 128), &mapk, &ctl->full, 64 * a, (int)h, c * C, (int)b);
+    };
+    // warp 0: item w's alpha, beta for tokens 2*lane, 2*lane+1 (1 and 0 past T)
+    float al[2] = {1.f, 1.f}, be[2] = {0.f, 0.f};
+    auto fetch_gates = [&](int64_t w) {
+        const int64_t bh = w / p.nchunks;
+        const int c = (int)(w % p.nchunks);
+        const int64_t b = bh / p.H, h = bh % p.H;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int64_t tt = (int64_t)c * C + 2 * lane + e;
+            const bool in = tt < p.T;
+            const int64_t idx = (b * p.T + (in ? tt : 0)) * p.H + h;
+            al[e] = in ? p.alpha[idx] : 1.f;
+            be[e] = in ? p.beta[idx] : 0.f;
         }
-        for (int i = lane; i < C; i += 32) {
-            const int64_t tt = (int64_t)t0 + i;
-            float al = 1.f, be = 0.f;
-            if (tt < p.T) {
-                const int64_t idx = (b * p.T + tt) * p.H + h;
-                al = p.alpha[idx];
-                be = p.beta[idx];
-            }
-            ctl->alpha[buf][i] = al;
-            ctl->beta[buf][i] = be;
-        }
-        mbar_arrive(&ctl->full[buf]);
     };
 
     constexpr uint32_t ID_KK = idesc_bf16(64, 64, false, false);
     int it = 0;
-    if (warp == 0 && (int64_t)blockIdx.x < items) issue(blockIdx.x, 0);
+    if (warp == 0 && (int64_t)blockIdx.x < items) {
+        if (lane == 0) load_k(blockIdx.x);
+        fetch_gates(blockIdx.x);
+    }
+    bool k_pending = (int64_t)blockIdx.x < items;   // a K copy is in flight (thread 0's view)
     for (int64_t w = blockIdx.x; w < items; w += gridDim.x, ++it) {
-        const int buf = it & 1;
+        if (warp == 0) {   // this item's gates (fetched one item ahead) into shared memory
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                ctl->alpha[2 * lane + e] = al[e];
+                ctl->beta[2 * lane + e] = be[e];
+            }
+        }
         if (tid == 0) ctl->stop = ctl->abort;   // one thread decides, everyone reads after the barrier
         bar_named(1, 128);
         if (ctl->stop) break;
-        if (warp == 0 && w + gridDim.x < items) issue(w + gridDim.x, buf ^ 1);
-        if (!mbar_wait(&ctl->full[buf], (uint32_t)(it >> 1) & 1u)) ctl->abort = 1;
+        if (!mbar_wait(&ctl->full, (uint32_t)it & 1u)) ctl->abort = 1;
+        if (tid == 0) k_pending = false;
         if (warp == 0)
-            ctl->fast = gate_scan(&ctl->alpha[buf][2 * lane], ctl->beta[buf], ctl->b2, ctl->gam, ctl->ginv,
-                                  nullptr, lane);
+            ctl->fast = gate_scan(&ctl->alpha[2 * lane], ctl->beta, ctl->b2, ctl->gam, ctl->ginv, nullptr, lane);
         if (tid == 32) {
             tc_fence_after_sync();
-            const uint32_t kb = tb + P_K + buf * 16384;
+            const uint32_t kb = tb + P_K;
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
                 umma_bf16(tmem, desc_k(kb, C * 128, kk), desc_k(kb, C * 128, kk), ID_KK, kk > 0);
@@ -404,21 +429,24 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         bar_named(1, 128);
         if (!mbar_wait(&ctl->mma, (uint32_t)it & 1u)) ctl->abort = 1;
         tc_fence_after_sync();
-        {   // A = diag(beta) (K K^T o Gamma o strict-lower); rows t = 16*warp + lane (lane < 16)
-            const int t = 16 * warp + lane;
-            const int ncols = (warp < 2) ? 32 : 64;
-            float x[64];
-            tmem_ld32(tq, *reinterpret_cast<float(*)[32]>(x));
-            if (warp >= 2) tmem_ld32(tq + 32, *reinterpret_cast<float(*)[32]>(x + 32));
-            tmem_wait_ld();
-            if (lane < 16) {
-                decay_mask_row<true>(x, t, ncols, ctl->beta[buf][t], ctl->fast != 0, ctl->gam, ctl->ginv,
-                                     ctl->b2);
-                float *arow = AF + t * AF_LD;
-#pragma unroll
-                for (int i = 0; i < 64; i += 4)
-                    *reinterpret_cast<float4 *>(arow + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        // the K buffer is free: start the next item's loads
+        if (warp == 0 && w + gridDim.x < items) {
+            if (lane == 0 && !ctl->abort) {
+                load_k(w + gridDim.x);
+                k_pending = true;
             }
+            fetch_gates(w + gridDim.x);
+        }
+        {   // A row t = 16*warp + (lane & 15), columns 32*(lane >> 4)..
+            const int t = 16 * warp + (lane & 15), col0 = 32 * (lane >> 4);
+            float x[32];
+            tmem_ld16x2_32<32>(tq, x);
+            tmem_wait_ld();
+            decay_mask32_strict(x, t, col0, ctl->beta[t], ctl->fast != 0, ctl->gam, ctl->ginv, ctl->b2);
+            float *arow = AF + t * AF_LD + col0;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4 *>(arow + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
         }
         tc_fence_before_sync();
         bar_named(1, 128);
@@ -437,16 +465,14 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
                 *reinterpret_cast<uint4 *>(dst + (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4)) = u;
             }
         }
-        bar_named(1, 128);   // AF, gates and the K buffer are reused by the next items
+        bar_named(1, 128);   // AF and the gates are reused by the next item
     }
     // let a prefetched copy land before the CTA exits
-    if (warp == 0 && lane == 0) {
-        const int64_t wn = (int64_t)blockIdx.x + (int64_t)it * gridDim.x;
-        if (wn < items) (void)mbar_wait(&ctl->full[it & 1], (uint32_t)(it >> 1) & 1u);
-    }
+    if (tid == 0 && k_pending) (void)mbar_wait(&ctl->full, (uint32_t)it & 1u);
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 64);
 }
+
 
 
 // Row t's 32 columns col0.. of the decayed, causally masked score matrix, in

@@ -199,6 +199,27 @@ inline SegPlan seg_plan(int rule, int64_t B, int64_t T, int64_t H, int64_t dv) {
     return sp;
 }
 
+// CTAs of `kernel` that can be resident on one SM at once, from its registers,
+// its shared memory and the TMEM columns each CTA allocates.  (The runtime's
+// occupancy query returns 1 for these tcgen05 kernels, although more fit.)
+inline int resident_per_sm(const void *kernel, int threads, int dyn_smem, int tmem_cols) {
+    int dev = 0, regs_sm = 65536, smem_sm = 233472, smem_res = 1024, thr_sm = 2048;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&smem_res, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return 1;
+    const int warps = (threads + 31) / 32;
+    const int regs_warp = (fa.numRegs * 32 + 255) / 256 * 256;   // allocated per warp in units of 256
+    int n = regs_warp > 0 ? regs_sm / (regs_warp * warps) : 1;
+    n = std::min(n, smem_sm / (dyn_smem + (int)fa.sharedSizeBytes + smem_res));
+    n = std::min(n, thr_sm / threads);
+    n = std::min(n, 512 / tmem_cols);
+    return std::max(n, 1);
+}
+
 // Device workspace the chunked path needs: the gated delta rule keeps the
 // per-chunk T = (I + A)^-1 operand images (8 KB per (batch, head, chunk));
 // sequence-parallel ELU+1 the partial state sums of its first pass; GLA needs
@@ -272,8 +293,11 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         pp.ws = static_cast<uint8_t *>(ws);
         const int64_t items = p.B * p.H * (int64_t)pp.nchunks;
         const int psmem = (int)((sizeof(gdn::PCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::P_END;
-        const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * 4);
         e = allow_smem((const void *)gdn_prep_kernel, psmem);
+        // one wave of resident CTAs walks all items (a second, partial wave
+        // would double the time)
+        const int per_sm = resident_per_sm((const void *)gdn_prep_kernel, gdn::PREP_THREADS, psmem, 64);
+        const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
         if (e == cudaSuccess) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.k, pp);
         const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::TEND;
         if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel, smem);

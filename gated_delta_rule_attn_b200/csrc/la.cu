@@ -164,8 +164,15 @@ bool make_map_4d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, 
 
 // Opt a kernel into more than 48 KB of dynamic shared memory (once per process
 // and device is enough; repeating it is harmless).
+// Opt the kernel in to `bytes` of dynamic shared memory and ask for the largest
+// shared-memory carveout, so that several CTAs of a small-footprint kernel can
+// be resident on one SM (and the occupancy query counts them).
 cudaError_t allow_smem(const void *kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+    return e;
 }
 }  // namespace la
 
