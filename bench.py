@@ -130,7 +130,7 @@ class ClockSampler:
                "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
                "display_clock_setting": 0x100}
 
-    def __init__(self, index: int, period: float = 0.05):
+    def __init__(self, index: int, period: float = 0.01):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self._stop = period, threading.Event()
         try:
