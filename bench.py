@@ -376,6 +376,8 @@ def run_gpu(args):
 
     # end to end through the host-buffer entry point (copies inside the timed region)
     out["e2e"] = run_e2e(torch, la, legs, min(K, args.e2e_steps), world)
+    if args.variants:
+        out["variants"] = run_variants(torch, la, workloads, K, hbm_peak, seed=rank)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(budget_s=args.cpu_seconds)
@@ -383,6 +385,41 @@ def run_gpu(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def run_variants(torch, la, workloads, K, hbm_peak, seed):
+    """The rule variants that run on the same kernels, at the prefill benchmark
+    shape (B=2, H=16, T=8192, d=128): DeltaNet (gated delta rule, alpha = 1),
+    RetNet (GLA, one constant decay per head), Lightning (GLA, g = 1).  Each is
+    timed K times with CUDA events, after 3 warm-up calls."""
+    spec = {"deltanet_prefill": ("gdn", dict(gdn_alpha="ones")),
+            "retnet_prefill": ("gla", dict(gla_gate="retnet")),
+            "lightning_prefill": ("gla", dict(gla_gate="ones"))}
+    res = {}
+    for name, (rule, kw) in spec.items():
+        p = workloads.make_problem(rule, 2, 8192, 16, 128, 128, seed=seed, **kw)
+        a = [None if t is None else t.cuda() for t in (p.q, p.k, p.v, p.g, p.beta)]
+        o = torch.empty(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
+        S = torch.empty(2, 16, 128, 128, device="cuda")
+        run = lambda: la.fwd(rule, *a, o=o, S_out=S)
+        for _ in range(3):
+            run()
+        stream = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            e0.record(stream)
+            run()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        la.check_device()
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / K
+        w = leg_work(rule + "_prefill")
+        gbs = w["bytes"] / (ms / 1e3) / 1e9
+        res[name] = {"ms": round(ms, 4), "tokens_per_s": round(w["tokens"] / (ms / 1e3)),
+                     "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4)}
+        del a, o, S
+    return res
 
 
 def run_e2e(torch, la, legs, steps, world):
@@ -519,6 +556,8 @@ def main():
     ap.add_argument("--profile-leg", choices=LEG_NAMES, default=None,
                     help="run one leg 3 + --reps times without timing (for ncu captures)")
     ap.add_argument("--reps", type=int, default=1)
+    ap.add_argument("--variants", action="store_true",
+                    help="also time DeltaNet, RetNet and Lightning prefill (same kernels) at B=2 H=16 T=8192")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

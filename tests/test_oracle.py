@@ -145,6 +145,24 @@ def test_gla_unit_gate_is_unnormalised_linear_attention():
     np.testing.assert_allclose(S[0, 0], S0[0, 0] + K.T @ V, rtol=1e-12)
 
 
+def test_gla_constant_decay_is_retention_closed_form():
+    """[SS] Retention: S_t = gamma S_{t-1} + k_t v_t^T with one constant gamma,
+    so S_t = gamma^(t+1) S0 + sum_{i<=t} gamma^(t-i) k_i v_i^T and the outputs are
+    the decayed causal score matrix (gamma^(t-i) (q_t . k_i)) applied to V plus
+    gamma^(t+1) S0^T q_t; the GLA recurrence with that gamma on every key dim."""
+    T, dk, dv, gam = 19, 4, 3, 0.8125
+    q, k, v = _rand(1, T, 1, dk), _rand(1, T, 1, dk), _rand(1, T, 1, dv)
+    S0 = _rand(1, 1, dk, dv)
+    o, S = oracle.gla_fwd(q, k, v, np.full((1, T, 1, dk), gam), S0)
+    t_idx = np.arange(T)
+    D = np.where(t_idx[:, None] >= t_idx[None, :], gam ** (t_idx[:, None] - t_idx[None, :]), 0.0)
+    Q, K, V = q[0, :, 0], k[0, :, 0], v[0, :, 0]
+    ref = ((Q @ K.T) * D) @ V + (gam ** (t_idx + 1))[:, None] * (Q @ S0[0, 0])
+    np.testing.assert_allclose(o[0, :, 0], ref, rtol=1e-11, atol=1e-12)
+    S_ref = gam ** T * S0[0, 0] + (K * (gam ** (T - 1 - t_idx))[:, None]).T @ V
+    np.testing.assert_allclose(S[0, 0], S_ref, rtol=1e-11, atol=1e-12)
+
+
 def test_gla_gate_scales_rows_of_state():
     """[LR] §2.2: g_t[i] multiplies row i (a key dim) of S; v = 0 isolates it."""
     dk, dv = 3, 2
@@ -186,6 +204,30 @@ def test_gdn_matches_transition_matrix_products():
         St = prod(0, t) @ S0[0, 0]
         for i in range(t + 1):
             St = St + prod(i + 1, t) @ np.outer(be[0, i, 0] * k[0, i, 0], v[0, i, 0])
+        np.testing.assert_allclose(o[0, t, 0], St.T @ q[0, t, 0], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S[0, 0], St, rtol=1e-11, atol=1e-12)
+
+
+def test_gdn_unit_alpha_is_delta_rule_products():
+    """[SS] Retention/Delta Rule: with alpha = 1 the gated rule is the delta rule
+    S_t = S_{t-1} + beta_t k_t (v_t - S_{t-1}^T k_t)^T, i.e. a product of the
+    rank-one corrections (I - beta_s k_s k_s^T) applied to S0 plus the written
+    values, evaluated here as dense products (no recurrence)."""
+    T, dk, dv = 10, 5, 3
+    q, k, v = _rand(1, T, 1, dk), _unit(_rand(1, T, 1, dk)), _rand(1, T, 1, dv)
+    be = rng.uniform(0.1, 1.0, (1, T, 1))
+    S0 = _rand(1, 1, dk, dv)
+    o, S = oracle.gdn_fwd(q, k, v, np.ones((1, T, 1)), be, S0)
+    E = [np.eye(dk) - be[0, s, 0] * np.outer(k[0, s, 0], k[0, s, 0]) for s in range(T)]
+    for t in range(T):
+        St = S0[0, 0].copy()
+        for s in range(t + 1):
+            St = E[s] @ St
+        for i in range(t + 1):
+            M = np.eye(dk)
+            for s in range(i + 1, t + 1):
+                M = E[s] @ M
+            St = St + M @ np.outer(be[0, i, 0] * k[0, i, 0], v[0, i, 0])
         np.testing.assert_allclose(o[0, t, 0], St.T @ q[0, t, 0], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(S[0, 0], St, rtol=1e-11, atol=1e-12)
 

@@ -84,15 +84,27 @@ def gdn_beta_from(x: torch.Tensor) -> torch.Tensor:
     return torch.sigmoid(x.double()).float()
 
 
+def retention_decay(H: int) -> torch.Tensor:
+    """One constant decay per head for the retention workloads: 1 - 2^-(5 + h mod 4)
+    (fp32, exact).  A synthetic choice spanning fast and slow heads."""
+    return torch.tensor([1.0 - 2.0 ** -(5 + h % 4) for h in range(H)], dtype=torch.float32)
+
+
 def make_problem(rule: str, B: int, T: int, H: int, dk: int, dv: int, *,
                  dtype: torch.dtype = torch.bfloat16, seed: int = 0,
                  init_state: str = "zero", eps: float = 1e-6,
-                 gla_gate: str = "softplus16", name: str = "") -> Problem:
+                 gla_gate: str = "softplus16", gdn_alpha: str = "sigmoid3",
+                 name: str = "") -> Problem:
     """Generic generator used by all prefill workloads and by the tests.
 
     ``init_state``: ``"zero"`` (S0=None, z0=None), ``"abs"`` (S0=|N(0,1)|,
     z0=1 for ELU), ``"normal"`` (S0=N(0,1)*0.1, z0=1+|N(0,1)| for ELU).
-    ``gla_gate``: ``"softplus16"`` (the workload recipe) or ``"ones"`` (g=1).
+    ``gla_gate``: ``"softplus16"`` (the workload recipe), ``"ones"`` (g=1: the
+    Lightning accumulation S_t = S_{t-1} + k_t v_t^T) or ``"retnet"`` (one
+    constant decay per head, 1 - 2^-(5 + h mod 4), on every key dim and token:
+    retention S_t = gamma S_{t-1} + k_t v_t^T).
+    ``gdn_alpha``: ``"sigmoid3"`` (the workload recipe) or ``"ones"`` (alpha=1:
+    the plain delta rule).
     """
     assert rule in RULES
     gen = _gen(seed)
@@ -103,11 +115,24 @@ def make_problem(rule: str, B: int, T: int, H: int, dk: int, dv: int, *,
     if rule == "gla":
         k = k / math.sqrt(dk)
         src = _randn(gen, B, T, H, dk)
-        g = gla_gate_from(src) if gla_gate == "softplus16" else torch.ones(B, T, H, dk)
+        if gla_gate == "softplus16":
+            g = gla_gate_from(src)
+        elif gla_gate == "ones":
+            g = torch.ones(B, T, H, dk)
+        elif gla_gate == "retnet":
+            g = retention_decay(H).view(1, 1, H, 1).expand(B, T, H, dk).contiguous()
+        else:
+            raise ValueError(gla_gate)
     elif rule == "gdn":
         q = _l2norm_last(q)
         k = _l2norm_last(k)
-        g = gdn_alpha_from(_randn(gen, B, T, H))
+        a_src = _randn(gen, B, T, H)
+        if gdn_alpha == "sigmoid3":
+            g = gdn_alpha_from(a_src)
+        elif gdn_alpha == "ones":
+            g = torch.ones(B, T, H)
+        else:
+            raise ValueError(gdn_alpha)
         beta = gdn_beta_from(_randn(gen, B, T, H))
     S0 = z0 = None
     if init_state == "abs":
