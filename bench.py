@@ -390,8 +390,9 @@ def run_gpu(args):
 def run_variants(torch, la, workloads, K, hbm_peak, seed):
     """The rule variants that run on the same kernels, at the prefill benchmark
     shape (B=2, H=16, T=8192, d=128): DeltaNet (gated delta rule, alpha = 1),
-    RetNet (GLA, one constant decay per head), Lightning (GLA, g = 1).  Each is
-    timed K times with CUDA events, after 3 warm-up calls."""
+    RetNet (GLA, one constant decay per head), Lightning (GLA, g = 1); and GLA /
+    gated-delta prefill of 32 packed variable-length sequences.  Each is timed K
+    times with CUDA events, after 3 warm-up calls."""
     spec = {"deltanet_prefill": ("gdn", dict(gdn_alpha="ones")),
             "retnet_prefill": ("gla", dict(gla_gate="retnet")),
             "lightning_prefill": ("gla", dict(gla_gate="ones"))}
@@ -418,6 +419,37 @@ def run_variants(torch, la, workloads, K, hbm_peak, seed):
         gbs = w["bytes"] / (ms / 1e3) / 1e9
         res[name] = {"ms": round(ms, 4), "tokens_per_s": round(w["tokens"] / (ms / 1e3)),
                      "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4)}
+        del a, o, S
+    # packed variable-length prefill: 32 sequences, lengths uniform in [1, 8192]
+    # (seeded), H=16, d=128, on one token axis
+    import numpy as np
+    lens = np.random.default_rng(1000 + seed).integers(1, 8193, size=32)
+    cu_h = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int64)
+    Ttot, Lmax = int(cu_h[-1]), int(lens.max())
+    for rule in ("gla", "gdn"):
+        p = workloads.make_problem(rule, 1, Ttot, 16, 128, 128, seed=seed)
+        a = [None if t is None else t.cuda() for t in (p.q, p.k, p.v, p.g, p.beta)]
+        cu = cu_h.cuda()
+        o = torch.empty(1, Ttot, 16, 128, dtype=torch.bfloat16, device="cuda")
+        S = torch.empty(32, 16, 128, 128, device="cuda")
+        run = lambda: la.fwd(rule, *a, o=o, S_out=S, cu_seqlens=cu, max_seqlen=Lmax)
+        for _ in range(3):
+            run()
+        stream = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            e0.record(stream)
+            run()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        la.check_device()
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / K
+        nbytes = prefill_bytes(rule, 1, Ttot, 16, 128, 128) + (32 - 1) * 16 * 128 * 128 * 4
+        gbs = nbytes / (ms / 1e3) / 1e9
+        res[f"packed_{rule}_prefill"] = {"ms": round(ms, 4), "tokens_per_s": round(Ttot / (ms / 1e3)),
+                                        "sequences": 32, "tokens": Ttot, "max_seqlen": Lmax,
+                                        "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4)}
         del a, o, S
     return res
 

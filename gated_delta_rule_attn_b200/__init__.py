@@ -16,6 +16,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libla_b200.so")
+ABI_VERSION = 2   # LA_ABI_VERSION of include/la.h that these struct layouts follow
 
 RULES = {"elu": 0, "gla": 1, "gdn": 2}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
@@ -43,7 +44,8 @@ class FwdArgs(ctypes.Structure):
                 ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("S0", ctypes.c_void_p),
                 ("z0", ctypes.c_void_p), ("eps", ctypes.c_float), ("o", ctypes.c_void_p),
                 ("S_out", ctypes.c_void_p), ("z_out", ctypes.c_void_p),
-                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("cu_seqlens", ctypes.c_void_p), ("max_seqlen", ctypes.c_int64)]
 
 
 class StepArgs(ctypes.Structure):
@@ -81,6 +83,9 @@ def lib():
                   L.la_fwd_host, L.la_check_device, L.la_fwd_noalloc):
             f.restype = ctypes.c_int
         L.la_abi_version.restype = ctypes.c_int
+        if L.la_abi_version() != ABI_VERSION:
+            raise ImportError(f"{LIB_PATH} has ABI version {L.la_abi_version()}, the binding expects "
+                              f"{ABI_VERSION}: rebuild it")
         _lib = L
     return _lib
 
@@ -109,9 +114,20 @@ def _need(t, name, device=True):
 
 
 def make_fwd_args(rule, q, k, v, g=None, beta=None, S0=None, z0=None, eps=1e-6,
-                  o=None, S_out=None, z_out=None) -> FwdArgs:
+                  o=None, S_out=None, z_out=None, cu_seqlens=None, max_seqlen=None) -> FwdArgs:
+    """Marshal tensors into la_fwd_args.  With ``cu_seqlens`` (int64 [B+1] on the
+    device) the token tensors are one packed axis [1, T, H, d] and B is the
+    number of sequences; ``max_seqlen`` bounds their lengths."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
+    if cu_seqlens is not None:
+        if B != 1:
+            raise ValueError("packed sequences take q, k, v as [1, T, H, d]")
+        if cu_seqlens.dtype != torch.int64 or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int64 tensor")
+        B = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("packed sequences need max_seqlen")
     a = FwdArgs()
     a.struct_size = ctypes.sizeof(FwdArgs)
     a.rule = RULES[rule]
@@ -124,6 +140,9 @@ def make_fwd_args(rule, q, k, v, g=None, beta=None, S0=None, z0=None, eps=1e-6,
     a.o = o.data_ptr() if o is not None else None
     a.S_out = S_out.data_ptr() if S_out is not None else None
     a.z_out = z_out.data_ptr() if z_out is not None else None
+    if cu_seqlens is not None:
+        a.cu_seqlens = cu_seqlens.data_ptr()
+        a.max_seqlen = int(max_seqlen)
     return a
 
 
@@ -142,24 +161,29 @@ def _workspace(device, stream_handle: int, nbytes: int):
 
 
 def fwd(rule: str, q, k, v, g=None, beta=None, S0=None, z0=None, eps: float = 1e-6,
-        o=None, S_out=None, z_out=None, stream=None, want_state: bool = True, workspace=None):
+        o=None, S_out=None, z_out=None, stream=None, want_state: bool = True, workspace=None,
+        cu_seqlens=None, max_seqlen=None):
     """Chunked prefill: returns (o, S_out, z_out-or-None). Enqueued on the current stream.
 
     ``workspace`` (a CUDA uint8 tensor of at least ``fwd_workspace_size`` bytes)
-    is allocated and cached per stream when not given."""
+    is allocated and cached per stream when not given.  ``cu_seqlens`` /
+    ``max_seqlen``: packed variable-length sequences (see ``make_fwd_args``);
+    the states are then [number of sequences, H, dk, dv]."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (S0, "S0"), (z0, "z0")):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (S0, "S0"), (z0, "z0"),
+                 (cu_seqlens, "cu_seqlens")):
         _need(t, n)
+    NS = B if cu_seqlens is None else cu_seqlens.numel() - 1   # sequences (state rows)
     if q.dtype != k.dtype or q.dtype != v.dtype:
         raise ValueError("q, k, v must share a dtype")
     if o is None:
         o = torch.empty(B, T, H, dv, dtype=q.dtype, device=q.device)
     if S_out is None and want_state:
-        S_out = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+        S_out = torch.empty(NS, H, dk, dv, dtype=torch.float32, device=q.device)
     if rule == "elu" and z_out is None and want_state:
-        z_out = torch.empty(B, H, dk, dtype=torch.float32, device=q.device)
-    a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, eps, o, S_out, z_out)
+        z_out = torch.empty(NS, H, dk, dtype=torch.float32, device=q.device)
+    a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, eps, o, S_out, z_out, cu_seqlens, max_seqlen)
     sh = _stream_handle(stream)
     n = ctypes.c_size_t()
     _check(lib().la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))

@@ -332,9 +332,11 @@ __device__ __forceinline__ void invert_unit_lower64(float *AF, float *TMP, int l
 
 struct GdnPrepParams {
     int64_t B, T, H;
-    int nchunks;
+    int nchunks;                  // chunks per (batch, head): ceil(max_seqlen / 64)
     const float *alpha, *beta;
-    uint8_t *ws;   // [B*H*nchunks][TT_BYTES]
+    uint8_t *ws;                  // [B*H*nchunks][TT_BYTES]
+    const int64_t *cu_seqlens;    // packed sequences, or nullptr (dense)
+    int64_t max_seqlen;           // = T for the dense layout
 };
 
 // One CTA handles (batch, head, chunk) items in a grid-stride loop.  The next
@@ -376,9 +378,10 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         const int64_t bh = w / p.nchunks;
         const int c = (int)(w % p.nchunks);
         const int64_t b = bh / p.H, h = bh % p.H;
+        const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, false);
         mbar_arrive_expect_tx(&ctl->full, 2u * C * 128u);
         for (int a = 0; a < KA; ++a)
-            tma_load_4d(tiles + P_K + a * (C * 128), &mapk, &ctl->full, 64 * a, (int)h, c * C, (int)b);
+            tma_load_4d(tiles + P_K + a * (C * 128), &mapk, &ctl->full, 64 * a, (int)h, sq.t0 + c * C, sq.b0);
     };
     // warp 0: item w's alpha, beta for tokens 2*lane, 2*lane+1 (1 and 0 past T)
     float al[2] = {1.f, 1.f}, be[2] = {0.f, 0.f};
@@ -386,11 +389,12 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         const int64_t bh = w / p.nchunks;
         const int c = (int)(w % p.nchunks);
         const int64_t b = bh / p.H, h = bh % p.H;
+        const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, false);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const int64_t tt = (int64_t)c * C + 2 * lane + e;
-            const bool in = tt < p.T;
-            const int64_t idx = (b * p.T + (in ? tt : 0)) * p.H + h;
+            const int64_t tt = (int64_t)c * C + 2 * lane + e;   // position in the sequence
+            const bool in = tt < sq.len;
+            const int64_t idx = (sq.row0 + (in ? tt : 0)) * p.H + h;
             al[e] = in ? p.alpha[idx] : 1.f;
             be[e] = in ? p.beta[idx] : 0.f;
         }
@@ -505,7 +509,11 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
     const int dvt = (int)(blockIdx.x % nslab);
     const int64_t bh = blockIdx.x / nslab;
     const int64_t b = bh / p.H, h = bh % p.H;
-    const int nchunks = (int)((p.T + C - 1) / C);
+    // this sequence's tokens (dense: all T of batch b); T images are stored for
+    // ceil(max_seqlen / 64) chunks per (batch, head)
+    const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, tid == 0 && h == 0 && dvt == 0);
+    const int nchunks = (int)((sq.len + C - 1) / C);
+    const int64_t ws_chunks = (p.max_seqlen + C - 1) / C;
 
     if (tid == 0) {
         for (int s = 0; s < NSTG; ++s) {
@@ -566,19 +574,19 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             int stop = (lane == 0) ? ctl->abort : 0;
             stop = __shfl_sync(0xffffffffu, stop, 0);
             if (stop) break;
-            const int t0 = c * C;
+            const int t0 = c * C;   // position in the sequence
             if (lane == 0) {
                 mbar_expect_tx(&ctl->full[s], 2u * KA * C * 128u + C * DVT * 2u + TT_BYTES);
                 uint8_t *qk = tiles + STG_QK + s * STG_QK_BYTES;
+                const int tm = sq.t0 + t0;   // tensor-map coordinate of the chunk's first token
 #pragma unroll
                 for (int a = 0; a < KA; ++a) {
-                    tma_load_4d(qk + a * QK_ACS, &maps.q, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
-                    tma_load_4d(qk + a * QK_ACS + 64 * 128, &maps.k, &ctl->full[s], 64 * a, (int)h, t0,
-                                (int)b);
+                    tma_load_4d(qk + a * QK_ACS, &maps.q, &ctl->full[s], 64 * a, (int)h, tm, sq.b0);
+                    tma_load_4d(qk + a * QK_ACS + 64 * 128, &maps.k, &ctl->full[s], 64 * a, (int)h, tm,
+                                sq.b0);
                 }
-                tma_load_4d(tiles + STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, t0,
-                            (int)b);
-                bulk_load(tiles + STG_TT + s * TT_BYTES, ws + (bh * nchunks + c) * (int64_t)TT_BYTES,
+                tma_load_4d(tiles + STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, tm, sq.b0);
+                bulk_load(tiles + STG_TT + s * TT_BYTES, ws + (bh * ws_chunks + c) * (int64_t)TT_BYTES,
                           TT_BYTES, &ctl->full[s]);
             }
             // the chunk's decay factors: b = log2 of the inclusive cumulative alpha,
@@ -587,9 +595,9 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int64_t tt = (int64_t)t0 + 2 * lane + e;
-                const bool in = tt < p.T;
-                al[e] = in ? p.g[(b * p.T + tt) * p.H + h] : 1.f;
-                ctl->bet[s][2 * lane + e] = in ? p.beta[(b * p.T + tt) * p.H + h] : 0.f;
+                const bool in = tt < sq.len;
+                al[e] = in ? p.g[(sq.row0 + tt) * p.H + h] : 1.f;
+                ctl->bet[s][2 * lane + e] = in ? p.beta[(sq.row0 + tt) * p.H + h] : 0.f;
             }
             const int fast = gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
             const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
@@ -615,7 +623,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         auto finish = [&](int j) {
             const int sj = j % NSTG, jb = j & 1;
             const int64_t tj = (int64_t)j * C;
-            const int nvalid = (int)min((int64_t)C, p.T - tj);
+            const int nvalid = (int)min((int64_t)C, sq.len - tj);
             if (!mbar_wait(&ctl->wready[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
             const float gam_o = ctl->gam[sj][ro & 63];   // read before the stage can be refilled
             bar_named(1, 128);
@@ -637,7 +645,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 tmem_wait_ld();
                 if (ro < nvalid) {
                     __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
-                                         ((b * p.T + tj + ro) * p.H + h) * p.dv + dvt * DVT;
+                                         ((sq.row0 + tj + ro) * p.H + h) * p.dv + dvt * DVT;
 #pragma unroll
                     for (int cc = 0; cc < 4; ++cc) {
                         uint4 u;

@@ -105,9 +105,11 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
     const int seg = (int)((blockIdx.x / nslab) % p.nseg);
     const int64_t bh = blockIdx.x / nslab / p.nseg;
     const int64_t b = bh / p.H, h = bh % p.H;
-    // this CTA's chunks: [cbase, cbase + nchunks) of the sequence
+    // this sequence's tokens (dense layout: all T of batch b; packed: its span of
+    // the token axis) and this CTA's chunks [cbase, cbase + nchunks) of it
+    const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, threadIdx.x == 0 && h == 0 && dvt == 0);
     const int cbase = seg * p.seg_chunks;
-    const int nchunks = (int)min((int64_t)p.seg_chunks, (p.T + C - 1) / C - cbase);
+    const int nchunks = (int)max((int64_t)0, min((int64_t)p.seg_chunks, (sq.len + C - 1) / C - cbase));
 
     auto stg = [&](int c) { return tiles + L::STG + (uint32_t)(c % NSTG) * L::STG_BYTES; };
 
@@ -163,14 +165,14 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         auto gate_load = [&](int c) {
             uint64_t *bar = &ctl->gfull[c & 1];
             mbar_arrive_expect_tx(bar, L::G_BYTES);
-            tma_load_4d(tiles + L::GT + (uint32_t)(c & 1) * L::G_BYTES, &maps.g, bar, 0, (int)h, (cbase + c) * C,
-                        (int)b);
+            tma_load_4d(tiles + L::GT + (uint32_t)(c & 1) * L::G_BYTES, &maps.g, bar, 0, (int)h,
+                        sq.t0 + (cbase + c) * C, sq.b0);
         };
         if (kGLA && leader)
             for (int c = 0; c < 2 && c < nchunks; ++c) gate_load(c);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTG;
-            const int nvalid = (int)min((int64_t)C, p.T - (int64_t)(cbase + c) * C);
+            const int nvalid = (int)min((int64_t)C, sq.len - (int64_t)(cbase + c) * C);
             if (leader) ctl->stopP = ctl->abort;
             bar_named(1, 256);
             if (ctl->stopP) break;
@@ -227,6 +229,13 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                         *reinterpret_cast<uint32_t *>(ka + off(h8 + i)) = pack_bf16x2(ks.x, ks.y);
                     }
                 }
+                // last chunk of a sequence: in a packed layout the rows past its
+                // end hold the next sequence's keys, which must not reach dS = K'^T V
+                if (nvalid < C) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (16 * qt + i >= nvalid) *reinterpret_cast<uint32_t *>(ka + off(i)) = 0u;
+                }
             } else {
                 // phi(Q), phi(K) in place (phi(k) = 0 past T), chunk sum of phi(k)
                 uint32_t qv[16], kv[16];
@@ -268,16 +277,16 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         auto load_chunk = [&](int c) {
             const int s = c % NSTG;
             uint8_t *st = stg(c);
-            const int t0 = (cbase + c) * C;
+            const int t0 = sq.t0 + (cbase + c) * C;   // tensor-map coordinate of the chunk's first token
             mbar_arrive_expect_tx(&ctl->full[s], 2u * L::Q_BYTES);
 #pragma unroll
             for (int a = 0; a < KA; ++a) {
-                tma_load_4d(st + a * (C * 128), &maps.q, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
-                tma_load_4d(st + L::Q_BYTES + a * L::K_ACS, &maps.k, &ctl->full[s], 64 * a, (int)h, t0, (int)b);
+                tma_load_4d(st + a * (C * 128), &maps.q, &ctl->full[s], 64 * a, (int)h, t0, sq.b0);
+                tma_load_4d(st + L::Q_BYTES + a * L::K_ACS, &maps.k, &ctl->full[s], 64 * a, (int)h, t0, sq.b0);
             }
             // the gate tile of chunk c+2 is loaded about one chunk period from
             // now: start bringing it into L2
-            if (kGLA && dvt == 0 && c + 2 < nchunks) tma_prefetch_l2_4d(&maps.g, 0, (int)h, t0 + 2 * C, (int)b);
+            if (kGLA && dvt == 0 && c + 2 < nchunks) tma_prefetch_l2_4d(&maps.g, 0, (int)h, t0 + 2 * C, sq.b0);
             issued = c;
         };
         // TMA of this CTA's V slab for chunk c
@@ -285,7 +294,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             const int j = c % L::NV;
             mbar_arrive_expect_tx(&ctl->vfull[j], L::V_BYTES);
             tma_load_4d(tiles + L::VR + (uint32_t)j * L::V_BYTES, &maps.v, &ctl->vfull[j], dvt * DVT, (int)h,
-                        (cbase + c) * C, (int)b);
+                        sq.t0 + (cbase + c) * C, sq.b0);
             issued_v = c;
         };
         if (a0) {
@@ -295,8 +304,8 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         for (int c = 0; c < nchunks; ++c) {
             const int bb = c & 1, j3 = c % 3;
             const uint32_t acc = L::C_ACC + 128u * (uint32_t)j3;
-            const int64_t t0 = (int64_t)(cbase + c) * C;
-            const int nvalid = (int)min((int64_t)C, p.T - t0);
+            const int64_t t0 = (int64_t)(cbase + c) * C;   // position in the sequence
+            const int nvalid = (int)min((int64_t)C, sq.len - t0);
             if (aborted(ctl)) break;
             if (!__all_sync(0xffffffffu, mbar_wait(&ctl->mP[j3], (uint32_t)(c / 3) & 1u))) {
                 ctl->abort = 1;
@@ -354,7 +363,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                         for (int jj = 0; jj < 16; ++jj) o[jj] *= inv;
                     }
                     __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
-                                         ((b * p.T + t0 + tr) * p.H + h) * p.dv + dvt * DVT + 16 * hf;
+                                         ((sq.row0 + t0 + tr) * p.H + h) * p.dv + dvt * DVT + 16 * hf;
 #pragma unroll
                     for (int cc = 0; cc < 2; ++cc) {
                         uint4 u;

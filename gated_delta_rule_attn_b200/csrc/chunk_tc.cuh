@@ -69,6 +69,11 @@ struct ChunkParams {
     // starts from S0 plus the partial sums in `agg` of segments < j
     int nseg = 1, nparts = 1, seg_chunks = 0;
     const float *agg = nullptr;
+    // packed sequences (tensors [1,T,H,*], sequence b = tokens [cu[b], cu[b+1]));
+    // nullptr = dense [B,T,H,*].  max_seqlen bounds every sequence's length (the
+    // launch sets it to T for the dense layout).
+    const int64_t *cu_seqlens = nullptr;
+    int64_t max_seqlen = 0;
 };
 
 namespace ck {
@@ -224,9 +229,14 @@ inline int resident_per_sm(const void *kernel, int threads, int dyn_smem, int tm
 // per-chunk T = (I + A)^-1 operand images (8 KB per (batch, head, chunk));
 // sequence-parallel ELU+1 the partial state sums of its first pass; GLA needs
 // none.
-inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv) {
+// `packed`: the sequences are packed on one token axis with lengths up to
+// max_seqlen (no sequence-parallel ELU+1 then).
+inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv,
+                                    bool packed = false, int64_t max_seqlen = 0) {
     if (T <= 0) return 0;
-    if (rule == kRuleGDN) return (size_t)(B * H * ((T + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;
+    const int64_t L = packed ? max_seqlen : T;
+    if (rule == kRuleGDN) return (size_t)(B * H * ((L + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;
+    if (packed) return 0;
     const SegPlan sp = seg_plan(rule, B, T, H, dv);
     if (sp.nseg < 2) return 0;
     return (size_t)(B * H * (sp.nseg - 1) * sp.nparts) * (size_t)(ck::DK * dv + ck::DK) * sizeof(float);
@@ -265,15 +275,20 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
     }
     Maps m;
     memset(&m, 0, sizeof(m));
-    bool okm = make_map_4d(&m.q, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, DK, 64, C,
+    const bool packed = p.cu_seqlens != nullptr;
+    const int64_t MB = packed ? 1 : p.B;   // outer extent of the 4-D tensor maps
+    bool okm = make_map_4d(&m.q, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, MB, p.T, p.H, DK, 64, C,
                            CU_TENSOR_MAP_SWIZZLE_128B) &&
-               make_map_4d(&m.k, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, DK, 64, C,
+               make_map_4d(&m.k, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, MB, p.T, p.H, DK, 64, C,
                            CU_TENSOR_MAP_SWIZZLE_128B) &&
-               make_map_4d(&m.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, p.dv, DVT, C,
+               make_map_4d(&m.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, MB, p.T, p.H, p.dv, DVT, C,
                            CU_TENSOR_MAP_SWIZZLE_64B);
     if (okm && rule == kRuleGLA)
-        okm = make_map_4d(&m.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.B, p.T, p.H, DK, DK, C,
+        okm = make_map_4d(&m.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, MB, p.T, p.H, DK, DK, C,
                           CU_TENSOR_MAP_SWIZZLE_NONE);
+    ChunkParams pq = p;
+    if (!packed) pq.max_seqlen = p.T;
+    const int64_t Lmax = pq.max_seqlen;
     if (!okm) {
         *err = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
         return 4;
@@ -281,15 +296,16 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
     const unsigned grid = (unsigned)(p.B * p.H * (p.dv / DVT));
     cudaError_t e;
     if (rule == kRuleGDN) {
-        const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv);
+        const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv, packed, Lmax);
         if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
             *err = "the gated delta rule needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
             return 8;
         }
         GdnPrepParams pp{};
         pp.B = p.B; pp.T = p.T; pp.H = p.H;
-        pp.nchunks = (int)((p.T + C - 1) / C);
+        pp.nchunks = (int)((Lmax + C - 1) / C);
         pp.alpha = p.g; pp.beta = p.beta;
+        pp.cu_seqlens = p.cu_seqlens; pp.max_seqlen = Lmax;
         pp.ws = static_cast<uint8_t *>(ws);
         const int64_t items = p.B * p.H * (int64_t)pp.nchunks;
         const int psmem = (int)((sizeof(gdn::PCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::P_END;
@@ -298,14 +314,15 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         // would double the time)
         const int per_sm = resident_per_sm((const void *)gdn_prep_kernel, gdn::PREP_THREADS, psmem, 64);
         const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
-        if (e == cudaSuccess) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.k, pp);
+        if (e == cudaSuccess && items > 0) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.k, pp);
         const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::TEND;
         if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel, smem);
         if (e == cudaSuccess)
-            chunk_gdn_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, p, static_cast<const uint8_t *>(ws));
+            chunk_gdn_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));
     } else {
-        const SegPlan sp = seg_plan(rule, p.B, p.T, p.H, p.dv);
-        ChunkParams q = p;
+        // packed sequences walk each sequence in one pass (no segments)
+        const SegPlan sp = packed ? SegPlan{1, 1, (int)((Lmax + C - 1) / C)} : seg_plan(rule, p.B, p.T, p.H, p.dv);
+        ChunkParams q = pq;
         if (sp.nseg > 1) {
             const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv);
             if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {

@@ -13,10 +13,33 @@ namespace la {
 
 // Device-wide error word (read and cleared by la_check_device).  The library is
 // one translation unit, so the definition lives here.
-enum : uint32_t { kErrTimeout = 1u, kErrRange = 2u };
+enum : uint32_t { kErrTimeout = 1u, kErrRange = 2u, kErrSeqlen = 4u };
 __device__ uint32_t g_error_word = 0;
 
 __device__ __forceinline__ void raise_error(uint32_t bit) { atomicOr(&g_error_word, bit); }
+
+// Where sequence b's tokens sit on the token axis: rows row0 .. row0+len-1 of a
+// [*, T, H, d] tensor viewed as rows of [H, d], and the (t, b) coordinates of its
+// first token for a 4-D tensor map.  Dense layout ([B, T, H, d], cu == nullptr):
+// row0 = b*T, len = T, map coordinates (0, b).  Packed layout (one token axis
+// of `total` tokens): row0 = cu[b], len = cu[b+1] - cu[b], map coordinates
+// (cu[b], 0).  Offsets are clamped into [0, total] and lengths to max_len, so a
+// bad offset array cannot move an access out of the tensors; `report` raises
+// kErrSeqlen when clamping changed anything.
+struct SeqSpan {
+    int64_t row0, len;
+    int t0, b0;
+};
+__device__ __forceinline__ SeqSpan seq_span(const int64_t *cu, int64_t b, int64_t T, int64_t max_len,
+                                            bool report) {
+    if (!cu) return SeqSpan{b * T, T, 0, (int)b};
+    const int64_t s_raw = cu[b], e_raw = cu[b + 1];
+    const int64_t s = s_raw < 0 ? 0 : (s_raw > T ? T : s_raw);
+    const int64_t e = e_raw < s ? s : (e_raw > T ? T : e_raw);
+    const int64_t len = e - s > max_len ? max_len : e - s;
+    if (report && (s != s_raw || e != e_raw || len != e - s)) raise_error(kErrSeqlen);
+    return SeqSpan{s, len, (int)s, 0};
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

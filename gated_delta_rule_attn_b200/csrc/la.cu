@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cstddef>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -182,7 +183,7 @@ bool uses_chunk_kernels(const la_fwd_args &a) { return a.dtype == LA_BF16 && a.d
 
 la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
     const Shape s{a.B, a.T, a.H, a.dk, a.dv};
-    if (a.T == 0) {
+    if (a.T == 0 || (a.cu_seqlens && a.max_seqlen == 0)) {   // no token in any sequence
         const size_t sb = (size_t)(s.B * s.H * s.dk * s.dv) * sizeof(float);
         const size_t zb = (size_t)(s.B * s.H * s.dk) * sizeof(float);
         if (a.S_out && a.S_out != a.S0) {
@@ -203,6 +204,7 @@ la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
         p.q = a.q; p.k = a.k; p.v = a.v; p.g = a.g; p.beta = a.beta;
         p.S0 = a.S0; p.z0 = a.z0; p.S_out = a.S_out; p.z_out = a.z_out;
         p.o = a.o; p.eps = a.eps;
+        p.cu_seqlens = a.cu_seqlens; p.max_seqlen = a.max_seqlen;
         std::string err;
         const la_status r =
             (la_status)la::launch_chunk_tc((int)a.rule, p, a.workspace, a.workspace_bytes, st, &err);
@@ -214,13 +216,26 @@ la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
     p.q = a.q; p.k = a.k; p.v = a.v; p.g = a.g; p.beta = a.beta;
     p.S_in = a.S0; p.S_out = a.S_out; p.z_in = a.z0; p.z_out = a.z_out;
     p.o = a.o; p.eps = a.eps;
+    p.cu_seqlens = a.cu_seqlens; p.max_seqlen = a.max_seqlen;
     return launch_recurrent(a.rule, p, a.dk, a.dv, a.dtype, st);
 }
 
-la_status validate_fwd(const la_fwd_args *a, bool device_ptrs) {
-    if (!a) return fail(LA_ERR_INVALID_ARG, "args is NULL");
-    if (a->struct_size < sizeof(la_fwd_args))
-        return fail(LA_ERR_INVALID_ARG, "struct_size smaller than sizeof(la_fwd_args)");
+// The caller's arguments as this library's la_fwd_args: a struct from an older
+// header (ABI version 1, without the packed-sequence fields) is accepted and the
+// missing fields read as NULL / 0.
+la_status load_fwd_args(const la_fwd_args *in, la_fwd_args *out) {
+    if (!in) return fail(LA_ERR_INVALID_ARG, "args is NULL");
+    constexpr size_t v1 = offsetof(la_fwd_args, cu_seqlens);
+    if (in->struct_size < v1)
+        return fail(LA_ERR_INVALID_ARG, "struct_size smaller than the version-1 la_fwd_args");
+    memset(out, 0, sizeof(*out));
+    memcpy(out, in, in->struct_size < sizeof(la_fwd_args) ? in->struct_size : sizeof(la_fwd_args));
+    out->struct_size = sizeof(la_fwd_args);
+    return LA_OK;
+}
+
+// `host_bufs`: the data pointers are host pointers (la_fwd_host).
+la_status validate_fwd(const la_fwd_args *a, bool device_ptrs, bool host_bufs = false) {
     const Shape s{a->B, a->T, a->H, a->dk, a->dv};
     la_status r = validate_common(a->rule, a->dtype, s);
     if (r != LA_OK) return r;
@@ -229,6 +244,14 @@ la_status validate_fwd(const la_fwd_args *a, bool device_ptrs) {
     if (a->T > 0 && (!a->q || !a->k || !a->v || !a->o))
         return fail(LA_ERR_INVALID_ARG, "q, k, v and o must be non-NULL when T > 0");
     if (!(a->eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+    if (a->cu_seqlens) {
+        if (host_bufs)
+            return fail(LA_ERR_UNSUPPORTED, "packed sequences (cu_seqlens) need device buffers: use la_fwd");
+        if (reinterpret_cast<uintptr_t>(a->cu_seqlens) & 7u)
+            return fail(LA_ERR_ALIGNMENT, "cu_seqlens must be 8-byte aligned");
+        if (a->max_seqlen < 0 || a->max_seqlen > a->T)
+            return fail(LA_ERR_INVALID_ARG, "packed sequences need 0 <= max_seqlen <= T");
+    }
     if (device_ptrs) {
         const void *ps[] = {a->q, a->k, a->v, a->g, a->beta, a->S0, a->z0, a->o, a->S_out, a->z_out};
         for (const void *p : ps)
@@ -241,16 +264,20 @@ la_status validate_fwd(const la_fwd_args *a, bool device_ptrs) {
 
 extern "C" {
 
-la_status la_fwd(const la_fwd_args *args, void *stream) {
-    la_status r = validate_fwd(args, true);
+la_status la_fwd(const la_fwd_args *in, void *stream) {
+    la_fwd_args A;
+    la_status r = load_fwd_args(in, &A);
     if (r != LA_OK) return r;
-    if (uses_chunk_kernels(*args)) {
-        const size_t need = la::chunk_workspace_bytes((int)args->rule, args->B, args->T, args->H, args->dv);
-        if (need && (!args->workspace || args->workspace_bytes < need || !aligned16(args->workspace)))
+    r = validate_fwd(&A, true);
+    if (r != LA_OK) return r;
+    if (uses_chunk_kernels(A)) {
+        const size_t need = la::chunk_workspace_bytes((int)A.rule, A.B, A.T, A.H, A.dv, A.cu_seqlens != nullptr,
+                                                      A.max_seqlen);
+        if (need && (!A.workspace || A.workspace_bytes < need || !aligned16(A.workspace)))
             return fail(LA_ERR_WORKSPACE,
                         "workspace missing, misaligned or smaller than la_fwd_workspace_size()");
     }
-    return launch_fwd(*args, static_cast<cudaStream_t>(stream));
+    return launch_fwd(A, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------
@@ -284,13 +311,16 @@ la_status noalloc_scratch(void **out) {
 }  // namespace
 
 la_status la_fwd_noalloc(const la_fwd_args *args, void *stream) {
-    la_status r = validate_fwd(args, true);
+    la_fwd_args a;
+    la_status r = load_fwd_args(args, &a);
     if (r != LA_OK) return r;
-    la_fwd_args a = *args;
+    r = validate_fwd(&a, true);
+    if (r != LA_OK) return r;
     a.workspace = nullptr;
     a.workspace_bytes = 0;
-    const size_t need =
-        uses_chunk_kernels(a) ? la::chunk_workspace_bytes((int)a.rule, a.B, a.T, a.H, a.dv) : 0;
+    const size_t need = uses_chunk_kernels(a) ? la::chunk_workspace_bytes((int)a.rule, a.B, a.T, a.H, a.dv,
+                                                                          a.cu_seqlens != nullptr, a.max_seqlen)
+                                              : 0;
     if (need > LA_NOALLOC_SCRATCH_BYTES)
         return fail(LA_ERR_WORKSPACE, "problem needs " + std::to_string(need) +
                                           " bytes of scratch; la_fwd_noalloc has " +
@@ -306,11 +336,14 @@ la_status la_fwd_noalloc(const la_fwd_args *args, void *stream) {
 
 la_status la_fwd_workspace_size(const la_fwd_args *args, size_t *bytes) {
     if (!bytes) return fail(LA_ERR_INVALID_ARG, "bytes is NULL");
-    la_status r = validate_fwd(args, false);
+    la_fwd_args a;
+    la_status r = load_fwd_args(args, &a);
     if (r != LA_OK) return r;
-    *bytes = uses_chunk_kernels(*args)
-                 ? la::chunk_workspace_bytes((int)args->rule, args->B, args->T, args->H, args->dv)
-                 : 0;
+    r = validate_fwd(&a, false);
+    if (r != LA_OK) return r;
+    *bytes = uses_chunk_kernels(a) ? la::chunk_workspace_bytes((int)a.rule, a.B, a.T, a.H, a.dv,
+                                                               a.cu_seqlens != nullptr, a.max_seqlen)
+                                   : 0;
     return ok();
 }
 
@@ -369,16 +402,23 @@ static void staging_layout(const la_fwd_args *a, StagingLayout *L) {
 
 la_status la_fwd_host_staging_size(const la_fwd_args *args, size_t *bytes) {
     if (!bytes) return fail(LA_ERR_INVALID_ARG, "bytes is NULL");
-    la_status r = validate_fwd(args, false);
+    la_fwd_args a;
+    la_status r = load_fwd_args(args, &a);
+    if (r != LA_OK) return r;
+    r = validate_fwd(&a, false, true);
     if (r != LA_OK) return r;
     StagingLayout L;
-    staging_layout(args, &L);
+    staging_layout(&a, &L);
     *bytes = L.total;
     return ok();
 }
 
-la_status la_fwd_host(const la_fwd_args *h, void *staging, size_t staging_bytes, void *stream) {
-    la_status r = validate_fwd(h, false);
+la_status la_fwd_host(const la_fwd_args *h_in, void *staging, size_t staging_bytes, void *stream) {
+    la_fwd_args H_args;
+    la_status r = load_fwd_args(h_in, &H_args);
+    if (r != LA_OK) return r;
+    const la_fwd_args *h = &H_args;
+    r = validate_fwd(h, false, true);
     if (r != LA_OK) return r;
     if (!staging || (reinterpret_cast<uintptr_t>(staging) & 255u))
         return fail(LA_ERR_ALIGNMENT, "staging must be a 256-byte aligned device buffer");
@@ -430,6 +470,10 @@ la_status la_check_device(void *stream, uint32_t *flags) {
     if (w & la::kErrTimeout) return fail(LA_ERR_TIMEOUT, "a bounded device wait ran out");
     if (w & la::kErrRange)
         return fail(LA_ERR_RANGE, "GLA cumulative gate inside a 64-token chunk fell below 1e-30");
+    if (w & la::kErrSeqlen)
+        return fail(LA_ERR_INVALID_ARG,
+                    "cu_seqlens: offsets out of order or outside [0, T], or a sequence longer than "
+                    "max_seqlen (clamped; those sequences' results are incomplete)");
     return ok();
 }
 

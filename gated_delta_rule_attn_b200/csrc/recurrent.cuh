@@ -40,6 +40,10 @@ struct RecurrentParams {
     float *z_out;               // ELU [B,H,dk] or null; may equal z_in
     void *o;                    // [B,T,H,dv]
     float eps;
+    // packed sequences: sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]) of
+    // one token axis of T tokens (tensors [1,T,H,*]); nullptr = dense layout
+    const int64_t *cu_seqlens = nullptr;
+    int64_t max_seqlen = 0;
 };
 
 __device__ __forceinline__ float elu_feature_precise(float x) {
@@ -85,8 +89,9 @@ __global__ void __launch_bounds__(256, 2) recurrent_kernel(const RecurrentParams
     const TIO *v = static_cast<const TIO *>(p.v);
     TIO *o = static_cast<TIO *>(p.o);
 
-    for (int64_t t = 0; t < T; ++t) {
-        const int64_t row = (b * T + t) * H + h;  // token row index into [B,T,H,*]
+    const SeqSpan sq = seq_span(p.cu_seqlens, b, T, p.max_seqlen, tid == 0 && h == 0);
+    for (int64_t t = 0; t < sq.len; ++t) {
+        const int64_t row = (sq.row0 + t) * H + h;  // token row index into [B,T,H,*] / [1,T,H,*]
         if (tid < DK) {
             float qx = to_f32(q[row * DK + tid]);
             float kx = to_f32(k[row * DK + tid]);

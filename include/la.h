@@ -40,7 +40,8 @@
  *     NULL = the legacy default stream) and returns immediately.  Arguments are
  *     validated on the host before any launch; an invalid call launches nothing.
  *   - Conditions detected on the device (a bounded wait that ran out, a GLA
- *     chunk whose cumulative gate leaves the fp32 range) set a device-wide error
+ *     chunk whose cumulative gate leaves the fp32 range, packed-sequence
+ *     offsets that are out of order or out of range) set a device-wide error
  *     word; la_check_device() reads and clears it.
  *   - Supported sizes: dk, dv in {32, 64, 128}; B, H >= 1; T >= 0.  T == 0
  *     writes S_out = S0 (or zeros) and z_out = z0 (or zeros).
@@ -56,7 +57,7 @@
 extern "C" {
 #endif
 
-#define LA_ABI_VERSION 1
+#define LA_ABI_VERSION 2
 
 typedef enum {
     LA_OK = 0,
@@ -99,6 +100,24 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *          one workspace must be ordered (same stream), otherwise they race.
  *          A missing or short workspace returns LA_ERR_WORKSPACE before any launch.
  * q/k/v/o must not overlap S_out/z_out.
+ *
+ * Packed variable-length sequences (fields appended in ABI version 2; a caller
+ * built against version 1 passes the smaller struct_size and gets the dense
+ * layout above):
+ *   cu_seqlens  device int64 [B+1], or NULL for the dense layout.  Sequence b
+ *          is tokens [cu_seqlens[b], cu_seqlens[b+1]) of ONE packed token axis:
+ *          q, k, g [1,T,H,*], v, o [1,T,H,dv], beta [1,T,H], with T the packed
+ *          length.  B counts sequences; S0/S_out/z0/z_out stay [B,H,...] and
+ *          every sequence starts from its own S0[b] (state reset at each
+ *          sequence start; the "verification matrix" of page "状态空间与线性注意力"
+ *          asks for exactly this reset).  Offsets must be nondecreasing, within
+ *          [0, T], 8-byte aligned.  Sequences may be empty.
+ *   max_seqlen  upper bound of cu_seqlens[b+1] - cu_seqlens[b] (0 <= max_seqlen
+ *          <= T); sizes the gated delta rule's workspace and the grid.
+ *   The offsets are read on the device only: offsets out of order or outside
+ *   [0, T], or a sequence longer than max_seqlen, are clamped to stay in bounds
+ *   and reported by la_check_device as LA_ERR_INVALID_ARG.  Packed sequences
+ *   are not accepted by la_fwd_host (LA_ERR_UNSUPPORTED).
  */
 typedef struct la_fwd_args {
     uint32_t struct_size;     /* = sizeof(la_fwd_args) */
@@ -116,6 +135,8 @@ typedef struct la_fwd_args {
     float *z_out;
     void *workspace;
     size_t workspace_bytes;
+    const int64_t *cu_seqlens;   /* ABI version 2 */
+    int64_t max_seqlen;          /* ABI version 2 */
 } la_fwd_args;
 
 /*

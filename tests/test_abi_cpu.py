@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.la_abi_version() == 1
+    assert L.la_abi_version() == 2
     assert L.la_status_string(0) == b"LA_OK"
     assert L.la_status_string(5) == b"LA_ERR_TIMEOUT"
     assert L.la_status_string(99) == b"LA_ERR_UNKNOWN"
@@ -146,3 +146,48 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 4, 1, 32, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         la.fwd("elu", q, q, q)
+
+
+# ---------------------------------------------------------------------------
+# Packed variable-length sequences (la_fwd_args fields of ABI version 2)
+# ---------------------------------------------------------------------------
+
+def test_version1_struct_size_still_accepted(L):
+    """A caller built against the version-1 header passes the smaller struct
+    (without cu_seqlens / max_seqlen) and gets the dense layout."""
+    a = args(T=130)
+    a.struct_size = la.FwdArgs.cu_seqlens.offset
+    a.cu_seqlens = 0xDEAD   # past the caller's struct: must be ignored
+    n = ctypes.c_size_t(0)
+    assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 1 * 2 * 3 * 8192
+    a.struct_size = la.FwdArgs.cu_seqlens.offset - 8
+    assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 1
+
+
+def test_packed_workspace_follows_max_seqlen(L):
+    """Gated delta rule: one 8 KB T image per (sequence, head, 64-token chunk of
+    the longest sequence); packed ELU+1 runs without segments (no workspace)."""
+    n = ctypes.c_size_t(0)
+    a = args(B=5, T=1000, H=2, cu_seqlens=FAKE, max_seqlen=300)
+    assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 5 * 2 * 5 * 8192
+    a = args("elu", B=1, T=40000, H=2, cu_seqlens=FAKE, max_seqlen=40000)
+    assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 0
+
+
+def test_packed_argument_checks(L):
+    bad_len = args(B=3, T=100, cu_seqlens=FAKE, max_seqlen=101)
+    assert L.la_fwd(ctypes.byref(bad_len), None) == 1
+    assert b"max_seqlen" in L.la_last_error_message()
+    neg = args(B=3, T=100, cu_seqlens=FAKE, max_seqlen=-1)
+    assert L.la_fwd(ctypes.byref(neg), None) == 1
+    mis = args(B=3, T=100, cu_seqlens=FAKE + 4, max_seqlen=50)
+    assert L.la_fwd(ctypes.byref(mis), None) == 3
+    # host buffers: packed sequences are not offered on la_fwd_host
+    h = args(B=3, T=100, cu_seqlens=FAKE, max_seqlen=50)
+    n = ctypes.c_size_t(0)
+    assert L.la_fwd_host_staging_size(ctypes.byref(h), ctypes.byref(n)) == 2
+    assert L.la_fwd_host(ctypes.byref(h), ctypes.c_void_p(FAKE), 1 << 30, None) == 2
+    assert b"la_fwd" in L.la_last_error_message()
