@@ -38,6 +38,7 @@ def _load():
         lib.oracle_elu.argtypes = [I, I, I, I, I, P, P, P, P, P, ctypes.c_double, P, P, P]
         lib.oracle_gla.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P]
         lib.oracle_gdn.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P]
+        lib.oracle_kda.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P]
         for f in (lib.oracle_elu, lib.oracle_gla, lib.oracle_gdn):
             f.restype = None
         _lib = lib
@@ -103,6 +104,19 @@ def gdn_fwd(q, k, v, alpha, beta, S0=None):
     return o, S
 
 
+def kda_fwd(q, k, v, alpha, beta, S0=None):
+    """KDA (per-key-channel retention alpha [B,T,H,dk] with the delta rule), dk x dv
+    state. Returns (o, S)."""
+    q, k, v, alpha, beta, S0 = map(_f64, (q, k, v, alpha, beta, S0))
+    B, T, H, dk, dv = _shape(q, v)
+    assert alpha.shape == (B, T, H, dk) and beta.shape == (B, T, H)
+    o = np.empty((B, T, H, dv))
+    S = np.empty((B, H, dk, dv))
+    _load().oracle_kda(B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                       _ptr(S0), _ptr(o), _ptr(S))
+    return o, S
+
+
 def fwd(problem):
     """Run the oracle on a ``workloads.Problem``; returns (o, S, z-or-None)."""
     p = problem
@@ -113,6 +127,9 @@ def fwd(problem):
         return o, S, None
     if p.rule == "gdn":
         o, S = gdn_fwd(p.q, p.k, p.v, p.g, p.beta, p.S0)
+        return o, S, None
+    if p.rule == "kda":
+        o, S = kda_fwd(p.q, p.k, p.v, p.g, p.beta, p.S0)
         return o, S, None
     raise ValueError(p.rule)
 
@@ -131,6 +148,9 @@ def step(rule: str, q, k, v, S, z=None, g=None, beta=None, eps: float = 1e-6):
         return o[:, 0], S2, None
     if rule == "gdn":
         o, S2 = gdn_fwd(q1, k1, v1, _f64(g)[:, None], _f64(beta)[:, None], S)
+        return o[:, 0], S2, None
+    if rule == "kda":
+        o, S2 = kda_fwd(q1, k1, v1, _f64(g)[:, None], _f64(beta)[:, None], S)
         return o[:, 0], S2, None
     raise ValueError(rule)
 

@@ -35,6 +35,11 @@
  *     orientation of "状态空间与线性注意力", section Retention、衰减与 Delta
  *     Rule; output o_t = S_t^T q_t read after the write, as in that page's
  *     KDA recurrent reference.
+ *   KDA (per-key-channel retention with the delta rule): "状态空间与线性注意力",
+ *     section KDA：逐通道遗忘与误差写入.  The old state is first decayed row by
+ *     row, Sbar = Diag(alpha_t) S_{t-1}; the residual of the decayed state's
+ *     prediction is then written, S_t = Sbar + beta_t k_t (v_t - Sbar^T k_t)^T;
+ *     o_t = S_t^T q_t.  alpha [B,T,H,dk], beta [B,T,H].
  */
 #include <math.h>
 #include <stdint.h>
@@ -164,4 +169,41 @@ void oracle_gdn(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
     }
 }
 
-int oracle_abi_version(void) { return 1; }
+/* KDA: decay each key row of the state, then the delta-rule write. */
+void oracle_kda(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                const double *q, const double *k, const double *v,
+                const double *alpha, const double *beta,
+                const double *S0, double *o, double *S_out) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H;
+        double *S = (double *)malloc(sizeof(double) * (size_t)(dk * dv + 2 * dv));
+        double *pred = S + dk * dv, *acc = pred + dv;
+        load_state(S, S0, b, h, H, dk * dv);
+        for (int64_t t = 0; t < T; ++t) {
+            const double *qt = q + IDX4(b, t, h, 0, T, H, dk);
+            const double *kt = k + IDX4(b, t, h, 0, T, H, dk);
+            const double *vt = v + IDX4(b, t, h, 0, T, H, dv);
+            const double *at = alpha + IDX4(b, t, h, 0, T, H, dk);
+            const double be = beta[IDX3(b, t, h, T, H)];
+            /* Sbar = Diag(alpha_t) S_{t-1} */
+            for (int64_t d = 0; d < dk; ++d)
+                for (int64_t j = 0; j < dv; ++j) S[d * dv + j] *= at[d];
+            /* pred = Sbar^T k_t, then S_t = Sbar + beta k (v - pred)^T */
+            for (int64_t j = 0; j < dv; ++j) pred[j] = 0.0;
+            for (int64_t d = 0; d < dk; ++d)
+                for (int64_t j = 0; j < dv; ++j) pred[j] += kt[d] * S[d * dv + j];
+            for (int64_t d = 0; d < dk; ++d)
+                for (int64_t j = 0; j < dv; ++j) S[d * dv + j] += be * kt[d] * (vt[j] - pred[j]);
+            /* o_t = S_t^T q_t */
+            for (int64_t j = 0; j < dv; ++j) acc[j] = 0.0;
+            for (int64_t d = 0; d < dk; ++d)
+                for (int64_t j = 0; j < dv; ++j) acc[j] += qt[d] * S[d * dv + j];
+            memcpy(o + IDX4(b, t, h, 0, T, H, dv), acc, sizeof(double) * (size_t)dv);
+        }
+        store_state(S_out, S, b, h, H, dk * dv);
+        free(S);
+    }
+}
+
+int oracle_abi_version(void) { return 2; }

@@ -232,6 +232,67 @@ def test_gdn_unit_alpha_is_delta_rule_products():
     np.testing.assert_allclose(S[0, 0], St, rtol=1e-11, atol=1e-12)
 
 
+def test_kda_matches_transition_matrix_products():
+    """[SS] KDA: decay, then the delta write on the decayed state, i.e.
+    S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T, evaluated
+    as dense transition products (an oracle that wrote before decaying, or
+    decayed the written term, fails this)."""
+    T, dk, dv = 9, 4, 3
+    q, k, v = _rand(1, T, 1, dk), _unit(_rand(1, T, 1, dk)), _rand(1, T, 1, dv)
+    a = rng.uniform(0.2, 1.0, (1, T, 1, dk))
+    be = rng.uniform(0.1, 1.0, (1, T, 1))
+    S0 = _rand(1, 1, dk, dv)
+    o, S = oracle.kda_fwd(q, k, v, a, be, S0)
+    A = [(np.eye(dk) - be[0, s, 0] * np.outer(k[0, s, 0], k[0, s, 0])) @ np.diag(a[0, s, 0])
+         for s in range(T)]
+
+    def prod(lo, hi):  # A_hi ... A_lo
+        M = np.eye(dk)
+        for s in range(lo, hi + 1):
+            M = A[s] @ M
+        return M
+
+    for t in range(T):
+        St = prod(0, t) @ S0[0, 0]
+        for i in range(t + 1):
+            St = St + prod(i + 1, t) @ np.outer(be[0, i, 0] * k[0, i, 0], v[0, i, 0])
+        np.testing.assert_allclose(o[0, t, 0], St.T @ q[0, t, 0], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S[0, 0], St, rtol=1e-11, atol=1e-12)
+
+
+def test_kda_with_one_retention_per_token_is_gated_delta_rule():
+    """alpha_t equal on every key channel: Diag(alpha_t) = alpha_t I commutes with
+    I - beta k k^T, so KDA is the gated delta rule ([SS] KDA vs [LS] GDN box)."""
+    B, T, H, dk, dv = 2, 17, 2, 5, 3
+    q, k, v = _rand(B, T, H, dk), _unit(_rand(B, T, H, dk)), _rand(B, T, H, dv)
+    a = rng.uniform(0.3, 1.0, (B, T, H))
+    be = rng.uniform(0.0, 1.0, (B, T, H))
+    S0 = _rand(B, H, dk, dv)
+    o1, S1 = oracle.kda_fwd(q, k, v, np.repeat(a[..., None], dk, axis=-1), be, S0)
+    o2, S2 = oracle.gdn_fwd(q, k, v, a, be, S0)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S1, S2, rtol=1e-12, atol=1e-13)
+
+
+def test_kda_zero_beta_is_channelwise_decay():
+    """beta = 0: S_t = Diag(prod_{s<=t} alpha_s) S0 and o_t = S_t^T q_t."""
+    T, dk, dv = 10, 4, 3
+    q, k, v = _rand(1, T, 1, dk), _rand(1, T, 1, dk), _rand(1, T, 1, dv)
+    a = rng.uniform(0.5, 1.0, (1, T, 1, dk))
+    S0 = _rand(1, 1, dk, dv)
+    o, S = oracle.kda_fwd(q, k, v, a, np.zeros((1, T, 1)), S0)
+    cum = np.cumprod(a[0, :, 0], axis=0)                     # [T, dk]
+    ref = np.einsum("td,dj,td->tj", q[0, :, 0], S0[0, 0], cum)
+    np.testing.assert_allclose(o[0, :, 0], ref, rtol=1e-12)
+    np.testing.assert_allclose(S[0, 0], cum[-1][:, None] * S0[0, 0], rtol=1e-12)
+
+
+def test_kda_workload_decay_is_bounded():
+    """The bounded log-decay keeps every retention in (e^-5, 1) ([SS] 有界 log-decay)."""
+    p = workloads.make_problem("kda", 2, 300, 3, 16, 8, seed=1)
+    assert float(p.g.min()) > math.exp(-5.0) and float(p.g.max()) < 1.0
+
+
 def test_gdn_zero_beta_is_pure_decay():
     """beta = 0: S_t = (prod alpha) S0 and o_t = (prod_{s<=t} alpha_s) S0^T q_t."""
     T, dk, dv = 12, 5, 4
@@ -313,11 +374,14 @@ def _run(rule, q, k, v, g, be, S0, z0):
     if rule == "gla":
         o, S = oracle.gla_fwd(q, k, v, g, S0)
         return o, S, None
+    if rule == "kda":
+        o, S = oracle.kda_fwd(q, k, v, g, be, S0)
+        return o, S, None
     o, S = oracle.gdn_fwd(q, k, v, g, be, S0)
     return o, S, None
 
 
-@pytest.mark.parametrize("rule", ["elu", "gla", "gdn"])
+@pytest.mark.parametrize("rule", ["elu", "gla", "gdn", "kda"])
 @pytest.mark.parametrize("tau", [0, 1, 7, 20, 29])
 def test_split_invariance_bitwise(rule, tau):
     """[SS] selective scan / KDA recurrent reference / 验证矩阵 (chunk boundary):
@@ -340,7 +404,7 @@ def test_split_invariance_bitwise(rule, tau):
         assert np.array_equal(z2, z)
 
 
-@pytest.mark.parametrize("rule", ["elu", "gla", "gdn"])
+@pytest.mark.parametrize("rule", ["elu", "gla", "gdn", "kda"])
 def test_sequences_are_independent(rule):
     """[SS] 验证矩阵 (reset: a batched run equals per-sample runs)."""
     p = workloads.make_problem(rule, 2, 10, 3, 4, 4, seed=5, init_state="normal")
@@ -357,7 +421,7 @@ def test_sequences_are_independent(rule):
             assert np.array_equal(S1[0, 0], S[b, h])
 
 
-@pytest.mark.parametrize("rule", ["elu", "gla", "gdn"])
+@pytest.mark.parametrize("rule", ["elu", "gla", "gdn", "kda"])
 def test_step_is_recurrence_at_T1(rule):
     """A decode step is one token of the recurrence: T steps of ``step`` equal
     one ``fwd`` over T tokens."""

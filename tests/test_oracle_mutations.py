@@ -34,6 +34,12 @@ MUTANTS = {
                                "const double a = beta[IDX3(b, t, h, T, H)];\n            const double be = alpha[IDX3(b, t, h, T, H)];"),
     "gdn_prediction_transposed": ("for (int64_t j = 0; j < dv; ++j) kS[j] += kt[d] * S[d * dv + j];",
                                   "for (int64_t j = 0; j < dv; ++j) kS[j] += kt[j % dk] * S[d * dv + j];"),
+    # KDA
+    "kda_decay_on_columns": ("S[d * dv + j] *= at[d];", "S[d * dv + j] *= at[j % dk];"),
+    "kda_decay_skipped": ("S[d * dv + j] *= at[d];", "S[d * dv + j] *= 1.0;"),
+    "kda_residual_sign": ("(vt[j] - pred[j])", "(vt[j] + pred[j])"),
+    "kda_write_not_scaled_by_beta": ("S[d * dv + j] += be * kt[d] * (vt[j] - pred[j]);",
+                                     "S[d * dv + j] += kt[d] * (vt[j] - pred[j]);"),
 }
 
 

@@ -29,7 +29,7 @@ from typing import Optional
 
 import torch
 
-RULES = ("elu", "gla", "gdn")
+RULES = ("elu", "gla", "gdn", "kda")
 
 
 @dataclass
@@ -84,6 +84,13 @@ def gdn_beta_from(x: torch.Tensor) -> torch.Tensor:
     return torch.sigmoid(x.double()).float()
 
 
+def kda_alpha_from(x: torch.Tensor, g_min: float = -5.0) -> torch.Tensor:
+    """Per-channel KDA retention with the bounded log-decay of page "状态空间与线性注意力"
+    (有界 log-decay): alpha = exp(g_min * sigmoid(x)) in (e^g_min, 1), the scale
+    e^A taken as 1; evaluated in fp64 and rounded once to fp32."""
+    return torch.exp(g_min * torch.sigmoid(x.double())).float()
+
+
 def retention_decay(H: int) -> torch.Tensor:
     """One constant decay per head for the retention workloads: 1 - 2^-(5 + h mod 4)
     (fp32, exact).  A synthetic choice spanning fast and slow heads."""
@@ -123,6 +130,11 @@ def make_problem(rule: str, B: int, T: int, H: int, dk: int, dv: int, *,
             g = retention_decay(H).view(1, 1, H, 1).expand(B, T, H, dk).contiguous()
         else:
             raise ValueError(gla_gate)
+    elif rule == "kda":
+        q = _l2norm_last(q)
+        k = _l2norm_last(k)
+        g = kda_alpha_from(_randn(gen, B, T, H, dk))
+        beta = gdn_beta_from(_randn(gen, B, T, H))
     elif rule == "gdn":
         q = _l2norm_last(q)
         k = _l2norm_last(k)
