@@ -387,11 +387,28 @@ def run_gpu(args):
         print(json.dumps(out), flush=True)
 
 
+def _time_calls(torch, run, K):
+    """Mean device time (ms) of K calls of ``run`` after 3 warm-up calls, CUDA
+    events on the current stream."""
+    for _ in range(3):
+        run()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return sum(e0.elapsed_time(e1) for e0, e1 in ev) / K
+
+
 def run_variants(torch, la, workloads, K, hbm_peak, seed):
     """The rule variants that run on the same kernels, at the prefill benchmark
     shape (B=2, H=16, T=8192, d=128): DeltaNet (gated delta rule, alpha = 1),
-    RetNet (GLA, one constant decay per head), Lightning (GLA, g = 1); and GLA /
-    gated-delta prefill of 32 packed variable-length sequences.  Each is timed K
+    RetNet (GLA, one constant decay per head), Lightning (GLA, g = 1); KDA
+    prefill and decode; and GLA / gated-delta prefill of 32 packed
+    variable-length sequences.  Each is timed K
     times with CUDA events, after 3 warm-up calls."""
     spec = {"deltanet_prefill": ("gdn", dict(gdn_alpha="ones")),
             "retnet_prefill": ("gla", dict(gla_gate="retnet")),
@@ -420,6 +437,31 @@ def run_variants(torch, la, workloads, K, hbm_peak, seed):
         res[name] = {"ms": round(ms, 4), "tokens_per_s": round(w["tokens"] / (ms / 1e3)),
                      "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4)}
         del a, o, S
+    # KDA (per-channel retention; recurrent kernel): prefill at the benchmark
+    # shape and one decode step on the [256,16,128,128] fp32 state
+    p = workloads.make_problem("kda", 2, 8192, 16, 128, 128, seed=seed)
+    a = [t.cuda() for t in (p.q, p.k, p.v, p.g, p.beta)]
+    o = torch.empty(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
+    S = torch.empty(2, 16, 128, 128, device="cuda")
+    Kk = max(2, min(K, 5))
+    ms = _time_calls(torch, lambda: la.fwd("kda", *a, o=o, S_out=S), Kk)
+    la.check_device()
+    w = prefill_bytes("gla", 2, 8192, 16, 128, 128) + 2 * 8192 * 16 * 4   # gla's bytes + beta
+    res["kda_prefill"] = {"ms": round(ms, 4), "tokens_per_s": round(2 * 8192 / (ms / 1e3)),
+                          "gbs": round(w / (ms / 1e3) / 1e9, 1), "hbm_frac": round(w / (ms / 1e3) / 1e9 / hbm_peak, 4),
+                          "kernel": "recurrent (CUDA cores; no chunked KDA kernel)", "timed_calls": Kk}
+    del a, o, S
+    Sd = workloads.decode_state(seed=seed).cuda()
+    pd = workloads.make_problem("kda", 256, 1, 16, 128, 128, seed=seed)
+    qd, kd, vd, gd = (x[:, 0].contiguous().cuda() for x in (pd.q, pd.k, pd.v, pd.g))
+    bd = pd.beta[:, 0].contiguous().cuda()
+    od = torch.empty(256, 16, 128, dtype=torch.bfloat16, device="cuda")
+    ms = _time_calls(torch, lambda: la.step("kda", qd, kd, vd, Sd, g=gd, beta=bd, o=od), K)
+    la.check_device()
+    wd = decode_bytes("gla", 256, 16, 128, 128) + 256 * 16 * 4   # gla's bytes + beta
+    res["kda_decode"] = {"ms": round(ms, 4), "gbs": round(wd / (ms / 1e3) / 1e9, 1),
+                         "hbm_frac": round(wd / (ms / 1e3) / 1e9 / hbm_peak, 4)}
+    del Sd
     # packed variable-length prefill: 32 sequences, lengths uniform in [1, 8192]
     # (seeded), H=16, d=128, on one token axis
     import numpy as np

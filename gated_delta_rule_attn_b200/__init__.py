@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libla_b200.so")
 ABI_VERSION = 2   # LA_ABI_VERSION of include/la.h that these struct layouts follow
 
-RULES = {"elu": 0, "gla": 1, "gdn": 2}
+RULES = {"elu": 0, "gla": 1, "gdn": 2, "kda": 3}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_ERR_ALIGNMENT",
           4: "LA_ERR_CUDA", 5: "LA_ERR_TIMEOUT", 6: "LA_ERR_RANGE", 7: "LA_ERR_INTERNAL",

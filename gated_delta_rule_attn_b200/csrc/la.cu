@@ -3,7 +3,7 @@
 //
 // Kernel selection for la_fwd:
 //   bf16, dk = 128           -> chunked tensor-core kernel (chunk_tc.cuh)
-//   fp32, or bf16 with dk < 128 -> per-token recurrent kernel (recurrent.cuh)
+//   fp32, or bf16 with dk < 128, or KDA -> per-token recurrent kernel (recurrent.cuh)
 // la_step always uses the recurrent kernel with T = 1 and the state in place.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -45,8 +45,8 @@ struct Shape {
 };
 
 la_status validate_common(la_rule rule, la_dtype dtype, const Shape &s) {
-    if (rule != LA_RULE_ELU && rule != LA_RULE_GLA && rule != LA_RULE_GDN)
-        return fail(LA_ERR_INVALID_ARG, "rule must be LA_RULE_ELU, LA_RULE_GLA or LA_RULE_GDN");
+    if (rule != LA_RULE_ELU && rule != LA_RULE_GLA && rule != LA_RULE_GDN && rule != LA_RULE_KDA)
+        return fail(LA_ERR_INVALID_ARG, "rule must be LA_RULE_ELU, LA_RULE_GLA, LA_RULE_GDN or LA_RULE_KDA");
     if (dtype != LA_F32 && dtype != LA_BF16)
         return fail(LA_ERR_INVALID_ARG, "dtype must be LA_F32 or LA_BF16");
     if (s.B < 1 || s.H < 1 || s.T < 0)
@@ -69,10 +69,12 @@ la_status validate_gates(la_rule rule, const float *g, const float *beta, const 
     } else {
         if (z0 || z1) return fail(LA_ERR_INVALID_ARG, "z0/z_out (and step z) are ELU-only");
         if (need && !g)
-            return fail(LA_ERR_INVALID_ARG, rule == LA_RULE_GLA ? "GLA needs the gate g"
-                                                                : "GDN needs alpha (g)");
+            return fail(LA_ERR_INVALID_ARG, rule == LA_RULE_GLA   ? "GLA needs the gate g"
+                                            : rule == LA_RULE_KDA ? "KDA needs alpha (g)"
+                                                                  : "GDN needs alpha (g)");
         if (rule == LA_RULE_GLA && beta) return fail(LA_ERR_INVALID_ARG, "GLA takes no beta");
-        if (need && rule == LA_RULE_GDN && !beta) return fail(LA_ERR_INVALID_ARG, "GDN needs beta");
+        if (need && (rule == LA_RULE_GDN || rule == LA_RULE_KDA) && !beta)
+            return fail(LA_ERR_INVALID_ARG, rule == LA_RULE_KDA ? "KDA needs beta" : "GDN needs beta");
     }
     return LA_OK;
 }
@@ -121,6 +123,7 @@ la_status launch_recurrent(la_rule rule, const la::RecurrentParams &p, int64_t d
     switch (rule) {
         case LA_RULE_ELU: return launch_rec_dk<la::kRuleELU>(p, dk, dv, dt, st);
         case LA_RULE_GLA: return launch_rec_dk<la::kRuleGLA>(p, dk, dv, dt, st);
+        case LA_RULE_KDA: return launch_rec_dk<la::kRuleKDA>(p, dk, dv, dt, st);
         default: return launch_rec_dk<la::kRuleGDN>(p, dk, dv, dt, st);
     }
 }
@@ -179,7 +182,10 @@ cudaError_t allow_smem(const void *kernel, int bytes) {
 
 namespace {
 
-bool uses_chunk_kernels(const la_fwd_args &a) { return a.dtype == LA_BF16 && a.dk == 128 && a.T > 0; }
+// KDA has no chunked kernel yet: every KDA prefill runs on the recurrent kernel.
+bool uses_chunk_kernels(const la_fwd_args &a) {
+    return a.dtype == LA_BF16 && a.dk == 128 && a.T > 0 && a.rule != LA_RULE_KDA;
+}
 
 la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
     const Shape s{a.B, a.T, a.H, a.dk, a.dv};
@@ -382,7 +388,7 @@ static void staging_layout(const la_fwd_args *a, StagingLayout *L) {
     const size_t es = elem_size(a->dtype);
     const size_t tok = (size_t)(a->B * a->T * a->H);
     size_t gb = 0;
-    if (a->g) gb = tok * (a->rule == LA_RULE_GLA ? (size_t)a->dk : 1) * 4;
+    if (a->g) gb = tok * (a->rule == LA_RULE_GLA || a->rule == LA_RULE_KDA ? (size_t)a->dk : 1) * 4;
     const size_t sb = (size_t)(a->B * a->H * a->dk * a->dv) * 4;
     const size_t zb = (size_t)(a->B * a->H * a->dk) * 4;
     const size_t wb = uses_chunk_kernels(*a)

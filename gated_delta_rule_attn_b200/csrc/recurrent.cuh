@@ -11,6 +11,9 @@
 //          S = alpha S + beta k u^T  (= alpha (I - beta k k^T) S + beta k v^T,
 //          page "线性注意力与 SSM", GDN box, dk x dv orientation),
 //          o = S^T q = alpha p + beta (q.k) u.
+//   KDA    Sbar = Diag(alpha) S (alpha per key channel), r = Sbar^T k,
+//          p = Sbar^T q, u = v - r, S = Sbar + beta k u^T, o = p + beta (q.k) u
+//          (page "状态空间与线性注意力", section KDA：逐通道遗忘与误差写入).
 //
 // Used for the decode step (T = 1, state in place: one streaming pass over S
 // with 128-bit loads and stores, warp-shuffle dot products and a cross-warp
@@ -27,7 +30,7 @@
 
 namespace la {
 
-enum : int { kRuleELU = 0, kRuleGLA = 1, kRuleGDN = 2 };
+enum : int { kRuleELU = 0, kRuleGLA = 1, kRuleGDN = 2, kRuleKDA = 3 };
 
 struct RecurrentParams {
     int64_t B, T, H;
@@ -101,21 +104,28 @@ __global__ void __launch_bounds__(256, 2) recurrent_kernel(const RecurrentParams
             }
             s_q[tid] = qx;
             s_k[tid] = kx;
-            if (RULE == kRuleGLA) s_g[tid] = p.g[row * DK + tid];
+            if (RULE == kRuleGLA || RULE == kRuleKDA) s_g[tid] = p.g[row * DK + tid];
         }
         if (tid < DV) s_v[tid] = to_f32(v[row * DV + tid]);
         if (RULE == kRuleGDN && tid == 0) {
             s_scal[0] = p.g[row];
             s_scal[1] = p.beta[row];
         }
+        if (RULE == kRuleKDA && tid == 0) {
+            s_scal[0] = 1.f;   // the decay is per key row (s_g), applied below
+            s_scal[1] = p.beta[row];
+        }
         __syncthreads();
 
-        if constexpr (RULE == kRuleGDN) {
+        if constexpr (RULE == kRuleGDN || RULE == kRuleKDA) {
             // r = S^T k and p = S^T q over this thread's rows, then across rows.
+            // KDA reads the decayed state Sbar = Diag(alpha) S: r = S^T (alpha o k),
+            // p = S^T (alpha o q) (one pass, no decayed copy).
             float4 pr = make_float4(0.f, 0.f, 0.f, 0.f), pp = pr;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                const float kd = s_k[rg * RPT + r], qd = s_q[rg * RPT + r];
+                const float ad = RULE == kRuleKDA ? s_g[rg * RPT + r] : 1.f;
+                const float kd = ad * s_k[rg * RPT + r], qd = ad * s_q[rg * RPT + r];
                 pr.x = fmaf(kd, s[r].x, pr.x); pr.y = fmaf(kd, s[r].y, pr.y);
                 pr.z = fmaf(kd, s[r].z, pr.z); pr.w = fmaf(kd, s[r].w, pr.w);
                 pp.x = fmaf(qd, s[r].x, pp.x); pp.y = fmaf(qd, s[r].y, pp.y);
@@ -155,10 +165,11 @@ __global__ void __launch_bounds__(256, 2) recurrent_kernel(const RecurrentParams
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const float bk = be * s_k[rg * RPT + r];
-                s[r].x = fmaf(al, s[r].x, bk * u[0]);
-                s[r].y = fmaf(al, s[r].y, bk * u[1]);
-                s[r].z = fmaf(al, s[r].z, bk * u[2]);
-                s[r].w = fmaf(al, s[r].w, bk * u[3]);
+                const float ar = RULE == kRuleKDA ? s_g[rg * RPT + r] : al;   // decay of row d
+                s[r].x = fmaf(ar, s[r].x, bk * u[0]);
+                s[r].y = fmaf(ar, s[r].y, bk * u[1]);
+                s[r].z = fmaf(ar, s[r].z, bk * u[2]);
+                s[r].w = fmaf(ar, s[r].w, bk * u[3]);
             }
             if (tid < DV) {
                 const float uj = s_v[tid] - al * s_vec[0][tid];

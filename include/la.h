@@ -71,7 +71,18 @@ typedef enum {
     LA_ERR_WORKSPACE = 8      /* workspace missing or smaller than la_fwd_workspace_size() */
 } la_status;
 
-typedef enum { LA_RULE_ELU = 0, LA_RULE_GLA = 1, LA_RULE_GDN = 2 } la_rule;
+/*
+ * Update rules (S is dk x dv; every output is read after its token's update):
+ *   ELU  normalised ELU+1 linear attention ("Linear / RNN 路线", §2.1)
+ *   GLA  S_t = Diag(g_t) S_{t-1} + k_t v_t^T ("Linear / RNN 路线", §2.2)
+ *   GDN  S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *        ("线性注意力与 SSM", GDN box, in the dk x dv orientation)
+ *   KDA  S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *        alpha_t per key channel ("状态空间与线性注意力", KDA：逐通道遗忘与误差写入).
+ *        KDA runs on the per-token recurrent kernel (CUDA cores) for every
+ *        dtype and size; it has no chunked tensor-core kernel yet.
+ */
+typedef enum { LA_RULE_ELU = 0, LA_RULE_GLA = 1, LA_RULE_GDN = 2, LA_RULE_KDA = 3 } la_rule;
 
 /* Element type of q, k, v and o.  Gates and the state are always fp32. */
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
@@ -81,8 +92,8 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *   q, k   [B,T,H,dk] of `dtype`
  *   v      [B,T,H,dv] of `dtype`
  *   g      GLA: gate [B,T,H,dk], every entry in (0,1];  GDN: alpha [B,T,H] in (0,1];
- *          ELU: must be NULL
- *   beta   GDN: [B,T,H] in [0,1];  others: NULL
+ *          KDA: alpha [B,T,H,dk] in (0,1] (per key channel);  ELU: must be NULL
+ *   beta   GDN, KDA: [B,T,H] in [0,1];  others: NULL
  *   S0     [B,H,dk,dv] initial state, or NULL for zeros
  *   z0     ELU: [B,H,dk] initial normaliser, or NULL for zeros; others: NULL
  *   eps    ELU: added to the denominator after the dot product; ignored otherwise
@@ -142,7 +153,8 @@ typedef struct la_fwd_args {
 /*
  * Decode arguments (one token per sequence, N = batch).  Device pointers.
  *   q, k [N,H,dk]; v, o [N,H,dv] of `dtype`
- *   g    GLA [N,H,dk] / GDN alpha [N,H] / ELU NULL;  beta GDN [N,H] / NULL
+ *   g    GLA [N,H,dk] / GDN alpha [N,H] / KDA alpha [N,H,dk] / ELU NULL;
+ *        beta GDN, KDA [N,H] / NULL
  *   S    [N,H,dk,dv] fp32, read and overwritten with the updated state
  *   z    ELU [N,H,dk] fp32, read and overwritten; NULL otherwise
  * The output is read from the state after this token's update.
