@@ -252,6 +252,27 @@ def leg_work(name):
                 flops=2.0 * 2 * 128 * 128 * 256 * 16)
 
 
+# ---------------------------------------------------------------------------
+# Multi-rank plumbing (one process per GPU; no collective on the data path)
+# ---------------------------------------------------------------------------
+
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum over all ranks of this rank's device times (ms): the
+    job takes as long as its slowest rank.  Identity without a process group."""
+    import torch
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, ms: float) -> float:
+    """Whole-job throughput under weak scaling: every rank processes its own
+    tokens_per_rank in the (max over ranks) time ms."""
+    return world * tokens_per_rank / (ms / 1e3)
+
+
 def run_profile_leg(args):
     """One leg only, `--reps` times with no timing: a small, fixed launch
     sequence for ncu captures (3 warm-up calls, then the reps)."""
@@ -319,11 +340,9 @@ def run_gpu(args):
     la.check_device()
 
     # max over ranks
-    if world > 1:
-        t = torch.tensor([total_ms] + [leg_ms[n] for n in legs.names], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t[0])
-        leg_ms = {n: float(t[i + 1]) for i, n in enumerate(legs.names)}
+    red = max_over_ranks(dist, [total_ms] + [leg_ms[n] for n in legs.names], "cuda")
+    total_ms = red[0]
+    leg_ms = {n: red[i + 1] for i, n in enumerate(legs.names)}
 
     hbm_peak, tc_peak, peak_kind = load_peaks()
     traffic = load_traffic()
@@ -339,7 +358,7 @@ def run_gpu(args):
     pre = ("gla_prefill", "gdn_prefill")
     pre_ms = sum(leg_ms[n] for n in pre)
     tokens = sum(leg_work(n)["tokens"] for n in pre)
-    value = world * tokens / (pre_ms / 1e3)
+    value = job_tokens_per_s(world, tokens, pre_ms)
     # roofline of the dominant kernel (longest leg)
     dom = max(legs.names, key=lambda n: leg_ms[n])
     w = leg_work(dom)
@@ -524,9 +543,10 @@ def run_e2e(torch, la, legs, steps, world):
         step()
     b.record(s)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
+    import torch.distributed as dist
+    ms = max_over_ranks(dist, [a.elapsed_time(b) / steps], "cuda")[0]
     tokens = 2 * 2 * 8192
-    return {"value": round(world * tokens / (ms / 1e3)), "unit": "tokens/s",
+    return {"value": round(job_tokens_per_s(world, tokens, ms)), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
             "ms_per_step": round(ms, 3), "api": "la_fwd_host (C ABI, pinned host buffers)"}
 
