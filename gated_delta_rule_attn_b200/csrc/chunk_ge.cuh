@@ -1,7 +1,12 @@
 // chunk_ge.cuh — GLA and normalized ELU+1 chunked prefill, warp-specialised and
 // software-pipelined across chunks.
 //
-// One CTA per (batch, head, 32-column value slab), 17 warps:
+// One CTA per (batch, head, value slab), 17 warps.  The slab is DVS = 32 value
+// columns (GLA) or 64 (ELU+1 when dv allows): a tcgen05 MMA costs about the same
+// issue time at N = 32 and N = 64, and the feature-map work per chunk does not
+// depend on the slab, so 64 columns per CTA halve both per value column (the
+// freed CTAs go to more sequence segments).  With DVS = 64 two accumulators fit
+// in TMEM instead of three.
 //   warps 0-7    prep: the feature map / gate scaling of q and k on CUDA cores.
 //                Thread (pr, qt) owns key dims 2pr, 2pr+1 of tokens 16qt..16qt+15
 //                (a warp covers a full 128-byte row per access, conflict-free).
@@ -38,19 +43,24 @@
 namespace la {
 namespace ck {
 
-template <int RULE>
+template <int RULE, int DVS_>
 struct GE {
     static constexpr bool kGLA = (RULE == kRuleGLA);
-    static constexpr int NSTG = kGLA ? 3 : 4;
+    static constexpr int DVS = DVS_;                  // value columns per CTA: 32 or 64
+    static constexpr int NSTG = (kGLA || DVS == 64) ? 3 : 4;
     static constexpr int NTHREADS = 544;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t C_ACC = 0;     // ACC[j] at 128 j: P (0-63), O (64-95), ELU den (96)
-    static constexpr uint32_t C_DS = 384;    // DS[b] at 384 + 32 b (M=128)
-    static constexpr int KR = kGLA ? 96 : 104;   // K tile rows: K' (0-63), S^T (64-95), ELU z^T (96), zeros
+    // TMEM: NACC accumulators ACC[j] at ACCS j: P (0-63), O (64..64+DVS-1),
+    // ELU den (64+DVS); then DS[b] at C_DS + DVS b (M=128)
+    static constexpr int NACC = DVS == 64 ? 2 : 3;
+    static constexpr uint32_t ACCS = DVS == 64 ? 160 : 128;
+    static constexpr uint32_t C_ACC = 0;
+    static constexpr uint32_t C_DS = NACC * ACCS;
+    static constexpr int KR = 64 + DVS + (kGLA ? 0 : 8);   // K tile rows: K', S^T, ELU z^T, zeros
     static constexpr uint32_t K_ACS = KR * 128;                // bytes per atom column of the K tile
     static constexpr uint32_t Q_BYTES = C * 128 * KA;           // [atom col][64 rows]
     static constexpr uint32_t K_BYTES = K_ACS * KA;
-    static constexpr uint32_t V_BYTES = C * DVT * 2;            // 64-byte swizzled [64][32]
+    static constexpr uint32_t V_BYTES = C * DVS * 2;            // [64][DVS], 64- or 128-byte swizzle
     static constexpr uint32_t STG_BYTES = Q_BYTES + K_BYTES;
     static constexpr int NV = 4;                                // V ring slots
     static constexpr uint32_t G_BYTES = C * DK * 4;             // GLA gate tile, fp32 [64][128]
@@ -86,10 +96,11 @@ __device__ __forceinline__ bool aborted(const GECtl *ctl) {
     return __any_sync(0xffffffffu, *reinterpret_cast<const volatile int *>(&ctl->abort) != 0);
 }
 
-template <int RULE>
+template <int RULE, int DVS>
 __global__ void __launch_bounds__(544, 1)
 chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
-    using L = GE<RULE>;
+    using L = GE<RULE, DVS>;
+    constexpr int NACC = L::NACC;
     constexpr bool kGLA = L::kGLA;
     constexpr int NSTG = L::NSTG;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -100,7 +111,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3;
-    const int nslab = (int)(p.dv / DVT);
+    const int nslab = (int)(p.dv / DVS);
     const int dvt = (int)(blockIdx.x % nslab);
     const int seg = (int)((blockIdx.x / nslab) % p.nseg);
     const int64_t bh = blockIdx.x / nslab / p.nseg;
@@ -293,7 +304,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         auto load_v = [&](int c) {
             const int j = c % L::NV;
             mbar_arrive_expect_tx(&ctl->vfull[j], L::V_BYTES);
-            tma_load_4d(tiles + L::VR + (uint32_t)j * L::V_BYTES, &maps.v, &ctl->vfull[j], dvt * DVT, (int)h,
+            tma_load_4d(tiles + L::VR + (uint32_t)j * L::V_BYTES, &maps.v, &ctl->vfull[j], dvt * DVS, (int)h,
                         sq.t0 + (cbase + c) * C, sq.b0);
             issued_v = c;
         };
@@ -302,12 +313,12 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             for (int c = 0; c < L::NV && c < nchunks; ++c) load_v(c);
         }
         for (int c = 0; c < nchunks; ++c) {
-            const int bb = c & 1, j3 = c % 3;
-            const uint32_t acc = L::C_ACC + 128u * (uint32_t)j3;
+            const int bb = c & 1, j3 = c % NACC;
+            const uint32_t acc = L::C_ACC + L::ACCS * (uint32_t)j3;
             const int64_t t0 = (int64_t)(cbase + c) * C;   // position in the sequence
             const int nvalid = (int)min((int64_t)C, sq.len - t0);
             if (aborted(ctl)) break;
-            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->mP[j3], (uint32_t)(c / 3) & 1u))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->mP[j3], (uint32_t)(c / NACC) & 1u))) {
                 ctl->abort = 1;
                 break;
             }
@@ -319,7 +330,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                 float x[32];
                 tmem_ld16x2_32<32>(tq + acc, x);
                 float dI[16];
-                if (!kGLA) tmem_ld16(tq + acc + 96, dI);
+                if (!kGLA) tmem_ld16(tq + acc + 64 + DVS, dI);
                 tmem_wait_ld();
                 float rs = 0.f;
 #pragma unroll
@@ -347,25 +358,27 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(&ctl->pA[bb]);
-            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->m3[j3], (uint32_t)(c / 3) & 1u))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->m3[j3], (uint32_t)(c / NACC) & 1u))) {
                 ctl->abort = 1;
                 break;
             }
             tc_fence_after_sync();
-            {
-                float o[16];
-                tmem_ld16x2_16<16>(tq + acc + 64, o);
+            {   // row tr, columns (DVS/2) hf .. of the slab
+                constexpr int OH = DVS / 2;
+                float o[OH];
+                if constexpr (DVS == 64) tmem_ld16x2_32<32>(tq + acc + 64, o);
+                else tmem_ld16x2_16<16>(tq + acc + 64, o);
                 tmem_wait_ld();
                 if (tr < nvalid) {
                     if (!kGLA) {
                         const float inv = 1.f / den;
 #pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) o[jj] *= inv;
+                        for (int jj = 0; jj < OH; ++jj) o[jj] *= inv;
                     }
                     __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
-                                         ((sq.row0 + t0 + tr) * p.H + h) * p.dv + dvt * DVT + 16 * hf;
+                                         ((sq.row0 + t0 + tr) * p.H + h) * p.dv + dvt * DVS + OH * hf;
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
+                    for (int cc = 0; cc < OH / 8; ++cc) {
                         uint4 u;
                         u.x = pack_bf16x2(o[8 * cc + 0], o[8 * cc + 1]);
                         u.y = pack_bf16x2(o[8 * cc + 2], o[8 * cc + 3]);
@@ -389,12 +402,12 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
     } else if (warp < 16) {
         // ------------------------------------------------------------------ group B
         const int d = 32 * quad + lane;             // state row (key dim)
-        float S[DVT];
+        float S[DVS];
         float z = 0.f;
         {
-            const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVT) : nullptr;
+            const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVS) : nullptr;
 #pragma unroll
-            for (int jj = 0; jj < DVT; jj += 4) {
+            for (int jj = 0; jj < DVS; jj += 4) {
                 float4 x = src ? *reinterpret_cast<const float4 *>(src + jj) : make_float4(0, 0, 0, 0);
                 S[jj] = x.x; S[jj + 1] = x.y; S[jj + 2] = x.z; S[jj + 3] = x.w;
             }
@@ -403,9 +416,9 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             const int64_t blk = (int64_t)DK * p.dv + DK;
             for (int i = 0; i < seg * p.nparts; ++i) {
                 const float *a = p.agg + (bh * (p.nseg - 1) * p.nparts + i) * blk;
-                const float *row = a + (int64_t)d * p.dv + dvt * DVT;
+                const float *row = a + (int64_t)d * p.dv + dvt * DVS;
 #pragma unroll
-                for (int jj = 0; jj < DVT; jj += 4) {
+                for (int jj = 0; jj < DVS; jj += 4) {
                     const float4 x = *reinterpret_cast<const float4 *>(row + jj);
                     S[jj] += x.x; S[jj + 1] += x.y; S[jj + 2] += x.z; S[jj + 3] += x.w;
                 }
@@ -417,14 +430,14 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             uint8_t *ka = tiles + L::STG + (uint32_t)s * L::STG_BYTES + L::Q_BYTES + (d >> 6) * L::K_ACS;
             const int dc = d & 63;
 #pragma unroll
-            for (int jj = 0; jj < DVT; ++jj) *elem(ka, 64 + jj, dc) = __float2bfloat16_rn(S[jj]);
-            if (!kGLA) *elem(ka, 96, dc) = __float2bfloat16_rn(z);
+            for (int jj = 0; jj < DVS; ++jj) *elem(ka, 64 + jj, dc) = __float2bfloat16_rn(S[jj]);
+            if (!kGLA) *elem(ka, 64 + DVS, dc) = __float2bfloat16_rn(z);
         };
         if (!kGLA) {   // rows 97..103 of every stage's K tile stay zero
             for (int s = 0; s < NSTG; ++s) {
                 uint8_t *ka = tiles + L::STG + (uint32_t)s * L::STG_BYTES + L::Q_BYTES + (d >> 6) * L::K_ACS;
 #pragma unroll
-                for (int r = 97; r < 104; ++r) *elem(ka, r, d & 63) = __float2bfloat16_rn(0.f);
+                for (int r = 64 + DVS + 1; r < L::KR; ++r) *elem(ka, r, d & 63) = __float2bfloat16_rn(0.f);
             }
         }
         write_state(0);
@@ -441,18 +454,21 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             }
             tc_fence_after_sync();
             {
-                float ds[DVT];
-                tmem_ld32(tq + L::C_DS + 32u * (uint32_t)bb, ds);
-                tmem_wait_ld();
                 const float g = ctl->gC[c & 3][d];
-                if (kGLA) {
 #pragma unroll
-                    for (int jj = 0; jj < DVT; ++jj) S[jj] = g * (S[jj] + ds[jj]);
-                } else {
+                for (int hh = 0; hh < DVS / 32; ++hh) {   // 32 columns of dS at a time
+                    float ds[32];
+                    tmem_ld32(tq + L::C_DS + (uint32_t)DVS * (uint32_t)bb + 32u * hh, ds);
+                    tmem_wait_ld();
+                    if (kGLA) {
 #pragma unroll
-                    for (int jj = 0; jj < DVT; ++jj) S[jj] += ds[jj];
-                    z += g;
+                        for (int jj = 0; jj < 32; ++jj) S[32 * hh + jj] = g * (S[32 * hh + jj] + ds[jj]);
+                    } else {
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) S[32 * hh + jj] += ds[jj];
+                    }
                 }
+                if (!kGLA) z += g;
             }
             if (c + 1 < nchunks) {
                 write_state((c + 1) % NSTG);
@@ -469,9 +485,9 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         }
         if (!ctl->abort && seg == p.nseg - 1) {
             if (p.S_out) {
-                float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVT);
+                float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVS);
 #pragma unroll
-                for (int jj = 0; jj < DVT; jj += 4)
+                for (int jj = 0; jj < DVS; jj += 4)
                     *reinterpret_cast<float4 *>(dst + jj) = make_float4(S[jj], S[jj + 1], S[jj + 2], S[jj + 3]);
             }
             if (!kGLA && p.z_out && dvt == 0) p.z_out[bh * DK + d] = z;
@@ -479,37 +495,41 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
     } else if (lane == 0) {
         // ------------------------------------------------------------------ MMA issue
         constexpr uint32_t ID1 = idesc_bf16(64, L::N1, false, false);
-        constexpr uint32_t ID2 = idesc_bf16(128, DVT, true, true);
-        constexpr uint32_t ID3 = idesc_bf16(64, DVT, false, true);
+        constexpr uint32_t ID2 = idesc_bf16(128, DVS, true, true);
+        constexpr uint32_t ID3 = idesc_bf16(64, DVS, false, true);
+        // V as the MN-major B operand: [64 tokens][DVS] with the 64-byte (DVS = 32)
+        // or 128-byte (DVS = 64) swizzle
+        auto vdesc = [&](uint32_t vb) { return DVS == 64 ? dmn128_0(vb, 8192u) : dmn64_0(vb); };
+        auto vstep = [&](uint64_t d0, int kk) { return DVS == 64 ? kstep_mn128(d0, kk) : kstep_mn64(d0, kk); };
         // MMA1(c): [P | O_inter (| den)] = Q'(c) [K'(c) ; S^T (; z^T)]^T, K = dk
         auto issue_mma1 = [&](int c) {
             const uint32_t qb = smem_u32(stg(c)), kb = qb + L::Q_BYTES;
             const uint64_t dq = dk0(qb), dkx = dk0(kb);
-            const uint32_t acc = tmem + L::C_ACC + 128u * (uint32_t)(c % 3);
+            const uint32_t acc = tmem + L::C_ACC + L::ACCS * (uint32_t)(c % NACC);
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
                 umma_bf16(acc, kstep_k(dq, C * 128, kk), kstep_k(dkx, L::K_ACS, kk), ID1, kk > 0);
-            umma_commit(&ctl->mP[c % 3]);
+            umma_commit(&ctl->mP[c % NACC]);
         };
         // MMA2(c): dS = K'(c)^T V(c), K = tokens
         auto issue_mma2 = [&](int c) {
             const uint32_t kb = smem_u32(stg(c)) + L::Q_BYTES, vb = tb + L::VR + (uint32_t)(c % L::NV) * L::V_BYTES;
-            const uint64_t du = dmn128_0(kb, L::K_ACS), dv = dmn64_0(vb);
-            const uint32_t ds = tmem + L::C_DS + 32u * (uint32_t)(c & 1);
+            const uint64_t du = dmn128_0(kb, L::K_ACS), dv = vdesc(vb);
+            const uint32_t ds = tmem + L::C_DS + (uint32_t)DVS * (uint32_t)(c & 1);
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(ds, kstep_mn128(du, kk), kstep_mn64(dv, kk), ID2, kk > 0);
+                umma_bf16(ds, kstep_mn128(du, kk), vstep(dv, kk), ID2, kk > 0);
             umma_commit(&ctl->mD[c & 1]);
         };
         // MMA3(c): O += P(c) V(c)
         auto issue_mma3 = [&](int c) {
             const uint32_t vb = tb + L::VR + (uint32_t)(c % L::NV) * L::V_BYTES;
-            const uint64_t dp = dk0(tb + L::PS + (uint32_t)(c & 1) * (C * 128)), dv = dmn64_0(vb);
-            const uint32_t acc = tmem + L::C_ACC + 128u * (uint32_t)(c % 3) + 64u;
+            const uint64_t dp = dk0(tb + L::PS + (uint32_t)(c & 1) * (C * 128)), dv = vdesc(vb);
+            const uint32_t acc = tmem + L::C_ACC + L::ACCS * (uint32_t)(c % NACC) + 64u;
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(acc, kstep_k(dp, C * 128, kk), kstep_mn64(dv, kk), ID3, 1u);
-            umma_commit(&ctl->m3[c % 3]);
+                umma_bf16(acc, kstep_k(dp, C * 128, kk), vstep(dv, kk), ID3, 1u);
+            umma_commit(&ctl->m3[c % NACC]);
         };
         auto ready = [&](bool w) {
             if (!w) ctl->abort = 1;
@@ -536,10 +556,11 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         for (int c = 0; c < nchunks && ok; ++c) {
             if (*reinterpret_cast<volatile int *>(&ctl->abort)) break;
             if (c + 1 < nchunks) {
-                // the state copy of chunk c is written (and DS[c&1] read); ACC[(c+1)%3]
-                // was released by the output epilogue of chunk c-2
+                // the state copy of chunk c is written (and DS[c&1] read); ACC[(c+1)%NACC]
+                // was released by the output epilogue of chunk c+1-NACC
                 ok = mbar_wait(&ctl->sB[c & 1], (uint32_t)(c >> 1) & 1u);
-                if (ok && c >= 2) ok = mbar_wait(&ctl->oA[(c + 1) % 3], (uint32_t)((c - 2) / 3) & 1u);
+                if (ok && c + 1 >= NACC)
+                    ok = mbar_wait(&ctl->oA[(c + 1) % NACC], (uint32_t)((c + 1 - NACC) / NACC) & 1u);
                 if (!ready(ok)) break;
                 issue_mma1(c + 1);
             }

@@ -188,12 +188,18 @@ struct SegPlan {
     int nseg = 1, nparts = 1, seg_chunks = 0;
 };
 
+// Value columns per CTA of the GLA / ELU chunked kernel: ELU+1 takes 64 when dv
+// allows (one CTA covers twice the columns for the same MMA instruction count
+// and the same feature-map work, and the freed CTAs go to more segments); GLA
+// keeps 32 (its 64-column variant would not fit the gate ring in shared memory).
+inline int ge_slab(int rule, int64_t dv) { return (rule == kRuleELU && dv % 64 == 0) ? 64 : ck::DVT; }
+
 inline SegPlan seg_plan(int rule, int64_t B, int64_t T, int64_t H, int64_t dv) {
     SegPlan sp;
     const int64_t nch = (T + ck::C - 1) / ck::C;
     sp.seg_chunks = (int)nch;
     if (rule != kRuleELU || nch < 16 || dv % ck::DVT != 0) return sp;
-    const int64_t sms = sm_count(), ctas = B * H * (dv / ck::DVT);
+    const int64_t sms = sm_count(), ctas = B * H * (dv / ge_slab(rule, dv));
     const int64_t nseg = std::min<int64_t>(sms / ctas, nch / 8);
     if (nseg < 2) return sp;
     sp.seg_chunks = (int)((nch + nseg - 1) / nseg);
@@ -243,14 +249,14 @@ inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, i
 }
 
 // GLA / ELU: one CTA per (batch, head, 32-column value slab).
-template <int RULE>
+template <int RULE, int DVS>
 cudaError_t launch_ge(const ck::Maps &m, const ChunkParams &p, cudaStream_t st) {
-    using L = ck::GE<RULE>;
+    using L = ck::GE<RULE, DVS>;
     const int smem = (int)((sizeof(ck::GECtl) + 1023) / 1024 * 1024) + 1024 + (int)L::END;
-    cudaError_t e = allow_smem((const void *)ck::chunk_ge_kernel<RULE>, smem);
+    cudaError_t e = allow_smem((const void *)ck::chunk_ge_kernel<RULE, DVS>, smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)(p.B * p.H * (p.dv / ck::DVT) * p.nseg);
-    ck::chunk_ge_kernel<RULE><<<grid, L::NTHREADS, smem, st>>>(m, p);
+    const unsigned grid = (unsigned)(p.B * p.H * (p.dv / DVS) * p.nseg);
+    ck::chunk_ge_kernel<RULE, DVS><<<grid, L::NTHREADS, smem, st>>>(m, p);
     return cudaGetLastError();
 }
 
@@ -341,7 +347,20 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
             q.agg = a.agg;
         }
         q.nseg = sp.nseg; q.nparts = sp.nparts; q.seg_chunks = sp.seg_chunks;
-        e = rule == kRuleGLA ? launch_ge<kRuleGLA>(m, q, st) : launch_ge<kRuleELU>(m, q, st);
+        if (rule == kRuleGLA) {
+            e = launch_ge<kRuleGLA, DVT>(m, q, st);
+        } else if (ge_slab(rule, p.dv) == 64) {
+            // 64-column V tiles with the 128-byte swizzle
+            Maps m64 = m;
+            if (!make_map_4d(&m64.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, MB, p.T, p.H, p.dv, 64, C,
+                             CU_TENSOR_MAP_SWIZZLE_128B)) {
+                *err = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
+                return 4;
+            }
+            e = launch_ge<kRuleELU, 64>(m64, q, st);
+        } else {
+            e = launch_ge<kRuleELU, DVT>(m, q, st);
+        }
     }
     if (e != cudaSuccess) {
         *err = std::string("chunk kernel launch: ") + cudaGetErrorString(e);
