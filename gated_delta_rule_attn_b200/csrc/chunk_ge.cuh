@@ -456,16 +456,16 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             {
                 const float g = ctl->gC[c & 3][d];
 #pragma unroll
-                for (int hh = 0; hh < DVS / 32; ++hh) {   // 32 columns of dS at a time
-                    float ds[32];
-                    tmem_ld32(tq + L::C_DS + (uint32_t)DVS * (uint32_t)bb + 32u * hh, ds);
+                for (int hh = 0; hh < DVS / 16; ++hh) {   // 16 columns of dS at a time
+                    float ds[16];
+                    tmem_ld16(tq + L::C_DS + (uint32_t)DVS * (uint32_t)bb + 16u * hh, ds);
                     tmem_wait_ld();
                     if (kGLA) {
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) S[32 * hh + jj] = g * (S[32 * hh + jj] + ds[jj]);
+                        for (int jj = 0; jj < 16; ++jj) S[16 * hh + jj] = g * (S[16 * hh + jj] + ds[jj]);
                     } else {
 #pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) S[32 * hh + jj] += ds[jj];
+                        for (int jj = 0; jj < 16; ++jj) S[16 * hh + jj] += ds[jj];
                     }
                 }
                 if (!kGLA) z += g;
