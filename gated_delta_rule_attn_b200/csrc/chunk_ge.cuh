@@ -62,14 +62,21 @@ struct GE {
     static constexpr uint32_t K_BYTES = K_ACS * KA;
     static constexpr uint32_t V_BYTES = C * DVS * 2;            // [64][DVS], 64- or 128-byte swizzle
     static constexpr uint32_t STG_BYTES = Q_BYTES + K_BYTES;
-    static constexpr int NV = 4;                                // V ring slots
+    // V ring slots and GLA gate slots: GLA with 64 columns keeps three q/k stages
+    // (the scarcer lead) by holding one gate tile, loaded as soon as the prep
+    // warps have the previous one in registers
+    static constexpr int NV = (kGLA && DVS == 64) ? 3 : 4;
+    static constexpr int NG = (kGLA && DVS == 64) ? 1 : 2;
     static constexpr uint32_t G_BYTES = C * DK * 4;             // GLA gate tile, fp32 [64][128]
     // tiles
     static constexpr uint32_t STG = 0;
     static constexpr uint32_t VR = STG + NSTG * STG_BYTES;      // V ring
-    static constexpr uint32_t GT = VR + NV * V_BYTES;           // GLA: two gate slots
-    static constexpr uint32_t PS = GT + (kGLA ? 2 * G_BYTES : 0);
+    static constexpr uint32_t GT = VR + NV * V_BYTES;           // GLA: NG gate slots
+    static constexpr uint32_t PS = GT + (kGLA ? NG * G_BYTES : 0);
     static constexpr uint32_t END = PS + 2 * C * 128;
+    // with the control block (5 KB) and the 1 KB alignment slack, within the
+    // 227 KB a CTA may use
+    static_assert(END + 6144 <= 232448, "chunk_ge_kernel tiles exceed shared memory");
     static constexpr int N1 = KR;
 };
 
@@ -171,27 +178,35 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         const int pr = lt & 63, qt = lt >> 6;
         const int a = pr >> 5;                                   // atom column
         const uint32_t cpos = (uint32_t)((pr & 31) >> 2), cin = (uint32_t)(pr & 3) << 2;
-        // GLA gate tile of chunk c into slot c & 1 (issued by prep thread 0 once
-        // every prep thread is done with the slot's previous chunk)
+        // GLA gate tile of chunk c into slot c % NG (issued by prep thread 0 once
+        // every prep thread is done with the slot's previous chunk: with two slots
+        // at the top of chunk c-1, with one as soon as chunk c-1's gates are in
+        // registers)
+        int g_issued = -1, g_used = -1;   // thread 0: last gate tiles loaded / seen landed
         auto gate_load = [&](int c) {
-            uint64_t *bar = &ctl->gfull[c & 1];
+            const int j = c % L::NG;
+            uint64_t *bar = &ctl->gfull[j];
             mbar_arrive_expect_tx(bar, L::G_BYTES);
-            tma_load_4d(tiles + L::GT + (uint32_t)(c & 1) * L::G_BYTES, &maps.g, bar, 0, (int)h,
+            tma_load_4d(tiles + L::GT + (uint32_t)j * L::G_BYTES, &maps.g, bar, 0, (int)h,
                         sq.t0 + (cbase + c) * C, sq.b0);
+            g_issued = c;
         };
         if (kGLA && leader)
-            for (int c = 0; c < 2 && c < nchunks; ++c) gate_load(c);
+            for (int c = 0; c < L::NG && c < nchunks; ++c) gate_load(c);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NSTG;
             const int nvalid = (int)min((int64_t)C, sq.len - (int64_t)(cbase + c) * C);
             if (leader) ctl->stopP = ctl->abort;
             bar_named(1, 256);
             if (ctl->stopP) break;
-            if (kGLA && leader && c >= 1 && c + 1 < nchunks) {
+            if (kGLA && L::NG == 2 && leader && c >= 1 && c + 1 < nchunks) {
                 fence_proxy_async_smem();
                 gate_load(c + 1);
             }
-            if (kGLA && !mbar_wait(&ctl->gfull[c & 1], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
+            if (kGLA) {
+                if (mbar_wait(&ctl->gfull[c % L::NG], (uint32_t)(c / L::NG) & 1u)) g_used = c;
+                else ctl->abort = 1;
+            }
             if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
             uint8_t *st = stg(c);
             uint8_t *qa = st + a * (C * 128), *ka = st + L::Q_BYTES + a * L::K_ACS;
@@ -202,7 +217,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             if constexpr (kGLA) {
                 // gamma_t = prod_{s<=t} g_s inside the chunk: local products over
                 // this thread's 16 tokens, then the product of the earlier quarters.
-                const uint8_t *G = tiles + L::GT + (uint32_t)(c & 1) * L::G_BYTES;   // fp32 [64][128]
+                const uint8_t *G = tiles + L::GT + (uint32_t)(c % L::NG) * L::G_BYTES;   // fp32 [64][128]
                 float2 gv[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -214,6 +229,10 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                 for (int i = 1; i < 16; ++i) gv[i] = __fmul2_rn(gv[i - 1], gv[i]);
                 ctl->tot[qt][pr] = gv[15];
                 bar_named(1, 256);
+                if (L::NG == 1 && leader && c + 1 < nchunks && !ctl->abort) {
+                    fence_proxy_async_smem();   // every prep thread holds chunk c's gates in registers
+                    gate_load(c + 1);
+                }
                 float2 pre = make_float2(1.f, 1.f);
                 for (int q2 = 0; q2 < qt; ++q2) pre = __fmul2_rn(pre, ctl->tot[q2][pr]);
                 if (qt == 3) {
@@ -278,6 +297,10 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->pfull[s]);
         }
+        // after an abort, let gate copies still in flight land before the CTA can exit
+        if (kGLA && leader)
+            for (int c = g_used + 1; c <= g_issued; ++c)
+                (void)mbar_wait(&ctl->gfull[c % L::NG], (uint32_t)(c / L::NG) & 1u);
     } else if (warp < 12) {
         // ------------------------------------------------------------------ group A
         const bool a0 = (tid == 256);
@@ -412,17 +435,22 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                 S[jj] = x.x; S[jj + 1] = x.y; S[jj + 2] = x.z; S[jj + 3] = x.w;
             }
             if (!kGLA && p.z0) z = p.z0[bh * DK + d];
-            // sequence-parallel ELU+1: add the contributions of the earlier segments
+            // sequence-parallel pass: fold the state through the token ranges of the
+            // earlier segments, in order (ELU+1: S += dS, z += dz; GLA: S <- D o S + dS)
             const int64_t blk = (int64_t)DK * p.dv + DK;
             for (int i = 0; i < seg * p.nparts; ++i) {
                 const float *a = p.agg + (bh * (p.nseg - 1) * p.nparts + i) * blk;
                 const float *row = a + (int64_t)d * p.dv + dvt * DVS;
+                const float dd = kGLA ? a[DK * p.dv + d] : 1.f;
 #pragma unroll
                 for (int jj = 0; jj < DVS; jj += 4) {
                     const float4 x = *reinterpret_cast<const float4 *>(row + jj);
-                    S[jj] += x.x; S[jj + 1] += x.y; S[jj + 2] += x.z; S[jj + 3] += x.w;
+                    S[jj] = fmaf(dd, S[jj], x.x);
+                    S[jj + 1] = fmaf(dd, S[jj + 1], x.y);
+                    S[jj + 2] = fmaf(dd, S[jj + 2], x.z);
+                    S[jj + 3] = fmaf(dd, S[jj + 3], x.w);
                 }
-                z += a[DK * p.dv + d];
+                if (!kGLA) z += a[DK * p.dv + d];
             }
         }
         // bf16 copy of S^T (and z^T) into rows 64.. of the K tile of stage s

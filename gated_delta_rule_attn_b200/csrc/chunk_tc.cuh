@@ -65,8 +65,8 @@ struct ChunkParams {
     float *S_out, *z_out;
     void *o;
     float eps;
-    // sequence-parallel ELU+1 (nseg > 1): segment j of every (batch, head)
-    // starts from S0 plus the partial sums in `agg` of segments < j
+    // sequence-parallel ELU+1 / GLA (nseg > 1): segment j of every (batch, head)
+    // starts from S0 folded through the range summaries in `agg` of segments < j
     int nseg = 1, nparts = 1, seg_chunks = 0;
     const float *agg = nullptr;
     // packed sequences (tensors [1,T,H,*], sequence b = tokens [cu[b], cu[b+1]));
@@ -180,25 +180,25 @@ inline int sm_count() {
     return n;
 }
 
-// Sequence parallelism for ELU+1: when the (batch, head, value slab) CTAs fill
-// only a fraction of the SMs, every sequence is cut into `nseg` segments of
-// `seg_chunks` chunks that run side by side; a first pass reduces the state
-// contributions of each segment but the last, in `nparts` pieces per segment.
+// Sequence parallelism for ELU+1 and GLA: when the (batch, head, value slab) CTAs
+// fill only a fraction of the SMs, every sequence is cut into `nseg` segments of
+// `seg_chunks` chunks that run side by side; a first pass summarises each
+// segment but the last, in `nparts` chunk ranges per segment, as the affine map
+// its tokens apply to the state (chunk_agg.cuh).
 struct SegPlan {
     int nseg = 1, nparts = 1, seg_chunks = 0;
 };
 
-// Value columns per CTA of the GLA / ELU chunked kernel: ELU+1 takes 64 when dv
-// allows (one CTA covers twice the columns for the same MMA instruction count
-// and the same feature-map work, and the freed CTAs go to more segments); GLA
-// keeps 32 (its 64-column variant would not fit the gate ring in shared memory).
-inline int ge_slab(int rule, int64_t dv) { return (rule == kRuleELU && dv % 64 == 0) ? 64 : ck::DVT; }
+// Value columns per CTA of the GLA / ELU chunked kernel: 64 when dv allows (one
+// CTA covers twice the columns for the same MMA instruction count and the same
+// feature-map or gate work, and the freed CTAs go to more segments), else 32.
+inline int ge_slab(int rule, int64_t dv) { (void)rule; return dv % 64 == 0 ? 64 : ck::DVT; }
 
 inline SegPlan seg_plan(int rule, int64_t B, int64_t T, int64_t H, int64_t dv) {
     SegPlan sp;
     const int64_t nch = (T + ck::C - 1) / ck::C;
     sp.seg_chunks = (int)nch;
-    if (rule != kRuleELU || nch < 16 || dv % ck::DVT != 0) return sp;
+    if ((rule != kRuleELU && rule != kRuleGLA) || nch < 16 || dv % ck::DVT != 0) return sp;
     const int64_t sms = sm_count(), ctas = B * H * (dv / ge_slab(rule, dv));
     const int64_t nseg = std::min<int64_t>(sms / ctas, nch / 8);
     if (nseg < 2) return sp;
@@ -233,10 +233,9 @@ inline int resident_per_sm(const void *kernel, int threads, int dyn_smem, int tm
 
 // Device workspace the chunked path needs: the gated delta rule keeps the
 // per-chunk T = (I + A)^-1 operand images (8 KB per (batch, head, chunk));
-// sequence-parallel ELU+1 the partial state sums of its first pass; GLA needs
-// none.
+// sequence-parallel ELU+1 and GLA the range summaries of their first pass.
 // `packed`: the sequences are packed on one token axis with lengths up to
-// max_seqlen (no sequence-parallel ELU+1 then).
+// max_seqlen (no sequence-parallel pass then).
 inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv,
                                     bool packed = false, int64_t max_seqlen = 0) {
     if (T <= 0) return 0;
@@ -260,16 +259,21 @@ cudaError_t launch_ge(const ck::Maps &m, const ChunkParams &p, cudaStream_t st) 
     return cudaGetLastError();
 }
 
-// First pass of sequence-parallel ELU+1.
-template <int DV>
+// First pass of sequence-parallel ELU+1 / GLA.
+template <int RULE, int DV>
 cudaError_t launch_agg(const ck::Maps &m, const AggParams &a, cudaStream_t st) {
-    using L = ck::AG<DV>;
+    using L = ck::AG<RULE, DV>;
     const int smem = (int)((sizeof(ck::AGCtl) + 1023) / 1024 * 1024) + 1024 + (int)L::END;
-    cudaError_t e = allow_smem((const void *)ck::chunk_agg_kernel<DV>, smem);
+    cudaError_t e = allow_smem((const void *)ck::chunk_agg_kernel<RULE, DV>, smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(a.B * a.H * (a.nseg - 1) * a.nparts);
-    ck::chunk_agg_kernel<DV><<<grid, 288, smem, st>>>(m, a);
+    ck::chunk_agg_kernel<RULE, DV><<<grid, 288, smem, st>>>(m, a);
     return cudaGetLastError();
+}
+template <int RULE>
+cudaError_t launch_agg_dv(const ck::Maps &m, const AggParams &a, cudaStream_t st) {
+    return a.dv == 32 ? launch_agg<RULE, 32>(m, a, st)
+         : a.dv == 64 ? launch_agg<RULE, 64>(m, a, st) : launch_agg<RULE, 128>(m, a, st);
 }
 
 inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_bytes, cudaStream_t st,
@@ -332,14 +336,14 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         if (sp.nseg > 1) {
             const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv);
             if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
-                *err = "sequence-parallel ELU+1 needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
+                *err = "sequence-parallel ELU+1 / GLA needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
                 return 8;
             }
             AggParams a{};
             a.B = p.B; a.T = p.T; a.H = p.H; a.dv = p.dv;
             a.agg = static_cast<float *>(ws);
             a.nseg = sp.nseg; a.nparts = sp.nparts; a.seg_chunks = sp.seg_chunks;
-            e = p.dv == 32 ? launch_agg<32>(m, a, st) : p.dv == 64 ? launch_agg<64>(m, a, st) : launch_agg<128>(m, a, st);
+            e = rule == kRuleGLA ? launch_agg_dv<kRuleGLA>(m, a, st) : launch_agg_dv<kRuleELU>(m, a, st);
             if (e != cudaSuccess) {
                 *err = std::string("chunk kernel launch: ") + cudaGetErrorString(e);
                 return 4;
@@ -347,9 +351,7 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
             q.agg = a.agg;
         }
         q.nseg = sp.nseg; q.nparts = sp.nparts; q.seg_chunks = sp.seg_chunks;
-        if (rule == kRuleGLA) {
-            e = launch_ge<kRuleGLA, DVT>(m, q, st);
-        } else if (ge_slab(rule, p.dv) == 64) {
+        if (ge_slab(rule, p.dv) == 64) {
             // 64-column V tiles with the 128-byte swizzle
             Maps m64 = m;
             if (!make_map_4d(&m64.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, MB, p.T, p.H, p.dv, 64, C,
@@ -357,9 +359,9 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
                 *err = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
                 return 4;
             }
-            e = launch_ge<kRuleELU, 64>(m64, q, st);
+            e = rule == kRuleGLA ? launch_ge<kRuleGLA, 64>(m64, q, st) : launch_ge<kRuleELU, 64>(m64, q, st);
         } else {
-            e = launch_ge<kRuleELU, DVT>(m, q, st);
+            e = rule == kRuleGLA ? launch_ge<kRuleGLA, DVT>(m, q, st) : launch_ge<kRuleELU, DVT>(m, q, st);
         }
     }
     if (e != cudaSuccess) {

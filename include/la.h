@@ -105,9 +105,11 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *          size is 0).  The gated delta rule on the tensor-core path (bf16,
  *          dk = 128) needs 8 KB per (batch, head, 64-token chunk): the chunk's
  *          T = (I + A)^-1 operand, written by a first kernel and read by the
- *          second within the same call.  ELU+1 over few heads and long sequences
- *          runs segment-parallel and keeps per-segment partial state sums there
- *          (dk*dv + dk floats per piece).  Calls that share
+ *          second within the same call.  ELU+1 and GLA over few heads and long
+ *          sequences run segment-parallel and keep there the summary of each
+ *          piece of every segment but the last (dk*dv + dk floats per piece: the
+ *          piece's state contribution and its normaliser sum or gate product).
+ *          Calls that share
  *          one workspace must be ordered (same stream), otherwise they race.
  *          A missing or short workspace returns LA_ERR_WORKSPACE before any launch.
  * q/k/v/o must not overlap S_out/z_out.

@@ -100,12 +100,13 @@ def test_null_args_and_workspace_query(L):
         assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
         assert n.value == 0
     assert L.la_fwd_workspace_size(ctypes.byref(args(dk=3)), ctypes.byref(n)) == 2
-    # long ELU+1 sequences over few heads run segment-parallel: the first pass
-    # keeps per-piece partial state sums (dk*dv + dk floats each).  Without a
-    # device the library plans for 148 SMs: 8 slab CTAs -> 8 segments of 8
-    # chunks, 2 pieces each.
-    assert L.la_fwd_workspace_size(ctypes.byref(args("elu", T=4096, H=2)), ctypes.byref(n)) == 0
-    assert n.value == 1 * 2 * 7 * 2 * (128 * 128 + 128) * 4
+    # long ELU+1 and GLA sequences over few heads run segment-parallel: the first
+    # pass keeps a summary per piece of every segment but the last (dk*dv + dk
+    # floats each).  Without a device the library plans for 148 SMs: 4 CTAs of
+    # 64 value columns -> 8 segments of 8 chunks, 2 pieces each.
+    for rule in ("elu", "gla"):
+        assert L.la_fwd_workspace_size(ctypes.byref(args(rule, T=4096, H=2)), ctypes.byref(n)) == 0
+        assert n.value == 1 * 2 * 7 * 2 * (128 * 128 + 128) * 4
 
 
 def test_step_validation(L):

@@ -158,6 +158,18 @@ def test_elu_sequence_parallel(la, B, H, T, dv):
     check(p, *run_gpu(la, p), TOL_BF16)
 
 
+@pytest.mark.parametrize("gate", ["softplus16", "retnet", "ones"])
+@pytest.mark.parametrize("B,H,T,dv", [(1, 2, 1500, 64), (1, 1, 4096 + 33, 32), (2, 1, 3000, 128)])
+def test_gla_sequence_parallel(la, B, H, T, dv, gate):
+    """GLA over few heads and long sequences runs segment-parallel: each segment
+    starts from S0 folded through the earlier segments' ranges, S <- D o S + dS
+    (D the range's gate product per key dim, from a first pass that walks each
+    range backwards).  With the retention gate and with g = 1 the initial state
+    and the early tokens still weigh on the last segment."""
+    p = workloads.make_problem("gla", B, T, H, 128, dv, seed=T + dv, init_state="normal", gla_gate=gate)
+    check(p, *run_gpu(la, p), TOL_BF16)
+
+
 @pytest.mark.parametrize("rule", ["elu", "gla", "gdn"])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_zero_length(la, rule, dtype):
