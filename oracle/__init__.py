@@ -12,7 +12,8 @@ upcast of the bf16/fp32 inputs) and calls the C functions.
 
 Pins: every function here is checked in ``tests/test_oracle.py`` against
 brute-force quadratic / transition-product forms, closed forms, the pages'
-worked delta-rule example and split invariance.
+worked delta-rule example and split invariance; ``head_rmsnorm`` against fixed
+points, scale invariance, a constant-row closed form and per-row independence.
 """
 from __future__ import annotations
 
@@ -39,6 +40,8 @@ def _load():
         lib.oracle_gla.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P]
         lib.oracle_gdn.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P]
         lib.oracle_kda.argtypes = [I, I, I, I, I, P, P, P, P, P, P, P, P]
+        lib.oracle_head_rmsnorm.argtypes = [I, I, P, P, ctypes.c_double, P]
+        lib.oracle_head_rmsnorm.restype = None
         for f in (lib.oracle_elu, lib.oracle_gla, lib.oracle_gdn):
             f.restype = None
         _lib = lib
@@ -132,6 +135,22 @@ def fwd(problem):
         o, S = kda_fwd(p.q, p.k, p.v, p.g, p.beta, p.S0)
         return o, S, None
     raise ValueError(p.rule)
+
+
+def head_rmsnorm(o, w=None, eps: float = 1e-6) -> np.ndarray:
+    """Head-wise RMS normalisation of an output array [..., dv] over its last
+    axis (Lightning's o_t = Norm(q_t^T S_t), "Linear / RNN 路线" §2.4; K3's
+    head-wise RMSNorm, "状态空间与线性注意力" KDA section): each row x becomes
+    w * x / sqrt(mean(x^2) + eps), w None = ones.  Returns a new fp64 array."""
+    x = _f64(o)
+    dv = x.shape[-1]
+    rows = int(np.prod(x.shape[:-1])) if x.ndim > 1 else 1
+    y = np.empty_like(x)
+    wd = _f64(w)
+    if wd is not None and wd.shape != (dv,):
+        raise ValueError("w must have shape [dv]")
+    _load().oracle_head_rmsnorm(rows, dv, _ptr(x), _ptr(wd), float(eps), _ptr(y))
+    return y
 
 
 def step(rule: str, q, k, v, S, z=None, g=None, beta=None, eps: float = 1e-6):

@@ -40,6 +40,12 @@
  *     row, Sbar = Diag(alpha_t) S_{t-1}; the residual of the decayed state's
  *     prediction is then written, S_t = Sbar + beta_t k_t (v_t - Sbar^T k_t)^T;
  *     o_t = S_t^T q_t.  alpha [B,T,H,dk], beta [B,T,H].
+ *   Output normalisation: Lightning attention reads o_t = Norm(q_t^T S_t)
+ *     with an RMSNorm at the output ("Linear / RNN 路线", §2.4); K3 applies a
+ *     head-wise RMSNorm to the recurrent output ("状态空间与线性注意力", KDA
+ *     section).  The pages name the norm without writing it out; the oracle
+ *     takes the root-mean-square normalisation of each (token, head) row over
+ *     its dv values, times an optional per-channel weight (oracle_head_rmsnorm).
  */
 #include <math.h>
 #include <stdint.h>
@@ -203,6 +209,19 @@ void oracle_kda(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
         }
         store_state(S_out, S, b, h, H, dk * dv);
         free(S);
+    }
+}
+
+/* Head-wise RMS normalisation: for each of `rows` rows x of dv values,
+ * y_j = w_j x_j / sqrt((1/dv) sum_i x_i^2 + eps), w NULL = all ones. */
+void oracle_head_rmsnorm(int64_t rows, int64_t dv, const double *x, const double *w, double eps,
+                         double *y) {
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *xr = x + r * dv;
+        double ss = 0.0;
+        for (int64_t j = 0; j < dv; ++j) ss += xr[j] * xr[j];
+        const double scale = 1.0 / sqrt(ss / (double)dv + eps);
+        for (int64_t j = 0; j < dv; ++j) y[r * dv + j] = xr[j] * scale * (w ? w[j] : 1.0);
     }
 }
 

@@ -442,3 +442,62 @@ def test_zero_length_returns_initial_state():
     o, S, _ = oracle.fwd(p)
     assert o.shape == (1, 0, 2, 4)
     assert np.array_equal(S, p.S0.double().numpy())
+
+
+# ---------------------------------------------------------------------------
+# Output RMS normalisation (Lightning's o_t = Norm(q_t^T S_t), page "Linear / RNN
+# 路线" §2.4; K3's head-wise RMSNorm of the recurrent output, page "状态空间与线性
+# 注意力", KDA section).  The pages name the norm; these pins fix what it does.
+# ---------------------------------------------------------------------------
+
+def test_rmsnorm_worked_row_by_hand():
+    """x = (3, 4, 0, 0): mean square 25/4, root 2.5, so y = (1.2, 1.6, 0, 0)."""
+    y = oracle.head_rmsnorm(np.array([3.0, 4.0, 0.0, 0.0]), eps=0.0)
+    np.testing.assert_allclose(y, [1.2, 1.6, 0.0, 0.0], rtol=0, atol=1e-15)
+
+
+def test_rmsnorm_unit_rows_are_fixed_points_and_weight_scales_channels():
+    """Rows of +-1 already have mean square 1: unchanged without a weight, and
+    multiplied channel by channel by the weight."""
+    rng = np.random.default_rng(0)
+    x = np.where(rng.random((5, 3, 64)) < 0.5, -1.0, 1.0)
+    np.testing.assert_array_equal(oracle.head_rmsnorm(x, eps=0.0), x)
+    w = rng.normal(size=64)
+    np.testing.assert_allclose(oracle.head_rmsnorm(x, w, eps=0.0), x * w, rtol=1e-15, atol=0)
+
+
+def test_rmsnorm_constant_row_closed_form():
+    """x = c * 1: every entry becomes c / sqrt(c^2 + eps)."""
+    for c, eps in ((-3.0, 0.5), (1e-3, 1e-6), (250.0, 1e-6)):
+        y = oracle.head_rmsnorm(np.full((2, 32), c), eps=eps)
+        np.testing.assert_allclose(y, c / math.sqrt(c * c + eps), rtol=1e-14)
+
+
+def test_rmsnorm_is_scale_invariant_without_eps():
+    rng = np.random.default_rng(1)
+    x = rng.normal(size=(4, 2, 128))
+    y = oracle.head_rmsnorm(x, eps=0.0)
+    for lam in (1e-3, 7.5, 1e4):
+        np.testing.assert_allclose(oracle.head_rmsnorm(lam * x, eps=0.0), y, rtol=1e-13, atol=1e-15)
+    # and every output row has mean square one
+    np.testing.assert_allclose((y * y).mean(axis=-1), 1.0, rtol=1e-13)
+
+
+def test_rmsnorm_normalises_each_row_on_its_own():
+    """Rows that are multiples of one row (per head and per token, at very
+    different scales) all normalise to the same row: the mean is taken over the
+    dv values of each row, not over heads or tokens."""
+    rng = np.random.default_rng(2)
+    base = rng.normal(size=64)
+    scales = np.array([[1.0, 10.0, 0.01], [3.0, 1e3, 0.5]])   # [tokens, heads]
+    x = scales[:, :, None] * base
+    y = oracle.head_rmsnorm(x, eps=0.0)
+    want = oracle.head_rmsnorm(base[None], eps=0.0)[0]
+    for t in range(2):
+        for h in range(3):
+            np.testing.assert_allclose(y[t, h], want, rtol=1e-13)
+
+
+def test_rmsnorm_zero_row_with_eps_stays_zero():
+    y = oracle.head_rmsnorm(np.zeros((3, 32)), w=np.arange(32.0), eps=1e-6)
+    np.testing.assert_array_equal(y, 0.0)

@@ -40,6 +40,13 @@ MUTANTS = {
     "kda_residual_sign": ("(vt[j] - pred[j])", "(vt[j] + pred[j])"),
     "kda_write_not_scaled_by_beta": ("S[d * dv + j] += be * kt[d] * (vt[j] - pred[j]);",
                                      "S[d * dv + j] += kt[d] * (vt[j] - pred[j]);"),
+    # output RMS normalisation
+    "norm_eps_outside_root": ("1.0 / sqrt(ss / (double)dv + eps)", "1.0 / (sqrt(ss / (double)dv) + eps)"),
+    "norm_sum_not_mean": ("1.0 / sqrt(ss / (double)dv + eps)", "1.0 / sqrt(ss + eps)"),
+    "norm_weight_ignored": ("xr[j] * scale * (w ? w[j] : 1.0)", "xr[j] * scale"),
+    "norm_over_all_rows": ("        double ss = 0.0;\n        for (int64_t j = 0; j < dv; ++j) ss += xr[j] * xr[j];",
+                           "        static double ss = 0.0;\n        for (int64_t j = 0; j < dv; ++j) ss += xr[j] * xr[j];"),
+    "norm_weight_per_row": ("xr[j] * scale * (w ? w[j] : 1.0)", "xr[j] * scale * (w ? w[r % dv] : 1.0)"),
 }
 
 
