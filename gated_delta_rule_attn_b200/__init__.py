@@ -16,7 +16,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libla_b200.so")
-ABI_VERSION = 2   # LA_ABI_VERSION of include/la.h that these struct layouts follow
+ABI_VERSION = 3   # LA_ABI_VERSION of include/la.h that these struct layouts follow
 
 RULES = {"elu": 0, "gla": 1, "gdn": 2, "kda": 3}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
@@ -45,7 +45,8 @@ class FwdArgs(ctypes.Structure):
                 ("z0", ctypes.c_void_p), ("eps", ctypes.c_float), ("o", ctypes.c_void_p),
                 ("S_out", ctypes.c_void_p), ("z_out", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
-                ("cu_seqlens", ctypes.c_void_p), ("max_seqlen", ctypes.c_int64)]
+                ("cu_seqlens", ctypes.c_void_p), ("max_seqlen", ctypes.c_int64),
+                ("out_norm", ctypes.c_int32), ("norm_eps", ctypes.c_float), ("norm_w", ctypes.c_void_p)]
 
 
 class StepArgs(ctypes.Structure):
@@ -54,7 +55,8 @@ class StepArgs(ctypes.Structure):
                 ("dv", ctypes.c_int64),
                 ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("g", ctypes.c_void_p), ("beta", ctypes.c_void_p), ("S", ctypes.c_void_p),
-                ("z", ctypes.c_void_p), ("eps", ctypes.c_float), ("o", ctypes.c_void_p)]
+                ("z", ctypes.c_void_p), ("eps", ctypes.c_float), ("o", ctypes.c_void_p),
+                ("out_norm", ctypes.c_int32), ("norm_eps", ctypes.c_float), ("norm_w", ctypes.c_void_p)]
 
 
 _lib = None
@@ -113,11 +115,21 @@ def _need(t, name, device=True):
         raise ValueError(f"{name} must be a CUDA tensor")
 
 
+def _set_norm(a, out_norm, norm_w, norm_eps):
+    """Output normalisation fields (la.h, ABI version 3)."""
+    a.out_norm = 1 if out_norm else 0
+    a.norm_eps = norm_eps
+    a.norm_w = norm_w.data_ptr() if norm_w is not None else None
+
+
 def make_fwd_args(rule, q, k, v, g=None, beta=None, S0=None, z0=None, eps=1e-6,
-                  o=None, S_out=None, z_out=None, cu_seqlens=None, max_seqlen=None) -> FwdArgs:
+                  o=None, S_out=None, z_out=None, cu_seqlens=None, max_seqlen=None,
+                  out_norm=False, norm_w=None, norm_eps=1e-6) -> FwdArgs:
     """Marshal tensors into la_fwd_args.  With ``cu_seqlens`` (int64 [B+1] on the
     device) the token tensors are one packed axis [1, T, H, d] and B is the
-    number of sequences; ``max_seqlen`` bounds their lengths."""
+    number of sequences; ``max_seqlen`` bounds their lengths.  ``out_norm``:
+    each (token, head) row of o is RMS-normalised over dv (weight ``norm_w``
+    fp32 [dv] or None, ``norm_eps`` > 0)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     if cu_seqlens is not None:
@@ -143,6 +155,7 @@ def make_fwd_args(rule, q, k, v, g=None, beta=None, S0=None, z0=None, eps=1e-6,
     if cu_seqlens is not None:
         a.cu_seqlens = cu_seqlens.data_ptr()
         a.max_seqlen = int(max_seqlen)
+    _set_norm(a, out_norm, norm_w, norm_eps)
     return a
 
 
@@ -162,17 +175,19 @@ def _workspace(device, stream_handle: int, nbytes: int):
 
 def fwd(rule: str, q, k, v, g=None, beta=None, S0=None, z0=None, eps: float = 1e-6,
         o=None, S_out=None, z_out=None, stream=None, want_state: bool = True, workspace=None,
-        cu_seqlens=None, max_seqlen=None):
+        cu_seqlens=None, max_seqlen=None, out_norm: bool = False, norm_w=None, norm_eps: float = 1e-6):
     """Chunked prefill: returns (o, S_out, z_out-or-None). Enqueued on the current stream.
 
     ``workspace`` (a CUDA uint8 tensor of at least ``fwd_workspace_size`` bytes)
     is allocated and cached per stream when not given.  ``cu_seqlens`` /
     ``max_seqlen``: packed variable-length sequences (see ``make_fwd_args``);
-    the states are then [number of sequences, H, dk, dv]."""
+    the states are then [number of sequences, H, dk, dv].  ``out_norm``,
+    ``norm_w``, ``norm_eps``: head-wise RMS normalisation of o (see
+    ``make_fwd_args``)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (S0, "S0"), (z0, "z0"),
-                 (cu_seqlens, "cu_seqlens")):
+                 (cu_seqlens, "cu_seqlens"), (norm_w, "norm_w")):
         _need(t, n)
     NS = B if cu_seqlens is None else cu_seqlens.numel() - 1   # sequences (state rows)
     if q.dtype != k.dtype or q.dtype != v.dtype:
@@ -183,7 +198,8 @@ def fwd(rule: str, q, k, v, g=None, beta=None, S0=None, z0=None, eps: float = 1e
         S_out = torch.empty(NS, H, dk, dv, dtype=torch.float32, device=q.device)
     if rule == "elu" and z_out is None and want_state:
         z_out = torch.empty(NS, H, dk, dtype=torch.float32, device=q.device)
-    a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, eps, o, S_out, z_out, cu_seqlens, max_seqlen)
+    a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, eps, o, S_out, z_out, cu_seqlens, max_seqlen,
+                      out_norm, norm_w, norm_eps)
     sh = _stream_handle(stream)
     n = ctypes.c_size_t()
     _check(lib().la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
@@ -202,11 +218,13 @@ def fwd_workspace_size(rule, q, k, v, g=None, beta=None, S0=None, z0=None) -> in
 
 
 def step(rule: str, q, k, v, S, z=None, g=None, beta=None, eps: float = 1e-6, o=None,
-         stream=None):
-    """Decode step: updates S (and z) in place, returns o [N,H,dv]."""
+         stream=None, out_norm: bool = False, norm_w=None, norm_eps: float = 1e-6):
+    """Decode step: updates S (and z) in place, returns o [N,H,dv] (RMS-normalised
+    per (sequence, head) over dv with ``out_norm``)."""
     N, H, dk = q.shape
     dv = v.shape[-1]
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (S, "S"), (z, "z")):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (S, "S"), (z, "z"),
+                 (norm_w, "norm_w")):
         _need(t, n)
     if o is None:
         o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
@@ -219,15 +237,17 @@ def step(rule: str, q, k, v, S, z=None, g=None, beta=None, eps: float = 1e-6, o=
                                             for t in (q, k, v, g, beta, S, z))
     a.eps = eps
     a.o = o.data_ptr()
+    _set_norm(a, out_norm, norm_w, norm_eps)
     _check(lib().la_step(ctypes.byref(a), _stream_handle(stream)))
     return o
 
 
-def host_staging_size(rule, q, k, v, g=None, beta=None, S0=None, z0=None, want_state=True) -> int:
+def host_staging_size(rule, q, k, v, g=None, beta=None, S0=None, z0=None, want_state=True,
+                      out_norm=False, norm_w=None, norm_eps=1e-6) -> int:
     """Bytes of device staging ``fwd_host`` needs for these host tensors."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
-    a = make_fwd_args(rule, q, k, v, g, beta, S0, z0)
+    a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, out_norm=out_norm, norm_w=norm_w, norm_eps=norm_eps)
     # output pointers only mark presence for the size computation
     a.o = 1
     a.S_out = 1 if want_state else None
@@ -238,14 +258,16 @@ def host_staging_size(rule, q, k, v, g=None, beta=None, S0=None, z0=None, want_s
 
 
 def fwd_host(rule: str, q, k, v, g=None, beta=None, S0=None, z0=None, eps: float = 1e-6,
-             o=None, S_out=None, z_out=None, staging=None, stream=None):
+             o=None, S_out=None, z_out=None, staging=None, stream=None,
+             out_norm: bool = False, norm_w=None, norm_eps: float = 1e-6):
     """la_fwd on host (CPU, ideally pinned) tensors through the C ABI: the library
     copies inputs into ``staging`` (a CUDA uint8 tensor), runs, copies outputs back
     and synchronises the stream.  Returns (o, S_out, z_out)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (g, "g"), (beta, "beta"), (S0, "S0"), (z0, "z0"),
-                 (o, "o"), (S_out, "S_out"), (z_out, "z_out")):
+                 (o, "o"), (S_out, "S_out"), (z_out, "z_out"), (norm_w, "norm_w")):
         _need(t, n, device=False)
-    a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, eps, o, S_out, z_out)
+    a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, eps, o, S_out, z_out,
+                      out_norm=out_norm, norm_w=norm_w, norm_eps=norm_eps)
     _check(lib().la_fwd_host(ctypes.byref(a), ctypes.c_void_p(staging.data_ptr()),
                              staging.numel(), _stream_handle(stream)))
     return o, S_out, z_out

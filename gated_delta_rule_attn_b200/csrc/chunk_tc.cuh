@@ -171,14 +171,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 
 namespace la {
 
-// Host launcher.  Returns an la_status value (0 = ok).
-inline int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-        n = 148;
-    return n;
-}
 
 // Sequence parallelism for ELU+1 and GLA: when the (batch, head, value slab) CTAs
 // fill only a fraction of the SMs, every sequence is cut into `nseg` segments of

@@ -329,4 +329,13 @@ __device__ __forceinline__ float2 elu_feature2(float2 x) {
 }
 
 
+// SMs of the current device (148 on B200; also the plan without a device).
+inline int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    return n;
+}
+
 }  // namespace la

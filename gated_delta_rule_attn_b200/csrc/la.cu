@@ -5,10 +5,13 @@
 //   bf16, dk = 128           -> chunked tensor-core kernel (chunk_tc.cuh)
 //   fp32, or bf16 with dk < 128, or KDA -> per-token recurrent kernel (recurrent.cuh)
 // la_step always uses the recurrent kernel with T = 1 and the state in place.
+// With out_norm set, a second pass normalises each (token, head) row of o
+// (out_norm.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstddef>
 #include <cstdio>
 #include <cstring>
@@ -19,6 +22,7 @@
 #include "device.cuh"
 #include "recurrent.cuh"
 #include "chunk_tc.cuh"
+#include "out_norm.cuh"
 
 namespace {
 
@@ -187,7 +191,29 @@ bool uses_chunk_kernels(const la_fwd_args &a) {
     return a.dtype == LA_BF16 && a.dk == 128 && a.T > 0 && a.rule != LA_RULE_KDA;
 }
 
-la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
+// Output normalisation arguments (ABI version 3), shared by la_fwd and la_step.
+la_status validate_norm(int32_t out_norm, float norm_eps, const float *norm_w, bool device_ptrs) {
+    if (out_norm != 0 && out_norm != 1) return fail(LA_ERR_INVALID_ARG, "out_norm must be 0 or 1");
+    if (!out_norm) return LA_OK;
+    if (!(norm_eps > 0.f) || !std::isfinite(norm_eps))
+        return fail(LA_ERR_INVALID_ARG, "out_norm needs a finite norm_eps > 0");
+    if (device_ptrs && norm_w && !aligned16(norm_w))
+        return fail(LA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
+    return LA_OK;
+}
+
+// In-place head-wise RMS normalisation of `rows` rows of dv values of o.
+la_status launch_norm(la_dtype dtype, void *o, int64_t rows, int64_t dv, const float *w, float eps,
+                      cudaStream_t st) {
+    const cudaError_t e =
+        dtype == LA_BF16
+            ? la::launch_out_rmsnorm(static_cast<__nv_bfloat16 *>(o), rows, dv, w, eps, st)
+            : la::launch_out_rmsnorm(static_cast<float *>(o), rows, dv, w, eps, st);
+    if (e != cudaSuccess) return fail(LA_ERR_CUDA, std::string("output norm launch: ") + cudaGetErrorString(e));
+    return ok();
+}
+
+la_status launch_fwd_core(const la_fwd_args &a, cudaStream_t st) {
     const Shape s{a.B, a.T, a.H, a.dk, a.dv};
     if (a.T == 0 || (a.cu_seqlens && a.max_seqlen == 0)) {   // no token in any sequence
         const size_t sb = (size_t)(s.B * s.H * s.dk * s.dv) * sizeof(float);
@@ -226,6 +252,14 @@ la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
     return launch_recurrent(a.rule, p, a.dk, a.dv, a.dtype, st);
 }
 
+la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
+    la_status r = launch_fwd_core(a, st);
+    if (r != LA_OK || !a.out_norm || a.T == 0) return r;
+    // o is [B,T,H,dv] dense or [1,T,H,dv] packed
+    const int64_t rows = (a.cu_seqlens ? a.T : a.B * a.T) * a.H;
+    return launch_norm(a.dtype, a.o, rows, a.dv, a.norm_w, a.norm_eps, st);
+}
+
 // The caller's arguments as this library's la_fwd_args: a struct from an older
 // header (ABI version 1, without the packed-sequence fields) is accepted and the
 // missing fields read as NULL / 0.
@@ -250,6 +284,8 @@ la_status validate_fwd(const la_fwd_args *a, bool device_ptrs, bool host_bufs = 
     if (a->T > 0 && (!a->q || !a->k || !a->v || !a->o))
         return fail(LA_ERR_INVALID_ARG, "q, k, v and o must be non-NULL when T > 0");
     if (!(a->eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+    r = validate_norm(a->out_norm, a->norm_eps, a->norm_w, device_ptrs);
+    if (r != LA_OK) return r;
     if (a->cu_seqlens) {
         if (host_bufs)
             return fail(LA_ERR_UNSUPPORTED, "packed sequences (cu_seqlens) need device buffers: use la_fwd");
@@ -353,10 +389,17 @@ la_status la_fwd_workspace_size(const la_fwd_args *args, size_t *bytes) {
     return ok();
 }
 
-la_status la_step(const la_step_args *a, void *stream) {
-    if (!a) return fail(LA_ERR_INVALID_ARG, "args is NULL");
-    if (a->struct_size < sizeof(la_step_args))
-        return fail(LA_ERR_INVALID_ARG, "struct_size smaller than sizeof(la_step_args)");
+la_status la_step(const la_step_args *in, void *stream) {
+    if (!in) return fail(LA_ERR_INVALID_ARG, "args is NULL");
+    // a struct from an ABI version-2 header ends at `o`: no output normalisation
+    constexpr size_t v2 = offsetof(la_step_args, out_norm);
+    if (in->struct_size < v2)
+        return fail(LA_ERR_INVALID_ARG, "struct_size smaller than the version-2 la_step_args");
+    la_step_args A;
+    memset(&A, 0, sizeof(A));
+    memcpy(&A, in, in->struct_size < sizeof(la_step_args) ? in->struct_size : sizeof(la_step_args));
+    A.struct_size = sizeof(la_step_args);
+    const la_step_args *a = &A;
     const Shape s{a->N, 1, a->H, a->dk, a->dv};
     la_status r = validate_common(a->rule, a->dtype, s);
     if (r != LA_OK) return r;
@@ -366,6 +409,8 @@ la_status la_step(const la_step_args *a, void *stream) {
         return fail(LA_ERR_INVALID_ARG, "q, k, v, o and S must be non-NULL");
     if (a->rule == LA_RULE_ELU && !a->z) return fail(LA_ERR_INVALID_ARG, "ELU decode needs z");
     if (!(a->eps >= 0.f)) return fail(LA_ERR_INVALID_ARG, "eps must be >= 0");
+    r = validate_norm(a->out_norm, a->norm_eps, a->norm_w, true);
+    if (r != LA_OK) return r;
     const void *ps[] = {a->q, a->k, a->v, a->g, a->beta, a->S, a->z, a->o};
     for (const void *p : ps)
         if (p && !aligned16(p)) return fail(LA_ERR_ALIGNMENT, "device pointers must be 16-byte aligned");
@@ -374,13 +419,17 @@ la_status la_step(const la_step_args *a, void *stream) {
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
     p.S_in = a->S; p.S_out = a->S; p.z_in = a->z; p.z_out = a->z;
     p.o = a->o; p.eps = a->eps;
-    return launch_recurrent(a->rule, p, a->dk, a->dv, a->dtype, static_cast<cudaStream_t>(stream));
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    r = launch_recurrent(a->rule, p, a->dk, a->dv, a->dtype, st);
+    if (r != LA_OK || !a->out_norm) return r;
+    return launch_norm(a->dtype, a->o, a->N * a->H, a->dv, a->norm_w, a->norm_eps, st);
 }
 
 // Host-buffer path: staging layout = each tensor at a 256-byte aligned offset.
+constexpr int kStaged = 12;
 struct StagingLayout {
-    size_t off[11];  // q k v g beta S0 z0 o S_out z_out workspace
-    size_t bytes[11];
+    size_t off[kStaged];  // q k v g beta S0 z0 o S_out z_out workspace norm_w
+    size_t bytes[kStaged];
     size_t total;
 };
 
@@ -394,11 +443,12 @@ static void staging_layout(const la_fwd_args *a, StagingLayout *L) {
     const size_t wb = uses_chunk_kernels(*a)
                           ? la::chunk_workspace_bytes((int)a->rule, a->B, a->T, a->H, a->dv)
                           : 0;
-    const size_t b[11] = {tok * a->dk * es, tok * a->dk * es, tok * a->dv * es, gb,
-                          a->beta ? tok * 4 : 0, a->S0 ? sb : 0, a->z0 ? zb : 0,
-                          tok * a->dv * es, a->S_out ? sb : 0, a->z_out ? zb : 0, wb};
+    const size_t nb = (a->out_norm && a->norm_w) ? (size_t)a->dv * 4 : 0;
+    const size_t b[kStaged] = {tok * a->dk * es, tok * a->dk * es, tok * a->dv * es, gb,
+                               a->beta ? tok * 4 : 0, a->S0 ? sb : 0, a->z0 ? zb : 0,
+                               tok * a->dv * es, a->S_out ? sb : 0, a->z_out ? zb : 0, wb, nb};
     size_t o = 0;
-    for (int i = 0; i < 11; ++i) {
+    for (int i = 0; i < kStaged; ++i) {
         L->off[i] = o;
         L->bytes[i] = b[i];
         o += (b[i] + 255) & ~(size_t)255;
@@ -433,11 +483,12 @@ la_status la_fwd_host(const la_fwd_args *h_in, void *staging, size_t staging_byt
     if (staging_bytes < L.total) return fail(LA_ERR_WORKSPACE, "staging buffer too small");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     char *base = static_cast<char *>(staging);
-    const void *src[7] = {h->q, h->k, h->v, h->g, h->beta, h->S0, h->z0};
-    void *dptr[11];
-    for (int i = 0; i < 11; ++i) dptr[i] = L.bytes[i] ? base + L.off[i] : nullptr;
-    for (int i = 0; i < 7; ++i) {
-        if (!L.bytes[i]) continue;
+    const void *src[kStaged] = {h->q, h->k, h->v, h->g, h->beta, h->S0, h->z0,
+                                nullptr, nullptr, nullptr, nullptr, h->norm_w};
+    void *dptr[kStaged];
+    for (int i = 0; i < kStaged; ++i) dptr[i] = L.bytes[i] ? base + L.off[i] : nullptr;
+    for (int i = 0; i < kStaged; ++i) {
+        if (!L.bytes[i] || !src[i]) continue;
         cudaError_t e = cudaMemcpyAsync(dptr[i], src[i], L.bytes[i], cudaMemcpyHostToDevice, st);
         if (e != cudaSuccess) return fail(LA_ERR_CUDA, std::string("H2D copy: ") + cudaGetErrorString(e));
     }
@@ -452,6 +503,7 @@ la_status la_fwd_host(const la_fwd_args *h_in, void *staging, size_t staging_byt
     d.z_out = static_cast<float *>(dptr[9]);
     d.workspace = dptr[10];
     d.workspace_bytes = L.bytes[10];
+    d.norm_w = static_cast<const float *>(dptr[11]);
     r = la_fwd(&d, stream);
     if (r != LA_OK) return r;
     void *dst[3] = {h->o, h->S_out, h->z_out};

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define LA_ABI_VERSION 2
+#define LA_ABI_VERSION 3
 
 typedef enum {
     LA_OK = 0,
@@ -131,6 +131,23 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *   [0, T], or a sequence longer than max_seqlen, are clamped to stay in bounds
  *   and reported by la_check_device as LA_ERR_INVALID_ARG.  Packed sequences
  *   are not accepted by la_fwd_host (LA_ERR_UNSUPPORTED).
+ *
+ * Output normalisation (fields appended in ABI version 3, in la_fwd_args and
+ * la_step_args; a caller built against an older header passes the older
+ * struct_size and gets none):
+ *   out_norm  0: o as above.  1: every (token, head) row of o is replaced by
+ *          its head-wise RMS normalisation, o_j <- w_j o_j / sqrt(mean_j o_j^2 +
+ *          norm_eps) over the dv values of the row: the output normalisation of
+ *          Lightning attention, o_t = Norm(q_t^T S_t) (page "Linear / RNN 路线",
+ *          §2.4, with GLA at g = 1), and the head-wise RMSNorm that K3 applies
+ *          to the recurrent output (page "状态空间与线性注意力", KDA section).
+ *          Applies to every rule.  The state and z are not affected.
+ *   norm_eps  > 0 (finite), added to the mean square before the square root.
+ *   norm_w    fp32 [dv] per-channel weight shared by the heads, or NULL (= 1);
+ *          16-byte aligned device pointer (host pointer for la_fwd_host).
+ *   The normalisation is a second pass over o on the same stream (a row spans
+ *   every value slab of the chunked kernels); it reads o as stored, so for bf16
+ *   problems it normalises the bf16-rounded output and rounds once more.
  */
 typedef struct la_fwd_args {
     uint32_t struct_size;     /* = sizeof(la_fwd_args) */
@@ -150,6 +167,9 @@ typedef struct la_fwd_args {
     size_t workspace_bytes;
     const int64_t *cu_seqlens;   /* ABI version 2 */
     int64_t max_seqlen;          /* ABI version 2 */
+    int32_t out_norm;            /* ABI version 3: output normalisation (below) */
+    float norm_eps;              /* ABI version 3 */
+    const float *norm_w;         /* ABI version 3 */
 } la_fwd_args;
 
 /*
@@ -159,7 +179,9 @@ typedef struct la_fwd_args {
  *        beta GDN, KDA [N,H] / NULL
  *   S    [N,H,dk,dv] fp32, read and overwritten with the updated state
  *   z    ELU [N,H,dk] fp32, read and overwritten; NULL otherwise
- * The output is read from the state after this token's update.
+ *   out_norm, norm_eps, norm_w  as in la_fwd_args (ABI version 3)
+ * The output is read from the state after this token's update.  A struct of
+ * ABI version 2 (struct_size up to `o`) is accepted, without normalisation.
  */
 typedef struct la_step_args {
     uint32_t struct_size;     /* = sizeof(la_step_args) */
@@ -173,6 +195,9 @@ typedef struct la_step_args {
     float *z;
     float eps;
     void *o;
+    int32_t out_norm;            /* ABI version 3: output normalisation (below) */
+    float norm_eps;              /* ABI version 3 */
+    const float *norm_w;         /* ABI version 3 */
 } la_step_args;
 
 /* Chunked prefill (see the struct above).  Asynchronous on `stream`. */

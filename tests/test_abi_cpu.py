@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.la_abi_version() == 2
+    assert L.la_abi_version() == 3
     assert L.la_status_string(0) == b"LA_OK"
     assert L.la_status_string(5) == b"LA_ERR_TIMEOUT"
     assert L.la_status_string(99) == b"LA_ERR_UNKNOWN"
@@ -192,3 +192,70 @@ def test_packed_argument_checks(L):
     assert L.la_fwd_host_staging_size(ctypes.byref(h), ctypes.byref(n)) == 2
     assert L.la_fwd_host(ctypes.byref(h), ctypes.c_void_p(FAKE), 1 << 30, None) == 2
     assert b"la_fwd" in L.la_last_error_message()
+
+
+# ---------------------------------------------------------------------------
+# Output normalisation (la_fwd_args / la_step_args fields of ABI version 3)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("kw,status,word", [
+    (dict(out_norm=2), 1, "out_norm"),
+    (dict(out_norm=1, norm_eps=0.0), 1, "norm_eps"),
+    (dict(out_norm=1, norm_eps=-1e-6), 1, "norm_eps"),
+    (dict(out_norm=1, norm_eps=float("inf")), 1, "norm_eps"),
+    (dict(out_norm=1, norm_eps=float("nan")), 1, "norm_eps"),
+    (dict(out_norm=1, norm_eps=1e-6, norm_w=FAKE + 4), 3, "aligned"),
+])
+def test_invalid_norm_arguments_rejected(L, kw, status, word):
+    r, msg = call(L, args("gla", T=8, **kw))
+    assert r == status and word in msg, msg
+
+
+def test_norm_fields_ignored_when_off_or_past_an_older_struct(L):
+    n = ctypes.c_size_t(7)
+    # out_norm = 0: norm_eps and norm_w are not looked at
+    a = args("gla", T=8, norm_eps=-5.0, norm_w=FAKE + 4)
+    assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    # a version-2 caller's struct ends before out_norm: garbage there is ignored
+    a = args("gla", T=8, out_norm=9)
+    a.struct_size = la.FwdArgs.out_norm.offset
+    assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+
+
+def step_args(**kw):
+    s = la.StepArgs()
+    s.struct_size = ctypes.sizeof(s)
+    s.rule, s.dtype, s.N, s.H, s.dk, s.dv = 2, 1, 4, 2, 128, 128
+    s.q = s.k = s.v = s.o = s.S = s.g = FAKE
+    for k, v in kw.items():
+        setattr(s, k, v)
+    return s
+
+
+def test_step_struct_versions_and_norm_checks(L):
+    # version-2 struct (ends at o): accepted, validation goes on (GDN needs beta)
+    s = step_args(out_norm=9)
+    s.struct_size = la.StepArgs.out_norm.offset
+    assert L.la_step(ctypes.byref(s), None) == 1
+    assert b"beta" in L.la_last_error_message()
+    s.struct_size = la.StepArgs.out_norm.offset - 8
+    assert L.la_step(ctypes.byref(s), None) == 1
+    assert b"struct_size" in L.la_last_error_message()
+    # full struct: the norm fields are checked
+    s = step_args(beta=FAKE, out_norm=1, norm_eps=0.0)
+    assert L.la_step(ctypes.byref(s), None) == 1
+    assert b"norm_eps" in L.la_last_error_message()
+    s = step_args(beta=FAKE, out_norm=1, norm_eps=1e-6, norm_w=FAKE + 8)
+    assert L.la_step(ctypes.byref(s), None) == 3
+
+
+def test_host_staging_holds_the_norm_weight(L):
+    a = args("gla", B=2, T=100, H=3, dk=64, dv=32, S0=FAKE, S_out=FAKE)
+    n0, n1 = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.la_fwd_host_staging_size(ctypes.byref(a), ctypes.byref(n0)) == 0
+    a.out_norm, a.norm_eps, a.norm_w = 1, 1e-6, FAKE + 4   # host pointer: no alignment rule
+    assert L.la_fwd_host_staging_size(ctypes.byref(a), ctypes.byref(n1)) == 0
+    assert n1.value == n0.value + 256   # 32 fp32 weights, padded to 256 bytes
+    a.norm_w = None
+    assert L.la_fwd_host_staging_size(ctypes.byref(a), ctypes.byref(n1)) == 0
+    assert n1.value == n0.value
