@@ -177,10 +177,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 LEG_NAMES = ["gla_prefill", "gdn_prefill", "elu_prefill", "gla_decode", "gdn_decode"]
-# kernels per call: GLA 1; gated delta rule 2 (T operand images, then the main
-# pass); ELU+1 at this shape 2 (segment sums, then the segment-parallel main
-# pass); each decode step 1
-LEG_LAUNCHES = {"gla_prefill": 1, "gdn_prefill": 2, "elu_prefill": 2, "gla_decode": 1, "gdn_decode": 1}
+# kernels per call: gated delta rule 2 (T operand images, then the main pass);
+# GLA and ELU+1 at these shapes 2 each (range summaries of the earlier sequence
+# segments, then the segment-parallel main pass); each decode step 1
+LEG_LAUNCHES = {"gla_prefill": 2, "gdn_prefill": 2, "elu_prefill": 2, "gla_decode": 1, "gdn_decode": 1}
 
 
 class Legs:
@@ -425,20 +425,23 @@ def _time_calls(torch, run, K):
 def run_variants(torch, la, workloads, K, hbm_peak, seed):
     """The rule variants that run on the same kernels, at the prefill benchmark
     shape (B=2, H=16, T=8192, d=128): DeltaNet (gated delta rule, alpha = 1),
-    RetNet (GLA, one constant decay per head), Lightning (GLA, g = 1); KDA
-    prefill and decode; and GLA / gated-delta prefill of 32 packed
-    variable-length sequences.  Each is timed K
+    RetNet (GLA, one constant decay per head), Lightning (GLA, g = 1) without
+    and with its output RMS normalisation; KDA prefill and decode; and GLA /
+    gated-delta prefill of 32 packed variable-length sequences.  Each is timed K
     times with CUDA events, after 3 warm-up calls."""
-    spec = {"deltanet_prefill": ("gdn", dict(gdn_alpha="ones")),
-            "retnet_prefill": ("gla", dict(gla_gate="retnet")),
-            "lightning_prefill": ("gla", dict(gla_gate="ones"))}
+    wn = torch.ones(128, device="cuda")
+    spec = {"deltanet_prefill": ("gdn", dict(gdn_alpha="ones"), {}),
+            "retnet_prefill": ("gla", dict(gla_gate="retnet"), {}),
+            "lightning_prefill": ("gla", dict(gla_gate="ones"), {}),
+            "lightning_norm_prefill": ("gla", dict(gla_gate="ones"),
+                                       dict(out_norm=True, norm_w=wn, norm_eps=1e-6))}
     res = {}
-    for name, (rule, kw) in spec.items():
+    for name, (rule, kw, fkw) in spec.items():
         p = workloads.make_problem(rule, 2, 8192, 16, 128, 128, seed=seed, **kw)
         a = [None if t is None else t.cuda() for t in (p.q, p.k, p.v, p.g, p.beta)]
         o = torch.empty(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
         S = torch.empty(2, 16, 128, 128, device="cuda")
-        run = lambda: la.fwd(rule, *a, o=o, S_out=S)
+        run = lambda: la.fwd(rule, *a, o=o, S_out=S, **fkw)
         for _ in range(3):
             run()
         stream = torch.cuda.current_stream()
@@ -456,6 +459,11 @@ def run_variants(torch, la, workloads, K, hbm_peak, seed):
         res[name] = {"ms": round(ms, 4), "tokens_per_s": round(w["tokens"] / (ms / 1e3)),
                      "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm_peak, 4)}
         del a, o, S
+    # the normalisation pass alone: o read and written once (bf16)
+    dn = res["lightning_norm_prefill"]["ms"] - res["lightning_prefill"]["ms"]
+    nb = 2 * (2 * 8192 * 16 * 128 * 2)
+    res["lightning_norm_prefill"]["norm_pass_ms"] = round(dn, 4)
+    res["lightning_norm_prefill"]["norm_pass_gbs"] = round(nb / (dn / 1e3) / 1e9, 1) if dn > 0 else None
     # KDA (per-channel retention; recurrent kernel): prefill at the benchmark
     # shape and one decode step on the [256,16,128,128] fp32 state
     p = workloads.make_problem("kda", 2, 8192, 16, 128, 128, seed=seed)
