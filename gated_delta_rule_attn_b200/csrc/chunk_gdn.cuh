@@ -64,6 +64,42 @@ constexpr uint32_t TWGS = TWS + 2 * 4096;            // gamma_C/gamma W
 constexpr uint32_t TSS = TWGS + 4096;                // 2 x S   [128][32] 64 B swizzle
 constexpr uint32_t TEND = TSS + 2 * 8192;
 
+}  // namespace gdn
+
+// KDA workspace item per (batch, head, chunk), written by kda_prep_kernel
+// (chunk_kda.cuh) and read by chunk_gdn_kernel<true>.
+namespace kda {
+constexpr uint32_t ITEM_T = 0;                 // T image, bf16 [64][64], 128-byte swizzled
+constexpr uint32_t ITEM_P = 8192;              // P image, bf16 [64][64], 128-byte swizzled
+constexpr uint32_t ITEM_GC = 16384;            // Gamma_C, fp32 [128]
+constexpr uint32_t ITEM_BYTES = 16384 + 512;
+}  // namespace kda
+
+namespace gdn {
+// Main-kernel shared memory of chunk_gdn_kernel<KDA>.  The gated delta rule
+// uses the tiles above.  KDA (chunk_kda.cuh) loads Qp = Q o Gamma and
+// Kp = K o Gamma in place of Q and K, plus Kc = K o Gamma_C / Gamma, the P image
+// (rows 0-63 of a per-stage [P ; 0] tile) and Gamma_C with every stage, so it
+// keeps 2 stages and needs neither the score tiles nor the gamma_C/gamma W copy.
+template <bool KDA>
+struct GL {
+    static constexpr int NSTG = KDA ? 2 : gdn::NSTG;
+    static constexpr uint32_t STG_QK = 0;                                       // [Q ; K] (KDA: [Qp ; Kp])
+    static constexpr uint32_t STG_KC = STG_QK + NSTG * STG_QK_BYTES;            // KDA: Kc [64][128]
+    static constexpr uint32_t STG_V = STG_KC + (KDA ? NSTG * 16384u : 0u);
+    static constexpr uint32_t STG_TT = STG_V + NSTG * 4096u;
+    static constexpr uint32_t STG_P = STG_TT + NSTG * TT_BYTES;                 // KDA: [P ; 0]
+    static constexpr uint32_t STG_GC = STG_P + (KDA ? NSTG * 16384u : 0u);      // KDA: Gamma_C fp32 [128]
+    static constexpr uint32_t TP = STG_GC + (KDA ? 1024u : 0u);                 // GDN: 2 x [P ; 0]
+    static constexpr uint32_t TR = TP + (KDA ? 0u : 2 * 16384u);
+    static constexpr uint32_t TWS = TR + 4096;
+    static constexpr uint32_t TWGS = TWS + 2 * 4096;                            // GDN only
+    static constexpr uint32_t TSS = TWGS + (KDA ? 0u : 4096u);
+    static constexpr uint32_t TEND = TSS + 2 * 8192;
+};
+static_assert(GL<false>::TEND == TEND && GL<false>::TP == TP && GL<false>::TSS == TSS,
+              "the gated delta rule's layout is the one above");
+
 // Prep-kernel shared memory.
 constexpr int AF_LD = 68;
 constexpr int TMP_LD = 36;
@@ -494,9 +530,16 @@ __device__ __forceinline__ void decay_mask32(float *x, int t, int col0, bool fas
     }
 }
 
+// KDA = true: the KDA main pass (chunk_kda.cuh has the algebra); maps.q, maps.k
+// and maps.kc then cover the prep kernel's Qp, Kp and Kc tensors and `ws` its
+// per-chunk items (T image, P image, Gamma_C).
+template <bool KDA>
 __global__ void __launch_bounds__(gdn::NTHREADS, 1)
 chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const uint8_t *ws) {
     using namespace gdn;
+    using L = gdn::GL<KDA>;
+    constexpr int NSTG = L::NSTG;
+    constexpr uint32_t ITEM = KDA ? kda::ITEM_BYTES : TT_BYTES;   // workspace bytes per chunk
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     GCtl *ctl = reinterpret_cast<GCtl *>(smem_raw);
     uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(GCtl) + (smem_u32(smem_raw) & 1023u)) -
@@ -540,10 +583,11 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         tmem_alloc(&ctl->tmem_base, TMEM_COLS);
         tc_fence_before_sync();
     }
-    // rows 64-127 of both [P ; 0] tiles stay zero
+    // rows 64-127 of both [P ; 0] tiles (KDA: of both stages' P tiles) stay zero
     for (int i = tid; i < 2 * 8192 / 16; i += NTHREADS) {
         const int tile = i / 512, off = (i % 512) * 16;
-        *reinterpret_cast<uint4 *>(tiles + TP + tile * 16384 + 8192 + off) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(tiles + (KDA ? L::STG_P : L::TP) + tile * 16384 + 8192 + off) =
+            make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -556,9 +600,9 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
     constexpr uint32_t ID_W = idesc_bf16(64, DVT, false, true);
     constexpr uint32_t ID_DS = idesc_bf16(128, DVT, true, true);
 
-    auto stage_qk = [&](int c) { return tb + STG_QK + (uint32_t)(c % NSTG) * STG_QK_BYTES; };
-    auto stage_v = [&](int c) { return tiles + STG_V + (uint32_t)(c % NSTG) * 4096u; };
-    auto stage_tt = [&](int c) { return tb + STG_TT + (uint32_t)(c % NSTG) * TT_BYTES; };
+    auto stage_qk = [&](int c) { return tb + L::STG_QK + (uint32_t)(c % NSTG) * STG_QK_BYTES; };
+    auto stage_v = [&](int c) { return tiles + L::STG_V + (uint32_t)(c % NSTG) * 4096u; };
+    auto stage_tt = [&](int c) { return tb + L::STG_TT + (uint32_t)(c % NSTG) * TT_BYTES; };
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
@@ -576,35 +620,52 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             if (stop) break;
             const int t0 = c * C;   // position in the sequence
             if (lane == 0) {
-                mbar_expect_tx(&ctl->full[s], 2u * KA * C * 128u + C * DVT * 2u + TT_BYTES);
-                uint8_t *qk = tiles + STG_QK + s * STG_QK_BYTES;
+                mbar_expect_tx(&ctl->full[s], KDA ? 3u * KA * C * 128u + C * DVT * 2u + 2u * TT_BYTES + 512u
+                                                  : 2u * KA * C * 128u + C * DVT * 2u + TT_BYTES);
+                uint8_t *qk = tiles + L::STG_QK + s * STG_QK_BYTES;
                 const int tm = sq.t0 + t0;   // tensor-map coordinate of the chunk's first token
 #pragma unroll
                 for (int a = 0; a < KA; ++a) {
                     tma_load_4d(qk + a * QK_ACS, &maps.q, &ctl->full[s], 64 * a, (int)h, tm, sq.b0);
                     tma_load_4d(qk + a * QK_ACS + 64 * 128, &maps.k, &ctl->full[s], 64 * a, (int)h, tm,
                                 sq.b0);
+                    if (KDA)
+                        tma_load_4d(tiles + L::STG_KC + s * 16384 + a * (C * 128), &maps.kc, &ctl->full[s],
+                                    64 * a, (int)h, tm, sq.b0);
                 }
-                tma_load_4d(tiles + STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, tm, sq.b0);
-                bulk_load(tiles + STG_TT + s * TT_BYTES, ws + (bh * ws_chunks + c) * (int64_t)TT_BYTES,
-                          TT_BYTES, &ctl->full[s]);
+                tma_load_4d(tiles + L::STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, tm, sq.b0);
+                const uint8_t *item = ws + (bh * ws_chunks + c) * (int64_t)ITEM;
+                bulk_load(tiles + L::STG_TT + s * TT_BYTES, item, TT_BYTES, &ctl->full[s]);
+                if (KDA) {
+                    bulk_load(tiles + L::STG_P + s * 16384, item + kda::ITEM_P, 8192, &ctl->full[s]);
+                    bulk_load(tiles + L::STG_GC + s * 512, item + kda::ITEM_GC, 512, &ctl->full[s]);
+                }
             }
-            // the chunk's decay factors: b = log2 of the inclusive cumulative alpha,
-            // gamma = 2^b, 1/gamma, gamma_C/gamma = 2^(b_63 - b); beta (0 past T)
-            float al[2];
+            if constexpr (KDA) {   // the decay factors come with the stage; betas (0 past T)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int64_t tt = (int64_t)t0 + 2 * lane + e;
-                const bool in = tt < sq.len;
-                al[e] = in ? p.g[(sq.row0 + tt) * p.H + h] : 1.f;
-                ctl->bet[s][2 * lane + e] = in ? p.beta[(sq.row0 + tt) * p.H + h] : 0.f;
+                for (int e = 0; e < 2; ++e) {
+                    const int64_t tt = (int64_t)t0 + 2 * lane + e;
+                    ctl->bet[s][2 * lane + e] = tt < sq.len ? p.beta[(sq.row0 + tt) * p.H + h] : 0.f;
+                }
+                __syncwarp();
+            } else {
+                // the chunk's decay factors: b = log2 of the inclusive cumulative alpha,
+                // gamma = 2^b, 1/gamma, gamma_C/gamma = 2^(b_63 - b); beta (0 past T)
+                float al[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int64_t tt = (int64_t)t0 + 2 * lane + e;
+                    const bool in = tt < sq.len;
+                    al[e] = in ? p.g[(sq.row0 + tt) * p.H + h] : 1.f;
+                    ctl->bet[s][2 * lane + e] = in ? p.beta[(sq.row0 + tt) * p.H + h] : 0.f;
+                }
+                const int fast = gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
+                const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
+                __syncwarp();
+                ctl->gct[s][2 * lane] = exp2f(blast - ctl->b2[s][2 * lane]);
+                ctl->gct[s][2 * lane + 1] = exp2f(blast - ctl->b2[s][2 * lane + 1]);
+                if (lane == 0) ctl->fast[s] = fast;
             }
-            const int fast = gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
-            const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
-            __syncwarp();
-            ctl->gct[s][2 * lane] = exp2f(blast - ctl->b2[s][2 * lane]);
-            ctl->gct[s][2 * lane + 1] = exp2f(blast - ctl->b2[s][2 * lane + 1]);
-            if (lane == 0) ctl->fast[s] = fast;
             mbar_arrive(&ctl->full[s]);
             issued = c + 1;
         }
@@ -625,11 +686,13 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             const int64_t tj = (int64_t)j * C;
             const int nvalid = (int)min((int64_t)C, sq.len - tj);
             if (!mbar_wait(&ctl->wready[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
-            const float gam_o = ctl->gam[sj][ro & 63];   // read before the stage can be refilled
+            // read before the stage can be refilled (KDA: X2 = Qp S0 already carries Gamma)
+            const float gam_o = KDA ? 1.f : ctl->gam[sj][ro & 63];
             bar_named(1, 128);
             if (leader) {
                 tc_fence_after_sync();
-                const uint32_t ps = tb + TP + (uint32_t)jb * 16384u, wsb = tb + TWS + (uint32_t)jb * 4096u;
+                const uint32_t ps = KDA ? tb + L::STG_P + (uint32_t)sj * 16384u : tb + L::TP + (uint32_t)jb * 16384u;
+                const uint32_t wsb = tb + L::TWS + (uint32_t)jb * 4096u;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     umma_bf16(tmem + C_PW + 32u * jb, desc_k(ps, 16384, kk), desc_mn64(wsb, kk), ID_XK, kk > 0);
@@ -678,36 +741,40 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             }
             // (the P tile and score accumulator of chunk c-2 were freed by finish(c-2))
             if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
-            if (leader) {
-                tc_fence_after_sync();
-                const uint32_t qk = stage_qk(c), kb = qk + 64 * 128;
+            if constexpr (KDA) {   // P arrived with the stage
+                if (c >= 1) finish(c - 1);
+            } else {
+                if (leader) {
+                    tc_fence_after_sync();
+                    const uint32_t qk = stage_qk(c), kb = qk + 64 * 128;
 #pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk)
-                    umma_bf16(tmem + C_SC + 64u * pb, desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk), ID_SC, kk > 0);
-                umma_commit(&ctl->l_done[pb]);
-            }
-            if (!mbar_wait(&ctl->l_done[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
-            tc_fence_after_sync();
-            {   // P row t, columns 32hf..32hf+31 -> bf16 rows 0-63 of [P ; 0]
-                float x[32];
-                tmem_ld16x2_32<32>(tq + C_SC + 64u * pb, x);
-                tmem_wait_ld();
-                decay_mask32(x, t, 32 * hf, ctl->fast[s] != 0, ctl->gam[s], ctl->ginv[s], ctl->b2[s]);
-                uint8_t *ps = tiles + TP + pb * 16384;
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint4 u;
-                    u.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
-                    u.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
-                    u.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
-                    u.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
-                    const int chunk = 4 * hf + cc;
-                    *reinterpret_cast<uint4 *>(ps + t * 128 + (((chunk ^ t) & 7) << 4)) = u;
+                    for (int kk = 0; kk < DK / 16; ++kk)
+                        umma_bf16(tmem + C_SC + 64u * pb, desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk), ID_SC, kk > 0);
+                    umma_commit(&ctl->l_done[pb]);
                 }
+                if (!mbar_wait(&ctl->l_done[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
+                tc_fence_after_sync();
+                {   // P row t, columns 32hf..32hf+31 -> bf16 rows 0-63 of [P ; 0]
+                    float x[32];
+                    tmem_ld16x2_32<32>(tq + C_SC + 64u * pb, x);
+                    tmem_wait_ld();
+                    decay_mask32(x, t, 32 * hf, ctl->fast[s] != 0, ctl->gam[s], ctl->ginv[s], ctl->b2[s]);
+                    uint8_t *ps = tiles + L::TP + pb * 16384;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        uint4 u;
+                        u.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
+                        u.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
+                        u.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
+                        u.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
+                        const int chunk = 4 * hf + cc;
+                        *reinterpret_cast<uint4 *>(ps + t * 128 + (((chunk ^ t) & 7) << 4)) = u;
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before_sync();
+                if (c >= 1) finish(c - 1);
             }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            if (c >= 1) finish(c - 1);
         }
         if (leader) umma_commit(&ctl->drain);
     } else {
@@ -725,12 +792,12 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 float4 x = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
                 S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
             }
-            store_row64(tiles + TSS, d, S);
+            store_row64(tiles + L::TSS, d, S);
         }
         fence_proxy_async_smem();
         bar_named(2, 128);
         // the bf16 copy of the state entering chunk c sits in buffer c & 1
-        auto ss_of = [&](int c) { return tb + TSS + (uint32_t)(c & 1) * 8192u; };
+        auto ss_of = [&](int c) { return tb + L::TSS + (uint32_t)(c & 1) * 8192u; };
         // [X2 ; KS] = [Q ; K] S0, K = dk
         auto issue_xk = [&](int c) {
             const uint32_t qk = stage_qk(c), ss = ss_of(c);
@@ -767,15 +834,17 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             ok = mbar_wait(&ctl->xk_done, (uint32_t)c & 1u) && ok;
             if (!ok) ctl->abort = 1;
             tc_fence_after_sync();
-            const float gC = ctl->gam[s][C - 1];
-            const float gct_r = ctl->gct[s][tr];
+            // decay of state row d over the chunk (KDA: per key channel)
+            const float gC = KDA ? reinterpret_cast<const float *>(tiles + L::STG_GC + s * 512)[d]
+                                 : ctl->gam[s][C - 1];
+            const float gct_r = KDA ? 1.f : ctl->gct[s][tr];
             if (quad >= 2) {   // R = diag(beta) (V - diag(gamma) KS): rows 64..127 of [X2 ; KS]
                 const int t = d - 64;
                 float ks[32];
                 tmem_ld32(tq + C_XK + 32u * pb, ks);
                 tmem_wait_ld();
                 const uint8_t *vt = stage_v(c);
-                const float be = ctl->bet[s][t], ga = ctl->gam[s][t];
+                const float be = ctl->bet[s][t], ga = KDA ? 1.f : ctl->gam[s][t];
                 float r[32];
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
@@ -789,7 +858,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                         r[j + 1] = be * fmaf(-ga, ks[j + 1], v2.y);
                     }
                 }
-                store_row64(tiles + TR, t, r);
+                store_row64(tiles + L::TR, t, r);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -799,7 +868,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 const uint32_t tt = stage_tt(c);
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + C_W, desc_k(tt, C * 128, kk), desc_mn64(tb + TR, kk), ID_W, kk > 0);
+                    umma_bf16(tmem + C_W, desc_k(tt, C * 128, kk), desc_mn64(tb + L::TR, kk), ID_W, kk > 0);
                 umma_commit(&ctl->w_done);
             }
             ok = mbar_wait(&ctl->w_done, (uint32_t)c & 1u);
@@ -808,13 +877,16 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             if (!ok) ctl->abort = 1;
             tc_fence_after_sync();
             {   // W and (gamma_C / gamma) W -> bf16, rows tr, columns 16 hf..
+                // (KDA: Kc carries Gamma_C / Gamma, and dS reads W itself)
                 float w[16], wg[16];
                 tmem_ld16x2_16<16>(tq + C_W, w);
                 tmem_wait_ld();
+                store_half64(L::TWS + (uint32_t)pb * 4096u, tr, w);
+                if (!KDA) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) wg[j] = w[j] * gct_r;
-                store_half64(TWS + (uint32_t)pb * 4096u, tr, w);
-                store_half64(TWGS, tr, wg);
+                    for (int j = 0; j < 16; ++j) wg[j] = w[j] * gct_r;
+                    store_half64(L::TWGS, tr, wg);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
@@ -822,10 +894,13 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             bar_named(2, 128);
             if (leader) {   // dS = K^T diag(gamma_C / gamma) W, K = tokens
                 tc_fence_after_sync();
-                const uint32_t kb = stage_qk(c) + 64 * 128;
+                // GDN: K^T (gamma_C/gamma W); KDA: Kc^T W
+                const uint32_t kb = KDA ? tb + L::STG_KC + (uint32_t)s * 16384u : stage_qk(c) + 64 * 128;
+                const uint32_t kacs = KDA ? (uint32_t)(C * 128) : QK_ACS;
+                const uint32_t wb = KDA ? tb + L::TWS + (uint32_t)pb * 4096u : tb + L::TWGS;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + C_DS, desc_mn128(kb, QK_ACS, kk), desc_mn64(tb + TWGS, kk), ID_DS, kk > 0);
+                    umma_bf16(tmem + C_DS, desc_mn128(kb, kacs, kk), desc_mn64(wb, kk), ID_DS, kk > 0);
                 umma_commit(&ctl->ds_done);
                 umma_commit(&ctl->empty[s]);
             }
@@ -837,7 +912,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < DVT; ++j) S[j] = fmaf(gC, S[j], ds[j]);
-                store_row64(tiles + TSS + (uint32_t)((c + 1) & 1) * 8192u, d, S);
+                store_row64(tiles + L::TSS + (uint32_t)((c + 1) & 1) * 8192u, d, S);
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();

@@ -147,6 +147,7 @@ __device__ __forceinline__ void store_out_row(void *o, const ChunkParams &p, int
 
 struct Maps {
     CUtensorMap q, k, v, g;
+    CUtensorMap kc;   // KDA: the prep kernel's Kc = K o Gamma_C / Gamma
 };
 
 __device__ __forceinline__ uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
@@ -166,6 +167,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 }  // namespace la
 
 #include "chunk_gdn.cuh"
+#include "chunk_kda.cuh"
 #include "chunk_ge.cuh"
 #include "chunk_agg.cuh"
 
@@ -223,16 +225,35 @@ inline int resident_per_sm(const void *kernel, int threads, int dyn_smem, int tm
     return std::max(n, 1);
 }
 
+// KDA workspace: the per-chunk items (T image, P image, Gamma_C), then the
+// Qp, Kp and Kc tensors [B,T,H,128] bf16, each at a 256-byte aligned offset.
+struct KdaWorkspace {
+    size_t items, qp, kp, kc, total;
+};
+inline KdaWorkspace kda_workspace(int64_t B, int64_t T, int64_t H) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    KdaWorkspace w{};
+    w.items = 0;
+    const size_t tensor = up((size_t)(B * T * H) * ck::DK * 2);
+    w.qp = up((size_t)(B * H * ((T + ck::C - 1) / ck::C)) * ck::kda::ITEM_BYTES);
+    w.kp = w.qp + tensor;
+    w.kc = w.kp + tensor;
+    w.total = w.kc + tensor;
+    return w;
+}
+
 // Device workspace the chunked path needs: the gated delta rule keeps the
-// per-chunk T = (I + A)^-1 operand images (8 KB per (batch, head, chunk));
-// sequence-parallel ELU+1 and GLA the range summaries of their first pass.
-// `packed`: the sequences are packed on one token axis with lengths up to
-// max_seqlen (no sequence-parallel pass then).
+// per-chunk T = (I + A)^-1 operand images (8 KB per (batch, head, chunk)); KDA
+// its prep kernel's items and scaled q/k tensors (dense layout only: packed KDA
+// runs on the recurrent kernel); sequence-parallel ELU+1 and GLA the range
+// summaries of their first pass.  `packed`: the sequences are packed on one
+// token axis with lengths up to max_seqlen (no sequence-parallel pass then).
 inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv,
                                     bool packed = false, int64_t max_seqlen = 0) {
     if (T <= 0) return 0;
     const int64_t L = packed ? max_seqlen : T;
     if (rule == kRuleGDN) return (size_t)(B * H * ((L + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;
+    if (rule == kRuleKDA) return packed ? 0 : kda_workspace(B, T, H).total;
     if (packed) return 0;
     const SegPlan sp = seg_plan(rule, B, T, H, dv);
     if (sp.nseg < 2) return 0;
@@ -297,7 +318,48 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
     }
     const unsigned grid = (unsigned)(p.B * p.H * (p.dv / DVT));
     cudaError_t e;
-    if (rule == kRuleGDN) {
+    if (rule == kRuleKDA) {
+        if (packed) {
+            *err = "the chunked KDA kernels take the dense layout";
+            return 2;
+        }
+        const KdaWorkspace kw = kda_workspace(p.B, p.T, p.H);
+        if (!ws || ws_bytes < kw.total || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
+            *err = "KDA needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
+            return 8;
+        }
+        uint8_t *w8 = static_cast<uint8_t *>(ws);
+        KdaPrepParams kp{};
+        kp.B = p.B; kp.T = p.T; kp.H = p.H;
+        kp.nchunks = (int)((p.T + C - 1) / C);
+        kp.q = static_cast<const __nv_bfloat16 *>(p.q);
+        kp.k = static_cast<const __nv_bfloat16 *>(p.k);
+        kp.alpha = p.g; kp.beta = p.beta;
+        kp.items = w8 + kw.items;
+        kp.qp = reinterpret_cast<__nv_bfloat16 *>(w8 + kw.qp);
+        kp.kp = reinterpret_cast<__nv_bfloat16 *>(w8 + kw.kp);
+        kp.kc = reinterpret_cast<__nv_bfloat16 *>(w8 + kw.kc);
+        Maps mk = m;
+        if (!make_map_4d(&mk.q, kp.qp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, DK, 64, C,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map_4d(&mk.k, kp.kp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, DK, 64, C,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_map_4d(&mk.kc, kp.kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, DK, 64, C,
+                         CU_TENSOR_MAP_SWIZZLE_128B)) {
+            *err = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
+            return 4;
+        }
+        const int64_t items = p.B * p.H * (int64_t)kp.nchunks;
+        const int psmem = (int)((sizeof(KCtl) + 1023) / 1024 * 1024) + 1024 + (int)kda::P_END;
+        e = allow_smem((const void *)kda_prep_kernel, psmem);
+        const int per_sm = resident_per_sm((const void *)kda_prep_kernel, kda::PREP_THREADS, psmem, 256);
+        const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
+        if (e == cudaSuccess) kda_prep_kernel<<<pgrid, kda::PREP_THREADS, psmem, st>>>(kp);
+        const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::GL<true>::TEND;
+        if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel<true>, smem);
+        if (e == cudaSuccess)
+            chunk_gdn_kernel<true><<<grid, gdn::NTHREADS, smem, st>>>(mk, pq, w8 + kw.items);
+    } else if (rule == kRuleGDN) {
         const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv, packed, Lmax);
         if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
             *err = "the gated delta rule needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
@@ -318,9 +380,9 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
         if (e == cudaSuccess && items > 0) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.k, pp);
         const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::TEND;
-        if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel, smem);
+        if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel<false>, smem);
         if (e == cudaSuccess)
-            chunk_gdn_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));
+            chunk_gdn_kernel<false><<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));
     } else {
         // packed sequences walk each sequence in one pass (no segments)
         const SegPlan sp = packed ? SegPlan{1, 1, (int)((Lmax + C - 1) / C)} : seg_plan(rule, p.B, p.T, p.H, p.dv);

@@ -2,8 +2,10 @@
 // kernel selection, the host-buffer entry point and the device error word.
 //
 // Kernel selection for la_fwd:
-//   bf16, dk = 128           -> chunked tensor-core kernel (chunk_tc.cuh)
-//   fp32, or bf16 with dk < 128, or KDA -> per-token recurrent kernel (recurrent.cuh)
+//   bf16, dk = 128           -> chunked tensor-core kernels (chunk_tc.cuh; KDA
+//                               with the dense layout only)
+//   fp32, or bf16 with dk < 128, or packed KDA -> per-token recurrent kernel
+//                               (recurrent.cuh)
 // la_step always uses the recurrent kernel with T = 1 and the state in place.
 // With out_norm set, a second pass normalises each (token, head) row of o
 // (out_norm.cuh).
@@ -186,9 +188,10 @@ cudaError_t allow_smem(const void *kernel, int bytes) {
 
 namespace {
 
-// KDA has no chunked kernel yet: every KDA prefill runs on the recurrent kernel.
+// Packed KDA sequences run on the recurrent kernel (the chunked KDA prep writes
+// scaled q/k tensors that a packed tail chunk would read past its sequence).
 bool uses_chunk_kernels(const la_fwd_args &a) {
-    return a.dtype == LA_BF16 && a.dk == 128 && a.T > 0 && a.rule != LA_RULE_KDA;
+    return a.dtype == LA_BF16 && a.dk == 128 && a.T > 0 && (a.rule != LA_RULE_KDA || !a.cu_seqlens);
 }
 
 // Output normalisation arguments (ABI version 3), shared by la_fwd and la_step.
@@ -527,7 +530,9 @@ la_status la_check_device(void *stream, uint32_t *flags) {
     if (flags) *flags = w;
     if (w & la::kErrTimeout) return fail(LA_ERR_TIMEOUT, "a bounded device wait ran out");
     if (w & la::kErrRange)
-        return fail(LA_ERR_RANGE, "GLA cumulative gate inside a 64-token chunk fell below 1e-30");
+        return fail(LA_ERR_RANGE,
+                    "a gate product left the chunked kernels' range (GLA: below 1e-30 inside a 64-token "
+                    "chunk; KDA: an 8-token retention product below 2^-60)");
     if (w & la::kErrSeqlen)
         return fail(LA_ERR_INVALID_ARG,
                     "cu_seqlens: offsets out of order or outside [0, T], or a sequence longer than "

@@ -66,7 +66,7 @@ typedef enum {
     LA_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned */
     LA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     LA_ERR_TIMEOUT = 5,       /* a bounded device-side wait ran out (la_check_device) */
-    LA_ERR_RANGE = 6,         /* GLA gate product left the fp32 range in a chunk (la_check_device) */
+    LA_ERR_RANGE = 6,         /* a gate product left a chunked kernel's range (la_check_device) */
     LA_ERR_INTERNAL = 7,
     LA_ERR_WORKSPACE = 8      /* workspace missing or smaller than la_fwd_workspace_size() */
 } la_status;
@@ -79,8 +79,12 @@ typedef enum {
  *        ("线性注意力与 SSM", GDN box, in the dk x dv orientation)
  *   KDA  S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
  *        alpha_t per key channel ("状态空间与线性注意力", KDA：逐通道遗忘与误差写入).
- *        KDA runs on the per-token recurrent kernel (CUDA cores) for every
- *        dtype and size; it has no chunked tensor-core kernel yet.
+ *        bf16 KDA with dk = 128 and the dense layout runs chunked on the tensor
+ *        cores, for retention whose product over any 8 consecutive tokens stays
+ *        >= 2^-60 per channel (the page's bounded log-decay, log alpha > -5,
+ *        satisfies this); outside that domain la_check_device reports
+ *        LA_ERR_RANGE.  fp32, dk < 128 and packed KDA run on the per-token
+ *        recurrent kernel (CUDA cores), which has no such domain.
  */
 typedef enum { LA_RULE_ELU = 0, LA_RULE_GLA = 1, LA_RULE_GDN = 2, LA_RULE_KDA = 3 } la_rule;
 
@@ -109,6 +113,10 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *          sequences run segment-parallel and keep there the summary of each
  *          piece of every segment but the last (dk*dv + dk floats per piece: the
  *          piece's state contribution and its normaliser sum or gate product).
+ *          Chunked KDA keeps 16.5 KB per (batch, head, chunk) (the T and P
+ *          operand images and the chunk's retention product) plus three bf16
+ *          [B,T,H,128] tensors: q and k scaled by the cumulative retention, and
+ *          k scaled by the retention from the token to its chunk's end.
  *          Calls that share
  *          one workspace must be ordered (same stream), otherwise they race.
  *          A missing or short workspace returns LA_ERR_WORKSPACE before any launch.
