@@ -639,6 +639,18 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 if (KDA) {
                     bulk_load(tiles + L::STG_P + s * 16384, item + kda::ITEM_P, 8192, &ctl->full[s]);
                     bulk_load(tiles + L::STG_GC + s * 512, item + kda::ITEM_GC, 512, &ctl->full[s]);
+                    // two stages leave about one chunk period for a load: start chunk
+                    // c+1's tiles and item on their way to L2 now
+                    if (c + 1 < nchunks) {
+#pragma unroll
+                        for (int a = 0; a < KA; ++a) {
+                            tma_prefetch_l2_4d(&maps.q, 64 * a, (int)h, tm + C, sq.b0);
+                            tma_prefetch_l2_4d(&maps.k, 64 * a, (int)h, tm + C, sq.b0);
+                            tma_prefetch_l2_4d(&maps.kc, 64 * a, (int)h, tm + C, sq.b0);
+                        }
+                        tma_prefetch_l2_4d(&maps.v, dvt * DVT, (int)h, tm + C, sq.b0);
+                        bulk_prefetch_l2(item + ITEM, ITEM);
+                    }
                 }
             }
             if constexpr (KDA) {   // the decay factors come with the stage; betas (0 past T)
@@ -690,6 +702,11 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             const float gam_o = KDA ? 1.f : ctl->gam[sj][ro & 63];
             bar_named(1, 128);
             if (leader) {
+                // KDA: P(j) came with stage j, which the state group has consumed
+                // (wready); this wait only makes the copy's completion visible to
+                // the issuing thread and returns at once (the stage cannot be
+                // refilled before PW(j) is committed below)
+                if (KDA && !mbar_wait(&ctl->full[sj], (uint32_t)(j / NSTG) & 1u)) ctl->abort = 1;
                 tc_fence_after_sync();
                 const uint32_t ps = KDA ? tb + L::STG_P + (uint32_t)sj * 16384u : tb + L::TP + (uint32_t)jb * 16384u;
                 const uint32_t wsb = tb + L::TWS + (uint32_t)jb * 4096u;
@@ -740,10 +757,12 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 break;
             }
             // (the P tile and score accumulator of chunk c-2 were freed by finish(c-2))
-            if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
-            if constexpr (KDA) {   // P arrived with the stage
+            if constexpr (KDA) {
+                // P comes with the stage; waiting here for stage c would hold PW(c-1),
+                // which frees the stage that chunk c+1 is loaded into (two stages)
                 if (c >= 1) finish(c - 1);
             } else {
+                if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
                 if (leader) {
                     tc_fence_after_sync();
                     const uint32_t qk = stage_qk(c), kb = qk + 64 * 128;

@@ -84,8 +84,11 @@ struct KdaPrepParams {
     __nv_bfloat16 *qp, *kp, *kc;      // [B,T,H,128]
 };
 
+// Four products as two packed fp32x2 multiplies.
 __device__ __forceinline__ float4 mul4(float4 a, float4 b) {
-    return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+    const float2 lo = __fmul2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y));
+    const float2 hi = __fmul2_rn(make_float2(a.z, a.w), make_float2(b.z, b.w));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
 }
 __device__ __forceinline__ float4 rcp4(float4 a) {
     return make_float4(rcp_approx(a.x), rcp_approx(a.y), rcp_approx(a.z), rcp_approx(a.w));
@@ -166,6 +169,23 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
         if (tid < 64) {
             const int64_t t = t0 + tid;
             ctl->beta[tid] = t < p.T ? p.beta[(b * p.T + t) * p.H + h] : 0.f;
+        }
+        {   // bring the next item's rows into L2 while this one is worked on: thread
+            // i < 64 the alpha row (512 B) of token i, thread 64 + i its q and k rows
+            const int64_t wn = w + gridDim.x;
+            if (wn < items) {
+                const int64_t bhn = wn / p.nchunks, bn = bhn / p.H, hn = bhn % p.H;
+                const int64_t tn = (int64_t)(wn % p.nchunks) * C + (tid & 63);
+                if (tn < p.T) {
+                    const int64_t row = ((bn * p.T + tn) * p.H + hn) * DK;
+                    if (tid < 64) {
+                        bulk_prefetch_l2(p.alpha + row, DK * 4);
+                    } else {
+                        bulk_prefetch_l2(p.q + row, DK * 2);
+                        bulk_prefetch_l2(p.k + row, DK * 2);
+                    }
+                }
+            }
         }
         // G_j = Gamma_t / Gamma_middle, in place of alpha: 1 / prod_{j+1..7} alpha
         // for j <= 7, prod_{8..j} alpha for j >= 8

@@ -122,6 +122,14 @@ __device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *map, int c
                  : "memory");
 }
 
+// L2 prefetch of `bytes` (a multiple of 16) at a 16-byte aligned global address
+// (no shared-memory destination, no barrier).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gptr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(gptr)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
