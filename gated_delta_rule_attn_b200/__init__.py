@@ -211,7 +211,11 @@ def fwd(rule: str, q, k, v, g=None, beta=None, S0=None, z0=None, eps: float = 1e
 
 
 def fwd_workspace_size(rule, q, k, v, g=None, beta=None, S0=None, z0=None) -> int:
+    """Bytes of workspace ``fwd`` needs for these inputs (shapes only are read)."""
     a = make_fwd_args(rule, q, k, v, g, beta, S0, z0)
+    # the query validates the arguments as la_fwd does, which needs a non-NULL o;
+    # no data is touched, so q's address stands in for it
+    a.o = a.q
     n = ctypes.c_size_t()
     _check(lib().la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
     return n.value

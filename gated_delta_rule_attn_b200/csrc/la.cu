@@ -216,7 +216,10 @@ la_status launch_norm(la_dtype dtype, void *o, int64_t rows, int64_t dv, const f
     return ok();
 }
 
-la_status launch_fwd_core(const la_fwd_args &a, cudaStream_t st) {
+// `recurrent`: run on the per-token recurrent kernel even where the chunked
+// kernels apply (la_fwd_noalloc for KDA problems whose chunked scratch exceeds
+// the library's array).
+la_status launch_fwd_core(const la_fwd_args &a, cudaStream_t st, bool recurrent) {
     const Shape s{a.B, a.T, a.H, a.dk, a.dv};
     if (a.T == 0 || (a.cu_seqlens && a.max_seqlen == 0)) {   // no token in any sequence
         const size_t sb = (size_t)(s.B * s.H * s.dk * s.dv) * sizeof(float);
@@ -233,7 +236,7 @@ la_status launch_fwd_core(const la_fwd_args &a, cudaStream_t st) {
         }
         return ok();
     }
-    if (uses_chunk_kernels(a)) {
+    if (!recurrent && uses_chunk_kernels(a)) {
         la::ChunkParams p{};
         p.B = a.B; p.T = a.T; p.H = a.H; p.dv = a.dv;
         p.q = a.q; p.k = a.k; p.v = a.v; p.g = a.g; p.beta = a.beta;
@@ -255,8 +258,8 @@ la_status launch_fwd_core(const la_fwd_args &a, cudaStream_t st) {
     return launch_recurrent(a.rule, p, a.dk, a.dv, a.dtype, st);
 }
 
-la_status launch_fwd(const la_fwd_args &a, cudaStream_t st) {
-    la_status r = launch_fwd_core(a, st);
+la_status launch_fwd(const la_fwd_args &a, cudaStream_t st, bool recurrent = false) {
+    la_status r = launch_fwd_core(a, st, recurrent);
     if (r != LA_OK || !a.out_norm || a.T == 0) return r;
     // o is [B,T,H,dv] dense or [1,T,H,dv] packed
     const int64_t rows = (a.cu_seqlens ? a.T : a.B * a.T) * a.H;
@@ -363,9 +366,13 @@ la_status la_fwd_noalloc(const la_fwd_args *args, void *stream) {
     if (r != LA_OK) return r;
     a.workspace = nullptr;
     a.workspace_bytes = 0;
-    const size_t need = uses_chunk_kernels(a) ? la::chunk_workspace_bytes((int)a.rule, a.B, a.T, a.H, a.dv,
-                                                                          a.cu_seqlens != nullptr, a.max_seqlen)
-                                              : 0;
+    size_t need = uses_chunk_kernels(a) ? la::chunk_workspace_bytes((int)a.rule, a.B, a.T, a.H, a.dv,
+                                                                    a.cu_seqlens != nullptr, a.max_seqlen)
+                                        : 0;
+    // KDA has a kernel that needs no scratch (the per-token recurrent one): a
+    // problem whose chunked scratch does not fit the array runs there instead
+    const bool recurrent = need > LA_NOALLOC_SCRATCH_BYTES && a.rule == LA_RULE_KDA;
+    if (recurrent) need = 0;
     if (need > LA_NOALLOC_SCRATCH_BYTES)
         return fail(LA_ERR_WORKSPACE, "problem needs " + std::to_string(need) +
                                           " bytes of scratch; la_fwd_noalloc has " +
@@ -376,7 +383,7 @@ la_status la_fwd_noalloc(const la_fwd_args *args, void *stream) {
         if (r != LA_OK) return r;
         a.workspace_bytes = LA_NOALLOC_SCRATCH_BYTES;
     }
-    return launch_fwd(a, static_cast<cudaStream_t>(stream));
+    return launch_fwd(a, static_cast<cudaStream_t>(stream), recurrent);
 }
 
 la_status la_fwd_workspace_size(const la_fwd_args *args, size_t *bytes) {

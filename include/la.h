@@ -251,6 +251,9 @@ la_status la_fwd_host(const la_fwd_args *host_args, void *staging, size_t stagin
  *     LA_NOALLOC_SCRATCH_BYTES, otherwise LA_ERR_WORKSPACE is returned before
  *     anything is launched.  For the gated delta rule that is 2048
  *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 8192.
+ *     KDA is the exception: a KDA problem whose chunked scratch does not fit
+ *     runs on the per-token recurrent kernel, which needs none (slower, same
+ *     results within the bf16 tolerance).
  *   - The first call on a device looks up the array's device address there
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.  Later calls on the device reuse the address.

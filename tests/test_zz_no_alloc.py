@@ -7,7 +7,9 @@ path needs.  la_fwd_noalloc uses the library's own fixed 16 MiB device array
 instead.  These tests call it through the C ABI and check that it gives what
 la_fwd gives, on two calls in a row with different inputs (the array keeps the
 previous call's contents), and that a problem needing more scratch than the
-array holds is refused before anything runs.
+array holds is refused before anything runs.  KDA, whose chunked path keeps
+scaled q/k tensors in the scratch, runs chunked when they fit and on the
+scratch-free recurrent kernel when they do not; both must match la_fwd.
 
 This file is named so that pytest collects it last.
 """
@@ -60,6 +62,33 @@ def test_noalloc_matches_la_fwd_on_two_calls():
         o = torch.empty_like(o_ref)
         S = torch.empty_like(S_ref)
         a = la.make_fwd_args("gdn", d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], None, 1e-6,
+                             o, S, None)
+        rc = L.la_fwd_noalloc(ctypes.byref(a), stream)
+        assert rc == 0, L.la_last_error_message()
+        torch.cuda.synchronize()
+        la.check_device()
+        assert _rel(o, o_ref) <= TOL
+        assert _rel(S, S_ref) <= TOL
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T", [300, 2048])
+def test_noalloc_kda_fits_or_runs_without_scratch(T):
+    """T=300 (B*H = 4) fits the array and runs chunked; T=2048 at H=16 needs
+    about 25 MB of chunked scratch and runs on the recurrent kernel."""
+    la = _lib()
+    L = la.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    H = 4 if T == 300 else 16
+    p = workloads.make_problem("kda", 1, T, H, 128, 128, seed=T, init_state="normal")
+    d = {n: getattr(p, n).cuda() for n in ("q", "k", "v", "g", "beta", "S0")}
+    o_ref, S_ref, _ = la.fwd("kda", d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert (la.fwd_workspace_size("kda", d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+            > (16 << 20)) == (T == 2048)
+    for _ in range(2):
+        o = torch.empty_like(o_ref)
+        S = torch.empty_like(S_ref)
+        a = la.make_fwd_args("kda", d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], None, 1e-6,
                              o, S, None)
         rc = L.la_fwd_noalloc(ctypes.byref(a), stream)
         assert rc == 0, L.la_last_error_message()
