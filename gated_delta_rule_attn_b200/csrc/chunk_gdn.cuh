@@ -624,14 +624,16 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                                                   : 2u * KA * C * 128u + C * DVT * 2u + TT_BYTES);
                 uint8_t *qk = tiles + L::STG_QK + s * STG_QK_BYTES;
                 const int tm = sq.t0 + t0;   // tensor-map coordinate of the chunk's first token
+                // q, k maps (KDA: the prep's qp, kp, kc, one row block per sequence
+                // even when packed): the chunk's first token at (tq, bq)
+                const int tq = KDA ? t0 : tm, bq = KDA ? (int)b : sq.b0;
 #pragma unroll
                 for (int a = 0; a < KA; ++a) {
-                    tma_load_4d(qk + a * QK_ACS, &maps.q, &ctl->full[s], 64 * a, (int)h, tm, sq.b0);
-                    tma_load_4d(qk + a * QK_ACS + 64 * 128, &maps.k, &ctl->full[s], 64 * a, (int)h, tm,
-                                sq.b0);
+                    tma_load_4d(qk + a * QK_ACS, &maps.q, &ctl->full[s], 64 * a, (int)h, tq, bq);
+                    tma_load_4d(qk + a * QK_ACS + 64 * 128, &maps.k, &ctl->full[s], 64 * a, (int)h, tq, bq);
                     if (KDA)
                         tma_load_4d(tiles + L::STG_KC + s * 16384 + a * (C * 128), &maps.kc, &ctl->full[s],
-                                    64 * a, (int)h, tm, sq.b0);
+                                    64 * a, (int)h, tq, bq);
                 }
                 tma_load_4d(tiles + L::STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, tm, sq.b0);
                 const uint8_t *item = ws + (bh * ws_chunks + c) * (int64_t)ITEM;
@@ -644,9 +646,9 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                     if (c + 1 < nchunks) {
 #pragma unroll
                         for (int a = 0; a < KA; ++a) {
-                            tma_prefetch_l2_4d(&maps.q, 64 * a, (int)h, tm + C, sq.b0);
-                            tma_prefetch_l2_4d(&maps.k, 64 * a, (int)h, tm + C, sq.b0);
-                            tma_prefetch_l2_4d(&maps.kc, 64 * a, (int)h, tm + C, sq.b0);
+                            tma_prefetch_l2_4d(&maps.q, 64 * a, (int)h, tq + C, bq);
+                            tma_prefetch_l2_4d(&maps.k, 64 * a, (int)h, tq + C, bq);
+                            tma_prefetch_l2_4d(&maps.kc, 64 * a, (int)h, tq + C, bq);
                         }
                         tma_prefetch_l2_4d(&maps.v, dvt * DVT, (int)h, tm + C, sq.b0);
                         bulk_prefetch_l2(item + ITEM, ITEM);

@@ -34,7 +34,11 @@
 //   per item: the T image and the P image (bf16, 128-byte swizzled [64][64], the
 //   shared-memory operand layout of chunk_gdn_kernel) and Gamma_C (fp32 [128]);
 //   per token: Qp = q o Gamma, Kp = k o Gamma, Kc = k o Gamma_C / Gamma as bf16
-//   [B,T,H,128] tensors, which chunk_gdn_kernel<true> loads by TMA in place of q, k.
+//   [B,Ls,H,128] tensors, which chunk_gdn_kernel<true> loads by TMA in place of q, k.
+//   Dense layout: Ls = T.  Packed sequences: one row block per sequence,
+//   Ls = 64 ceil(max_seqlen / 64), so a sequence's tail chunk owns its padding
+//   rows, which are written as zeros (the next sequence's tokens never appear
+//   in its chunks).
 // Warp w owns sub-chunk w: lane l holds key channels 4l..4l+3 of its 16 tokens.
 #pragma once
 
@@ -77,11 +81,14 @@ struct KCtl {
 
 struct KdaPrepParams {
     int64_t B, T, H;
-    int nchunks;                      // ceil(T / 64)
-    const __nv_bfloat16 *q, *k;       // [B,T,H,128]
-    const float *alpha, *beta;        // [B,T,H,128], [B,T,H]
+    int nchunks;                      // chunks per (sequence, head): ceil(max_seqlen / 64)
+    int64_t Ls;                       // token extent of qp, kp, kc: T, or 64 nchunks when packed
+    const __nv_bfloat16 *q, *k;       // [B,T,H,128] (packed: [1,T,H,128])
+    const float *alpha, *beta;        // [B,T,H,128], [B,T,H] (packed: [1,T,H,*])
     uint8_t *items;                   // [B*H*nchunks][ITEM_BYTES]
-    __nv_bfloat16 *qp, *kp, *kc;      // [B,T,H,128]
+    __nv_bfloat16 *qp, *kp, *kc;      // [B,Ls,H,128]
+    const int64_t *cu_seqlens;        // packed sequences, or nullptr (dense)
+    int64_t max_seqlen;               // = T for the dense layout
 };
 
 // Four products as two packed fp32x2 multiplies.
@@ -144,15 +151,20 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
     const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lanes
     constexpr uint32_t ID_S = idesc_bf16(128, 64, false, false);
 
-    int it = 0;
-    for (int64_t w = blockIdx.x; w < items; w += gridDim.x, ++it) {
+    int it = 0;   // items processed (one MMA commit each): the mbarrier phase
+    for (int64_t w = blockIdx.x; w < items; w += gridDim.x) {
         const int64_t bh = w / p.nchunks;
         const int c = (int)(w % p.nchunks);
         const int64_t b = bh / p.H, h = bh % p.H;
-        const int64_t t0 = (int64_t)c * C;
+        const int64_t t0 = (int64_t)c * C;   // position in the sequence
+        const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, false);
         if (tid == 0) ctl->stop = ctl->abort;   // one thread decides, everyone reads after the barrier
         bar_named(1, 128);
         if (ctl->stop) break;
+        if (t0 >= sq.len) continue;   // past this packed sequence's last chunk (uniform over the CTA)
+        // rows of qp, kp, kc this item writes: the sequence's tokens, plus (packed)
+        // the padding rows of its tail chunk, as zeros
+        const int64_t wlen = p.cu_seqlens ? p.Ls : sq.len;
 
         // (1) loads: alpha (1 past T), q and k (0 past T) of this thread's 16 tokens x 4 channels
         float4 g[16];
@@ -160,24 +172,25 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int64_t t = t0 + 16 * sc + j;
-            const bool valid = t < p.T;
-            const int64_t row = ((b * p.T + (valid ? t : 0)) * p.H + h) * DK + d0;
+            const bool valid = t < sq.len;
+            const int64_t row = ((sq.row0 + (valid ? t : 0)) * p.H + h) * DK + d0;
             g[j] = valid ? __ldg(reinterpret_cast<const float4 *>(p.alpha + row)) : make_float4(1.f, 1.f, 1.f, 1.f);
             qr[j] = valid ? __ldg(reinterpret_cast<const uint2 *>(p.q + row)) : make_uint2(0u, 0u);
             kr[j] = valid ? __ldg(reinterpret_cast<const uint2 *>(p.k + row)) : make_uint2(0u, 0u);
         }
         if (tid < 64) {
             const int64_t t = t0 + tid;
-            ctl->beta[tid] = t < p.T ? p.beta[(b * p.T + t) * p.H + h] : 0.f;
+            ctl->beta[tid] = t < sq.len ? p.beta[(sq.row0 + t) * p.H + h] : 0.f;
         }
         {   // bring the next item's rows into L2 while this one is worked on: thread
             // i < 64 the alpha row (512 B) of token i, thread 64 + i its q and k rows
             const int64_t wn = w + gridDim.x;
             if (wn < items) {
                 const int64_t bhn = wn / p.nchunks, bn = bhn / p.H, hn = bhn % p.H;
+                const SeqSpan sn = seq_span(p.cu_seqlens, bn, p.T, p.max_seqlen, false);
                 const int64_t tn = (int64_t)(wn % p.nchunks) * C + (tid & 63);
-                if (tn < p.T) {
-                    const int64_t row = ((bn * p.T + tn) * p.H + hn) * DK;
+                if (tn < sn.len) {
+                    const int64_t row = ((sn.row0 + tn) * p.H + hn) * DK;
                     if (tid < 64) {
                         bulk_prefetch_l2(p.alpha + row, DK * 4);
                     } else {
@@ -251,12 +264,14 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
 #pragma unroll
             for (int a = 0; a < 4; ++a)
                 if (a > sc) st4_sw128(tiles + P_KR + a * KR_BYTES, KR_ACS, 16 * sc + j, d0, mul4(kf, mul4(Hd, mk[a])));
-            if (t < p.T) {
-                const int64_t row = ((b * p.T + t) * p.H + h) * DK + d0;
+            if (t < wlen) {
+                const int64_t row = ((b * p.Ls + t) * p.H + h) * DK + d0;
                 const float4 Gg = mul4(Gd, gm);   // Gamma_t
-                *reinterpret_cast<uint2 *>(p.qp + row) = f32_to_bf16x4(mul4(qf, Gg));
-                *reinterpret_cast<uint2 *>(p.kp + row) = f32_to_bf16x4(mul4(kf, Gg));
-                *reinterpret_cast<uint2 *>(p.kc + row) = f32_to_bf16x4(mul4(kf, mul4(Hd, cm)));   // Gamma_C / Gamma_t
+                const bool in = t < sq.len;
+                *reinterpret_cast<uint2 *>(p.qp + row) = in ? f32_to_bf16x4(mul4(qf, Gg)) : make_uint2(0u, 0u);
+                *reinterpret_cast<uint2 *>(p.kp + row) = in ? f32_to_bf16x4(mul4(kf, Gg)) : make_uint2(0u, 0u);
+                *reinterpret_cast<uint2 *>(p.kc + row) =   // Gamma_C / Gamma_t
+                    in ? f32_to_bf16x4(mul4(kf, mul4(Hd, cm))) : make_uint2(0u, 0u);
             }
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0) raise_error(kErrRange);
@@ -276,6 +291,7 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
             umma_commit(&ctl->mma);
         }
         if (!mbar_wait(&ctl->mma, (uint32_t)it & 1u)) ctl->abort = 1;
+        ++it;
         tc_fence_after_sync();
 
         // (5) lane l < 16: P row of token 16w + l; lane l >= 16: A row of token 16w + l - 16.

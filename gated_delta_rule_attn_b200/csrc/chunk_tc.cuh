@@ -226,7 +226,9 @@ inline int resident_per_sm(const void *kernel, int threads, int dyn_smem, int tm
 }
 
 // KDA workspace: the per-chunk items (T image, P image, Gamma_C), then the
-// Qp, Kp and Kc tensors [B,T,H,128] bf16, each at a 256-byte aligned offset.
+// Qp, Kp and Kc tensors [B,Ls,H,128] bf16, each at a 256-byte aligned offset
+// (Ls = T dense; 64 ceil(max_seqlen / 64) for packed sequences, one row block
+// per sequence).
 struct KdaWorkspace {
     size_t items, qp, kp, kc, total;
 };
@@ -244,8 +246,7 @@ inline KdaWorkspace kda_workspace(int64_t B, int64_t T, int64_t H) {
 
 // Device workspace the chunked path needs: the gated delta rule keeps the
 // per-chunk T = (I + A)^-1 operand images (8 KB per (batch, head, chunk)); KDA
-// its prep kernel's items and scaled q/k tensors (dense layout only: packed KDA
-// runs on the recurrent kernel); sequence-parallel ELU+1 and GLA the range
+// its prep kernel's items and scaled q/k tensors; sequence-parallel ELU+1 and GLA the range
 // summaries of their first pass.  `packed`: the sequences are packed on one
 // token axis with lengths up to max_seqlen (no sequence-parallel pass then).
 inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv,
@@ -253,7 +254,7 @@ inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, i
     if (T <= 0) return 0;
     const int64_t L = packed ? max_seqlen : T;
     if (rule == kRuleGDN) return (size_t)(B * H * ((L + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;
-    if (rule == kRuleKDA) return packed ? 0 : kda_workspace(B, T, H).total;
+    if (rule == kRuleKDA) return kda_workspace(B, packed ? (L + ck::C - 1) / ck::C * ck::C : T, H).total;
     if (packed) return 0;
     const SegPlan sp = seg_plan(rule, B, T, H, dv);
     if (sp.nseg < 2) return 0;
@@ -319,11 +320,9 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
     const unsigned grid = (unsigned)(p.B * p.H * (p.dv / DVT));
     cudaError_t e;
     if (rule == kRuleKDA) {
-        if (packed) {
-            *err = "the chunked KDA kernels take the dense layout";
-            return 2;
-        }
-        const KdaWorkspace kw = kda_workspace(p.B, p.T, p.H);
+        const int nch = (int)((Lmax + C - 1) / C);
+        const int64_t Ls = packed ? (int64_t)nch * C : p.T;
+        const KdaWorkspace kw = kda_workspace(p.B, Ls, p.H);
         if (!ws || ws_bytes < kw.total || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
             *err = "KDA needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
             return 8;
@@ -331,7 +330,10 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         uint8_t *w8 = static_cast<uint8_t *>(ws);
         KdaPrepParams kp{};
         kp.B = p.B; kp.T = p.T; kp.H = p.H;
-        kp.nchunks = (int)((p.T + C - 1) / C);
+        kp.nchunks = nch;
+        kp.Ls = Ls;
+        kp.cu_seqlens = p.cu_seqlens;
+        kp.max_seqlen = Lmax;
         kp.q = static_cast<const __nv_bfloat16 *>(p.q);
         kp.k = static_cast<const __nv_bfloat16 *>(p.k);
         kp.alpha = p.g; kp.beta = p.beta;
@@ -340,11 +342,11 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         kp.kp = reinterpret_cast<__nv_bfloat16 *>(w8 + kw.kp);
         kp.kc = reinterpret_cast<__nv_bfloat16 *>(w8 + kw.kc);
         Maps mk = m;
-        if (!make_map_4d(&mk.q, kp.qp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, DK, 64, C,
+        if (!make_map_4d(&mk.q, kp.qp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, Ls, p.H, DK, 64, C,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map_4d(&mk.k, kp.kp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, DK, 64, C,
+            !make_map_4d(&mk.k, kp.kp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, Ls, p.H, DK, 64, C,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map_4d(&mk.kc, kp.kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, p.T, p.H, DK, 64, C,
+            !make_map_4d(&mk.kc, kp.kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, Ls, p.H, DK, 64, C,
                          CU_TENSOR_MAP_SWIZZLE_128B)) {
             *err = "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)";
             return 4;

@@ -2,10 +2,8 @@
 // kernel selection, the host-buffer entry point and the device error word.
 //
 // Kernel selection for la_fwd:
-//   bf16, dk = 128           -> chunked tensor-core kernels (chunk_tc.cuh; KDA
-//                               with the dense layout only)
-//   fp32, or bf16 with dk < 128, or packed KDA -> per-token recurrent kernel
-//                               (recurrent.cuh)
+//   bf16, dk = 128           -> chunked tensor-core kernels (chunk_tc.cuh)
+//   fp32, or bf16 with dk < 128 -> per-token recurrent kernel (recurrent.cuh)
 // la_step always uses the recurrent kernel with T = 1 and the state in place.
 // With out_norm set, a second pass normalises each (token, head) row of o
 // (out_norm.cuh).
@@ -188,10 +186,8 @@ cudaError_t allow_smem(const void *kernel, int bytes) {
 
 namespace {
 
-// Packed KDA sequences run on the recurrent kernel (the chunked KDA prep writes
-// scaled q/k tensors that a packed tail chunk would read past its sequence).
 bool uses_chunk_kernels(const la_fwd_args &a) {
-    return a.dtype == LA_BF16 && a.dk == 128 && a.T > 0 && (a.rule != LA_RULE_KDA || !a.cu_seqlens);
+    return a.dtype == LA_BF16 && a.dk == 128 && a.T > 0;
 }
 
 // Output normalisation arguments (ABI version 3), shared by la_fwd and la_step.

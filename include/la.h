@@ -79,12 +79,12 @@ typedef enum {
  *        ("线性注意力与 SSM", GDN box, in the dk x dv orientation)
  *   KDA  S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
  *        alpha_t per key channel ("状态空间与线性注意力", KDA：逐通道遗忘与误差写入).
- *        bf16 KDA with dk = 128 and the dense layout runs chunked on the tensor
+ *        bf16 KDA with dk = 128 (dense or packed) runs chunked on the tensor
  *        cores, for retention whose product over any 8 consecutive tokens stays
  *        >= 2^-60 per channel (the page's bounded log-decay, log alpha > -5,
  *        satisfies this); outside that domain la_check_device reports
- *        LA_ERR_RANGE.  fp32, dk < 128 and packed KDA run on the per-token
- *        recurrent kernel (CUDA cores), which has no such domain.
+ *        LA_ERR_RANGE.  fp32 and dk < 128 KDA run on the per-token recurrent
+ *        kernel (CUDA cores), which has no such domain.
  */
 typedef enum { LA_RULE_ELU = 0, LA_RULE_GLA = 1, LA_RULE_GDN = 2, LA_RULE_KDA = 3 } la_rule;
 
@@ -115,8 +115,10 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *          piece's state contribution and its normaliser sum or gate product).
  *          Chunked KDA keeps 16.5 KB per (batch, head, chunk) (the T and P
  *          operand images and the chunk's retention product) plus three bf16
- *          [B,T,H,128] tensors: q and k scaled by the cumulative retention, and
- *          k scaled by the retention from the token to its chunk's end.
+ *          [B,Ls,H,128] tensors: q and k scaled by the cumulative retention, and
+ *          k scaled by the retention from the token to its chunk's end (Ls = T;
+ *          with packed sequences Ls = 64 ceil(max_seqlen / 64), one row block
+ *          per sequence).
  *          Calls that share
  *          one workspace must be ordered (same stream), otherwise they race.
  *          A missing or short workspace returns LA_ERR_WORKSPACE before any launch.

@@ -8,7 +8,9 @@ library's own dense call on every sequence alone: the chunked kernels start
 chunks at each sequence's first token, so a packed run does exactly the dense
 run's arithmetic and the results must agree bit for bit.  Offsets that are out
 of order, out of range or longer than max_seqlen are clamped on the device (no
-access leaves the tensors) and reported by la_check_device.
+access leaves the tensors) and reported by la_check_device.  KDA's chunked path
+keeps its scaled q/k in one row block per sequence (the tail chunk's padding
+rows zero), so it too matches its dense calls bit for bit.
 """
 import ctypes
 
@@ -47,7 +49,7 @@ def run_packed(la, rule, packed, cu, max_seqlen):
     return o, S, z
 
 
-@pytest.mark.parametrize("rule", ["elu", "gla", "gdn"])
+@pytest.mark.parametrize("rule", ["elu", "gla", "gdn", "kda"])
 @pytest.mark.parametrize("dk,dv,dtype", [(128, 64, torch.bfloat16), (128, 128, torch.bfloat16),
                                          (32, 32, torch.float32), (64, 32, torch.bfloat16)])
 def test_packed_matches_oracle_per_sequence(la, rule, dk, dv, dtype):
@@ -65,7 +67,7 @@ def test_packed_matches_oracle_per_sequence(la, rule, dk, dv, dtype):
             assert rel_err(z[i:i + 1].cpu().numpy(), rz) <= tol, f"sequence {i}: z"
 
 
-@pytest.mark.parametrize("rule", ["elu", "gla", "gdn"])
+@pytest.mark.parametrize("rule", ["elu", "gla", "gdn", "kda"])
 def test_packed_equals_dense_calls_bitwise(la, rule):
     """Chunked tensor-core path (bf16, dk = 128): every sequence's outputs and
     final state are bit-identical to a dense call on that sequence alone."""
@@ -82,7 +84,7 @@ def test_packed_equals_dense_calls_bitwise(la, rule):
             assert torch.equal(z[i:i + 1], zd), f"sequence {i}: z differs from the dense call"
 
 
-@pytest.mark.parametrize("rule", ["gla", "gdn"])
+@pytest.mark.parametrize("rule", ["gla", "gdn", "kda"])
 def test_packed_many_sequences_full_width(la, rule):
     """Sixteen heads and 24 sequences of mixed lengths (the decode-batch shape
     of a serving prefill), checked on a few sequences."""
@@ -99,7 +101,7 @@ def test_packed_many_sequences_full_width(la, rule):
         assert rel_err(S[i:i + 1].cpu().numpy(), rS) <= TOL_BF16
 
 
-@pytest.mark.parametrize("rule", ["gla", "gdn"])
+@pytest.mark.parametrize("rule", ["gla", "gdn", "kda"])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_bad_offsets_are_clamped_and_reported(la, rule, dtype):
     """Offsets out of order and beyond T, and a sequence longer than max_seqlen:
