@@ -180,7 +180,11 @@ LEG_NAMES = ["gla_prefill", "gdn_prefill", "elu_prefill", "gla_decode", "gdn_dec
 # kernels per call: gated delta rule 2 (T operand images, then the main pass);
 # GLA and ELU+1 at these shapes 2 each (range summaries of the earlier sequence
 # segments, then the segment-parallel main pass); each decode step 1
-LEG_LAUNCHES = {"gla_prefill": 2, "gdn_prefill": 2, "elu_prefill": 2, "gla_decode": 1, "gdn_decode": 1}
+LEG_LAUNCHES = {"gla_prefill": 2, "gdn_prefill": 2, "elu_prefill": 2, "gla_decode": 1, "gdn_decode": 1,
+                "kda_prefill": 2}
+# legs that --profile-leg can run but the timed step does not: KDA prefill at the
+# prefill benchmark shape (prep kernel, then the KDA main pass)
+PROFILE_ONLY_LEGS = ["kda_prefill"]
 
 
 class Legs:
@@ -209,6 +213,11 @@ class Legs:
             self.o_elu = e(1, 32768, 16, 64, dtype=torch.bfloat16, device="cuda")
             self.S_elu = e(1, 16, 128, 64, device="cuda")
             self.z_elu = e(1, 16, 128, device="cuda")
+        if "kda_prefill" in want:
+            kda = self.host["kda"] = workloads.make_problem("kda", 2, 8192, 16, 128, 128, seed=seed)
+            self.kda = {k: dev(getattr(kda, k)) for k in ("q", "k", "v", "g", "beta")}
+            self.o_kda = e(2, 8192, 16, 128, dtype=torch.bfloat16, device="cuda")
+            self.S_kda = e(2, 16, 128, 128, device="cuda")
         if want & {"gla_decode", "gdn_decode"}:
             self.S_dec = workloads.decode_state(seed=seed).cuda()
             self.dec_gla = [x.cuda() for x in workloads.decode_steps("gla", 1, seed=seed)[0]]
@@ -224,6 +233,9 @@ class Legs:
         elif name == "gdn_prefill":
             a = self.gdn
             la.fwd("gdn", a["q"], a["k"], a["v"], a["g"], a["beta"], o=self.o_gdn, S_out=self.S_gdn)
+        elif name == "kda_prefill":
+            a = self.kda
+            la.fwd("kda", a["q"], a["k"], a["v"], a["g"], a["beta"], o=self.o_kda, S_out=self.S_kda)
         elif name == "elu_prefill":
             a = self.elu
             la.fwd("elu", a["q"], a["k"], a["v"], S0=a["S0"], z0=a["z0"], eps=1e-6, o=self.o_elu,
@@ -656,7 +668,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-leg", choices=LEG_NAMES, default=None,
+    ap.add_argument("--profile-leg", choices=LEG_NAMES + PROFILE_ONLY_LEGS, default=None,
                     help="run one leg 3 + --reps times without timing (for ncu captures)")
     ap.add_argument("--reps", type=int, default=1)
     ap.add_argument("--variants", action="store_true",
