@@ -1,20 +1,21 @@
 // chunk_gdn.cuh — gated delta rule, chunked prefill: two kernels.
 //
 // gdn_prep_kernel (fully parallel over (batch, head, chunk)): for each 64-token
-//   chunk, the state-independent triangular system of the WY / UT form:
-//     A = diag(beta) (K K^T o Gamma o strict-lower)   (K K^T on tcgen05),
+//   chunk, the state-independent parts, from one M=128 MMA [Q ; K] K^T:
+//     P = Q K^T o Gamma o M                            (rows 0-63),
+//     A = diag(beta) (K K^T o Gamma o strict-lower)    (rows 64-127),
 //     T = (I + A)^-1   (16x16 diagonal blocks by substitution, then two levels of
 //                       block merges on mma.sync tf32),
-//   and writes T as a bf16 operand image (128-byte swizzled, exactly as the main
-//   kernel's shared memory wants it) to the workspace: 8 KB per (batch, head,
-//   chunk).
+//   and writes T and P as bf16 operand images (128-byte swizzled, exactly as the
+//   main kernel's shared memory wants them) to the workspace: 16 KB per (batch,
+//   head, chunk).  Computing P here keeps Q K^T out of the main kernel's tensor
+//   pipe, where its 8 instructions would queue ahead of the recurrence's MMAs.
 //
 // chunk_gdn_kernel (one CTA per (batch, head, 32-column value slab), 9 warps):
-//   warp 0      producer: TMA loads of q, k, v and a bulk copy of the chunk's
-//               T image (3 stages); the chunk's decay factors and betas;
-//   warps 1-4   "score" group: P = (Q K^T) o Gamma o M  (tcgen05, M=64) ->
-//               bf16 tile [P ; 0] for chunk c, then, one chunk behind the state
-//               group, PW = [P ; 0] W and O = diag(gamma) X2 + PW for chunk c-1;
+//   warp 0      producer: TMA loads of q, k, v and bulk copies of the chunk's
+//               T and P images (3 stages); the chunk's decay factors and betas;
+//   warps 1-4   "output" group: as soon as the state group has W of chunk c,
+//               PW = [P ; 0] W and O = diag(gamma) X2 + PW;
 //   warps 5-8   "state" group, the recurrence across chunks.  With
 //               W = U - W_k S0 = T diag(beta) (V - diag(gamma) K S0):
 //                 [X2 ; KS] = [Q ; K] S0        (one M=128 MMA chain, S0 bf16),
@@ -42,45 +43,41 @@ namespace gdn {
 constexpr int NSTG = 3;
 constexpr int NTHREADS = 288;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM columns of the main kernel
-constexpr uint32_t C_SC = 0;     // 2 x 64, M=64  scores Q K^T
+// TMEM columns of the main kernel (columns 0-127 unused)
 constexpr uint32_t C_XK = 128;   // 2 x 32, M=128 [Q ; K] S0
 constexpr uint32_t C_W = 192;    // 32,     M=64  W = T R
 constexpr uint32_t C_DS = 224;   // 32,     M=128 dS
 constexpr uint32_t C_PW = 256;   // 2 x 32, M=128 [P ; 0] W (rows 0-63)
 
 constexpr uint32_t TT_BYTES = 8192;                  // T, bf16 [64][64]
+// Workspace item per (batch, head, chunk), written by the prep kernel: the T and
+// P operand images, bf16 [64][64], 128-byte swizzled as the main kernel's
+// shared memory wants them (KDA appends Gamma_C)
+constexpr uint32_t ITEM_T = 0;
+constexpr uint32_t ITEM_P = 8192;
+constexpr uint32_t ITEM_BYTES = 16384;
 
-// Main-kernel shared-memory tiles (byte offsets from a 1 KB aligned base).
 constexpr uint32_t QK_ACS = 128 * 128;               // one atom column: Q rows 0-63, K rows 64-127
-constexpr uint32_t STG_QK = 0;                       // NSTG x 2 atom columns
 constexpr uint32_t STG_QK_BYTES = 2 * QK_ACS;
-constexpr uint32_t STG_V = STG_QK + NSTG * STG_QK_BYTES;   // NSTG x [64][32] bf16, 64 B swizzle
-constexpr uint32_t STG_TT = STG_V + NSTG * 4096;           // NSTG x T
-constexpr uint32_t TP = STG_TT + NSTG * TT_BYTES;    // 2 x [P ; 0] [128][64] bf16 (rows 64-127 zero)
-constexpr uint32_t TR = TP + 2 * 16384;              // R       [64][32] 64 B swizzle
-constexpr uint32_t TWS = TR + 4096;                  // 2 x W
-constexpr uint32_t TWGS = TWS + 2 * 4096;            // gamma_C/gamma W
-constexpr uint32_t TSS = TWGS + 4096;                // 2 x S   [128][32] 64 B swizzle
-constexpr uint32_t TEND = TSS + 2 * 8192;
 
 }  // namespace gdn
 
 // KDA workspace item per (batch, head, chunk), written by kda_prep_kernel
-// (chunk_kda.cuh) and read by chunk_gdn_kernel<true>.
+// (chunk_kda.cuh) and read by chunk_gdn_kernel<true>: the gated delta rule's
+// item, then Gamma_C.
 namespace kda {
-constexpr uint32_t ITEM_T = 0;                 // T image, bf16 [64][64], 128-byte swizzled
-constexpr uint32_t ITEM_P = 8192;              // P image, bf16 [64][64], 128-byte swizzled
-constexpr uint32_t ITEM_GC = 16384;            // Gamma_C, fp32 [128]
+constexpr uint32_t ITEM_T = gdn::ITEM_T;      // T image
+constexpr uint32_t ITEM_P = gdn::ITEM_P;      // P image
+constexpr uint32_t ITEM_GC = 16384;           // Gamma_C, fp32 [128]
 constexpr uint32_t ITEM_BYTES = 16384 + 512;
 }  // namespace kda
 
 namespace gdn {
-// Main-kernel shared memory of chunk_gdn_kernel<KDA>.  The gated delta rule
-// uses the tiles above.  KDA (chunk_kda.cuh) loads Qp = Q o Gamma and
-// Kp = K o Gamma in place of Q and K, plus Kc = K o Gamma_C / Gamma, the P image
-// (rows 0-63 of a per-stage [P ; 0] tile) and Gamma_C with every stage, so it
-// keeps 2 stages and needs neither the score tiles nor the gamma_C/gamma W copy.
+// Main-kernel shared memory of chunk_gdn_kernel<KDA> (byte offsets from a 1 KB
+// aligned base).  Every stage holds [Q ; K] (KDA: [Qp ; Kp], plus Kc), a V slab
+// ([64][32] bf16, 64-byte swizzle), T, and the P image in rows 0-63 of a
+// [P ; 0] tile whose rows 64-127 stay zero (KDA: and Gamma_C).  KDA keeps 2
+// stages and needs no gamma_C/gamma W copy.
 template <bool KDA>
 struct GL {
     static constexpr int NSTG = KDA ? 2 : gdn::NSTG;
@@ -88,30 +85,28 @@ struct GL {
     static constexpr uint32_t STG_KC = STG_QK + NSTG * STG_QK_BYTES;            // KDA: Kc [64][128]
     static constexpr uint32_t STG_V = STG_KC + (KDA ? NSTG * 16384u : 0u);
     static constexpr uint32_t STG_TT = STG_V + NSTG * 4096u;
-    static constexpr uint32_t STG_P = STG_TT + NSTG * TT_BYTES;                 // KDA: [P ; 0]
-    static constexpr uint32_t STG_GC = STG_P + (KDA ? NSTG * 16384u : 0u);      // KDA: Gamma_C fp32 [128]
-    static constexpr uint32_t TP = STG_GC + (KDA ? 1024u : 0u);                 // GDN: 2 x [P ; 0]
-    static constexpr uint32_t TR = TP + (KDA ? 0u : 2 * 16384u);
-    static constexpr uint32_t TWS = TR + 4096;
-    static constexpr uint32_t TWGS = TWS + 2 * 4096;                            // GDN only
-    static constexpr uint32_t TSS = TWGS + (KDA ? 0u : 4096u);
+    static constexpr uint32_t STG_P = STG_TT + NSTG * TT_BYTES;                 // [P ; 0]
+    static constexpr uint32_t STG_GC = STG_P + NSTG * 16384u;                   // KDA: Gamma_C fp32 [128]
+    static constexpr uint32_t TR = STG_GC + (KDA ? 1024u : 0u);                 // R [64][32] 64 B swizzle
+    static constexpr uint32_t TWS = TR + 4096;                                  // 2 x W
+    static constexpr uint32_t TWGS = TWS + 2 * 4096;                            // GDN: gamma_C/gamma W
+    static constexpr uint32_t TSS = TWGS + (KDA ? 0u : 4096u);                  // 2 x S [128][32] 64 B swizzle
     static constexpr uint32_t TEND = TSS + 2 * 8192;
 };
-static_assert(GL<false>::TEND == TEND && GL<false>::TP == TP && GL<false>::TSS == TSS,
-              "the gated delta rule's layout is the one above");
 
 // Prep-kernel shared memory.
 constexpr int AF_LD = 68;
 constexpr int TMP_LD = 36;
-constexpr uint32_t P_K = 0;                          // K [64][128] bf16
-constexpr uint32_t P_AF = 16384;                     // A, then T, fp32 [64][AF_LD]
+constexpr uint32_t P_QK = 0;                         // [Q ; K]: 2 atom columns of 128 rows (Q 0-63, K 64-127)
+constexpr uint32_t P_AF = 2 * QK_ACS;                // A, then T, fp32 [64][AF_LD]
 constexpr uint32_t P_TMP = P_AF + 64 * AF_LD * 4;    // fp32 scratch [32][TMP_LD]
-constexpr uint32_t P_END = P_TMP + 32 * TMP_LD * 4;
+constexpr uint32_t P_END = P_TMP + 32 * TMP_LD * 4;   // the control block follows
+static_assert(P_END % 16 == 0, "the prep kernel's control block must be 16-byte aligned");
 constexpr int PREP_THREADS = 128;
 
 struct GCtl {
     uint64_t full[NSTG], empty[NSTG];
-    uint64_t l_done[2], wready[2], pw_done[2], oA[2], xk_done, w_done, ds_done, drain;
+    uint64_t wready[2], pw_done[2], oA[2], xk_done, w_done, ds_done, drain;
     uint32_t tmem_base;
     int abort, stopS, stopL[2];
     int fast[NSTG];
@@ -229,21 +224,6 @@ __device__ __forceinline__ int gate_scan(const float *al, const float *beta, flo
     }
     const float last = __shfl_sync(0xffffffffu, e1, 31);
     return last >= -120.f ? 1 : 0;
-}
-
-// Row t's 32 columns col0.. of A = diag(beta) (K K^T o Gamma o strict-lower), in
-// place: x_i <- x_i * rowf * gamma_t / gamma_i for i < t, 0 on and above the diagonal.
-__device__ __forceinline__ void decay_mask32_strict(float *x, int t, int col0, float rowf, bool fast,
-                                                    const float *gam, const float *ginv, const float *b2) {
-    if (fast) {
-        const float rs = rowf * gam[t];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = (col0 + j < t) ? x[j] * rs * ginv[col0 + j] : 0.f;
-    } else {
-        const float bt = b2[t];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = (col0 + j < t) ? x[j] * rowf * exp2f(bt - b2[col0 + j]) : 0.f;
-    }
 }
 
 // Row t of the decayed, masked score matrix from 64 raw scores x (in place):
@@ -370,23 +350,24 @@ struct GdnPrepParams {
     int64_t B, T, H;
     int nchunks;                  // chunks per (batch, head): ceil(max_seqlen / 64)
     const float *alpha, *beta;
-    uint8_t *ws;                  // [B*H*nchunks][TT_BYTES]
+    uint8_t *ws;                  // [B*H*nchunks][ITEM_BYTES]
     const int64_t *cu_seqlens;    // packed sequences, or nullptr (dense)
     int64_t max_seqlen;           // = T for the dense layout
 };
 
 // One CTA handles (batch, head, chunk) items in a grid-stride loop.  The next
-// item's K tile is loaded (TMA) as soon as this item's K K^T MMA has read the
-// buffer, and its alpha and beta are fetched into registers at the same point,
-// so neither load is waited for.  The grid is sized to the CTAs that are
-// resident at once.
+// item's [Q ; K] tile is loaded (TMA) as soon as this item's [Q ; K] K^T MMA has
+// read the buffer, and its alpha and beta are fetched into registers at the same
+// point, so neither load is waited for.  The grid is sized to the CTAs that are
+// resident at once: 4 per SM, with the control block after the tiles (no
+// rounding of it to 1 KB), 57 KB of shared memory and 128 registers per thread.
 __global__ void __launch_bounds__(gdn::PREP_THREADS, 4)
-gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p) {
+gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant__ CUtensorMap mapk,
+                const GdnPrepParams p) {
     using namespace gdn;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    PCtl *ctl = reinterpret_cast<PCtl *>(smem_raw);
-    uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(PCtl) + (smem_u32(smem_raw) & 1023u)) -
-                     (smem_u32(smem_raw) & 1023u);
+    uint8_t *tiles = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);   // 1 KB aligned
+    PCtl *ctl = reinterpret_cast<PCtl *>(tiles + P_END);
     const uint32_t tb = smem_u32(tiles);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t items = p.B * p.H * (int64_t)p.nchunks;
@@ -398,6 +379,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         mbar_init(&ctl->mma, 1);
         ctl->abort = 0;
         fence_barrier_init();
+        tma_prefetch_desc(&mapq);
         tma_prefetch_desc(&mapk);
     }
     if (warp == 0) {
@@ -409,15 +391,19 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tq = tmem + ((uint32_t)(32 * warp) << 16);
 
-    // warp 0, lane 0: TMA of item w's K tile
+    // warp 0, lane 0: TMA of item w's [Q ; K] tile (Q rows 0-63, K rows 64-127 of
+    // each 64-column atom)
     auto load_k = [&](int64_t w) {
         const int64_t bh = w / p.nchunks;
         const int c = (int)(w % p.nchunks);
         const int64_t b = bh / p.H, h = bh % p.H;
         const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, false);
-        mbar_arrive_expect_tx(&ctl->full, 2u * C * 128u);
-        for (int a = 0; a < KA; ++a)
-            tma_load_4d(tiles + P_K + a * (C * 128), &mapk, &ctl->full, 64 * a, (int)h, sq.t0 + c * C, sq.b0);
+        mbar_arrive_expect_tx(&ctl->full, 2u * KA * C * 128u);
+        for (int a = 0; a < KA; ++a) {
+            tma_load_4d(tiles + P_QK + a * QK_ACS, &mapq, &ctl->full, 64 * a, (int)h, sq.t0 + c * C, sq.b0);
+            tma_load_4d(tiles + P_QK + a * QK_ACS + 64 * 128, &mapk, &ctl->full, 64 * a, (int)h, sq.t0 + c * C,
+                        sq.b0);
+        }
     };
     // warp 0: item w's alpha, beta for tokens 2*lane, 2*lane+1 (1 and 0 past T)
     float al[2] = {1.f, 1.f}, be[2] = {0.f, 0.f};
@@ -436,7 +422,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         }
     };
 
-    constexpr uint32_t ID_KK = idesc_bf16(64, 64, false, false);
+    constexpr uint32_t ID_QK = idesc_bf16(128, 64, false, false);
     int it = 0;
     if (warp == 0 && (int64_t)blockIdx.x < items) {
         if (lane == 0) load_k(blockIdx.x);
@@ -458,12 +444,12 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         if (tid == 0) k_pending = false;
         if (warp == 0)
             ctl->fast = gate_scan(&ctl->alpha[2 * lane], ctl->beta, ctl->b2, ctl->gam, ctl->ginv, nullptr, lane);
-        if (tid == 32) {
+        if (tid == 32) {   // [Q ; K] K^T: rows 0-63 Q K^T, rows 64-127 K K^T
             tc_fence_after_sync();
-            const uint32_t kb = tb + P_K;
+            const uint32_t qk = tb + P_QK, kb = qk + 64 * 128;
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem, desc_k(kb, C * 128, kk), desc_k(kb, C * 128, kk), ID_KK, kk > 0);
+                umma_bf16(tmem, desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk), ID_QK, kk > 0);
             umma_commit(&ctl->mma);
         }
         bar_named(1, 128);
@@ -477,16 +463,34 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
             }
             fetch_gates(w + gridDim.x);
         }
-        {   // A row t = 16*warp + (lane & 15), columns 32*(lane >> 4)..
-            const int t = 16 * warp + (lane & 15), col0 = 32 * (lane >> 4);
-            float x[32];
-            tmem_ld16x2_32<32>(tq, x);
+        {   // row r = tid of the M=128 accumulator: warps 0-1 the P row of token r
+            // (inclusive mask, to the item's P image), warps 2-3 the A row of token
+            // r - 64 (strict mask, times beta, to AF)
+            const int t = tid & 63;
+            float x[64];
+            tmem_ld32(tq, *reinterpret_cast<float(*)[32]>(x));
+            tmem_ld32(tq + 32u, *reinterpret_cast<float(*)[32]>(x + 32));
             tmem_wait_ld();
-            decay_mask32_strict(x, t, col0, ctl->beta[t], ctl->fast != 0, ctl->gam, ctl->ginv, ctl->b2);
-            float *arow = AF + t * AF_LD + col0;
+            if (warp < 2) {
+                decay_mask_row<false>(x, t, t < 32 ? 32 : 64, 1.f, ctl->fast != 0, ctl->gam, ctl->ginv, ctl->b2);
+                uint8_t *dst = p.ws + w * (int64_t)ITEM_BYTES + ITEM_P + (uint32_t)t * 128u;
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(arow + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint4 u;
+                    u.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
+                    u.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
+                    u.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
+                    u.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
+                    *reinterpret_cast<uint4 *>(dst + (uint32_t)(((cc ^ t) & 7) << 4)) = u;
+                }
+            } else {
+                decay_mask_row<true>(x, t, t < 32 ? 32 : 64, ctl->beta[t], ctl->fast != 0, ctl->gam, ctl->ginv,
+                                     ctl->b2);
+                float *arow = AF + t * AF_LD;
+#pragma unroll
+                for (int i = 0; i < 64; i += 4)
+                    *reinterpret_cast<float4 *>(arow + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+            }
         }
         tc_fence_before_sync();
         bar_named(1, 128);
@@ -494,7 +498,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
         {   // T -> workspace, a 128-byte swizzled [64][64] bf16 image
             const int t = tid >> 1, hh = tid & 1;
             const float *Trow = AF + t * AF_LD + 32 * hh;
-            uint8_t *dst = p.ws + w * (int64_t)TT_BYTES;
+            uint8_t *dst = p.ws + w * (int64_t)ITEM_BYTES + ITEM_T;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
                 uint4 u;
@@ -515,21 +519,6 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapk, const GdnPrepParams p)
 
 
 
-// Row t's 32 columns col0.. of the decayed, causally masked score matrix, in
-// place: x_i <- x_i * gamma_t / gamma_i for i <= t, 0 above the diagonal.
-__device__ __forceinline__ void decay_mask32(float *x, int t, int col0, bool fast, const float *gam,
-                                             const float *ginv, const float *b2) {
-    if (fast) {
-        const float gt = gam[t];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = (col0 + j <= t) ? x[j] * gt * ginv[col0 + j] : 0.f;
-    } else {
-        const float bt = b2[t];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = (col0 + j <= t) ? x[j] * exp2f(bt - b2[col0 + j]) : 0.f;
-    }
-}
-
 // KDA = true: the KDA main pass (chunk_kda.cuh has the algebra); maps.q, maps.k
 // and maps.kc then cover the prep kernel's Qp, Kp and Kc tensors and `ws` its
 // per-chunk items (T image, P image, Gamma_C).
@@ -539,7 +528,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
     using namespace gdn;
     using L = gdn::GL<KDA>;
     constexpr int NSTG = L::NSTG;
-    constexpr uint32_t ITEM = KDA ? kda::ITEM_BYTES : TT_BYTES;   // workspace bytes per chunk
+    constexpr uint32_t ITEM = KDA ? kda::ITEM_BYTES : ITEM_BYTES;   // workspace bytes per chunk
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     GCtl *ctl = reinterpret_cast<GCtl *>(smem_raw);
     uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(GCtl) + (smem_u32(smem_raw) & 1023u)) -
@@ -564,7 +553,6 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             mbar_init(&ctl->empty[s], 2);   // the state group's and the score group's MMAs
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&ctl->l_done[i], 1);
             mbar_init(&ctl->wready[i], 128);
             mbar_init(&ctl->pw_done[i], 1);
             mbar_init(&ctl->oA[i], 128);
@@ -583,11 +571,10 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         tmem_alloc(&ctl->tmem_base, TMEM_COLS);
         tc_fence_before_sync();
     }
-    // rows 64-127 of both [P ; 0] tiles (KDA: of both stages' P tiles) stay zero
-    for (int i = tid; i < 2 * 8192 / 16; i += NTHREADS) {
+    // rows 64-127 of every stage's [P ; 0] tile stay zero
+    for (int i = tid; i < NSTG * 8192 / 16; i += NTHREADS) {
         const int tile = i / 512, off = (i % 512) * 16;
-        *reinterpret_cast<uint4 *>(tiles + (KDA ? L::STG_P : L::TP) + tile * 16384 + 8192 + off) =
-            make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(tiles + L::STG_P + tile * 16384 + 8192 + off) = make_uint4(0, 0, 0, 0);
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -595,7 +582,6 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16);   // this warp's TMEM lanes
 
-    constexpr uint32_t ID_SC = idesc_bf16(64, 64, false, false);
     constexpr uint32_t ID_XK = idesc_bf16(128, DVT, false, true);
     constexpr uint32_t ID_W = idesc_bf16(64, DVT, false, true);
     constexpr uint32_t ID_DS = idesc_bf16(128, DVT, true, true);
@@ -621,7 +607,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             const int t0 = c * C;   // position in the sequence
             if (lane == 0) {
                 mbar_expect_tx(&ctl->full[s], KDA ? 3u * KA * C * 128u + C * DVT * 2u + 2u * TT_BYTES + 512u
-                                                  : 2u * KA * C * 128u + C * DVT * 2u + TT_BYTES);
+                                                  : 2u * KA * C * 128u + C * DVT * 2u + 2u * TT_BYTES);
                 uint8_t *qk = tiles + L::STG_QK + s * STG_QK_BYTES;
                 const int tm = sq.t0 + t0;   // tensor-map coordinate of the chunk's first token
                 // q, k maps (KDA: the prep's qp, kp, kc, one row block per sequence
@@ -637,9 +623,9 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
                 }
                 tma_load_4d(tiles + L::STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, tm, sq.b0);
                 const uint8_t *item = ws + (bh * ws_chunks + c) * (int64_t)ITEM;
-                bulk_load(tiles + L::STG_TT + s * TT_BYTES, item, TT_BYTES, &ctl->full[s]);
+                bulk_load(tiles + L::STG_TT + s * TT_BYTES, item + ITEM_T, TT_BYTES, &ctl->full[s]);
+                bulk_load(tiles + L::STG_P + s * 16384, item + ITEM_P, 8192, &ctl->full[s]);
                 if (KDA) {
-                    bulk_load(tiles + L::STG_P + s * 16384, item + kda::ITEM_P, 8192, &ctl->full[s]);
                     bulk_load(tiles + L::STG_GC + s * 512, item + kda::ITEM_GC, 512, &ctl->full[s]);
                     // two stages leave about one chunk period for a load: start chunk
                     // c+1's tiles and item on their way to L2 now
@@ -688,11 +674,10 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             for (int c = (issued > NSTG ? issued - NSTG : 0); c < issued; ++c)
                 (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
     } else if (warp < 5) {
-        // ------------------------------------------------------------------ score group
+        // ------------------------------------------------------------------ output group
         const int lt = tid - 32;
         const bool leader = (lt == 0);
-        const int t = 16 * quad + (lane & 15), hf = lane >> 4;   // M=64 row, column half
-        const int ro = 32 * quad + lane;                          // M=128 row: output rows 0-63 in quads 0, 1
+        const int ro = 32 * quad + lane;   // M=128 row: output rows 0-63 in quads 0, 1
         // PW = [P ; 0] W and O = diag(gamma) X2 + PW of chunk j, X2 = rows 0-63 of [X2 ; KS]
         // (a failed wait sets the abort flag; every thread still takes every barrier)
         auto finish = [&](int j) {
@@ -704,13 +689,13 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             const float gam_o = KDA ? 1.f : ctl->gam[sj][ro & 63];
             bar_named(1, 128);
             if (leader) {
-                // KDA: P(j) came with stage j, which the state group has consumed
-                // (wready); this wait only makes the copy's completion visible to
-                // the issuing thread and returns at once (the stage cannot be
-                // refilled before PW(j) is committed below)
-                if (KDA && !mbar_wait(&ctl->full[sj], (uint32_t)(j / NSTG) & 1u)) ctl->abort = 1;
+                // P(j) came with stage j, which the state group has consumed (wready);
+                // this wait only makes the copy's completion visible to the issuing
+                // thread and returns at once (the stage cannot be refilled before
+                // PW(j) is committed below)
+                if (!mbar_wait(&ctl->full[sj], (uint32_t)(j / NSTG) & 1u)) ctl->abort = 1;
                 tc_fence_after_sync();
-                const uint32_t ps = KDA ? tb + L::STG_P + (uint32_t)sj * 16384u : tb + L::TP + (uint32_t)jb * 16384u;
+                const uint32_t ps = tb + L::STG_P + (uint32_t)sj * 16384u;
                 const uint32_t wsb = tb + L::TWS + (uint32_t)jb * 4096u;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
@@ -746,56 +731,18 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
             tc_fence_before_sync();
             mbar_arrive(&ctl->oA[jb]);
         };
-        // iteration c: P of chunk c (c < nchunks), then PW and O of chunk c-1.
-        // The stop flag alternates between two words so that the leader's write
-        // for iteration c+1 cannot reach a thread still reading iteration c's.
-        for (int c = 0; c <= nchunks; ++c) {
-            const int s = c % NSTG, pb = c & 1;
+        // one chunk per iteration, in order, each as soon as the state group has its
+        // W (P comes with the stage, so nothing else is waited for: a wait for a
+        // later stage here would hold PW, which frees that stage for a later
+        // chunk's loads).  The stop flag alternates between two words so that the
+        // leader's write for iteration j+1 cannot reach a thread still reading
+        // iteration j's.
+        for (int j = 0; j < nchunks; ++j) {
+            const int pb = j & 1;
             if (leader) ctl->stopL[pb] = ctl->abort;
             bar_named(1, 128);
             if (ctl->stopL[pb]) break;
-            if (c == nchunks) {
-                if (c >= 1) finish(c - 1);
-                break;
-            }
-            // (the P tile and score accumulator of chunk c-2 were freed by finish(c-2))
-            if constexpr (KDA) {
-                // P comes with the stage; waiting here for stage c would hold PW(c-1),
-                // which frees the stage that chunk c+1 is loaded into (two stages)
-                if (c >= 1) finish(c - 1);
-            } else {
-                if (!mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u)) ctl->abort = 1;
-                if (leader) {
-                    tc_fence_after_sync();
-                    const uint32_t qk = stage_qk(c), kb = qk + 64 * 128;
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk)
-                        umma_bf16(tmem + C_SC + 64u * pb, desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk), ID_SC, kk > 0);
-                    umma_commit(&ctl->l_done[pb]);
-                }
-                if (!mbar_wait(&ctl->l_done[pb], (uint32_t)(c >> 1) & 1u)) ctl->abort = 1;
-                tc_fence_after_sync();
-                {   // P row t, columns 32hf..32hf+31 -> bf16 rows 0-63 of [P ; 0]
-                    float x[32];
-                    tmem_ld16x2_32<32>(tq + C_SC + 64u * pb, x);
-                    tmem_wait_ld();
-                    decay_mask32(x, t, 32 * hf, ctl->fast[s] != 0, ctl->gam[s], ctl->ginv[s], ctl->b2[s]);
-                    uint8_t *ps = tiles + L::TP + pb * 16384;
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        uint4 u;
-                        u.x = pack_bf16x2(x[8 * cc + 0], x[8 * cc + 1]);
-                        u.y = pack_bf16x2(x[8 * cc + 2], x[8 * cc + 3]);
-                        u.z = pack_bf16x2(x[8 * cc + 4], x[8 * cc + 5]);
-                        u.w = pack_bf16x2(x[8 * cc + 6], x[8 * cc + 7]);
-                        const int chunk = 4 * hf + cc;
-                        *reinterpret_cast<uint4 *>(ps + t * 128 + (((chunk ^ t) & 7) << 4)) = u;
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before_sync();
-                if (c >= 1) finish(c - 1);
-            }
+            finish(j);
         }
         if (leader) umma_commit(&ctl->drain);
     } else {

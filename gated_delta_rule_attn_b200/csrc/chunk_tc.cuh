@@ -245,7 +245,7 @@ inline KdaWorkspace kda_workspace(int64_t B, int64_t T, int64_t H) {
 }
 
 // Device workspace the chunked path needs: the gated delta rule keeps the
-// per-chunk T = (I + A)^-1 operand images (8 KB per (batch, head, chunk)); KDA
+// per-chunk T = (I + A)^-1 and P operand images (16 KB per (batch, head, chunk)); KDA
 // its prep kernel's items and scaled q/k tensors; sequence-parallel ELU+1 and GLA the range
 // summaries of their first pass.  `packed`: the sequences are packed on one
 // token axis with lengths up to max_seqlen (no sequence-parallel pass then).
@@ -253,7 +253,7 @@ inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, i
                                     bool packed = false, int64_t max_seqlen = 0) {
     if (T <= 0) return 0;
     const int64_t L = packed ? max_seqlen : T;
-    if (rule == kRuleGDN) return (size_t)(B * H * ((L + ck::C - 1) / ck::C)) * ck::gdn::TT_BYTES;
+    if (rule == kRuleGDN) return (size_t)(B * H * ((L + ck::C - 1) / ck::C)) * ck::gdn::ITEM_BYTES;
     if (rule == kRuleKDA) return kda_workspace(B, packed ? (L + ck::C - 1) / ck::C * ck::C : T, H).total;
     if (packed) return 0;
     const SegPlan sp = seg_plan(rule, B, T, H, dv);
@@ -374,14 +374,15 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         pp.cu_seqlens = p.cu_seqlens; pp.max_seqlen = Lmax;
         pp.ws = static_cast<uint8_t *>(ws);
         const int64_t items = p.B * p.H * (int64_t)pp.nchunks;
-        const int psmem = (int)((sizeof(gdn::PCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::P_END;
+        // tiles (1 KB aligned from a base that may sit anywhere), then the control block
+        const int psmem = 1023 + (int)gdn::P_END + (int)((sizeof(gdn::PCtl) + 15) / 16 * 16);
         e = allow_smem((const void *)gdn_prep_kernel, psmem);
         // one wave of resident CTAs walks all items (a second, partial wave
         // would double the time)
         const int per_sm = resident_per_sm((const void *)gdn_prep_kernel, gdn::PREP_THREADS, psmem, 64);
         const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
-        if (e == cudaSuccess && items > 0) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.k, pp);
-        const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::TEND;
+        if (e == cudaSuccess && items > 0) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.q, m.k, pp);
+        const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::GL<false>::TEND;
         if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel<false>, smem);
         if (e == cudaSuccess)
             chunk_gdn_kernel<false><<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));

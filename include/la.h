@@ -107,9 +107,9 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *   workspace / workspace_bytes: device scratch of at least
  *          la_fwd_workspace_size() bytes, 16-byte aligned (may be NULL when that
  *          size is 0).  The gated delta rule on the tensor-core path (bf16,
- *          dk = 128) needs 8 KB per (batch, head, 64-token chunk): the chunk's
- *          T = (I + A)^-1 operand, written by a first kernel and read by the
- *          second within the same call.  ELU+1 and GLA over few heads and long
+ *          dk = 128) needs 16 KB per (batch, head, 64-token chunk): the chunk's
+ *          T = (I + A)^-1 and masked, decayed score operands, written by a first
+ *          kernel and read by the second within the same call.  ELU+1 and GLA over few heads and long
  *          sequences run segment-parallel and keep there the summary of each
  *          piece of every segment but the last (dk*dv + dk floats per piece: the
  *          piece's state contribution and its normaliser sum or gate product).
@@ -251,8 +251,8 @@ la_status la_fwd_host(const la_fwd_args *host_args, void *staging, size_t stagin
  *
  *   - The problem's scratch need (la_fwd_workspace_size) must be at most
  *     LA_NOALLOC_SCRATCH_BYTES, otherwise LA_ERR_WORKSPACE is returned before
- *     anything is launched.  For the gated delta rule that is 2048
- *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 8192.
+ *     anything is launched.  For the gated delta rule that is 1024
+ *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 4096.
  *     KDA is the exception: a KDA problem whose chunked scratch does not fit
  *     runs on the per-token recurrent kernel, which needs none (slower, same
  *     results within the bf16 tolerance).
