@@ -14,7 +14,10 @@ headers, not from the kernels:
   cumulative retention Gamma, and the pairwise factors Gamma_t / Gamma_i formed
   as the KDA prep kernel forms them: per 16-token sub-chunk, relative to its
   middle token, from products of alpha and one reciprocal, with the
-  cross-sub-chunk factors as products of sub-chunk products.
+  cross-sub-chunk factors as products of sub-chunk products;
+* GLA (page "Linear / RNN 路线", §2.2): Qt = Q o gamma, Kt = K / gamma with gamma
+  the cumulative gate inside the chunk, and the segment summaries (D, dS) of the
+  segment-parallel two-pass prefill folded in order; ELU+1 (§2.1): segment sums.
 
 A dropped term, a wrong reference token or a transposed operand in these
 derivations makes the chunked result differ from the recurrence by far more
@@ -179,3 +182,88 @@ def test_kda_subchunk_factors_recover_pairwise_decay():
             a, s = t // SUB, i // SUB
             mid = np.ones(4) if s == a else U[s] * np.prod(L[s + 1:a], axis=0) * D[a]
             np.testing.assert_allclose(G[t] * Hh[i] * mid, gam[t] / gam[i], rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# GLA and ELU+1: the chunk form and the segment summaries of the two-pass,
+# segment-parallel prefill (page "Linear / RNN 路线", §2.1 and §2.2: over a range
+# of tokens both recurrences are affine in the state entering it)
+# ---------------------------------------------------------------------------
+
+def gla_chunked(q, k, v, g, S0):
+    """gamma_t = prod_{s<=t} g_s inside the chunk (per key dim); Qt = Q o gamma,
+    Kt = K / gamma; O = Qt S0 + ((Qt Kt^T) o M) V; S <- diag(gamma_C)(S0 + Kt^T V)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    S_out = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else S0[b, h].copy()
+            for c0 in range(0, T, C):
+                n = min(C, T - c0)
+                Q, K, V = (_chunk(x, b, h, c0, n, 0.0, x.shape[-1]) for x in (q, k, v))
+                G = _chunk(g, b, h, c0, n, 1.0, dk)
+                gam = np.cumprod(G, axis=0)
+                Qt, Kt = Q * gam, K / gam
+                O = Qt @ S + np.tril(Qt @ Kt.T) @ V
+                S = gam[-1][:, None] * (S + Kt.T @ V)
+                o[b, c0:c0 + n, h] = O[:n]
+            S_out[b, h] = S
+    return o, S_out
+
+
+def gla_segment_summary(k, v, g):
+    """(D, dS) of a token range: S_end = diag(D) S_in + dS with D = prod g and
+    dS = sum_t diag(prod_{s>t} g_s) k_t v_t^T, walked backwards as the first pass
+    walks it (every factor <= 1)."""
+    L, dk = k.shape
+    R = np.ones(dk)
+    dS = np.zeros((dk, v.shape[-1]))
+    for t in range(L - 1, -1, -1):
+        dS += (R * k[t])[:, None] * v[t][None, :]
+        R = R * g[t]
+    return R, dS
+
+
+@pytest.mark.parametrize("T", [1, 37, 64, 200])
+def test_gla_chunk_form_equals_recurrence(T):
+    p = workloads.make_problem("gla", 2, T, 2, 16, 8, seed=T + 3, init_state="normal")
+    ro, rS, _ = oracle.fwd(p)
+    o, S = gla_chunked(*(_f64(x) for x in (p.q, p.k, p.v, p.g, p.S0)))
+    assert _rel(o, ro) < 1e-12 and _rel(S, rS) < 1e-12
+
+
+@pytest.mark.parametrize("cuts", [(100,), (64, 128), (7, 150, 151)])
+def test_gla_segments_fold_to_the_recurrence(cuts):
+    """Summaries of every segment but the last, folded in order (S <- D o S + dS),
+    give each segment's initial state; running each segment from it reproduces
+    the whole-sequence outputs and final state."""
+    T = 200
+    p = workloads.make_problem("gla", 1, T, 1, 16, 8, seed=11, init_state="normal")
+    q, k, v, g, S0 = (_f64(x) for x in (p.q, p.k, p.v, p.g, p.S0))
+    ro, rS, _ = oracle.fwd(p)
+    edges = (0,) + tuple(cuts) + (T,)
+    S = S0[0, 0].copy()
+    for a, b_ in zip(edges[:-1], edges[1:]):
+        sub = lambda x: x[:, a:b_]
+        o, _ = gla_chunked(sub(q), sub(k), sub(v), sub(g), S[None, None])
+        assert _rel(o, ro[:, a:b_]) < 1e-12
+        D, dS = gla_segment_summary(k[0, a:b_, 0], v[0, a:b_, 0], g[0, a:b_, 0])
+        S = D[:, None] * S + dS
+    assert _rel(S[None, None], rS) < 1e-12
+
+
+def test_elu_segments_fold_to_the_recurrence():
+    """ELU+1: a range adds phi(K)^T V to S and sum phi(k) to z; folding the
+    segment sums in order gives the final (S, z) of the recurrence."""
+    T = 150
+    p = workloads.make_problem("elu", 1, T, 1, 16, 8, seed=12, init_state="abs")
+    ro, rS, rz = oracle.fwd(p)
+    k, v = _f64(p.k)[0, :, 0], _f64(p.v)[0, :, 0]
+    phi = np.where(k > 0, k + 1.0, np.exp(k))
+    S, z = _f64(p.S0)[0, 0].copy(), _f64(p.z0)[0, 0].copy()
+    for a, b_ in ((0, 40), (40, 41), (41, 150)):
+        S = S + phi[a:b_].T @ v[a:b_]
+        z = z + phi[a:b_].sum(axis=0)
+    assert _rel(S[None, None], rS) < 1e-12 and _rel(z[None, None], rz) < 1e-12
