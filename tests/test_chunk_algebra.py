@@ -267,3 +267,48 @@ def test_elu_segments_fold_to_the_recurrence():
         S = S + phi[a:b_].T @ v[a:b_]
         z = z + phi[a:b_].sum(axis=0)
     assert _rel(S[None, None], rS) < 1e-12 and _rel(z[None, None], rz) < 1e-12
+
+
+def gdn_one_mma_chain(q, k, v, alpha, beta, S0):
+    """The gated delta rule with the state-dependent work of a chunk reduced to
+    products with S0 whose other factors are precomputable per chunk:
+      U = T diag(beta) V,  W_k = T diag(beta gamma) K,  (W = U - W_k S0)
+      G = K^T diag(gamma_C/gamma) W_k,  D = K^T diag(gamma_C/gamma) U,
+      S <- gamma_C S0 + D - G S0,
+      O = (diag(gamma) Q - P W_k) S0 + P U,  P = (Q K^T) o Gamma o M."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    S_out = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else S0[b, h].copy()
+            for c0 in range(0, T, C):
+                n = min(C, T - c0)
+                Q, K, V = (_chunk(x, b, h, c0, n, 0.0, x.shape[-1]) for x in (q, k, v))
+                al = _chunk(alpha[..., None], b, h, c0, n, 1.0, 1)[:, 0]
+                be = _chunk(beta[..., None], b, h, c0, n, 0.0, 1)[:, 0]
+                gam = np.cumprod(al)
+                Gam = np.tril(gam[:, None] / gam[None, :])
+                Tm = np.linalg.inv(np.eye(C) + be[:, None] * np.tril(K @ K.T * Gam, -1))
+                U = Tm @ (be[:, None] * V)
+                Wk = Tm @ ((be * gam)[:, None] * K)
+                Kd = (gam[-1] / gam)[:, None] * K
+                G, D = Kd.T @ Wk, Kd.T @ U
+                P = Q @ K.T * Gam
+                Qe = gam[:, None] * Q - P @ Wk
+                O = Qe @ S + P @ U
+                S = gam[-1] * S + D - G @ S
+                o[b, c0:c0 + n, h] = O[:n]
+            S_out[b, h] = S
+    return o, S_out
+
+
+@pytest.mark.parametrize("T", [1, 37, 130])
+def test_gdn_one_mma_chain_form_equals_recurrence(T):
+    """The chain form proposed as the next gated-delta kernel (one MMA per chunk
+    on the recurrence) is exact."""
+    p = workloads.make_problem("gdn", 2, T, 2, 16, 8, seed=T + 5, init_state="normal")
+    ro, rS, _ = oracle.fwd(p)
+    o, S = gdn_one_mma_chain(*(_f64(x) for x in (p.q, p.k, p.v, p.g, p.beta, p.S0)))
+    assert _rel(o, ro) < 1e-12 and _rel(S, rS) < 1e-12
