@@ -312,3 +312,67 @@ def test_gdn_one_mma_chain_form_equals_recurrence(T):
     ro, rS, _ = oracle.fwd(p)
     o, S = gdn_one_mma_chain(*(_f64(x) for x in (p.q, p.k, p.v, p.g, p.beta, p.S0)))
     assert _rel(o, ro) < 1e-12 and _rel(S, rS) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Rounding model: bf16 wherever a tensor-core operand is read, fp32 for the
+# accumulators and the carried state (the precision of the kernels), for the
+# gated delta rule's current chain and for the one-MMA chain above
+# ---------------------------------------------------------------------------
+
+def _bf(x):
+    import torch
+    return torch.from_numpy(np.asarray(x, np.float32)).bfloat16().float().numpy().astype(np.float64)
+
+
+def _f32(x):
+    return np.asarray(x, np.float32).astype(np.float64)
+
+
+def gdn_rounded(q, k, v, alpha, beta, one_mma):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    S_out = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv))
+            for c0 in range(0, T, C):
+                n = min(C, T - c0)
+                Q, K, V = (_chunk(x, b, h, c0, n, 0.0, x.shape[-1]) for x in (q, k, v))
+                al = _chunk(alpha[..., None], b, h, c0, n, 1.0, 1)[:, 0]
+                be = _chunk(beta[..., None], b, h, c0, n, 0.0, 1)[:, 0]
+                gam = _f32(np.cumprod(al))
+                Gam = np.tril(gam[:, None] / gam[None, :])
+                Tm = _f32(np.linalg.inv(np.eye(C) + be[:, None] * np.tril(_f32(K @ K.T) * Gam, -1)))
+                P = _bf(_f32(Q @ K.T) * Gam)
+                Sb = _bf(S)
+                if not one_mma:   # [Q ; K] S0 -> R -> W = T R -> dS (the kernels of this library)
+                    R = _bf(be[:, None] * (V - gam[:, None] * _f32(K @ Sb)))
+                    W = _f32(_bf(Tm) @ R)
+                    O = gam[:, None] * _f32(Q @ Sb) + _f32(P @ _bf(W))
+                    S = _f32(gam[-1] * S + _f32(K.T @ _bf(W * (gam[-1] / gam)[:, None])))
+                else:             # S <- gamma_C S + D - G S,  O = Qe S + P U
+                    U = _f32(Tm @ (be[:, None] * V))
+                    Wk = _f32(Tm @ ((be * gam)[:, None] * K))
+                    Kd = _bf((gam[-1] / gam)[:, None] * K)
+                    G, D = _bf(_f32(Kd.T @ _bf(Wk))), _f32(Kd.T @ _bf(U))
+                    Qe = _bf(gam[:, None] * Q - _f32(P @ _bf(Wk)))
+                    O = _f32(Qe @ Sb) + _f32(P @ _bf(U))
+                    S = _f32(gam[-1] * S + D - _f32(G @ Sb))
+                o[b, c0:c0 + n, h] = _bf(O)[:n]
+            S_out[b, h] = S
+    return o, S_out
+
+
+@pytest.mark.parametrize("alpha", ["sigmoid3", "ones"])
+def test_gdn_chain_forms_meet_the_bf16_bound_under_the_rounding_model(alpha):
+    """Both chain forms stay well inside the bf16 bound (2e-2) at d = 128 over 16
+    chunks: the current one (the GPU measures 4.4-5.4e-3 on this workload) and
+    the one-MMA form, whose bf16 G multiplies the state every chunk."""
+    p = workloads.make_problem("gdn", 1, 1024, 1, 128, 128, seed=4, gdn_alpha=alpha)
+    ro, rS, _ = oracle.fwd(p)
+    args = [_f64(x) for x in (p.q, p.k, p.v, p.g, p.beta)]
+    for one_mma in (False, True):
+        o, S = gdn_rounded(*args, one_mma)
+        assert _rel(o, ro) < 1e-2 and _rel(S, rS) < 1e-2, (one_mma, _rel(o, ro), _rel(S, rS))
