@@ -2,8 +2,8 @@
  * la.h — C ABI of the B200 (sm_100a) causal linear-attention library.
  *
  * The library computes the causal linear-attention forward that folds a
- * sequence into a fixed dk x dv matrix state per (batch, head), for three
- * update rules:
+ * sequence into a fixed dk x dv matrix state per (batch, head), for these
+ * update rules (KDA, the fourth, is described with la_rule below):
  *
  *   LA_RULE_ELU  normalized ELU+1 linear attention
  *       S_t = S_{t-1} + phi(k_t) v_t^T,  z_t = z_{t-1} + phi(k_t),
@@ -26,11 +26,15 @@
  *            optional initial state, all outputs and the final state returned).
  *   la_step  one decode token per sequence, state updated in place.
  *   la_fwd_host  la_fwd on HOST buffers: copies in, runs, copies out.
+ *   la_fwd_noalloc  la_fwd with a library-owned scratch array (no allocation).
+ *   la_check_device  reads and clears the device-side error word.
  *
  * Conventions (all entry points)
  *   - Layouts are dense row-major: q,k [B,T,H,dk]; v,o [B,T,H,dv]; GLA gate
- *     [B,T,H,dk] fp32; GDN alpha,beta [B,T,H] fp32; state [B,H,dk,dv] fp32 with
- *     rows = key dims; ELU normaliser z [B,H,dk] fp32.  Decode drops the T axis.
+ *     [B,T,H,dk] fp32; GDN alpha,beta [B,T,H] fp32; KDA alpha [B,T,H,dk] and
+ *     beta [B,T,H] fp32; state [B,H,dk,dv] fp32 with rows = key dims; ELU
+ *     normaliser z [B,H,dk] fp32.  Decode drops the T axis.  Packed sequences
+ *     (la_fwd_args.cu_seqlens) put the token tensors on one axis [1,T,H,*].
  *   - Device pointers must be 16-byte aligned.  The library reads and writes
  *     only the buffers it is given, never allocates or frees device memory,
  *     never synchronises the stream (except la_check_device / la_fwd_host,
@@ -40,9 +44,10 @@
  *     NULL = the legacy default stream) and returns immediately.  Arguments are
  *     validated on the host before any launch; an invalid call launches nothing.
  *   - Conditions detected on the device (a bounded wait that ran out, a GLA
- *     chunk whose cumulative gate leaves the fp32 range, packed-sequence
- *     offsets that are out of order or out of range) set a device-wide error
- *     word; la_check_device() reads and clears it.
+ *     chunk whose cumulative gate or a KDA sub-chunk whose retention product
+ *     leaves the chunked kernels' range, packed-sequence offsets that are out
+ *     of order or out of range) set a device-wide error word;
+ *     la_check_device() reads and clears it.
  *   - Supported sizes: dk, dv in {32, 64, 128}; B, H >= 1; T >= 0.  T == 0
  *     writes S_out = S0 (or zeros) and z_out = z0 (or zeros).
  *   - There is no CPU fallback: every result comes from a CUDA kernel.
@@ -272,8 +277,10 @@ la_status la_fwd_noalloc(const la_fwd_args *args, void *stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device error word set by
- * earlier kernels.  Returns LA_OK, LA_ERR_TIMEOUT, LA_ERR_RANGE or LA_ERR_CUDA.
- * `flags` (may be NULL) receives the raw word (bit 0 timeout, bit 1 range).
+ * earlier kernels.  Returns LA_OK, LA_ERR_TIMEOUT, LA_ERR_RANGE,
+ * LA_ERR_INVALID_ARG (packed-sequence offsets that had to be clamped) or
+ * LA_ERR_CUDA.  `flags` (may be NULL) receives the raw word (bit 0 timeout,
+ * bit 1 range, bit 2 clamped offsets).
  */
 la_status la_check_device(void *stream, uint32_t *flags);
 
