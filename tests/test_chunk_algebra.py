@@ -376,3 +376,16 @@ def test_gdn_chain_forms_meet_the_bf16_bound_under_the_rounding_model(alpha):
     for one_mma in (False, True):
         o, S = gdn_rounded(*args, one_mma)
         assert _rel(o, ro) < 1e-2 and _rel(S, rS) < 1e-2, (one_mma, _rel(o, ro), _rel(S, rS))
+
+
+def test_kda_benchmark_workload_is_inside_the_chunked_domain():
+    """The chunked KDA kernel needs every 8-token retention product (the halves of
+    each 16-token sub-chunk, aligned at multiples of 8 in a dense sequence) to be
+    >= 2^-60 per channel.  The benchmark's KDA workload (B=2 H=16 T=8192 d=128,
+    seed 0) satisfies it with margin, so its timing never runs into the range
+    report."""
+    p = workloads.make_problem("kda", 2, 8192, 16, 128, 128, seed=0)
+    la = np.log2(p.g.double().numpy())                      # [B, T, H, dk]
+    halves = la.reshape(2, 8192 // 8, 8, 16, 128).sum(axis=2)
+    assert halves.min() >= -60.0
+    assert halves.min() < -20.0   # the decay is strong: the sub-chunk factors matter
