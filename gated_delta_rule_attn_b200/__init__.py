@@ -24,10 +24,10 @@ STATUS = {0: "LA_OK", 1: "LA_ERR_INVALID_ARG", 2: "LA_ERR_UNSUPPORTED", 3: "LA_E
           4: "LA_ERR_CUDA", 5: "LA_ERR_TIMEOUT", 6: "LA_ERR_RANGE", 7: "LA_ERR_INTERNAL",
           8: "LA_ERR_WORKSPACE"}
 
-# Symbols include/la.h declares (checked by the CPU test suite).
+# Symbols include/la.h and include/la_testing.h declare (checked by the CPU test suite).
 EXPORTS = ("la_fwd", "la_fwd_workspace_size", "la_step", "la_fwd_host_staging_size",
            "la_fwd_host", "la_check_device", "la_status_string", "la_last_error_message",
-           "la_abi_version", "la_fwd_noalloc")
+           "la_abi_version", "la_fwd_noalloc", "la_testing_set_wait_limit")
 
 
 class LAError(RuntimeError):
@@ -78,6 +78,8 @@ def lib():
         L.la_fwd_host.argtypes = [ctypes.POINTER(FwdArgs), P, ctypes.c_size_t, P]
         L.la_check_device.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
         L.la_fwd_noalloc.argtypes = [ctypes.POINTER(FwdArgs), P]
+        L.la_testing_set_wait_limit.argtypes = [ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
+        L.la_testing_set_wait_limit.restype = ctypes.c_int
         L.la_status_string.argtypes = [ctypes.c_int]
         L.la_status_string.restype = ctypes.c_char_p
         L.la_last_error_message.restype = ctypes.c_char_p

@@ -24,7 +24,7 @@ FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + [os.path.join(ROOT, "include", "la.h")])
+                  + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

@@ -232,10 +232,11 @@ chunk_agg_kernel(const __grid_constant__ Maps maps, const AggParams p) {
         umma_commit(&ctl->done);
         if (ctl->abort)   // let copies still in flight land before the CTA exits
             for (int c = (issued - NSTG + 1 > 0 ? issued - NSTG + 1 : 0); c <= issued; ++c)
-                (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
+                (void)mbar_drain(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
     }
     if (warp < 4) {   // dS rows out: thread d = key dim
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&ctl->done, 0u));
+        // the long limit: TMEM is released below, so every MMA must have finished
+        const bool ok = __all_sync(0xffffffffu, mbar_drain(&ctl->done, 0u));
         tc_fence_after_sync();
         const int d = 32 * warp + lane;
         const uint32_t tq = tmem + ((uint32_t)(32 * warp) << 16);

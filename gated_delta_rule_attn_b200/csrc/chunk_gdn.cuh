@@ -116,7 +116,7 @@ struct GCtl {
 };
 
 struct PCtl {
-    uint64_t full, mma;
+    uint64_t full, mma, drain;
     uint32_t tmem_base;
     int abort, stop, fast;
     float alpha[64], beta[64];
@@ -377,6 +377,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
     if (tid == 0) {
         mbar_init(&ctl->full, 1);
         mbar_init(&ctl->mma, 1);
+        mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_barrier_init();
         tma_prefetch_desc(&mapq);
@@ -511,9 +512,16 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
         }
         bar_named(1, 128);   // AF and the gates are reused by the next item
     }
-    // let a prefetched copy land before the CTA exits
-    if (tid == 0 && k_pending) (void)mbar_wait(&ctl->full, (uint32_t)it & 1u);
+    // let a prefetched copy land and every MMA finish before the CTA frees TMEM
+    // and exits (these two waits keep the long limit even after a timeout)
+    if (tid == 0 && k_pending) (void)mbar_drain(&ctl->full, (uint32_t)it & 1u);
+    if (tid == 32) {
+        umma_commit(&ctl->drain);
+        (void)mbar_drain(&ctl->drain, 0u);
+    }
+    tc_fence_before_sync();
     __syncthreads();
+    tc_fence_after_sync();
     if (warp == 0) tmem_dealloc(tmem, 64);
 }
 
@@ -672,7 +680,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         // let copies still in flight land before the CTA can exit
         if (lane == 0)
             for (int c = (issued > NSTG ? issued - NSTG : 0); c < issued; ++c)
-                (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
+                (void)mbar_drain(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
     } else if (warp < 5) {
         // ------------------------------------------------------------------ output group
         const int lt = tid - 32;
@@ -897,7 +905,7 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
         }
         if (leader) {   // every MMA issued by either group has finished before TMEM is released
             umma_commit(&ctl->drain);
-            (void)mbar_wait(&ctl->drain, 0u);
+            (void)mbar_drain(&ctl->drain, 0u);
         }
         if (!ctl->abort && p.S_out) {
             float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVT);

@@ -300,7 +300,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         // after an abort, let gate copies still in flight land before the CTA can exit
         if (kGLA && leader)
             for (int c = g_used + 1; c <= g_issued; ++c)
-                (void)mbar_wait(&ctl->gfull[c % L::NG], (uint32_t)(c / L::NG) & 1u);
+                (void)mbar_drain(&ctl->gfull[c % L::NG], (uint32_t)(c / L::NG) & 1u);
     } else if (warp < 12) {
         // ------------------------------------------------------------------ group A
         const bool a0 = (tid == 256);
@@ -418,9 +418,9 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         }
         if (a0 && ctl->abort) {   // let copies still in flight land before the CTA exits
             for (int c = (issued - NSTG + 1 > 0 ? issued - NSTG + 1 : 0); c <= issued; ++c)
-                (void)mbar_wait(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
+                (void)mbar_drain(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
             for (int c = (issued_v - L::NV + 1 > 0 ? issued_v - L::NV + 1 : 0); c <= issued_v; ++c)
-                (void)mbar_wait(&ctl->vfull[c % L::NV], (uint32_t)(c / L::NV) & 1u);
+                (void)mbar_drain(&ctl->vfull[c % L::NV], (uint32_t)(c / L::NV) & 1u);
         }
     } else if (warp < 16) {
         // ------------------------------------------------------------------ group B
@@ -601,7 +601,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         }
         // every MMA issued so far has finished before TMEM is released
         umma_commit(&ctl->drain);
-        (void)mbar_wait(&ctl->drain, 0u);
+        (void)mbar_drain(&ctl->drain, 0u);
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);

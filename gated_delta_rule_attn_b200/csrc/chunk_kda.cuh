@@ -69,7 +69,7 @@ constexpr float kDown = 5.421010862427522e-20f;        // 2^-64
 }  // namespace kda
 
 struct KCtl {
-    uint64_t mma;
+    uint64_t mma, drain;
     uint32_t tmem_base;
     int abort, stop;
     // per sub-chunk and key channel: the product of alpha over its tokens up to
@@ -132,6 +132,7 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
 
     if (tid == 0) {
         mbar_init(&ctl->mma, 1);
+        mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_barrier_init();
     }
@@ -356,7 +357,15 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
         }
         bar_named(1, 128);   // AF aliases [Qs ; Ks], which the next item rewrites
     }
+    // every MMA has finished before TMEM is released (a long wait even after a
+    // timeout ended the loop)
+    if (tid == 0) {
+        umma_commit(&ctl->drain);
+        (void)mbar_drain(&ctl->drain, 0u);
+    }
+    tc_fence_before_sync();
     __syncthreads();
+    tc_fence_after_sync();
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 

@@ -82,18 +82,60 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Spin limit for every wait in this library: about one second at boost clock.
 constexpr long long kWaitLimitCycles = 2000000000LL;
 
-// Bounded wait on an mbarrier phase.  Returns false (and raises kErrTimeout) if
-// the phase did not complete within kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// The limit ordinary waits use, in constant memory (a cached read per wait).  It
+// is kWaitLimitCycles unless the library's testing hook (la_testing_set_wait_limit)
+// shortened it so that a test makes waits run out and exercises the abort paths.
+// A suspended try_wait may sleep until its phase completes, so a shortened limit
+// is enforced by non-blocking polls instead.  Drain waits, which guard the
+// release of TMEM and the exit of a CTA with copies in flight, always keep
+// kWaitLimitCycles.
+__constant__ long long g_wait_limit = kWaitLimitCycles;
+
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, long long limit) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             raise_error(kErrTimeout);
             return false;
         }
     }
     return true;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false (and raises kErrTimeout) if
+// the phase did not complete within g_wait_limit cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_test(bar, parity)) return true;   // the phase is done: no limit needed
+    const long long limit = g_wait_limit;
+    if (limit >= kWaitLimitCycles) return mbar_wait_for(bar, parity, limit);
+    const long long t0 = clock64();
+    while (!mbar_test(bar, parity)) {
+        if (clock64() - t0 > limit) {
+            raise_error(kErrTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+// Wait for asynchronous work this CTA issued (copies, MMAs) before it frees the
+// resources that work uses; bounded by kWaitLimitCycles whatever g_wait_limit is.
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_for(bar, parity, kWaitLimitCycles);
 }
 
 // ---------------------------------------------------------------------------

@@ -19,6 +19,7 @@
 #include <string>
 
 #include "la.h"
+#include "la_testing.h"
 #include "device.cuh"
 #include "recurrent.cuh"
 #include "chunk_tc.cuh"
@@ -330,26 +331,69 @@ la_status la_fwd(const la_fwd_args *in, void *stream) {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
+// The array's device address in the calling thread's current CUDA context,
+// cached per context.  A context is named by its driver-assigned ID
+// (cuCtxGetId), which is never reused within a process: after
+// cudaDeviceReset, or under a context the caller created, the address is
+// looked up again instead of reusing one from a context that no longer holds
+// the array.  Without the driver entry points the address is looked up on every
+// call (cudaGetSymbolAddress allocates nothing).
 std::mutex g_noalloc_mu;
-constexpr int kMaxDevices = 256;
-void *g_noalloc_ptr[kMaxDevices] = {};
+constexpr int kNoallocCache = 64;
+struct NoallocEntry {
+    unsigned long long ctx_id;
+    void *ptr;
+};
+NoallocEntry g_noalloc_cache[kNoallocCache];
+int g_noalloc_used = 0, g_noalloc_next = 0;
 
-// Device address of g_noalloc_scratch on the current device (looked up once
-// per device; the host-side symbol itself is not a device address).
+using PfnCtxGetCurrent = CUresult (*)(CUcontext *);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long *);
+
+void *driver_fn(const char *name) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return p;
+}
+
+// ID of the calling thread's current context (false if it cannot be read).
+bool current_context_id(unsigned long long *id) {
+    static PfnCtxGetCurrent get_current = nullptr;
+    static PfnCtxGetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        get_current = reinterpret_cast<PfnCtxGetCurrent>(driver_fn("cuCtxGetCurrent"));
+        get_id = reinterpret_cast<PfnCtxGetId>(driver_fn("cuCtxGetId"));
+    });
+    CUcontext ctx = nullptr;
+    return get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+           get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 la_status noalloc_scratch(void **out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return fail(LA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return fail(LA_ERR_UNSUPPORTED, "device ordinal out of range");
+    // no context current yet (the runtime binds the primary one lazily): the
+    // lookup below binds it, and the next call finds it named
+    unsigned long long id = 0;
+    const bool named = current_context_id(&id);
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess || !p)
-            return fail(LA_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
-        g_noalloc_ptr[dev] = p;
+    if (named)
+        for (int i = 0; i < g_noalloc_used; ++i)
+            if (g_noalloc_cache[i].ctx_id == id) {
+                *out = g_noalloc_cache[i].ptr;
+                return LA_OK;
+            }
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+        return fail(LA_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    if (named) {
+        const int slot = g_noalloc_used < kNoallocCache ? g_noalloc_used++ : (g_noalloc_next++ % kNoallocCache);
+        g_noalloc_cache[slot] = NoallocEntry{id, p};
     }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return LA_OK;
 }
 }  // namespace
@@ -561,5 +605,14 @@ const char *la_status_string(la_status s) {
 const char *la_last_error_message(void) { return g_last_error.c_str(); }
 
 int la_abi_version(void) { return LA_ABI_VERSION; }
+
+la_status la_testing_set_wait_limit(int64_t cycles, int64_t *previous) {
+    long long prev = 0, next = cycles > 0 ? (long long)cycles : la::kWaitLimitCycles;
+    cudaError_t e = cudaMemcpyFromSymbol(&prev, la::g_wait_limit, sizeof(prev));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(la::g_wait_limit, &next, sizeof(next));
+    if (e != cudaSuccess) return fail(LA_ERR_CUDA, std::string("wait limit: ") + cudaGetErrorString(e));
+    if (previous) *previous = (int64_t)prev;
+    return ok();
+}
 
 }  // extern "C"

@@ -258,17 +258,24 @@ la_status la_fwd_host(const la_fwd_args *host_args, void *staging, size_t stagin
  *     LA_NOALLOC_SCRATCH_BYTES, otherwise LA_ERR_WORKSPACE is returned before
  *     anything is launched.  For the gated delta rule that is 1024
  *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 4096.
+ *     ELU+1 and GLA use the array when they split long sequences of few heads
+ *     into segments (the segment summaries, dk*dv + dk floats per piece); the
+ *     number of pieces is bounded by the SM count, so that need always fits.
  *     KDA is the exception: a KDA problem whose chunked scratch does not fit
  *     runs on the per-token recurrent kernel, which needs none (slower, same
  *     results within the bf16 tolerance).
- *   - The first call on a device looks up the array's device address there
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.  Later calls on the device reuse the address.
+ *   - The array's device address is looked up (cudaGetSymbolAddress) in the
+ *     calling thread's current CUDA context on the first call made under that
+ *     context and reused by later calls under it; a new context (another
+ *     device, a context the caller created, or the primary context again after
+ *     cudaDeviceReset) gets its own lookup.  Make the first call under a
+ *     context before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents; the
  *     kernels write every scratch byte they read within the same call, so no
  *     clearing is needed.  Calls that overlap on the GPU (different streams
- *     without ordering, or several host threads) race on the array: serialise
- *     them.
+ *     without ordering, or several host threads) race on the array, for every
+ *     rule that uses it (the gated delta rule, KDA, segment-parallel ELU+1 and
+ *     GLA): serialise them.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  * Otherwise identical to la_fwd (validation, status codes, asynchrony).
  */

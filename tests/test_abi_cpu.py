@@ -1,10 +1,11 @@
 """Host-side checks of the C ABI (no GPU needed, no kernel launched).
 
-* the library loads and exports every function ``include/la.h`` declares;
+* the library loads and exports every function ``include/*.h`` declares;
 * invalid arguments are rejected on the host with the documented status codes
   before anything is launched (the pointers below are never dereferenced).
 """
 import ctypes
+import glob
 import os
 import re
 
@@ -23,7 +24,7 @@ def L():
 
 
 def declared_functions():
-    text = open(os.path.join(ROOT, "include", "la.h")).read()
+    text = "".join(open(p).read() for p in sorted(glob.glob(os.path.join(ROOT, "include", "*.h"))))
     return sorted(set(re.findall(r"^\s*(?:la_status|const char \*|int)\s*(la_\w+)\s*\(", text, re.M)))
 
 
