@@ -8,15 +8,17 @@ its exact output.  The library normalises its stored (bf16-rounded for bf16
 problems) output and rounds once more.  The state is not touched by the
 normalisation: it must equal, bit for bit, the state of the same call without it.
 
-Bound.  The output bound (max|o - o_ref| / max|o_ref|) applies to the output
-before normalisation, checked on the same call without ``out_norm``.  Dividing a
-row by its RMS sigma multiplies that row's absolute error by about
-(1 + max|o_row| / sigma) / sigma, to first order; a row whose RMS is a small
-fraction of the largest (KDA's per-channel retention produces such rows) is
-ill-conditioned, whatever the method.  So each normalised row must agree with
-the reference within one relative rounding of the normalised scale (the same
-tolerance, times max|y_ref|) plus that propagation of its own measured
-un-normalised error (times 1.5 for second-order terms).
+Bounds.  Every rule but KDA: the normalised output is held to the fixed bf16
+(2e-2) or fp32 (1e-4) bound against the oracle's normalised output, like any
+other output.  KDA: its per-channel retention leaves rows whose RMS is a small
+fraction of the largest, and dividing a row by its RMS sigma multiplies the
+row's absolute error by about (1 + max|o_row| / sigma) / sigma to first order,
+whatever the method.  So a KDA row may differ from the reference by one rounding
+of the normalised scale (the tolerance times max|y_ref|) plus that propagation
+of the un-normalised error budget, the tolerance times max|o_ref| (which the
+un-normalised output is held to first), with the row's conditioning taken from
+the oracle's output (times 1.5 for second-order terms).  No part of the bound
+comes from the GPU's own measured error.
 """
 import numpy as np
 import pytest
@@ -53,20 +55,22 @@ def check_norm(la, p, w, tol, norm_eps=EPS_N):
     # the output bound, before normalisation
     op = o_plain.float().cpu().numpy().astype(np.float64)
     assert rel_err(op, ro) <= tol, f"{p.name}: un-normalised o rel err {rel_err(op, ro):.3e}"
-    # each normalised row: one rounding of the normalised scale plus the first-order
-    # propagation of the row's own un-normalised error through w o / sigma
     y = o.float().cpu().numpy().astype(np.float64)
     assert np.all(np.isfinite(y))
-    wmax = 1.0 if w is None else float(w.abs().max())
-    sigma = np.sqrt((ro ** 2).mean(axis=-1) + norm_eps)
-    d_o = np.abs(op - ro).max(axis=-1)
-    cond = (1.0 + np.abs(ro).max(axis=-1) / sigma) / sigma
-    bound = tol * np.abs(want).max() + 1.5 * wmax * d_o * cond
-    dy = np.abs(y - want).max(axis=-1)
-    worst = np.unravel_index(np.argmax(dy / bound), dy.shape)
-    assert np.all(dy <= bound), (f"{p.name}: normalised row {worst} off by {dy[worst]:.3e} "
-                                 f"> bound {bound[worst]:.3e}")
     e = rel_err(y, want)
+    if p.rule != "kda":
+        assert e <= tol, f"{p.name}: normalised o rel err {e:.3e} > {tol}"
+    else:
+        # each row: one rounding of the normalised scale plus the first-order
+        # propagation of the un-normalised error budget through w o / sigma
+        wmax = 1.0 if w is None else float(w.abs().max())
+        sigma = np.sqrt((ro ** 2).mean(axis=-1) + norm_eps)
+        cond = (1.0 + np.abs(ro).max(axis=-1) / sigma) / sigma
+        bound = tol * np.abs(want).max() + 1.5 * wmax * (tol * np.abs(ro).max()) * cond
+        dy = np.abs(y - want).max(axis=-1)
+        worst = np.unravel_index(np.argmax(dy / bound), dy.shape)
+        assert np.all(dy <= bound), (f"{p.name}: normalised row {worst} off by {dy[worst]:.3e} "
+                                     f"> bound {bound[worst]:.3e}")
     assert torch.equal(S, S_plain)
     if z is not None:
         assert torch.equal(z, z_plain)
@@ -139,19 +143,16 @@ def test_packed_sequences_with_norm(la):
         assert rel_err(S[i:i + 1].cpu().numpy(), rS) <= TOL_BF16
 
 
-def test_lightning_full_size_sampled(la):
+def test_lightning_full_size(la):
     """B=2, H=16, T=8192, d=128 (the prefill benchmark shape) with g = 1 and the
-    norm, heads (0,3) and (1,15) against the oracle."""
+    norm, every head against the oracle at the fixed bound."""
     p = workloads.make_problem("gla", 2, 8192, 16, 128, 128, gla_gate="ones", seed=3)
     w = weight(128, 1)
     o, S, _ = run(la, p, w)
-    o = o.float().cpu().numpy()
-    for b, h in ((0, 3), (1, 15)):
-        sp = sub_heads(p, [b], [h])
-        ro, rS, _ = oracle.fwd(sp)
-        want = oracle.head_rmsnorm(ro, w.double().numpy(), EPS_N)
-        assert rel_err(o[[b]][:, :, [h]], want) <= TOL_BF16
-        assert rel_err(S[[b]][:, [h]].cpu().numpy(), rS) <= TOL_BF16
+    ro, rS, _ = oracle.fwd(p)
+    want = oracle.head_rmsnorm(ro, w.double().numpy(), EPS_N)
+    assert rel_err(o.float().cpu().numpy(), want) <= TOL_BF16
+    assert rel_err(S.cpu().numpy(), rS) <= TOL_BF16
 
 
 def test_host_buffers_with_norm_match_device(la):

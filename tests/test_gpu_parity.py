@@ -3,8 +3,7 @@ same seeded inputs.
 
 Metric (per tensor): max|x - ref| / max|ref|.  Bounds: 1e-4 for fp32 inputs,
 2e-2 for bf16 inputs with fp32 accumulation (outputs and final state each).
-Full-size workloads are checked on a sample of (batch, head) sequences, which
-are independent, so the oracle computes them exactly.
+The full-size workloads are checked on every (batch, head) sequence.
 """
 import numpy as np
 import pytest
@@ -88,26 +87,31 @@ def test_gla_prefill_full(la):
     check(p, *run_gpu(la, p), TOL_BF16)
 
 
-def test_gla_prefill_long_sampled(la):
+def test_gla_prefill_long_full(la):
+    """GLA at the prefill benchmark shape, B=2 H=16 T=8192 d=128, every head."""
     p = workloads.gla_prefill(B=2, H=16, T=8192)
-    check(p, *run_gpu(la, p), TOL_BF16, heads=([0, 1], [0, 7, 15]))
+    check(p, *run_gpu(la, p), TOL_BF16)
 
 
-def test_elu_long_sampled(la):
+def test_elu_long_full(la):
+    """Normalized ELU+1 at the pages' worked shape, B=1 H=16 N=32768 dphi=128 dv=64,
+    with S0 >= 0 and z0 = 1 carried in, every head."""
     p = workloads.elu_long()
-    check(p, *run_gpu(la, p), TOL_BF16, heads=([0], [0, 5, 15]))
+    check(p, *run_gpu(la, p), TOL_BF16)
 
 
-def test_gdn_prefill_sampled(la):
+def test_gdn_prefill_full(la):
+    """The gated delta rule at B=2 H=16 T=8192 d=128, every head."""
     p = workloads.gdn_prefill()
-    check(p, *run_gpu(la, p), TOL_BF16, heads=([0, 1], [0, 9, 15]))
+    check(p, *run_gpu(la, p), TOL_BF16)
 
 
 def test_gdn_split_invariance_at_3000(la):
     """Scan [0,3000), carry the state, scan [3000,8192): matches the oracle's whole
-    scan and the GPU's whole scan (page "状态空间与线性注意力", chunk boundaries)."""
+    scan and the GPU's whole scan (page "状态空间与线性注意力", chunk boundaries),
+    every head."""
     p = workloads.gdn_prefill()
-    hs = ([0, 1], [0, 9, 15])
+    hs = None
     t = to_dev(p)
     o_w, S_w, _ = la.fwd("gdn", t["q"], t["k"], t["v"], t["g"], t["beta"])
     tau = 3000
