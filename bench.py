@@ -629,8 +629,26 @@ def cpu_baseline(budget_s: float = 15.0):
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    if rank != 0:
-        return
+    dist = None
+    if world > 1:
+        # the ranks meet once at the end (gloo: CPU only), so they finish together;
+        # rank 0 alone does the work and prints the line
+        import torch.distributed as dist
+        from datetime import timedelta
+        if not dist.is_initialized():
+            dist.init_process_group("gloo", timeout=timedelta(minutes=10))
+        else:
+            dist = None   # the caller owns the group
+    try:
+        if rank == 0:
+            _reference_line(args, world)
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+def _reference_line(args, world):
     import oracle
     T = args.ref_tokens
     for _ in range(args.warmup):
@@ -658,7 +676,30 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
-def main():
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, argv):
+    """One rank started by launch_ranks: the environment a torchrun launch gives
+    it (one process per GPU, rendezvous on 127.0.0.1), then the bench itself."""
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    main(argv)
+
+
+def launch_ranks(world: int, argv) -> None:
+    """`--gpus N` without a launcher: start N ranks (spawned processes, one per
+    GPU) and wait for them; a rank that fails fails the launch."""
+    import torch.multiprocessing as mp
+    mp.start_processes(_rank_main, args=(world, free_port(), argv), nprocs=world, join=True,
+                       start_method="spawn")
+
+
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
@@ -673,9 +714,22 @@ def main():
     ap.add_argument("--reps", type=int, default=1)
     ap.add_argument("--variants", action="store_true",
                     help="also time DeltaNet, RetNet and Lightning prefill (same kernels) at B=2 H=16 T=8192")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    launched = "WORLD_SIZE" in os.environ
+    if args.gpus < 1:
+        sys.exit("bench.py: --gpus must be >= 1")
+    if launched and int(os.environ["WORLD_SIZE"]) != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but the launcher started WORLD_SIZE={os.environ['WORLD_SIZE']} ranks")
+    if args.gpus > 1 and not launched:
+        if args.impl == "cuda" and not args.profile_leg:
+            import torch
+            have = torch.cuda.device_count()
+            if have < args.gpus:
+                sys.exit(f"bench.py: --gpus {args.gpus} needs {args.gpus} CUDA devices, this node has {have}")
+        launch_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv))
+        return
     if args.profile_leg:
         run_profile_leg(args)
     elif args.impl == "reference":

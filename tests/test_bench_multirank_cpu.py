@@ -5,7 +5,9 @@ With N GPUs the bench runs one process per GPU, each on its own sequences
 barrier and the maximum of the per-rank device times, and the whole-job value
 counts every rank's tokens over that maximum.  The reference arm runs on rank
 0 alone; the other ranks exit without work.  These tests drive exactly those
-functions from two gloo ranks.
+functions from two gloo ranks, and drive ``bench.py --gpus 2`` itself: without
+a launcher it starts its two ranks (torchrun's environment, 127.0.0.1), and it
+refuses to run on fewer CUDA devices than asked for.
 """
 import io
 import json
@@ -86,3 +88,41 @@ def test_reference_arm_runs_on_rank_zero_only(tmp_path):
     line = json.loads(out0[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def _bench(*argv, timeout=300):
+    import subprocess
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        env.pop(k, None)
+    env["OMP_NUM_THREADS"] = "2"
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *argv], cwd=ROOT, env=env,
+                          capture_output=True, text=True, timeout=timeout)
+
+
+def test_gpus_flag_launches_the_ranks_itself():
+    """`bench.py --gpus 2` without torchrun starts two ranks (torchrun's
+    environment, rendezvous on 127.0.0.1; the reference arm meets over gloo) and
+    prints one line, from rank 0, for the whole job."""
+    r = _bench("--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--ref-tokens", "16")
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+def test_gpus_flag_refuses_missing_devices():
+    """The CUDA arm refuses, instead of running on fewer GPUs, when the node has
+    fewer CUDA devices than --gpus asks for (none here)."""
+    r = _bench("--gpus", "2", "--steps", "1")
+    assert r.returncode != 0
+    assert "needs 2 CUDA devices" in r.stderr
+    assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_gpus_flag_must_match_the_launcher():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="4", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "WORLD_SIZE=4" in r.stderr
