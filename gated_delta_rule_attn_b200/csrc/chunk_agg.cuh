@@ -35,6 +35,8 @@ struct AggParams {
     int64_t B, T, H, dv;
     float *agg;     // [B*H][nseg-1][nparts] blocks of DK*dv (dS, row-major) + DK (dz or D) floats
     int nseg, nparts, seg_chunks;
+    uint32_t *seq_flags = nullptr;   // GLA: see ChunkParams
+    uint32_t call_id = 0;
 };
 
 namespace ck {
@@ -164,6 +166,11 @@ chunk_agg_kernel(const __grid_constant__ Maps maps, const AggParams p) {
                 const float2 gc = __fmul2_rn(__fmul2_rn(ctl->tot[0][pr], ctl->tot[1][pr]),
                                              __fmul2_rn(ctl->tot[2][pr], ctl->tot[3][pr]));
                 zacc = __fmul2_rn(zacc, gc);
+                // a chunk the main pass cannot take in its chunked form: the
+                // sequence is recomputed by the recurrent kernel (these summaries
+                // stay exact: every factor above is <= 1)
+                if (qt == 0 && p.seq_flags && !(fminf(gc.x, gc.y) >= kGlaMinChunkGate))
+                    p.seq_flags[bh] = p.call_id;
             } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {

@@ -95,6 +95,7 @@ struct GECtl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort, stopP;
+    int seqfail;                     // GLA: a chunk of this CTA left the chunked form's range
     alignas(16) float gC[4][128];    // GLA: gamma at chunk end per key dim; ELU: chunk sum of phi(k)
     alignas(16) float2 tot[4][64];   // prep: per-quarter gate products (GLA) / sums of phi(k) (ELU)
 };
@@ -151,6 +152,7 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         mbar_init(&ctl->s0, 128);
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
+        ctl->seqfail = 0;
         fence_barrier_init();
         tma_prefetch_desc(&maps.q);
         tma_prefetch_desc(&maps.k);
@@ -238,7 +240,12 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
                 if (qt == 3) {
                     const float2 gc = __fmul2_rn(pre, gv[15]);
                     *reinterpret_cast<float2 *>(&ctl->gC[c & 3][2 * pr]) = gc;
-                    if (!(fminf(gc.x, gc.y) >= 1e-30f)) raise_error(kErrRange);
+                    // out of the chunked form's range: this CTA's results for the
+                    // sequence are discarded and the recurrent kernel recomputes it
+                    if (!(fminf(gc.x, gc.y) >= kGlaMinChunkGate)) {
+                        ctl->seqfail = 1;
+                        if (p.seq_flags) p.seq_flags[bh] = p.call_id;
+                    }
                 }
                 // Qt = Q o gamma, Kt = K / gamma (both in place), 8 tokens at a time
 #pragma unroll
@@ -511,7 +518,12 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             tc_fence_before_sync();
             mbar_arrive(&ctl->sB[bb]);
         }
-        if (!ctl->abort && seg == p.nseg - 1) {
+        // a sequence flagged here or, for the earlier segments, by the summary
+        // pass keeps S_out untouched (S0 may alias it): the recurrent kernel
+        // recomputes it from S0
+        const bool flagged = kGLA && (*reinterpret_cast<volatile int *>(&ctl->seqfail) != 0 ||
+                                      (p.seq_flags && p.seq_flags[bh] == p.call_id));
+        if (!ctl->abort && seg == p.nseg - 1 && !flagged) {
             if (p.S_out) {
                 float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVS);
 #pragma unroll
@@ -603,6 +615,9 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         umma_commit(&ctl->drain);
         (void)mbar_drain(&ctl->drain, 0u);
     }
+    // GLA: the exact recomputation kernel that follows may be scheduled now (it
+    // waits for this grid's completion before reading anything)
+    if (kGLA) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
 }

@@ -46,6 +46,7 @@
 #pragma once
 
 #include <algorithm>
+#include <atomic>
 #include <string>
 
 #include "device.cuh"
@@ -74,7 +75,20 @@ struct ChunkParams {
     // launch sets it to T for the dense layout).
     const int64_t *cu_seqlens = nullptr;
     int64_t max_seqlen = 0;
+    // GLA: per-sequence flags in the workspace.  A sequence with a chunk whose
+    // gate product leaves the chunked form's range gets seq_flags[b*H + h] =
+    // call_id (an ID unique to the call, so the flags need no clearing); the
+    // chunked kernels then leave its final state unwritten and the recurrent
+    // kernel recomputes the sequence exactly.
+    uint32_t *seq_flags = nullptr;
+    uint32_t call_id = 0;
 };
+
+// Smallest per-key-dim gate product over one 64-token chunk that GLA's chunked
+// form handles: it scales keys by 1 / (the gate product from the chunk's start),
+// which for products >= 2^-120 stays a normal fp32 and bf16 number (as does
+// q times the product).
+constexpr float kGlaMinChunkGate = 0x1p-120f;
 
 namespace ck {
 
@@ -244,21 +258,29 @@ inline KdaWorkspace kda_workspace(int64_t B, int64_t T, int64_t H) {
     return w;
 }
 
+// Segment summaries of sequence-parallel ELU+1 / GLA (none when packed).
+inline size_t chunk_agg_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv, bool packed) {
+    if (packed || (rule != kRuleELU && rule != kRuleGLA)) return 0;
+    const SegPlan sp = seg_plan(rule, B, T, H, dv);
+    if (sp.nseg < 2) return 0;
+    return (size_t)(B * H * (sp.nseg - 1) * sp.nparts) * (size_t)(ck::DK * dv + ck::DK) * sizeof(float);
+}
+// GLA's per-sequence flags (uint32 per (batch, head)), after the summaries.
+inline size_t gla_flag_bytes(int64_t B, int64_t H) { return ((size_t)(B * H) * 4 + 255) & ~(size_t)255; }
+
 // Device workspace the chunked path needs: the gated delta rule keeps the
 // per-chunk T = (I + A)^-1 and P operand images (16 KB per (batch, head, chunk)); KDA
 // its prep kernel's items and scaled q/k tensors; sequence-parallel ELU+1 and GLA the range
-// summaries of their first pass.  `packed`: the sequences are packed on one
-// token axis with lengths up to max_seqlen (no sequence-parallel pass then).
+// summaries of their first pass; GLA its per-sequence range flags.  `packed`: the
+// sequences are packed on one token axis with lengths up to max_seqlen (no
+// sequence-parallel pass then).
 inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t dv,
                                     bool packed = false, int64_t max_seqlen = 0) {
     if (T <= 0) return 0;
     const int64_t L = packed ? max_seqlen : T;
     if (rule == kRuleGDN) return (size_t)(B * H * ((L + ck::C - 1) / ck::C)) * ck::gdn::ITEM_BYTES;
     if (rule == kRuleKDA) return kda_workspace(B, packed ? (L + ck::C - 1) / ck::C * ck::C : T, H).total;
-    if (packed) return 0;
-    const SegPlan sp = seg_plan(rule, B, T, H, dv);
-    if (sp.nseg < 2) return 0;
-    return (size_t)(B * H * (sp.nseg - 1) * sp.nparts) * (size_t)(ck::DK * dv + ck::DK) * sizeof(float);
+    return chunk_agg_bytes(rule, B, T, H, dv, packed) + (rule == kRuleGLA ? gla_flag_bytes(B, H) : 0);
 }
 
 // GLA / ELU: one CTA per (batch, head, 32-column value slab).
@@ -288,6 +310,34 @@ template <int RULE>
 cudaError_t launch_agg_dv(const ck::Maps &m, const AggParams &a, cudaStream_t st) {
     return a.dv == 32 ? launch_agg<RULE, 32>(m, a, st)
          : a.dv == 64 ? launch_agg<RULE, 64>(m, a, st) : launch_agg<RULE, 128>(m, a, st);
+}
+
+// The recurrent kernel over the GLA sequences flagged in p.seq_flags for this call.
+inline cudaError_t launch_gla_recompute(const ChunkParams &p, cudaStream_t st) {
+    RecurrentParams r{};
+    r.B = p.B; r.T = p.T; r.H = p.H;
+    r.q = p.q; r.k = p.k; r.v = p.v; r.g = p.g; r.beta = nullptr;
+    r.S_in = p.S0; r.S_out = p.S_out; r.z_in = nullptr; r.z_out = nullptr;
+    r.o = p.o; r.eps = p.eps;
+    r.cu_seqlens = p.cu_seqlens; r.max_seqlen = p.max_seqlen;
+    r.seq_flags = p.seq_flags; r.call_id = p.call_id;
+    // a programmatic dependent launch: scheduled as the chunked kernel's CTAs
+    // finish instead of after a full kernel boundary (the kernel waits for that
+    // grid's completion before it reads the flags)
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(p.B * p.H));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    switch (p.dv) {
+        case 32: return cudaLaunchKernelEx(&cfg, recurrent_kernel<kRuleGLA, 128, 32, __nv_bfloat16>, r);
+        case 64: return cudaLaunchKernelEx(&cfg, recurrent_kernel<kRuleGLA, 128, 64, __nv_bfloat16>, r);
+        default: return cudaLaunchKernelEx(&cfg, recurrent_kernel<kRuleGLA, 128, 128, __nv_bfloat16>, r);
+    }
 }
 
 inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_bytes, cudaStream_t st,
@@ -390,16 +440,28 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         // packed sequences walk each sequence in one pass (no segments)
         const SegPlan sp = packed ? SegPlan{1, 1, (int)((Lmax + C - 1) / C)} : seg_plan(rule, p.B, p.T, p.H, p.dv);
         ChunkParams q = pq;
+        const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv, packed, Lmax);
+        if (need && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u))) {
+            *err = rule == kRuleGLA ? "GLA needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes"
+                                    : "sequence-parallel ELU+1 needs a 16-byte aligned workspace of "
+                                      "la_fwd_workspace_size() bytes";
+            return 8;
+        }
+        if (rule == kRuleGLA) {
+            // flags after the summaries; a call ID that no earlier call used
+            static std::atomic<uint32_t> next_call{0};
+            uint32_t id = next_call.fetch_add(1) + 1u;
+            if (id == 0u) id = next_call.fetch_add(1) + 1u;
+            q.seq_flags = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) +
+                                                       chunk_agg_bytes(rule, p.B, p.T, p.H, p.dv, packed));
+            q.call_id = id;
+        }
         if (sp.nseg > 1) {
-            const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv);
-            if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
-                *err = "sequence-parallel ELU+1 / GLA needs a 16-byte aligned workspace of la_fwd_workspace_size() bytes";
-                return 8;
-            }
             AggParams a{};
             a.B = p.B; a.T = p.T; a.H = p.H; a.dv = p.dv;
             a.agg = static_cast<float *>(ws);
             a.nseg = sp.nseg; a.nparts = sp.nparts; a.seg_chunks = sp.seg_chunks;
+            a.seq_flags = q.seq_flags; a.call_id = q.call_id;
             e = rule == kRuleGLA ? launch_agg_dv<kRuleGLA>(m, a, st) : launch_agg_dv<kRuleELU>(m, a, st);
             if (e != cudaSuccess) {
                 *err = std::string("chunk kernel launch: ") + cudaGetErrorString(e);
@@ -420,6 +482,10 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         } else {
             e = rule == kRuleGLA ? launch_ge<kRuleGLA, DVT>(m, q, st) : launch_ge<kRuleELU, DVT>(m, q, st);
         }
+        // GLA sequences with a chunk out of the chunked form's range: recomputed
+        // exactly by the per-token recurrent kernel from S0 (every other CTA exits
+        // at once)
+        if (e == cudaSuccess && rule == kRuleGLA) e = launch_gla_recompute(q, st);
     }
     if (e != cudaSuccess) {
         *err = std::string("chunk kernel launch: ") + cudaGetErrorString(e);

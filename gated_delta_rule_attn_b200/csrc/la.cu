@@ -578,8 +578,8 @@ la_status la_check_device(void *stream, uint32_t *flags) {
     if (w & la::kErrTimeout) return fail(LA_ERR_TIMEOUT, "a bounded device wait ran out");
     if (w & la::kErrRange)
         return fail(LA_ERR_RANGE,
-                    "a gate product left the chunked kernels' range (GLA: below 1e-30 inside a 64-token "
-                    "chunk; KDA: an 8-token retention product below 2^-60)");
+                    "a KDA retention product left the chunked kernels' range (an 8-token product "
+                    "below 2^-60)");
     if (w & la::kErrSeqlen)
         return fail(LA_ERR_INVALID_ARG,
                     "cu_seqlens: offsets out of order or outside [0, T], or a sequence longer than "

@@ -47,6 +47,10 @@ struct RecurrentParams {
     // one token axis of T tokens (tensors [1,T,H,*]); nullptr = dense layout
     const int64_t *cu_seqlens = nullptr;
     int64_t max_seqlen = 0;
+    // set: only the sequences (b, h) with seq_flags[b*H + h] == call_id run (the
+    // exact recomputation of GLA sequences the chunked kernels could not take)
+    const uint32_t *seq_flags = nullptr;
+    uint32_t call_id = 0;
 };
 
 __device__ __forceinline__ float elu_feature_precise(float x) {
@@ -71,6 +75,12 @@ __global__ void __launch_bounds__(256, 2) recurrent_kernel(const RecurrentParams
     const int tid = threadIdx.x;
     const int cg = tid % CG, rg = tid / CG;
     const int64_t bh = blockIdx.x;
+    if (p.seq_flags) {
+        // launched as a programmatic dependent of the chunked kernel: wait for it
+        // to finish (and its writes to be visible) before reading its flags
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (p.seq_flags[bh] != p.call_id) return;   // uniform over the CTA
+    }
     const int64_t b = bh / p.H, h = bh % p.H;
     const int64_t H = p.H, T = p.T;
 

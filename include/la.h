@@ -43,11 +43,10 @@
  *   - Each call enqueues work on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream) and returns immediately.  Arguments are
  *     validated on the host before any launch; an invalid call launches nothing.
- *   - Conditions detected on the device (a bounded wait that ran out, a GLA
- *     chunk whose cumulative gate or a KDA sub-chunk whose retention product
- *     leaves the chunked kernels' range, packed-sequence offsets that are out
- *     of order or out of range) set a device-wide error word;
- *     la_check_device() reads and clears it.
+ *   - Conditions detected on the device (a bounded wait that ran out, a KDA
+ *     sub-chunk whose retention product leaves the chunked kernels' range,
+ *     packed-sequence offsets that are out of order or out of range) set a
+ *     device-wide error word; la_check_device() reads and clears it.
  *   - Supported sizes: dk, dv in {32, 64, 128}; B, H >= 1; T >= 0.  T == 0
  *     writes S_out = S0 (or zeros) and z_out = z0 (or zeros).
  *   - There is no CPU fallback: every result comes from a CUDA kernel.
@@ -79,7 +78,11 @@ typedef enum {
 /*
  * Update rules (S is dk x dv; every output is read after its token's update):
  *   ELU  normalised ELU+1 linear attention ("Linear / RNN 路线", §2.1)
- *   GLA  S_t = Diag(g_t) S_{t-1} + k_t v_t^T ("Linear / RNN 路线", §2.2)
+ *   GLA  S_t = Diag(g_t) S_{t-1} + k_t v_t^T ("Linear / RNN 路线", §2.2),
+ *        for every g in (0, 1].  bf16 GLA with dk = 128 runs chunked on the
+ *        tensor cores; a sequence with a 64-token chunk whose gate product falls
+ *        below 2^-120 in some key dim (the chunked form's range) is recomputed
+ *        within the same call by the per-token recurrent kernel (exact, slower).
  *   GDN  S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
  *        ("线性注意力与 SSM", GDN box, in the dk x dv orientation)
  *   KDA  S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
@@ -118,6 +121,8 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *          sequences run segment-parallel and keep there the summary of each
  *          piece of every segment but the last (dk*dv + dk floats per piece: the
  *          piece's state contribution and its normaliser sum or gate product).
+ *          Chunked GLA also keeps one 4-byte flag per (batch, head) there (a
+ *          sequence to recompute, see la_rule), so its workspace is never 0.
  *          Chunked KDA keeps 16.5 KB per (batch, head, chunk) (the T and P
  *          operand images and the chunk's retention product) plus three bf16
  *          [B,Ls,H,128] tensors: q and k scaled by the cumulative retention, and
@@ -284,7 +289,7 @@ la_status la_fwd_noalloc(const la_fwd_args *args, void *stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device error word set by
- * earlier kernels.  Returns LA_OK, LA_ERR_TIMEOUT, LA_ERR_RANGE,
+ * earlier kernels.  Returns LA_OK, LA_ERR_TIMEOUT, LA_ERR_RANGE (KDA only),
  * LA_ERR_INVALID_ARG (packed-sequence offsets that had to be clamped) or
  * LA_ERR_CUDA.  `flags` (may be NULL) receives the raw word (bit 0 timeout,
  * bit 1 range, bit 2 clamped offsets).

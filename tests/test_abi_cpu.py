@@ -98,17 +98,22 @@ def test_null_args_and_workspace_query(L):
     # (batch, head, 64-token chunk)
     assert L.la_fwd_workspace_size(ctypes.byref(args(T=130)), ctypes.byref(n)) == 0
     assert n.value == 1 * 2 * 3 * 16384
-    for a in (args("gla"), args("elu"), args(dtype=0), args(dk=64), args(T=0)):
+    for a in (args("elu"), args(dtype=0), args(dk=64), args(T=0), args("gla", dtype=0)):
         assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
         assert n.value == 0
+    # chunked GLA: one uint32 range flag per (batch, head), in 256-byte units
+    assert L.la_fwd_workspace_size(ctypes.byref(args("gla")), ctypes.byref(n)) == 0
+    assert n.value == 256
+    assert L.la_fwd_workspace_size(ctypes.byref(args("gla", B=9, H=16)), ctypes.byref(n)) == 0
+    assert n.value == 768
     assert L.la_fwd_workspace_size(ctypes.byref(args(dk=3)), ctypes.byref(n)) == 2
     # long ELU+1 and GLA sequences over few heads run segment-parallel: the first
     # pass keeps a summary per piece of every segment but the last (dk*dv + dk
     # floats each).  Without a device the library plans for 148 SMs: 4 CTAs of
     # 64 value columns -> 8 segments of 8 chunks, 2 pieces each.
-    for rule in ("elu", "gla"):
+    for rule, flags in (("elu", 0), ("gla", 256)):
         assert L.la_fwd_workspace_size(ctypes.byref(args(rule, T=4096, H=2)), ctypes.byref(n)) == 0
-        assert n.value == 1 * 2 * 7 * 2 * (128 * 128 + 128) * 4
+        assert n.value == 1 * 2 * 7 * 2 * (128 * 128 + 128) * 4 + flags
 
 
 def test_kda_workspace_query():
