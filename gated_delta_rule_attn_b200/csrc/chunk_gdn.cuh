@@ -1,28 +1,25 @@
-// chunk_gdn.cuh — gated delta rule, chunked prefill: two kernels.
+// chunk_gdn.cuh — gated delta rule, chunked prefill: two kernels (and the
+// templated main pass that KDA shares, chunk_gdn_kernel<true>).
 //
 // gdn_prep_kernel (fully parallel over (batch, head, chunk)): for each 64-token
 //   chunk, the state-independent parts, from one M=128 MMA [Q ; K] K^T:
-//     P = Q K^T o Gamma o M                            (rows 0-63),
-//     A = diag(beta) (K K^T o Gamma o strict-lower)    (rows 64-127),
+//     P = Q K^T o Gamma o M                            (the Q rows),
+//     A = diag(beta) (K K^T o Gamma o strict-lower)    (the K rows),
 //     T = (I + A)^-1   (16x16 diagonal blocks by substitution, then two levels of
 //                       block merges on mma.sync tf32),
-//   and writes T and P as bf16 operand images (128-byte swizzled, exactly as the
-//   main kernel's shared memory wants them) to the workspace: 16 KB per (batch,
-//   head, chunk).  Computing P here keeps Q K^T out of the main kernel's tensor
-//   pipe, where its 8 instructions would queue ahead of the recurrence's MMAs.
+//     U = T diag(beta gamma) K                         (one M=64, N=128 MMA),
+//   and writes T diag(beta), P and -U as bf16 operand images (128-byte
+//   swizzled, exactly as the main kernel's shared memory wants them) to the
+//   workspace: 32 KB per (batch, head, chunk).
 //
-// chunk_gdn_kernel (one CTA per (batch, head, 32-column value slab), 9 warps):
-//   warp 0      producer: TMA loads of q, k, v and bulk copies of the chunk's
-//               T and P images (3 stages); the chunk's decay factors and betas;
-//   warps 1-4   "output" group: as soon as the state group has W of chunk c,
-//               PW = [P ; 0] W and O = diag(gamma) X2 + PW;
-//   warps 5-8   "state" group, the recurrence across chunks.  With
-//               W = U - W_k S0 = T diag(beta) (V - diag(gamma) K S0):
-//                 [X2 ; KS] = [Q ; K] S0        (one M=128 MMA chain, S0 bf16),
-//                 R = diag(beta) (V - diag(gamma) KS)   (bf16),
-//                 W = T R,
-//                 dS = K^T diag(gamma_C/gamma) W,
-//                 S <- gamma_C S + dS (fp32, one state row per thread).
+// gdn_main_kernel (one CTA per (batch, head, 32-column value slab), 9 warps):
+//   with W = T diag(beta) (V - diag(gamma) K S0) = T diag(beta) V - U S0,
+//     [X2 ; W] = [0 ; T diag(beta)] V + [Q ; -U] S0   (one accumulator; the first
+//                                                     product off the recurrence),
+//     dS = K^T diag(gamma_C/gamma) W,  S <- gamma_C S + dS   (fp32, one state row
+//                                                     per thread),
+//     O = diag(gamma) X2 + [P ; K0] W   (rows 0-63).
+//   Two MMA round trips per chunk on the recurrence ([Q ; -U] S0, then dS).
 // The derivation of the WY / UT form is in chunk_tc.cuh's header.
 //
 // Pairwise decays Gamma_ti = gamma_t / gamma_i (i <= t) are products of
@@ -33,6 +30,8 @@
 // Hand-offs use mbarriers (TMA transactions, tcgen05.commit, thread arrivals)
 // and named barriers inside a group; every wait is bounded.
 #pragma once
+
+#include <cstddef>
 
 #include "device.cuh"
 
@@ -50,12 +49,15 @@ constexpr uint32_t C_DS = 224;   // 32,     M=128 dS
 constexpr uint32_t C_PW = 256;   // 2 x 32, M=128 [P ; 0] W (rows 0-63)
 
 constexpr uint32_t TT_BYTES = 8192;                  // T, bf16 [64][64]
-// Workspace item per (batch, head, chunk), written by the prep kernel: the T and
-// P operand images, bf16 [64][64], 128-byte swizzled as the main kernel's
-// shared memory wants them (KDA appends Gamma_C)
+// Workspace item per (batch, head, chunk), written by the prep kernel: operand
+// images, bf16, 128-byte swizzled exactly as the main kernel's shared memory
+// wants them: T diag(beta) [64][64], P [64][64] and -U = -T diag(beta gamma) K as
+// two [64][64] blocks (key columns 0-63, 64-127).  KDA's item (chunk_kda.cuh)
+// shares the T and P offsets (its T image is T itself) and appends Gamma_C.
 constexpr uint32_t ITEM_T = 0;
 constexpr uint32_t ITEM_P = 8192;
-constexpr uint32_t ITEM_BYTES = 16384;
+constexpr uint32_t ITEM_U = 16384;
+constexpr uint32_t ITEM_BYTES = 32768;
 
 constexpr uint32_t QK_ACS = 128 * 128;               // one atom column: Q rows 0-63, K rows 64-127
 constexpr uint32_t STG_QK_BYTES = 2 * QK_ACS;
@@ -94,15 +96,22 @@ struct GL {
     static constexpr uint32_t TEND = TSS + 2 * 8192;
 };
 
-// Prep-kernel shared memory.
+// Prep-kernel shared memory.  Each of the two 64-column atom columns of q and k
+// holds three [64][64] blocks, K0 | Q | K1: item i's K lands in slot i & 1, so
+// that [K0 ; Q] (even items) or [Q ; K1] (odd items) is one M=128 operand, and
+// the next item's K can be loaded while this item's -U MMA still reads its own.
 constexpr int AF_LD = 68;
 constexpr int TMP_LD = 36;
-constexpr uint32_t P_QK = 0;                         // [Q ; K]: 2 atom columns of 128 rows (Q 0-63, K 64-127)
-constexpr uint32_t P_AF = 2 * QK_ACS;                // A, then T, fp32 [64][AF_LD]
+constexpr uint32_t P_ACS = 3 * 8192;                 // atom column: K0 | Q | K1
+constexpr uint32_t P_Q = 8192;                       // Q block within an atom column
+constexpr uint32_t P_AF = 2 * P_ACS;                 // A, then T, fp32 [64][AF_LD]; then the
+                                                     // T diag(beta gamma) operand image (bf16)
 constexpr uint32_t P_TMP = P_AF + 64 * AF_LD * 4;    // fp32 scratch [32][TMP_LD]
 constexpr uint32_t P_END = P_TMP + 32 * TMP_LD * 4;   // the control block follows
 static_assert(P_END % 16 == 0, "the prep kernel's control block must be 16-byte aligned");
+static_assert(P_AF % 1024 == 0, "the operand image in AF must be 1 KB aligned");
 constexpr int PREP_THREADS = 128;
+constexpr uint32_t PREP_TMEM_COLS = 128;
 
 struct GCtl {
     uint64_t full[NSTG], empty[NSTG];
@@ -116,12 +125,15 @@ struct GCtl {
 };
 
 struct PCtl {
-    uint64_t full, mma, drain;
+    uint64_t full, mma, mma_u, drain;
     uint32_t tmem_base;
     int abort, stop, fast;
+    // 16-byte aligned (the block starts 16-byte aligned and the fields before
+    // take 48 bytes): read as float4
     float alpha[64], beta[64];
     float gam[64], ginv[64], b2[64];
 };
+static_assert(offsetof(PCtl, alpha) % 16 == 0, "PCtl's gate arrays are read as float4");
 
 
 // ---- mma.sync m16n8k8 tf32 (fp32 accumulate) used for the block merges ----
@@ -228,25 +240,48 @@ __device__ __forceinline__ int gate_scan(const float *al, const float *beta, flo
 
 // Row t of the decayed, masked score matrix from 64 raw scores x (in place):
 //   x_i <- x_i * rowf * gamma_t / gamma_i  for i <= t (i < t if strict), else 0.
-// ncols = 32 when only the first 32 columns can be unmasked (t < 32).
+// ncols = 32 when only the first 32 columns can be unmasked (t < 32).  gam, ginv
+// and b2 are 16-byte aligned shared arrays, read four at a time.
 template <bool STRICT>
 __device__ __forceinline__ void decay_mask_row(float *x, int t, int ncols, float rowf, bool fast,
                                                const float *gam, const float *ginv, const float *b2) {
     if (fast) {
         const float rs = rowf * gam[t];
+        const float4 *g4 = reinterpret_cast<const float4 *>(ginv);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            if (i >= ncols) { x[i] = 0.f; continue; }
-            const bool keep = STRICT ? (i < t) : (i <= t);
-            x[i] = keep ? x[i] * rs * ginv[i] : 0.f;
+        for (int i4 = 0; i4 < 16; ++i4) {
+            if (4 * i4 >= ncols) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[4 * i4 + e] = 0.f;
+                continue;
+            }
+            const float4 g = g4[i4];
+            const float gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = 4 * i4 + e;
+                const bool keep = STRICT ? (i < t) : (i <= t);
+                x[i] = keep ? x[i] * (rs * gv[e]) : 0.f;
+            }
         }
     } else {
         const float bt = b2[t];
+        const float4 *b4 = reinterpret_cast<const float4 *>(b2);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            if (i >= ncols) { x[i] = 0.f; continue; }
-            const bool keep = STRICT ? (i < t) : (i <= t);
-            x[i] = keep ? x[i] * rowf * exp2f(bt - b2[i]) : 0.f;
+        for (int i4 = 0; i4 < 16; ++i4) {
+            if (4 * i4 >= ncols) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[4 * i4 + e] = 0.f;
+                continue;
+            }
+            const float4 g = b4[i4];
+            const float gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = 4 * i4 + e;
+                const bool keep = STRICT ? (i < t) : (i <= t);
+                x[i] = keep ? x[i] * (rowf * exp2f(bt - gv[e])) : 0.f;
+            }
         }
     }
 }
@@ -356,12 +391,16 @@ struct GdnPrepParams {
 };
 
 // One CTA handles (batch, head, chunk) items in a grid-stride loop.  The next
-// item's [Q ; K] tile is loaded (TMA) as soon as this item's [Q ; K] K^T MMA has
-// read the buffer, and its alpha and beta are fetched into registers at the same
-// point, so neither load is waited for.  The grid is sized to the CTAs that are
-// resident at once: 4 per SM, with the control block after the tiles (no
-// rounding of it to 1 KB), 57 KB of shared memory and 128 registers per thread.
-__global__ void __launch_bounds__(gdn::PREP_THREADS, 4)
+// item's Q and K are loaded (TMA) as soon as this item's [Q ; K] K^T MMA has
+// read Q (K goes to the other K slot), and its alpha and beta are fetched into
+// registers at the same point, so neither load is waited for.  The grid is
+// sized to the CTAs that are resident at once (3 per SM: 71 KB of shared
+// memory, 128 TMEM columns).
+//
+// Per item: [Q ; K] K^T -> P (to the item) and A; T = (I + A)^-1; the item's
+// T diag(beta) image; then -U = -(T diag(beta gamma)) K as one M=64, N=128 MMA
+// whose A operand is written over AF, and its image.
+__global__ void __launch_bounds__(gdn::PREP_THREADS, 3)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant__ CUtensorMap mapk,
                 const GdnPrepParams p) {
     using namespace gdn;
@@ -377,6 +416,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
     if (tid == 0) {
         mbar_init(&ctl->full, 1);
         mbar_init(&ctl->mma, 1);
+        mbar_init(&ctl->mma_u, 1);
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_barrier_init();
@@ -384,7 +424,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
         tma_prefetch_desc(&mapk);
     }
     if (warp == 0) {
-        tmem_alloc(&ctl->tmem_base, 64);
+        tmem_alloc(&ctl->tmem_base, PREP_TMEM_COLS);
         tc_fence_before_sync();
     }
     __syncthreads();
@@ -392,87 +432,101 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tq = tmem + ((uint32_t)(32 * warp) << 16);
 
-    // warp 0, lane 0: TMA of item w's [Q ; K] tile (Q rows 0-63, K rows 64-127 of
-    // each 64-column atom)
-    auto load_k = [&](int64_t w) {
-        const int64_t bh = w / p.nchunks;
-        const int c = (int)(w % p.nchunks);
-        const int64_t b = bh / p.H, h = bh % p.H;
-        const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, false);
+    // item w -> (batch, head, chunk); item counts stay below 2^32 (a workspace of
+    // 32 KB per item could not exist otherwise), so 32-bit divisions suffice
+    struct ItemPos { int64_t b, h; int c; };
+    auto item_pos = [&](int64_t w) {
+        const uint32_t wu = (uint32_t)w, nch = (uint32_t)p.nchunks, H = (uint32_t)p.H;
+        const uint32_t bh = wu / nch;
+        return ItemPos{(int64_t)(bh / H), (int64_t)(bh % H), (int)(wu - bh * nch)};
+    };
+    // warp 2, lane 0: TMA of item w's Q (the Q blocks) and K (K slot `slot`)
+    auto load_qk = [&](int64_t w, int slot) {
+        const ItemPos ip = item_pos(w);
+        const int64_t h = ip.h;
+        const int c = ip.c;
+        const SeqSpan sq = seq_span(p.cu_seqlens, ip.b, p.T, p.max_seqlen, false);
         mbar_arrive_expect_tx(&ctl->full, 2u * KA * C * 128u);
         for (int a = 0; a < KA; ++a) {
-            tma_load_4d(tiles + P_QK + a * QK_ACS, &mapq, &ctl->full, 64 * a, (int)h, sq.t0 + c * C, sq.b0);
-            tma_load_4d(tiles + P_QK + a * QK_ACS + 64 * 128, &mapk, &ctl->full, 64 * a, (int)h, sq.t0 + c * C,
+            tma_load_4d(tiles + a * P_ACS + P_Q, &mapq, &ctl->full, 64 * a, (int)h, sq.t0 + c * C, sq.b0);
+            tma_load_4d(tiles + a * P_ACS + 16384u * slot, &mapk, &ctl->full, 64 * a, (int)h, sq.t0 + c * C,
                         sq.b0);
         }
     };
-    // warp 0: item w's alpha, beta for tokens 2*lane, 2*lane+1 (1 and 0 past T)
+    // warp 2: item w's alpha, beta for tokens 2*lane, 2*lane+1, loaded unconditionally
+    // (a clamped index) so that nothing waits for them before their use one item
+    // later, where tokens past T take alpha = 1 and beta = 0
     float al[2] = {1.f, 1.f}, be[2] = {0.f, 0.f};
+    bool gin[2] = {false, false};
     auto fetch_gates = [&](int64_t w) {
-        const int64_t bh = w / p.nchunks;
-        const int c = (int)(w % p.nchunks);
-        const int64_t b = bh / p.H, h = bh % p.H;
-        const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, false);
+        const ItemPos ip = item_pos(w);
+        const int64_t h = ip.h;
+        const int c = ip.c;
+        const SeqSpan sq = seq_span(p.cu_seqlens, ip.b, p.T, p.max_seqlen, false);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int64_t tt = (int64_t)c * C + 2 * lane + e;   // position in the sequence
-            const bool in = tt < sq.len;
-            const int64_t idx = (sq.row0 + (in ? tt : 0)) * p.H + h;
-            al[e] = in ? p.alpha[idx] : 1.f;
-            be[e] = in ? p.beta[idx] : 0.f;
+            gin[e] = tt < sq.len;
+            const int64_t idx = gin[e] ? (sq.row0 + tt) * p.H + h : 0;   // element 0 always exists
+            al[e] = __ldg(p.alpha + idx);
+            be[e] = __ldg(p.beta + idx);
         }
     };
 
     constexpr uint32_t ID_QK = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t ID_U = idesc_bf16(64, 128, false, true);
     int it = 0;
-    if (warp == 0 && (int64_t)blockIdx.x < items) {
-        if (lane == 0) load_k(blockIdx.x);
+    if (warp == 2 && (int64_t)blockIdx.x < items) {
+        if (lane == 0) load_qk(blockIdx.x, 0);
         fetch_gates(blockIdx.x);
     }
-    bool k_pending = (int64_t)blockIdx.x < items;   // a K copy is in flight (thread 0's view)
+    bool k_pending = (int64_t)blockIdx.x < items;   // a copy is in flight (thread 64's view)
     for (int64_t w = blockIdx.x; w < items; w += gridDim.x, ++it) {
-        if (warp == 0) {   // this item's gates (fetched one item ahead) into shared memory
+        const int slot = it & 1;                      // this item's K slot
+        const uint32_t kslot = tb + 16384u * (uint32_t)slot;
+        if (warp == 2) {   // this item's gates (fetched one item ahead) into shared memory
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                ctl->alpha[2 * lane + e] = al[e];
-                ctl->beta[2 * lane + e] = be[e];
+                ctl->alpha[2 * lane + e] = gin[e] ? al[e] : 1.f;
+                ctl->beta[2 * lane + e] = gin[e] ? be[e] : 0.f;
             }
         }
         if (tid == 0) ctl->stop = ctl->abort;   // one thread decides, everyone reads after the barrier
         bar_named(1, 128);
         if (ctl->stop) break;
         if (!mbar_wait(&ctl->full, (uint32_t)it & 1u)) ctl->abort = 1;
-        if (tid == 0) k_pending = false;
+        if (tid == 64) k_pending = false;
         if (warp == 0)
             ctl->fast = gate_scan(&ctl->alpha[2 * lane], ctl->beta, ctl->b2, ctl->gam, ctl->ginv, nullptr, lane);
-        if (tid == 32) {   // [Q ; K] K^T: rows 0-63 Q K^T, rows 64-127 K K^T
+        if (tid == 32) {   // [K0 ; Q] K^T (even items) or [Q ; K1] K^T (odd items)
             tc_fence_after_sync();
-            const uint32_t qk = tb + P_QK, kb = qk + 64 * 128;
+            const uint32_t a0 = tb + 8192u * (uint32_t)slot;
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem, desc_k(qk, QK_ACS, kk), desc_k(kb, QK_ACS, kk), ID_QK, kk > 0);
+                umma_bf16(tmem, desc_k(a0, P_ACS, kk), desc_k(kslot, P_ACS, kk), ID_QK, kk > 0);
             umma_commit(&ctl->mma);
         }
         bar_named(1, 128);
         if (!mbar_wait(&ctl->mma, (uint32_t)it & 1u)) ctl->abort = 1;
         tc_fence_after_sync();
-        // the K buffer is free: start the next item's loads
-        if (warp == 0 && w + gridDim.x < items) {
+        // Q and the other K slot are free: start the next item's loads
+        if (warp == 2 && w + gridDim.x < items) {
             if (lane == 0 && !ctl->abort) {
-                load_k(w + gridDim.x);
+                load_qk(w + gridDim.x, slot ^ 1);
                 k_pending = true;
             }
             fetch_gates(w + gridDim.x);
         }
-        {   // row r = tid of the M=128 accumulator: warps 0-1 the P row of token r
-            // (inclusive mask, to the item's P image), warps 2-3 the A row of token
-            // r - 64 (strict mask, times beta, to AF)
+        {   // row r = tid of the M=128 accumulator: the rows of Q give the P row of
+            // token r & 63 (inclusive mask, to the item's P image), the rows of K the
+            // A row of token r & 63 (strict mask, times beta, to AF)
             const int t = tid & 63;
+            const bool prow = (warp < 2) == (slot == 1);
             float x[64];
             tmem_ld32(tq, *reinterpret_cast<float(*)[32]>(x));
             tmem_ld32(tq + 32u, *reinterpret_cast<float(*)[32]>(x + 32));
             tmem_wait_ld();
-            if (warp < 2) {
+            if (prow) {
                 decay_mask_row<false>(x, t, t < 32 ? 32 : 64, 1.f, ctl->fast != 0, ctl->gam, ctl->ginv, ctl->b2);
                 uint8_t *dst = p.ws + w * (int64_t)ITEM_BYTES + ITEM_P + (uint32_t)t * 128u;
 #pragma unroll
@@ -496,25 +550,79 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
         tc_fence_before_sync();
         bar_named(1, 128);
         invert_unit_lower64(AF, TMP, tid, lane, 1, 2);
-        {   // T -> workspace, a 128-byte swizzled [64][64] bf16 image
+        {   // T diag(beta) -> the item; T diag(beta gamma) -> the -U MMA's A operand,
+            // written over AF once every thread has read its part of T
             const int t = tid >> 1, hh = tid & 1;
-            const float *Trow = AF + t * AF_LD + 32 * hh;
+            const float4 *Trow = reinterpret_cast<const float4 *>(AF + t * AF_LD + 32 * hh);
+            const float4 *be4 = reinterpret_cast<const float4 *>(ctl->beta + 32 * hh);
+            const float4 *ga4 = reinterpret_cast<const float4 *>(ctl->gam + 32 * hh);
             uint8_t *dst = p.ws + w * (int64_t)ITEM_BYTES + ITEM_T;
+            uint4 ug[4];
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-                uint4 u;
-                uint32_t *pu = &u.x;
+                float tv[8], bv[8], gv[8];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) pu[e] = pack_bf16x2(Trow[8 * cc + 2 * e], Trow[8 * cc + 2 * e + 1]);
+                for (int hq = 0; hq < 2; ++hq) {
+                    const float4 a = Trow[2 * cc + hq], bb = be4[2 * cc + hq], g = ga4[2 * cc + hq];
+                    tv[4 * hq] = a.x; tv[4 * hq + 1] = a.y; tv[4 * hq + 2] = a.z; tv[4 * hq + 3] = a.w;
+                    bv[4 * hq] = bb.x; bv[4 * hq + 1] = bb.y; bv[4 * hq + 2] = bb.z; bv[4 * hq + 3] = bb.w;
+                    gv[4 * hq] = g.x; gv[4 * hq + 1] = g.y; gv[4 * hq + 2] = g.z; gv[4 * hq + 3] = g.w;
+                }
+                uint4 u;
+                uint32_t *pu = &u.x, *pg = &ug[cc].x;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    pu[e] = pack_bf16x2(tv[2 * e] * bv[2 * e], tv[2 * e + 1] * bv[2 * e + 1]);
+                    pg[e] = pack_bf16x2(tv[2 * e] * (bv[2 * e] * gv[2 * e]),
+                                        tv[2 * e + 1] * (bv[2 * e + 1] * gv[2 * e + 1]));
+                }
                 const int chunk = 4 * hh + cc;
                 *reinterpret_cast<uint4 *>(dst + (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4)) = u;
             }
+            bar_named(1, 128);   // every read of T is done
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int chunk = 4 * hh + cc;
+                *reinterpret_cast<uint4 *>(tiles + P_AF + (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4)) =
+                    ug[cc];
+            }
         }
-        bar_named(1, 128);   // AF and the gates are reused by the next item
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        bar_named(1, 128);
+        if (tid == 32) {   // U = (T diag(beta gamma)) K: M=64 tokens, N=128 key columns, K=64 tokens
+            tc_fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_bf16(tmem, desc_k(tb + P_AF, C * 128, kk), desc_mn128(kslot, P_ACS, kk), ID_U, kk > 0);
+            umma_commit(&ctl->mma_u);
+        }
+        if (!mbar_wait(&ctl->mma_u, (uint32_t)it & 1u)) ctl->abort = 1;
+        tc_fence_after_sync();
+        {   // -U -> the item: row tr = 16 warp + (lane & 15) of the M=64 accumulator,
+            // key columns 64 hf .. 64 hf + 63 = block hf of the image
+            const int tr = 16 * warp + (lane & 15), hf = lane >> 4;
+            float x[64];
+            tmem_ld16x2_32<64>(tq, *reinterpret_cast<float(*)[32]>(x));
+            tmem_ld16x2_32<64>(tq + 32u, *reinterpret_cast<float(*)[32]>(x + 32));
+            tmem_wait_ld();
+            uint8_t *dst = p.ws + w * (int64_t)ITEM_BYTES + ITEM_U + (uint32_t)hf * 8192u + (uint32_t)tr * 128u;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                uint4 u;
+                u.x = pack_bf16x2(-x[8 * cc + 0], -x[8 * cc + 1]);
+                u.y = pack_bf16x2(-x[8 * cc + 2], -x[8 * cc + 3]);
+                u.z = pack_bf16x2(-x[8 * cc + 4], -x[8 * cc + 5]);
+                u.w = pack_bf16x2(-x[8 * cc + 6], -x[8 * cc + 7]);
+                *reinterpret_cast<uint4 *>(dst + (uint32_t)(((cc ^ tr) & 7) << 4)) = u;
+            }
+        }
+        tc_fence_before_sync();
+        bar_named(1, 128);   // AF, TMEM and the gates are reused by the next item
     }
     // let a prefetched copy land and every MMA finish before the CTA frees TMEM
     // and exits (these two waits keep the long limit even after a timeout)
-    if (tid == 0 && k_pending) (void)mbar_drain(&ctl->full, (uint32_t)it & 1u);
+    if (tid == 64 && k_pending) (void)mbar_drain(&ctl->full, (uint32_t)it & 1u);
     if (tid == 32) {
         umma_commit(&ctl->drain);
         (void)mbar_drain(&ctl->drain, 0u);
@@ -522,7 +630,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    if (warp == 0) tmem_dealloc(tmem, 64);
+    if (warp == 0) tmem_dealloc(tmem, PREP_TMEM_COLS);
 }
 
 
@@ -916,6 +1024,377 @@ chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const u
     }
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+namespace gdn {
+// Shared memory of gdn_main_kernel (byte offsets from a 1 KB aligned base).
+//   ring A, 2 stages: [Q ; -U] as two atom columns of 128 rows (Q rows 0-63 from
+//     q by TMA, -U rows 64-127 from the item), the A operand of
+//     [X2 ; W] += [Q ; -U] S0;
+//   ring B, 3 stages: Z | T diag(beta) | P | K | V, where [Z ; T diag(beta)] is
+//     the A operand of [X2 ; W] = [0 ; T diag(beta)] V (Z stays zero), [P ; K0]
+//     that of PW (rows 64-127, the first K block, give rows of the accumulator
+//     that are never read) and K that of dS = K^T diag(gamma_C / gamma) W;
+//   W (2 buffers) and diag(gamma_C / gamma) W, bf16 [64][32], and S0, bf16
+//     [128][32], all with the 64-byte swizzle.
+struct ML {
+    static constexpr int NA = 2, NB = 3;
+    static constexpr uint32_t A_BYTES = 2 * QK_ACS;
+    static constexpr uint32_t B_Z = 0, B_T = 8192, B_P = 16384, B_K = 24576, B_V = 40960;
+    static constexpr uint32_t B_BYTES = 45056;
+    static constexpr uint32_t SA = 0;
+    static constexpr uint32_t SB = SA + NA * A_BYTES;
+    static constexpr uint32_t TWS = SB + NB * B_BYTES;
+    static constexpr uint32_t TWGS = TWS + 2 * 4096;
+    static constexpr uint32_t TSS = TWGS + 4096;
+    static constexpr uint32_t TEND = TSS + 8192;
+};
+// TMEM columns of gdn_main_kernel
+constexpr uint32_t M_TMEM_COLS = 256;
+constexpr uint32_t M_XW = 0;    // 2 x 32, M=128 [X2 ; W] (chunk c in buffer c & 1)
+constexpr uint32_t M_DS = 64;   // 32,     M=128 dS
+constexpr uint32_t M_PW = 96;   // 2 x 32, M=128 [P ; K0] W (rows 0-63)
+
+struct MCtl {
+    uint64_t fullA[ML::NA], emptyA[ML::NA], fullB[ML::NB], emptyB[ML::NB];
+    uint64_t wready[2], pw_done[2], w0_done[2], xk_done, ds_done, drain;
+    uint32_t tmem_base;
+    int abort, stopS, stopL[2];
+    // per ring-B stage: b = log2 of the inclusive cumulative alpha, gamma = 2^b,
+    // 1/gamma and gamma_C / gamma (written by the producer)
+    float b2[ML::NB][64], gam[ML::NB][64], ginv[ML::NB][64], gct[ML::NB][64];
+};
+}  // namespace gdn
+
+// The gated delta rule's main pass (one CTA per (batch, head, 32-column value
+// slab), 9 warps).  With the item's T diag(beta) and -U, the state enters a
+// chunk's work through one MMA chain whose accumulator already holds the
+// state-independent part:
+//   [X2 ; W] = [0 ; T diag(beta)] V + [Q ; -U] S0      (X2 = Q S0)
+//   dS = K^T diag(gamma_C / gamma) W,   S <- gamma_C S + dS   (fp32 carry)
+//   O  = diag(gamma) X2 + P W.
+//   warp 0      producer: ring A (Q by TMA, -U from the item) and ring B (K, V
+//               by TMA; T diag(beta), P from the item; the decay factors);
+//   warps 1-4   output group: PW = [P ; K0] W and O, then the accumulator of
+//               the chunk after next: [0 ; T diag(beta)] V;
+//   warps 5-8   state group: W -> bf16 (and diag(gamma_C / gamma) W), dS, the
+//               state update, and [Q ; -U] S0 of the next chunk.
+__global__ void __launch_bounds__(gdn::NTHREADS, 1)
+gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const uint8_t *ws) {
+    using namespace gdn;
+    using L = ML;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    MCtl *ctl = reinterpret_cast<MCtl *>(smem_raw);
+    uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(MCtl) + (smem_u32(smem_raw) & 1023u)) -
+                     (smem_u32(smem_raw) & 1023u);
+    const uint32_t tb = smem_u32(tiles);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3;
+    const int nslab = (int)(p.dv / DVT);
+    const int dvt = (int)(blockIdx.x % nslab);
+    const int64_t bh = blockIdx.x / nslab;
+    const int64_t b = bh / p.H, h = bh % p.H;
+    // this sequence's tokens (dense: all T of batch b); items are stored for
+    // ceil(max_seqlen / 64) chunks per (batch, head)
+    const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, tid == 0 && h == 0 && dvt == 0);
+    const int nchunks = (int)((sq.len + C - 1) / C);
+    const int64_t ws_chunks = (p.max_seqlen + C - 1) / C;
+
+    if (tid == 0) {
+        for (int s = 0; s < L::NA; ++s) {
+            mbar_init(&ctl->fullA[s], 1);
+            mbar_init(&ctl->emptyA[s], 1);   // [Q ; -U] S0 has read the stage
+        }
+        for (int s = 0; s < L::NB; ++s) {
+            mbar_init(&ctl->fullB[s], 32);
+            mbar_init(&ctl->emptyB[s], 2);   // dS and PW have read the stage
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->wready[i], 128);
+            mbar_init(&ctl->pw_done[i], 1);
+            mbar_init(&ctl->w0_done[i], 1);
+        }
+        mbar_init(&ctl->xk_done, 1);
+        mbar_init(&ctl->ds_done, 1);
+        mbar_init(&ctl->drain, 2);   // one commit from each MMA-issuing thread
+        ctl->abort = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&maps.q);
+        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(&maps.v);
+    }
+    if (warp == 0) {
+        tmem_alloc(&ctl->tmem_base, M_TMEM_COLS);
+        tc_fence_before_sync();
+    }
+    for (int i = tid; i < L::NB * 8192 / 16; i += NTHREADS) {   // the Z blocks stay zero
+        const int st = i / 512, off = (i % 512) * 16;
+        *reinterpret_cast<uint4 *>(tiles + L::SB + st * L::B_BYTES + L::B_Z + off) = make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = ctl->tmem_base;
+    const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16);   // this warp's TMEM lanes
+
+    constexpr uint32_t ID_XW = idesc_bf16(128, DVT, false, true);
+    constexpr uint32_t ID_DS = idesc_bf16(128, DVT, true, true);
+    auto stage_a = [&](int c) { return L::SA + (uint32_t)(c & 1) * L::A_BYTES; };
+    auto stage_b = [&](int c) { return L::SB + (uint32_t)(c % L::NB) * L::B_BYTES; };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        float al[2] = {1.f, 1.f};   // the alphas of the chunk to be issued next
+        auto fetch = [&](int c) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int64_t tt = (int64_t)c * C + 2 * lane + e;
+                al[e] = tt < sq.len ? p.g[(sq.row0 + tt) * p.H + h] : 1.f;
+            }
+        };
+        // whole warp: wait (if `need`) until the slot's last readers are done; false
+        // once the CTA is aborting (lane 0 decides, so the warp leaves together)
+        auto acquire = [&](uint64_t *bar, uint32_t parity, bool need) {
+            if (need) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(bar, parity);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok && lane == 0) ctl->abort = 1;
+            }
+            const int stop = (lane == 0) ? ctl->abort : 0;
+            return __shfl_sync(0xffffffffu, stop, 0) == 0;
+        };
+        if (nchunks > 0) fetch(0);
+        int issuedA = 0, issuedB = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int tm = sq.t0 + c * C;   // tensor-map coordinate of the chunk's first token
+            const uint8_t *item = ws + (bh * ws_chunks + c) * (int64_t)ITEM_BYTES;
+            const int a = c & 1, s = c % L::NB;
+            if (!acquire(&ctl->emptyA[a], (uint32_t)((c >> 1) - 1) & 1u, c >= L::NA)) break;
+            if (lane == 0) {
+                uint8_t *qa = tiles + stage_a(c);
+                mbar_arrive_expect_tx(&ctl->fullA[a], 2u * KA * C * 128u);
+#pragma unroll
+                for (int ka = 0; ka < KA; ++ka) {
+                    tma_load_4d(qa + ka * QK_ACS, &maps.q, &ctl->fullA[a], 64 * ka, (int)h, tm, sq.b0);
+                    bulk_load(qa + ka * QK_ACS + 64 * 128, item + ITEM_U + ka * 8192, 8192, &ctl->fullA[a]);
+                }
+            }
+            issuedA = c + 1;
+            if (!acquire(&ctl->emptyB[s], (uint32_t)((c / L::NB) - 1) & 1u, c >= L::NB)) break;
+            if (lane == 0) {
+                uint8_t *sb = tiles + stage_b(c);
+                mbar_expect_tx(&ctl->fullB[s], KA * C * 128u + C * DVT * 2u + 2u * TT_BYTES);
+#pragma unroll
+                for (int ka = 0; ka < KA; ++ka)
+                    tma_load_4d(sb + L::B_K + ka * 8192, &maps.k, &ctl->fullB[s], 64 * ka, (int)h, tm, sq.b0);
+                tma_load_4d(sb + L::B_V, &maps.v, &ctl->fullB[s], dvt * DVT, (int)h, tm, sq.b0);
+                bulk_load(sb + L::B_T, item + ITEM_T, TT_BYTES, &ctl->fullB[s]);
+                bulk_load(sb + L::B_P, item + ITEM_P, TT_BYTES, &ctl->fullB[s]);
+            }
+            // the chunk's decay factors: gamma = 2^b, gamma_C / gamma = 2^(b_63 - b)
+            (void)gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
+            const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
+            __syncwarp();
+            ctl->gct[s][2 * lane] = exp2f(blast - ctl->b2[s][2 * lane]);
+            ctl->gct[s][2 * lane + 1] = exp2f(blast - ctl->b2[s][2 * lane + 1]);
+            if (c + 1 < nchunks) fetch(c + 1);   // in flight while the next slots free up
+            mbar_arrive(&ctl->fullB[s]);
+            issuedB = c + 1;
+        }
+        // let copies still in flight land before the CTA can exit
+        if (lane == 0) {
+            for (int c = (issuedA > L::NA ? issuedA - L::NA : 0); c < issuedA; ++c)
+                (void)mbar_drain(&ctl->fullA[c & 1], (uint32_t)(c >> 1) & 1u);
+            for (int c = (issuedB > L::NB ? issuedB - L::NB : 0); c < issuedB; ++c)
+                (void)mbar_drain(&ctl->fullB[c % L::NB], (uint32_t)(c / L::NB) & 1u);
+        }
+    } else if (warp < 5) {
+        // ------------------------------------------------------------------ output group
+        const int lt = tid - 32;
+        const bool leader = (lt == 0);
+        const int ro = 32 * quad + lane;   // M=128 row: output rows 0-63 in quads 0, 1
+        // [X2 ; W] = [0 ; T diag(beta)] V of chunk c
+        auto issue_w0 = [&](int c) {
+            const uint32_t zb = tb + stage_b(c) + L::B_Z, vb = tb + stage_b(c) + L::B_V;
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_bf16(tmem + M_XW + 32u * (uint32_t)(c & 1), desc_k(zb, 16384, kk), desc_mn64(vb, kk), ID_XW,
+                          kk > 0);
+            umma_commit(&ctl->w0_done[c & 1]);
+        };
+        if (leader)   // chunks 0 and 1 into the two accumulator buffers
+            for (int c = 0; c < 2 && c < nchunks; ++c) {
+                if (!mbar_wait(&ctl->fullB[c], 0u)) ctl->abort = 1;
+                tc_fence_after_sync();
+                issue_w0(c);
+            }
+        // PW = [P ; K0] W and O = diag(gamma) X2 + PW of chunk j (a failed wait sets
+        // the abort flag; every thread still takes every barrier)
+        auto finish = [&](int j) {
+            const int sj = j % L::NB, jb = j & 1;
+            const int64_t tj = (int64_t)j * C;
+            const int nvalid = (int)min((int64_t)C, sq.len - tj);
+            if (!mbar_wait(&ctl->wready[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
+            const float gam_o = ctl->gam[sj][ro & 63];   // read before the stage can be refilled
+            bar_named(1, 128);
+            if (leader) {
+                // stage j landed long ago (the state group has its W); the wait makes the
+                // copy's completion visible to this thread
+                if (!mbar_wait(&ctl->fullB[sj], (uint32_t)(j / L::NB) & 1u)) ctl->abort = 1;
+                tc_fence_after_sync();
+                const uint32_t ps = tb + stage_b(j) + L::B_P;
+                const uint32_t wsb = tb + L::TWS + (uint32_t)jb * 4096u;
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + M_PW + 32u * jb, desc_k(ps, 16384, kk), desc_mn64(wsb, kk), ID_XW, kk > 0);
+                umma_commit(&ctl->pw_done[jb]);
+                umma_commit(&ctl->emptyB[sj]);
+            }
+            if (!mbar_wait(&ctl->pw_done[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
+            tc_fence_after_sync();
+            if (quad < 2) {
+                float x2[32], pw[32];
+                tmem_ld32(tq + M_XW + 32u * jb, x2);
+                tmem_ld32(tq + M_PW + 32u * jb, pw);
+                tmem_wait_ld();
+                if (ro < nvalid) {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
+                                         ((sq.row0 + tj + ro) * p.H + h) * p.dv + dvt * DVT;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        uint4 u;
+                        u.x = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 0], pw[8 * cc + 0]),
+                                          fmaf(gam_o, x2[8 * cc + 1], pw[8 * cc + 1]));
+                        u.y = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 2], pw[8 * cc + 2]),
+                                          fmaf(gam_o, x2[8 * cc + 3], pw[8 * cc + 3]));
+                        u.z = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 4], pw[8 * cc + 4]),
+                                          fmaf(gam_o, x2[8 * cc + 5], pw[8 * cc + 5]));
+                        u.w = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 6], pw[8 * cc + 6]),
+                                          fmaf(gam_o, x2[8 * cc + 7], pw[8 * cc + 7]));
+                        reinterpret_cast<uint4 *>(dst)[cc] = u;
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            bar_named(1, 128);   // X2 and PW of buffer jb are read
+            if (leader && j + 2 < nchunks) {
+                // chunk j+2's [0 ; T diag(beta)] V into the buffer just read (the state
+                // group read W of chunk j from it before wready)
+                if (!mbar_wait(&ctl->fullB[(j + 2) % L::NB], (uint32_t)((j + 2) / L::NB) & 1u)) ctl->abort = 1;
+                tc_fence_after_sync();
+                issue_w0(j + 2);
+            }
+        };
+        for (int j = 0; j < nchunks; ++j) {
+            const int pb = j & 1;
+            if (leader) ctl->stopL[pb] = ctl->abort;
+            bar_named(1, 128);
+            if (ctl->stopL[pb]) break;
+            finish(j);
+        }
+        if (leader) umma_commit(&ctl->drain);
+    } else {
+        // ------------------------------------------------------------------ state group
+        const int st = tid - 160;
+        const bool leader = (st == 0);
+        const int d = 32 * quad + lane;   // state row
+        float S[DVT];
+        {
+            const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVT) : nullptr;
+#pragma unroll
+            for (int j = 0; j < DVT; j += 4) {
+                float4 x = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
+                S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+            }
+            store_row64(tiles + L::TSS, d, S);
+        }
+        fence_proxy_async_smem();
+        bar_named(2, 128);
+        // [X2 ; W] += [Q ; -U] S0 of chunk c, once [0 ; T diag(beta)] V of chunk c is
+        // in the accumulator and the ring-A stage has landed
+        auto issue_xk = [&](int c) {
+            bool ok = mbar_wait(&ctl->w0_done[c & 1], (uint32_t)(c >> 1) & 1u);
+            ok = mbar_wait(&ctl->fullA[c & 1], (uint32_t)(c >> 1) & 1u) && ok;
+            if (!ok) ctl->abort = 1;
+            tc_fence_after_sync();
+            const uint32_t qa = tb + stage_a(c);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk)
+                umma_bf16(tmem + M_XW + 32u * (uint32_t)(c & 1), desc_k(qa, QK_ACS, kk),
+                          desc_mn64(tb + L::TSS, kk), ID_XW, 1u);
+            umma_commit(&ctl->xk_done);
+            umma_commit(&ctl->emptyA[c & 1]);
+        };
+        if (leader && nchunks > 0) issue_xk(0);
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % L::NB, pb = c & 1;
+            if (leader) ctl->stopS = ctl->abort;
+            bar_named(2, 128);
+            if (ctl->stopS) break;
+            bool ok = mbar_wait(&ctl->fullB[s], (uint32_t)(c / L::NB) & 1u);
+            ok = mbar_wait(&ctl->xk_done, (uint32_t)c & 1u) && ok;
+            if (!ok) ctl->abort = 1;
+            tc_fence_after_sync();
+            const float gC = ctl->gam[s][C - 1];   // read before the stage can be refilled
+            if (quad >= 2) {   // W row t -> bf16 W (for PW) and diag(gamma_C / gamma) W (for dS)
+                const int t = d - 64;
+                // PW of chunk c-2 has read W buffer pb
+                if (c >= 2 && !mbar_wait(&ctl->pw_done[pb], (uint32_t)((c - 2) >> 1) & 1u)) ctl->abort = 1;
+                float w[32];
+                tmem_ld32(tq + M_XW + 32u * pb, w);
+                const float g = ctl->gct[s][t];
+                tmem_wait_ld();
+                store_row64(tiles + L::TWS + (uint32_t)pb * 4096u, t, w);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) w[j] *= g;
+                store_row64(tiles + L::TWGS, t, w);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            mbar_arrive(&ctl->wready[pb]);   // the output group may issue PW(c)
+            bar_named(2, 128);
+            if (leader) {   // dS = K^T diag(gamma_C / gamma) W, K = tokens
+                tc_fence_after_sync();
+                const uint32_t kb = tb + stage_b(c) + L::B_K;
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    umma_bf16(tmem + M_DS, desc_mn128(kb, C * 128, kk), desc_mn64(tb + L::TWGS, kk), ID_DS, kk > 0);
+                umma_commit(&ctl->ds_done);
+                umma_commit(&ctl->emptyB[s]);
+            }
+            if (!mbar_wait(&ctl->ds_done, (uint32_t)c & 1u)) ctl->abort = 1;
+            tc_fence_after_sync();
+            {   // S <- gamma_C S + dS, then its bf16 copy for chunk c+1 ([Q ; -U] S0 of
+                // chunk c has finished: xk_done)
+                float ds[DVT];
+                tmem_ld32(tq + M_DS, ds);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < DVT; ++j) S[j] = fmaf(gC, S[j], ds[j]);
+                store_row64(tiles + L::TSS, d, S);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before_sync();
+            bar_named(2, 128);
+            if (leader && c + 1 < nchunks) issue_xk(c + 1);
+        }
+        if (leader) {   // every MMA issued by either group has finished before TMEM is released
+            umma_commit(&ctl->drain);
+            (void)mbar_drain(&ctl->drain, 0u);
+        }
+        if (!ctl->abort && p.S_out) {
+            float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVT);
+#pragma unroll
+            for (int j = 0; j < DVT; j += 4)
+                *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 0) tmem_dealloc(tmem, M_TMEM_COLS);
 }
 
 }  // namespace ck

@@ -429,13 +429,14 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         e = allow_smem((const void *)gdn_prep_kernel, psmem);
         // one wave of resident CTAs walks all items (a second, partial wave
         // would double the time)
-        const int per_sm = resident_per_sm((const void *)gdn_prep_kernel, gdn::PREP_THREADS, psmem, 64);
+        const int per_sm =
+            resident_per_sm((const void *)gdn_prep_kernel, gdn::PREP_THREADS, psmem, (int)gdn::PREP_TMEM_COLS);
         const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
         if (e == cudaSuccess && items > 0) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.q, m.k, pp);
-        const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::GL<false>::TEND;
-        if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel<false>, smem);
+        const int smem = (int)((sizeof(gdn::MCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::ML::TEND;
+        if (e == cudaSuccess) e = allow_smem((const void *)gdn_main_kernel, smem);
         if (e == cudaSuccess)
-            chunk_gdn_kernel<false><<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));
+            gdn_main_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));
     } else {
         // packed sequences walk each sequence in one pass (no segments)
         const SegPlan sp = packed ? SegPlan{1, 1, (int)((Lmax + C - 1) / C)} : seg_plan(rule, p.B, p.T, p.H, p.dv);

@@ -115,9 +115,10 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *   workspace / workspace_bytes: device scratch of at least
  *          la_fwd_workspace_size() bytes, 16-byte aligned (may be NULL when that
  *          size is 0).  The gated delta rule on the tensor-core path (bf16,
- *          dk = 128) needs 16 KB per (batch, head, 64-token chunk): the chunk's
- *          T = (I + A)^-1 and masked, decayed score operands, written by a first
- *          kernel and read by the second within the same call.  ELU+1 and GLA over few heads and long
+ *          dk = 128) needs 32 KB per (batch, head, 64-token chunk): the chunk's
+ *          T diag(beta) (T = (I + A)^-1), masked decayed score and
+ *          -T diag(beta gamma) K operands, written by a first kernel and read by
+ *          the second within the same call.  ELU+1 and GLA over few heads and long
  *          sequences run segment-parallel and keep there the summary of each
  *          piece of every segment but the last (dk*dv + dk floats per piece: the
  *          piece's state contribution and its normaliser sum or gate product).
@@ -261,8 +262,8 @@ la_status la_fwd_host(const la_fwd_args *host_args, void *staging, size_t stagin
  *
  *   - The problem's scratch need (la_fwd_workspace_size) must be at most
  *     LA_NOALLOC_SCRATCH_BYTES, otherwise LA_ERR_WORKSPACE is returned before
- *     anything is launched.  For the gated delta rule that is 1024
- *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 4096.
+ *     anything is launched.  For the gated delta rule that is 512
+ *     (batch x head x 64-token chunk) units, e.g. B*H = 16 up to T = 2048.
  *     ELU+1 and GLA use the array when they split long sequences of few heads
  *     into segments (the segment summaries, dk*dv + dk floats per piece); the
  *     number of pieces is bounded by the SM count, so that need always fits.

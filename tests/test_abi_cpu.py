@@ -94,10 +94,10 @@ def test_rule_specific_gate_checks(L):
 def test_null_args_and_workspace_query(L):
     assert L.la_fwd(None, None) == 1
     n = ctypes.c_size_t(123)
-    # gated delta rule, bf16, dk=128: the 8 KB T and 8 KB P operand images per
-    # (batch, head, 64-token chunk)
+    # gated delta rule, bf16, dk=128: the 8 KB T diag(beta), 8 KB P and 16 KB -U
+    # operand images per (batch, head, 64-token chunk)
     assert L.la_fwd_workspace_size(ctypes.byref(args(T=130)), ctypes.byref(n)) == 0
-    assert n.value == 1 * 2 * 3 * 16384
+    assert n.value == 1 * 2 * 3 * 32768
     for a in (args("elu"), args(dtype=0), args(dk=64), args(T=0), args("gla", dtype=0)):
         assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
         assert n.value == 0
@@ -188,19 +188,19 @@ def test_version1_struct_size_still_accepted(L):
     a.cu_seqlens = 0xDEAD   # past the caller's struct: must be ignored
     n = ctypes.c_size_t(0)
     assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
-    assert n.value == 1 * 2 * 3 * 16384
+    assert n.value == 1 * 2 * 3 * 32768
     a.struct_size = la.FwdArgs.cu_seqlens.offset - 8
     assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 1
 
 
 def test_packed_workspace_follows_max_seqlen(L):
-    """Gated delta rule: the 16 KB T and P images per (sequence, head, 64-token
-    chunk of the longest sequence); packed ELU+1 runs without segments (no
-    workspace)."""
+    """Gated delta rule: the 32 KB of operand images per (sequence, head,
+    64-token chunk of the longest sequence); packed ELU+1 runs without segments
+    (no workspace)."""
     n = ctypes.c_size_t(0)
     a = args(B=5, T=1000, H=2, cu_seqlens=FAKE, max_seqlen=300)
     assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
-    assert n.value == 5 * 2 * 5 * 16384
+    assert n.value == 5 * 2 * 5 * 32768
     a = args("elu", B=1, T=40000, H=2, cu_seqlens=FAKE, max_seqlen=40000)
     assert L.la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
     assert n.value == 0

@@ -81,7 +81,7 @@ def test_oversized_problem_refused_on_host():
     a = la.FwdArgs()
     a.struct_size = ctypes.sizeof(a)
     a.rule, a.dtype = 2, 1
-    a.B, a.T, a.H, a.dk, a.dv = 1, 64 * 65, 32, 128, 128      # 2080 chunk units > 1024
+    a.B, a.T, a.H, a.dk, a.dv = 1, 64 * 65, 32, 128, 128      # 2080 chunk units > 512
     a.q = a.k = a.v = a.o = a.g = a.beta = 0x10000
     assert L.la_fwd_noalloc(ctypes.byref(a), None) == 8
     assert b"la_fwd_noalloc" in L.la_last_error_message()
