@@ -177,10 +177,12 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 LEG_NAMES = ["gla_prefill", "gdn_prefill", "elu_prefill", "gla_decode", "gdn_decode"]
-# kernels per call: gated delta rule 2 (T operand images, then the main pass);
-# GLA and ELU+1 at these shapes 2 each (range summaries of the earlier sequence
-# segments, then the segment-parallel main pass); each decode step 1
-LEG_LAUNCHES = {"gla_prefill": 2, "gdn_prefill": 2, "elu_prefill": 2, "gla_decode": 1, "gdn_decode": 1,
+# kernels per call: gated delta rule 2 (operand images, then the main pass);
+# ELU+1 at its shape 2 (summaries of the earlier sequence segments, then the
+# segment-parallel main pass); GLA 3 (the same two, then the per-token kernel
+# over the sequences the chunked form flagged, launched dependent on the main
+# pass and exiting at once when none is flagged); each decode step 1
+LEG_LAUNCHES = {"gla_prefill": 3, "gdn_prefill": 2, "elu_prefill": 2, "gla_decode": 1, "gdn_decode": 1,
                 "kda_prefill": 2}
 # legs that --profile-leg can run but the timed step does not: KDA prefill at the
 # prefill benchmark shape (prep kernel, then the KDA main pass)

@@ -5,8 +5,9 @@ applies (page "状态空间与线性注意力", KDA section).
 
 Reference: the fp64 oracle's recurrence followed by ``oracle.head_rmsnorm`` on
 its exact output.  The library normalises its stored (bf16-rounded for bf16
-problems) output and rounds once more.  The state is not touched by the
-normalisation: it must equal, bit for bit, the state of the same call without it.
+problems) output in a second pass and rounds once more.  The state is not
+touched by the normalisation: it must equal, bit for bit, the state of the same
+call without it.
 
 Bounds.  Every rule but KDA: the normalised output is held to the fixed bf16
 (2e-2) or fp32 (1e-4) bound against the oracle's normalised output, like any
@@ -96,6 +97,26 @@ def test_norm_every_rule_and_path(la, rule, dk, dv, dtype):
     check_norm(la, p, weight(dv, 3), TOL_F32 if dtype == torch.float32 else TOL_BF16)
 
 
+@pytest.mark.parametrize("rule,T", [("elu", 300), ("elu", 3000), ("gla", 777)])
+def test_norm_over_two_value_slabs(la, rule, T):
+    """dv = 128: each row spans two 64-column value slabs of the chunked kernel
+    (T = 3000 over 3 heads also runs segment-parallel)."""
+    kw = {"gla_gate": "ones"} if rule == "gla" else {}
+    p = workloads.make_problem(rule, 1, T, 3, 128, 128, seed=T + 1, init_state="normal", **kw)
+    check_norm(la, p, weight(128, T), TOL_BF16)
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+def test_norm_on_recomputed_gla_sequences(la, dv):
+    """GLA gates of 0.02 take every chunk out of the chunked form's range: the
+    sequences are recomputed by the per-token kernel before the normalisation
+    pass."""
+    p = workloads.make_problem("gla", 2, 300, 2, 128, dv, seed=dv, init_state="normal")
+    p = workloads.Problem("gla", p.q, p.k, p.v, torch.full((2, 300, 2, 128), 0.02), None, p.S0, None, p.eps,
+                          f"gla_0.02_norm_dv{dv}")
+    check_norm(la, p, weight(dv, 4), TOL_BF16)
+
+
 def test_norm_eps_matters_for_small_rows(la):
     """A large eps against an output of small RMS scales the rows down rather than
     up to unit RMS; the library follows the oracle there too."""
@@ -122,14 +143,15 @@ def test_decode_step_with_norm(la, rule, variant):
     assert rel_err(S.cpu().numpy(), S_ref) <= TOL_BF16
 
 
-def test_packed_sequences_with_norm(la):
+@pytest.mark.parametrize("dv", [64, 128])
+def test_packed_sequences_with_norm(la, dv):
     lengths = [70, 0, 3, 200]
-    parts = [workloads.make_problem("gla", 1, L, 2, 128, 64, gla_gate="ones", seed=80 + i, init_state="normal")
+    parts = [workloads.make_problem("gla", 1, L, 2, 128, dv, gla_gate="ones", seed=80 + i, init_state="normal")
              for i, L in enumerate(lengths)]
     cat = lambda n: torch.cat([getattr(p, n) for p in parts], dim=1).contiguous().cuda()
     S0 = torch.cat([p.S0 for p in parts], dim=0).contiguous().cuda()
     cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int64).cuda()
-    w = weight(64, 8)
+    w = weight(dv, 8)
     o, S, _ = la.fwd("gla", cat("q"), cat("k"), cat("v"), cat("g"), S0=S0, cu_seqlens=cu,
                      max_seqlen=max(lengths), out_norm=True, norm_w=w.cuda(), norm_eps=EPS_N)
     torch.cuda.synchronize()
