@@ -96,14 +96,13 @@ struct GL {
     static constexpr uint32_t TEND = TSS + 2 * 8192;
 };
 
-// Prep-kernel shared memory.  Each of the two 64-column atom columns of q and k
-// holds three [64][64] blocks, K0 | Q | K1: item i's K lands in slot i & 1, so
-// that [K0 ; Q] (even items) or [Q ; K1] (odd items) is one M=128 operand, and
-// the next item's K can be loaded while this item's -U MMA still reads its own.
+// Prep-kernel shared memory: [Q ; K] as two atom columns of 128 rows (Q rows
+// 0-63, K rows 64-127), one M=128 operand.  The next item's Q is loaded once
+// this item's [Q ; K] K^T has read it, its K once the -U MMA has.
 constexpr int AF_LD = 68;
 constexpr int TMP_LD = 36;
-constexpr uint32_t P_ACS = 3 * 8192;                 // atom column: K0 | Q | K1
-constexpr uint32_t P_Q = 8192;                       // Q block within an atom column
+constexpr uint32_t P_ACS = QK_ACS;                   // atom column: Q | K
+constexpr uint32_t P_K = 8192;                       // K block within an atom column
 constexpr uint32_t P_AF = 2 * P_ACS;                 // A, then T, fp32 [64][AF_LD]; then the
                                                      // T diag(beta gamma) operand image (bf16)
 constexpr uint32_t P_TMP = P_AF + 64 * AF_LD * 4;    // fp32 scratch [32][TMP_LD]
@@ -112,6 +111,7 @@ static_assert(P_END % 16 == 0, "the prep kernel's control block must be 16-byte 
 static_assert(P_AF % 1024 == 0, "the operand image in AF must be 1 KB aligned");
 constexpr int PREP_THREADS = 128;
 constexpr uint32_t PREP_TMEM_COLS = 128;
+constexpr int PREP_CTAS_PER_SM = 4;
 
 struct GCtl {
     uint64_t full[NSTG], empty[NSTG];
@@ -125,12 +125,11 @@ struct GCtl {
 };
 
 struct PCtl {
-    uint64_t full, mma, mma_u, drain;
+    uint64_t qfull, kfull, mma, mma_u, drain;
     uint32_t tmem_base;
     int abort, stop, fast;
-    // 16-byte aligned (the block starts 16-byte aligned and the fields before
-    // take 48 bytes): read as float4
-    float alpha[64], beta[64];
+    // read as float4 (the block itself starts 16-byte aligned)
+    alignas(16) float alpha[64], beta[64];
     float gam[64], ginv[64], b2[64];
 };
 static_assert(offsetof(PCtl, alpha) % 16 == 0, "PCtl's gate arrays are read as float4");
@@ -391,16 +390,16 @@ struct GdnPrepParams {
 };
 
 // One CTA handles (batch, head, chunk) items in a grid-stride loop.  The next
-// item's Q and K are loaded (TMA) as soon as this item's [Q ; K] K^T MMA has
-// read Q (K goes to the other K slot), and its alpha and beta are fetched into
-// registers at the same point, so neither load is waited for.  The grid is
-// sized to the CTAs that are resident at once (3 per SM: 71 KB of shared
-// memory, 128 TMEM columns).
+// item's Q is loaded (TMA) as soon as this item's [Q ; K] K^T MMA has read it,
+// its alpha and beta are fetched into registers at the same point, and its K
+// once this item's -U MMA has read K.  The grid is sized to the CTAs that are
+// resident at once (4 per SM: 55 KB of shared memory, 128 TMEM columns), so
+// that the other CTAs of an SM cover a load still in flight.
 //
 // Per item: [Q ; K] K^T -> P (to the item) and A; T = (I + A)^-1; the item's
 // T diag(beta) image; then -U = -(T diag(beta gamma)) K as one M=64, N=128 MMA
 // whose A operand is written over AF, and its image.
-__global__ void __launch_bounds__(gdn::PREP_THREADS, 3)
+__global__ void __launch_bounds__(gdn::PREP_THREADS, gdn::PREP_CTAS_PER_SM)
 gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant__ CUtensorMap mapk,
                 const GdnPrepParams p) {
     using namespace gdn;
@@ -414,7 +413,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
     float *TMP = reinterpret_cast<float *>(tiles + P_TMP);
 
     if (tid == 0) {
-        mbar_init(&ctl->full, 1);
+        mbar_init(&ctl->qfull, 1);
+        mbar_init(&ctl->kfull, 1);
         mbar_init(&ctl->mma, 1);
         mbar_init(&ctl->mma_u, 1);
         mbar_init(&ctl->drain, 1);
@@ -440,18 +440,15 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
         const uint32_t bh = wu / nch;
         return ItemPos{(int64_t)(bh / H), (int64_t)(bh % H), (int)(wu - bh * nch)};
     };
-    // warp 2, lane 0: TMA of item w's Q (the Q blocks) and K (K slot `slot`)
-    auto load_qk = [&](int64_t w, int slot) {
+    // warp 2, lane 0: TMA of item w's Q (kq = 0) or K (kq = 1)
+    auto load_half = [&](int64_t w, int kq) {
         const ItemPos ip = item_pos(w);
-        const int64_t h = ip.h;
-        const int c = ip.c;
         const SeqSpan sq = seq_span(p.cu_seqlens, ip.b, p.T, p.max_seqlen, false);
-        mbar_arrive_expect_tx(&ctl->full, 2u * KA * C * 128u);
-        for (int a = 0; a < KA; ++a) {
-            tma_load_4d(tiles + a * P_ACS + P_Q, &mapq, &ctl->full, 64 * a, (int)h, sq.t0 + c * C, sq.b0);
-            tma_load_4d(tiles + a * P_ACS + 16384u * slot, &mapk, &ctl->full, 64 * a, (int)h, sq.t0 + c * C,
-                        sq.b0);
-        }
+        uint64_t *bar = kq ? &ctl->kfull : &ctl->qfull;
+        mbar_arrive_expect_tx(bar, KA * C * 128u);
+        for (int a = 0; a < KA; ++a)
+            tma_load_4d(tiles + a * P_ACS + (kq ? P_K : 0u), kq ? &mapk : &mapq, bar, 64 * a, (int)ip.h,
+                        sq.t0 + ip.c * C, sq.b0);
     };
     // warp 2: item w's alpha, beta for tokens 2*lane, 2*lane+1, loaded unconditionally
     // (a clamped index) so that nothing waits for them before their use one item
@@ -477,13 +474,16 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
     constexpr uint32_t ID_U = idesc_bf16(64, 128, false, true);
     int it = 0;
     if (warp == 2 && (int64_t)blockIdx.x < items) {
-        if (lane == 0) load_qk(blockIdx.x, 0);
+        if (lane == 0) {
+            load_half(blockIdx.x, 0);
+            load_half(blockIdx.x, 1);
+        }
         fetch_gates(blockIdx.x);
     }
-    bool k_pending = (int64_t)blockIdx.x < items;   // a copy is in flight (thread 64's view)
+    // copies in flight (thread 64's view)
+    bool q_pending = (int64_t)blockIdx.x < items, k_pending = q_pending;
+    const uint32_t kb = tb + P_K;   // the K rows (atom column 0)
     for (int64_t w = blockIdx.x; w < items; w += gridDim.x, ++it) {
-        const int slot = it & 1;                      // this item's K slot
-        const uint32_t kslot = tb + 16384u * (uint32_t)slot;
         if (warp == 2) {   // this item's gates (fetched one item ahead) into shared memory
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -494,34 +494,35 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
         if (tid == 0) ctl->stop = ctl->abort;   // one thread decides, everyone reads after the barrier
         bar_named(1, 128);
         if (ctl->stop) break;
-        if (!mbar_wait(&ctl->full, (uint32_t)it & 1u)) ctl->abort = 1;
-        if (tid == 64) k_pending = false;
+        bool landed = mbar_wait(&ctl->qfull, (uint32_t)it & 1u);
+        landed = mbar_wait(&ctl->kfull, (uint32_t)it & 1u) && landed;
+        if (!landed) ctl->abort = 1;
+        if (tid == 64) q_pending = k_pending = false;
         if (warp == 0)
             ctl->fast = gate_scan(&ctl->alpha[2 * lane], ctl->beta, ctl->b2, ctl->gam, ctl->ginv, nullptr, lane);
-        if (tid == 32) {   // [K0 ; Q] K^T (even items) or [Q ; K1] K^T (odd items)
+        if (tid == 32) {   // [Q ; K] K^T: rows 0-63 Q K^T, rows 64-127 K K^T
             tc_fence_after_sync();
-            const uint32_t a0 = tb + 8192u * (uint32_t)slot;
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem, desc_k(a0, P_ACS, kk), desc_k(kslot, P_ACS, kk), ID_QK, kk > 0);
+                umma_bf16(tmem, desc_k(tb, P_ACS, kk), desc_k(kb, P_ACS, kk), ID_QK, kk > 0);
             umma_commit(&ctl->mma);
         }
         bar_named(1, 128);
         if (!mbar_wait(&ctl->mma, (uint32_t)it & 1u)) ctl->abort = 1;
         tc_fence_after_sync();
-        // Q and the other K slot are free: start the next item's loads
+        // Q is free: start the next item's Q and gates
         if (warp == 2 && w + gridDim.x < items) {
             if (lane == 0 && !ctl->abort) {
-                load_qk(w + gridDim.x, slot ^ 1);
-                k_pending = true;
+                load_half(w + gridDim.x, 0);
+                q_pending = true;
             }
             fetch_gates(w + gridDim.x);
         }
-        {   // row r = tid of the M=128 accumulator: the rows of Q give the P row of
-            // token r & 63 (inclusive mask, to the item's P image), the rows of K the
-            // A row of token r & 63 (strict mask, times beta, to AF)
+        {   // row r = tid of the M=128 accumulator: warps 0-1 the P row of token r
+            // (inclusive mask, to the item's P image), warps 2-3 the A row of token
+            // r - 64 (strict mask, times beta, to AF)
             const int t = tid & 63;
-            const bool prow = (warp < 2) == (slot == 1);
+            const bool prow = warp < 2;
             float x[64];
             tmem_ld32(tq, *reinterpret_cast<float(*)[32]>(x));
             tmem_ld32(tq + 32u, *reinterpret_cast<float(*)[32]>(x + 32));
@@ -594,11 +595,16 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
             tc_fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
-                umma_bf16(tmem, desc_k(tb + P_AF, C * 128, kk), desc_mn128(kslot, P_ACS, kk), ID_U, kk > 0);
+                umma_bf16(tmem, desc_k(tb + P_AF, C * 128, kk), desc_mn128(kb, P_ACS, kk), ID_U, kk > 0);
             umma_commit(&ctl->mma_u);
         }
         if (!mbar_wait(&ctl->mma_u, (uint32_t)it & 1u)) ctl->abort = 1;
         tc_fence_after_sync();
+        // K is free: the next item's K
+        if (tid == 64 && w + gridDim.x < items && !ctl->abort) {
+            load_half(w + gridDim.x, 1);
+            k_pending = true;
+        }
         {   // -U -> the item: row tr = 16 warp + (lane & 15) of the M=64 accumulator,
             // key columns 64 hf .. 64 hf + 63 = block hf of the image
             const int tr = 16 * warp + (lane & 15), hf = lane >> 4;
@@ -622,7 +628,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
     }
     // let a prefetched copy land and every MMA finish before the CTA frees TMEM
     // and exits (these two waits keep the long limit even after a timeout)
-    if (tid == 64 && k_pending) (void)mbar_drain(&ctl->full, (uint32_t)it & 1u);
+    if (tid == 64 && q_pending) (void)mbar_drain(&ctl->qfull, (uint32_t)it & 1u);
+    if (tid == 64 && k_pending) (void)mbar_drain(&ctl->kfull, (uint32_t)it & 1u);
     if (tid == 32) {
         umma_commit(&ctl->drain);
         (void)mbar_drain(&ctl->drain, 0u);
