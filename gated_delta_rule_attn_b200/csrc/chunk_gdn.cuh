@@ -1,5 +1,5 @@
-// chunk_gdn.cuh — gated delta rule, chunked prefill: two kernels (and the
-// templated main pass that KDA shares, chunk_gdn_kernel<true>).
+// chunk_gdn.cuh — gated delta rule, chunked prefill: two kernels (the main pass
+// is templated: KDA runs it on its own prep kernel's outputs, gdn_main_kernel<true>).
 //
 // gdn_prep_kernel (fully parallel over (batch, head, chunk)): for each 64-token
 //   chunk, the state-independent parts, from one M=128 MMA [Q ; K] K^T:
@@ -39,63 +39,36 @@ namespace la {
 namespace ck {
 namespace gdn {
 
-constexpr int NSTG = 3;
-constexpr int NTHREADS = 288;
-constexpr uint32_t TMEM_COLS = 512;
-// TMEM columns of the main kernel (columns 0-127 unused)
-constexpr uint32_t C_XK = 128;   // 2 x 32, M=128 [Q ; K] S0
-constexpr uint32_t C_W = 192;    // 32,     M=64  W = T R
-constexpr uint32_t C_DS = 224;   // 32,     M=128 dS
-constexpr uint32_t C_PW = 256;   // 2 x 32, M=128 [P ; 0] W (rows 0-63)
+constexpr int NTHREADS = 288;   // the main pass: producer, output group, state group
 
 constexpr uint32_t TT_BYTES = 8192;                  // T, bf16 [64][64]
 // Workspace item per (batch, head, chunk), written by the prep kernel: operand
 // images, bf16, 128-byte swizzled exactly as the main kernel's shared memory
 // wants them: T diag(beta) [64][64], P [64][64] and -U = -T diag(beta gamma) K as
 // two [64][64] blocks (key columns 0-63, 64-127).  KDA's item (chunk_kda.cuh)
-// shares the T and P offsets (its T image is T itself) and appends Gamma_C.
+// has the same three images (its U is T diag(beta) (K o Gamma)) and appends
+// Gamma_C.
 constexpr uint32_t ITEM_T = 0;
 constexpr uint32_t ITEM_P = 8192;
 constexpr uint32_t ITEM_U = 16384;
 constexpr uint32_t ITEM_BYTES = 32768;
 
 constexpr uint32_t QK_ACS = 128 * 128;               // one atom column: Q rows 0-63, K rows 64-127
-constexpr uint32_t STG_QK_BYTES = 2 * QK_ACS;
 
 }  // namespace gdn
 
 // KDA workspace item per (batch, head, chunk), written by kda_prep_kernel
-// (chunk_kda.cuh) and read by chunk_gdn_kernel<true>: the gated delta rule's
+// (chunk_kda.cuh) and read by gdn_main_kernel<true>: the gated delta rule's
 // item, then Gamma_C.
 namespace kda {
-constexpr uint32_t ITEM_T = gdn::ITEM_T;      // T image
+constexpr uint32_t ITEM_T = gdn::ITEM_T;      // T diag(beta) image
 constexpr uint32_t ITEM_P = gdn::ITEM_P;      // P image
-constexpr uint32_t ITEM_GC = 16384;           // Gamma_C, fp32 [128]
-constexpr uint32_t ITEM_BYTES = 16384 + 512;
+constexpr uint32_t ITEM_U = gdn::ITEM_U;      // -U = -T diag(beta) (K o Gamma), two [64][64] blocks
+constexpr uint32_t ITEM_GC = 32768;           // Gamma_C, fp32 [128]
+constexpr uint32_t ITEM_BYTES = 32768 + 512;
 }  // namespace kda
 
 namespace gdn {
-// Main-kernel shared memory of chunk_gdn_kernel<KDA> (byte offsets from a 1 KB
-// aligned base).  Every stage holds [Q ; K] (KDA: [Qp ; Kp], plus Kc), a V slab
-// ([64][32] bf16, 64-byte swizzle), T, and the P image in rows 0-63 of a
-// [P ; 0] tile whose rows 64-127 stay zero (KDA: and Gamma_C).  KDA keeps 2
-// stages and needs no gamma_C/gamma W copy.
-template <bool KDA>
-struct GL {
-    static constexpr int NSTG = KDA ? 2 : gdn::NSTG;
-    static constexpr uint32_t STG_QK = 0;                                       // [Q ; K] (KDA: [Qp ; Kp])
-    static constexpr uint32_t STG_KC = STG_QK + NSTG * STG_QK_BYTES;            // KDA: Kc [64][128]
-    static constexpr uint32_t STG_V = STG_KC + (KDA ? NSTG * 16384u : 0u);
-    static constexpr uint32_t STG_TT = STG_V + NSTG * 4096u;
-    static constexpr uint32_t STG_P = STG_TT + NSTG * TT_BYTES;                 // [P ; 0]
-    static constexpr uint32_t STG_GC = STG_P + NSTG * 16384u;                   // KDA: Gamma_C fp32 [128]
-    static constexpr uint32_t TR = STG_GC + (KDA ? 1024u : 0u);                 // R [64][32] 64 B swizzle
-    static constexpr uint32_t TWS = TR + 4096;                                  // 2 x W
-    static constexpr uint32_t TWGS = TWS + 2 * 4096;                            // GDN: gamma_C/gamma W
-    static constexpr uint32_t TSS = TWGS + (KDA ? 0u : 4096u);                  // 2 x S [128][32] 64 B swizzle
-    static constexpr uint32_t TEND = TSS + 2 * 8192;
-};
-
 // Prep-kernel shared memory: [Q ; K] as two atom columns of 128 rows (Q rows
 // 0-63, K rows 64-127), one M=128 operand.  The next item's Q is loaded once
 // this item's [Q ; K] K^T has read it, its K once the -U MMA has.
@@ -112,17 +85,6 @@ static_assert(P_AF % 1024 == 0, "the operand image in AF must be 1 KB aligned");
 constexpr int PREP_THREADS = 128;
 constexpr uint32_t PREP_TMEM_COLS = 128;
 constexpr int PREP_CTAS_PER_SM = 4;
-
-struct GCtl {
-    uint64_t full[NSTG], empty[NSTG];
-    uint64_t wready[2], pw_done[2], oA[2], xk_done, w_done, ds_done, drain;
-    uint32_t tmem_base;
-    int abort, stopS, stopL[2];
-    int fast[NSTG];
-    // per stage: b = log2 of the inclusive cumulative alpha, gamma = 2^b,
-    // 1/gamma, gamma_C/gamma and beta (written by the producer)
-    float b2[NSTG][64], gam[NSTG][64], ginv[NSTG][64], gct[NSTG][64], bet[NSTG][64];
-};
 
 struct PCtl {
     uint64_t qfull, kfull, mma, mma_u, drain;
@@ -642,397 +604,6 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
 
 
 
-// KDA = true: the KDA main pass (chunk_kda.cuh has the algebra); maps.q, maps.k
-// and maps.kc then cover the prep kernel's Qp, Kp and Kc tensors and `ws` its
-// per-chunk items (T image, P image, Gamma_C).
-template <bool KDA>
-__global__ void __launch_bounds__(gdn::NTHREADS, 1)
-chunk_gdn_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const uint8_t *ws) {
-    using namespace gdn;
-    using L = gdn::GL<KDA>;
-    constexpr int NSTG = L::NSTG;
-    constexpr uint32_t ITEM = KDA ? kda::ITEM_BYTES : ITEM_BYTES;   // workspace bytes per chunk
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    GCtl *ctl = reinterpret_cast<GCtl *>(smem_raw);
-    uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(GCtl) + (smem_u32(smem_raw) & 1023u)) -
-                     (smem_u32(smem_raw) & 1023u);
-    const uint32_t tb = smem_u32(tiles);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3;
-    const int nslab = (int)(p.dv / DVT);
-    const int dvt = (int)(blockIdx.x % nslab);
-    const int64_t bh = blockIdx.x / nslab;
-    const int64_t b = bh / p.H, h = bh % p.H;
-    // this sequence's tokens (dense: all T of batch b); T images are stored for
-    // ceil(max_seqlen / 64) chunks per (batch, head)
-    const SeqSpan sq = seq_span(p.cu_seqlens, b, p.T, p.max_seqlen, tid == 0 && h == 0 && dvt == 0);
-    const int nchunks = (int)((sq.len + C - 1) / C);
-    const int64_t ws_chunks = (p.max_seqlen + C - 1) / C;
-
-    if (tid == 0) {
-        for (int s = 0; s < NSTG; ++s) {
-            mbar_init(&ctl->full[s], 32);
-            mbar_init(&ctl->empty[s], 2);   // the state group's and the score group's MMAs
-        }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&ctl->wready[i], 128);
-            mbar_init(&ctl->pw_done[i], 1);
-            mbar_init(&ctl->oA[i], 128);
-        }
-        mbar_init(&ctl->xk_done, 1);
-        mbar_init(&ctl->w_done, 1);
-        mbar_init(&ctl->ds_done, 1);
-        mbar_init(&ctl->drain, 2);   // one commit from each MMA-issuing thread
-        ctl->abort = 0;
-        fence_barrier_init();
-        tma_prefetch_desc(&maps.q);
-        tma_prefetch_desc(&maps.k);
-        tma_prefetch_desc(&maps.v);
-    }
-    if (warp == 0) {
-        tmem_alloc(&ctl->tmem_base, TMEM_COLS);
-        tc_fence_before_sync();
-    }
-    // rows 64-127 of every stage's [P ; 0] tile stay zero
-    for (int i = tid; i < NSTG * 8192 / 16; i += NTHREADS) {
-        const int tile = i / 512, off = (i % 512) * 16;
-        *reinterpret_cast<uint4 *>(tiles + L::STG_P + tile * 16384 + 8192 + off) = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem = ctl->tmem_base;
-    const uint32_t tq = tmem + ((uint32_t)(32 * quad) << 16);   // this warp's TMEM lanes
-
-    constexpr uint32_t ID_XK = idesc_bf16(128, DVT, false, true);
-    constexpr uint32_t ID_W = idesc_bf16(64, DVT, false, true);
-    constexpr uint32_t ID_DS = idesc_bf16(128, DVT, true, true);
-
-    auto stage_qk = [&](int c) { return tb + L::STG_QK + (uint32_t)(c % NSTG) * STG_QK_BYTES; };
-    auto stage_v = [&](int c) { return tiles + L::STG_V + (uint32_t)(c % NSTG) * 4096u; };
-    auto stage_tt = [&](int c) { return tb + L::STG_TT + (uint32_t)(c % NSTG) * TT_BYTES; };
-
-    if (warp == 0) {
-        // ------------------------------------------------------------------ producer
-        int issued = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % NSTG;
-            if (c >= NSTG) {   // the stage's last readers are done
-                int ok = 1;
-                if (lane == 0) ok = mbar_wait(&ctl->empty[s], (uint32_t)((c / NSTG) - 1) & 1u);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok && lane == 0) ctl->abort = 1;
-            }
-            int stop = (lane == 0) ? ctl->abort : 0;
-            stop = __shfl_sync(0xffffffffu, stop, 0);
-            if (stop) break;
-            const int t0 = c * C;   // position in the sequence
-            if (lane == 0) {
-                mbar_expect_tx(&ctl->full[s], KDA ? 3u * KA * C * 128u + C * DVT * 2u + 2u * TT_BYTES + 512u
-                                                  : 2u * KA * C * 128u + C * DVT * 2u + 2u * TT_BYTES);
-                uint8_t *qk = tiles + L::STG_QK + s * STG_QK_BYTES;
-                const int tm = sq.t0 + t0;   // tensor-map coordinate of the chunk's first token
-                // q, k maps (KDA: the prep's qp, kp, kc, one row block per sequence
-                // even when packed): the chunk's first token at (tq, bq)
-                const int tq = KDA ? t0 : tm, bq = KDA ? (int)b : sq.b0;
-#pragma unroll
-                for (int a = 0; a < KA; ++a) {
-                    tma_load_4d(qk + a * QK_ACS, &maps.q, &ctl->full[s], 64 * a, (int)h, tq, bq);
-                    tma_load_4d(qk + a * QK_ACS + 64 * 128, &maps.k, &ctl->full[s], 64 * a, (int)h, tq, bq);
-                    if (KDA)
-                        tma_load_4d(tiles + L::STG_KC + s * 16384 + a * (C * 128), &maps.kc, &ctl->full[s],
-                                    64 * a, (int)h, tq, bq);
-                }
-                tma_load_4d(tiles + L::STG_V + s * 4096, &maps.v, &ctl->full[s], dvt * DVT, (int)h, tm, sq.b0);
-                const uint8_t *item = ws + (bh * ws_chunks + c) * (int64_t)ITEM;
-                bulk_load(tiles + L::STG_TT + s * TT_BYTES, item + ITEM_T, TT_BYTES, &ctl->full[s]);
-                bulk_load(tiles + L::STG_P + s * 16384, item + ITEM_P, 8192, &ctl->full[s]);
-                if (KDA) {
-                    bulk_load(tiles + L::STG_GC + s * 512, item + kda::ITEM_GC, 512, &ctl->full[s]);
-                    // two stages leave about one chunk period for a load: start chunk
-                    // c+1's tiles and item on their way to L2 now
-                    if (c + 1 < nchunks) {
-#pragma unroll
-                        for (int a = 0; a < KA; ++a) {
-                            tma_prefetch_l2_4d(&maps.q, 64 * a, (int)h, tq + C, bq);
-                            tma_prefetch_l2_4d(&maps.k, 64 * a, (int)h, tq + C, bq);
-                            tma_prefetch_l2_4d(&maps.kc, 64 * a, (int)h, tq + C, bq);
-                        }
-                        tma_prefetch_l2_4d(&maps.v, dvt * DVT, (int)h, tm + C, sq.b0);
-                        bulk_prefetch_l2(item + ITEM, ITEM);
-                    }
-                }
-            }
-            if constexpr (KDA) {   // the decay factors come with the stage; betas (0 past T)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int64_t tt = (int64_t)t0 + 2 * lane + e;
-                    ctl->bet[s][2 * lane + e] = tt < sq.len ? p.beta[(sq.row0 + tt) * p.H + h] : 0.f;
-                }
-                __syncwarp();
-            } else {
-                // the chunk's decay factors: b = log2 of the inclusive cumulative alpha,
-                // gamma = 2^b, 1/gamma, gamma_C/gamma = 2^(b_63 - b); beta (0 past T)
-                float al[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int64_t tt = (int64_t)t0 + 2 * lane + e;
-                    const bool in = tt < sq.len;
-                    al[e] = in ? p.g[(sq.row0 + tt) * p.H + h] : 1.f;
-                    ctl->bet[s][2 * lane + e] = in ? p.beta[(sq.row0 + tt) * p.H + h] : 0.f;
-                }
-                const int fast = gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
-                const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
-                __syncwarp();
-                ctl->gct[s][2 * lane] = exp2f(blast - ctl->b2[s][2 * lane]);
-                ctl->gct[s][2 * lane + 1] = exp2f(blast - ctl->b2[s][2 * lane + 1]);
-                if (lane == 0) ctl->fast[s] = fast;
-            }
-            mbar_arrive(&ctl->full[s]);
-            issued = c + 1;
-        }
-        // let copies still in flight land before the CTA can exit
-        if (lane == 0)
-            for (int c = (issued > NSTG ? issued - NSTG : 0); c < issued; ++c)
-                (void)mbar_drain(&ctl->full[c % NSTG], (uint32_t)(c / NSTG) & 1u);
-    } else if (warp < 5) {
-        // ------------------------------------------------------------------ output group
-        const int lt = tid - 32;
-        const bool leader = (lt == 0);
-        const int ro = 32 * quad + lane;   // M=128 row: output rows 0-63 in quads 0, 1
-        // PW = [P ; 0] W and O = diag(gamma) X2 + PW of chunk j, X2 = rows 0-63 of [X2 ; KS]
-        // (a failed wait sets the abort flag; every thread still takes every barrier)
-        auto finish = [&](int j) {
-            const int sj = j % NSTG, jb = j & 1;
-            const int64_t tj = (int64_t)j * C;
-            const int nvalid = (int)min((int64_t)C, sq.len - tj);
-            if (!mbar_wait(&ctl->wready[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
-            // read before the stage can be refilled (KDA: X2 = Qp S0 already carries Gamma)
-            const float gam_o = KDA ? 1.f : ctl->gam[sj][ro & 63];
-            bar_named(1, 128);
-            if (leader) {
-                // P(j) came with stage j, which the state group has consumed (wready);
-                // this wait only makes the copy's completion visible to the issuing
-                // thread and returns at once (the stage cannot be refilled before
-                // PW(j) is committed below)
-                if (!mbar_wait(&ctl->full[sj], (uint32_t)(j / NSTG) & 1u)) ctl->abort = 1;
-                tc_fence_after_sync();
-                const uint32_t ps = tb + L::STG_P + (uint32_t)sj * 16384u;
-                const uint32_t wsb = tb + L::TWS + (uint32_t)jb * 4096u;
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + C_PW + 32u * jb, desc_k(ps, 16384, kk), desc_mn64(wsb, kk), ID_XK, kk > 0);
-                umma_commit(&ctl->pw_done[jb]);
-                umma_commit(&ctl->empty[sj]);
-            }
-            if (!mbar_wait(&ctl->pw_done[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
-            tc_fence_after_sync();
-            if (quad < 2) {
-                float x2[32], pw[32];
-                tmem_ld32(tq + C_XK + 32u * jb, x2);
-                tmem_ld32(tq + C_PW + 32u * jb, pw);
-                tmem_wait_ld();
-                if (ro < nvalid) {
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.o) +
-                                         ((sq.row0 + tj + ro) * p.H + h) * p.dv + dvt * DVT;
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        uint4 u;
-                        u.x = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 0], pw[8 * cc + 0]),
-                                          fmaf(gam_o, x2[8 * cc + 1], pw[8 * cc + 1]));
-                        u.y = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 2], pw[8 * cc + 2]),
-                                          fmaf(gam_o, x2[8 * cc + 3], pw[8 * cc + 3]));
-                        u.z = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 4], pw[8 * cc + 4]),
-                                          fmaf(gam_o, x2[8 * cc + 5], pw[8 * cc + 5]));
-                        u.w = pack_bf16x2(fmaf(gam_o, x2[8 * cc + 6], pw[8 * cc + 6]),
-                                          fmaf(gam_o, x2[8 * cc + 7], pw[8 * cc + 7]));
-                        reinterpret_cast<uint4 *>(dst)[cc] = u;
-                    }
-                }
-            }
-            tc_fence_before_sync();
-            mbar_arrive(&ctl->oA[jb]);
-        };
-        // one chunk per iteration, in order, each as soon as the state group has its
-        // W (P comes with the stage, so nothing else is waited for: a wait for a
-        // later stage here would hold PW, which frees that stage for a later
-        // chunk's loads).  The stop flag alternates between two words so that the
-        // leader's write for iteration j+1 cannot reach a thread still reading
-        // iteration j's.
-        for (int j = 0; j < nchunks; ++j) {
-            const int pb = j & 1;
-            if (leader) ctl->stopL[pb] = ctl->abort;
-            bar_named(1, 128);
-            if (ctl->stopL[pb]) break;
-            finish(j);
-        }
-        if (leader) umma_commit(&ctl->drain);
-    } else {
-        // ------------------------------------------------------------------ state group
-        const int st = tid - 160;
-        const bool leader = (st == 0);
-        const int d = 32 * quad + lane;               // row of the M=128 accumulators (state row)
-        const int tr = 16 * quad + (lane & 15);       // row of the M=64 accumulator W
-        const int hf = lane >> 4;                     // which 16 of W's 32 columns
-        float S[DVT];
-        {
-            const float *src = p.S0 ? p.S0 + ((bh * DK + d) * p.dv + dvt * DVT) : nullptr;
-#pragma unroll
-            for (int j = 0; j < DVT; j += 4) {
-                float4 x = src ? *reinterpret_cast<const float4 *>(src + j) : make_float4(0, 0, 0, 0);
-                S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-            }
-            store_row64(tiles + L::TSS, d, S);
-        }
-        fence_proxy_async_smem();
-        bar_named(2, 128);
-        // the bf16 copy of the state entering chunk c sits in buffer c & 1
-        auto ss_of = [&](int c) { return tb + L::TSS + (uint32_t)(c & 1) * 8192u; };
-        // [X2 ; KS] = [Q ; K] S0, K = dk
-        auto issue_xk = [&](int c) {
-            const uint32_t qk = stage_qk(c), ss = ss_of(c);
-#pragma unroll
-            for (int kk = 0; kk < DK / 16; ++kk)
-                umma_bf16(tmem + C_XK + 32u * (c & 1), desc_k(qk, QK_ACS, kk), desc_mn64(ss, kk), ID_XK, kk > 0);
-            umma_commit(&ctl->xk_done);
-        };
-        // half row (16 columns, 2 chunks of 16 B) of a [rows][32] bf16 tile, 64-byte swizzle
-        auto store_half64 = [&](uint32_t tile_off, int r, const float *x16) {
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c = 2 * hf + cc;
-                uint4 u;
-                u.x = pack_bf16x2(x16[8 * cc + 0], x16[8 * cc + 1]);
-                u.y = pack_bf16x2(x16[8 * cc + 2], x16[8 * cc + 3]);
-                u.z = pack_bf16x2(x16[8 * cc + 4], x16[8 * cc + 5]);
-                u.w = pack_bf16x2(x16[8 * cc + 6], x16[8 * cc + 7]);
-                *reinterpret_cast<uint4 *>(tiles + tile_off + r * 64 + (((c ^ (r >> 1)) & 3) << 4)) = u;
-            }
-        };
-        if (leader && nchunks > 0) {
-            if (!mbar_wait(&ctl->full[0], 0u)) ctl->abort = 1;
-            tc_fence_after_sync();
-            issue_xk(0);
-        }
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % NSTG, pb = c & 1;
-            if (leader) ctl->stopS = ctl->abort;
-            bar_named(2, 128);
-            if (ctl->stopS) break;
-            // the stage landed (V, T and the decay factors are read directly)
-            bool ok = mbar_wait(&ctl->full[s], (uint32_t)(c / NSTG) & 1u);
-            ok = mbar_wait(&ctl->xk_done, (uint32_t)c & 1u) && ok;
-            if (!ok) ctl->abort = 1;
-            tc_fence_after_sync();
-            // decay of state row d over the chunk (KDA: per key channel)
-            const float gC = KDA ? reinterpret_cast<const float *>(tiles + L::STG_GC + s * 512)[d]
-                                 : ctl->gam[s][C - 1];
-            const float gct_r = KDA ? 1.f : ctl->gct[s][tr];
-            if (quad >= 2) {   // R = diag(beta) (V - diag(gamma) KS): rows 64..127 of [X2 ; KS]
-                const int t = d - 64;
-                float ks[32];
-                tmem_ld32(tq + C_XK + 32u * pb, ks);
-                tmem_wait_ld();
-                const uint8_t *vt = stage_v(c);
-                const float be = ctl->bet[s][t], ga = KDA ? 1.f : ctl->gam[s][t];
-                float r[32];
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const uint4 u = *reinterpret_cast<const uint4 *>(vt + t * 64 + (((cc ^ (t >> 1)) & 3) << 4));
-                    const uint32_t *w = &u.x;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 v2 = unpack_bf16x2(w[e]);
-                        const int j = 8 * cc + 2 * e;
-                        r[j] = be * fmaf(-ga, ks[j], v2.x);
-                        r[j + 1] = be * fmaf(-ga, ks[j + 1], v2.y);
-                    }
-                }
-                store_row64(tiles + L::TR, t, r);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            bar_named(2, 128);
-            if (leader) {   // W = T R, K = tokens
-                tc_fence_after_sync();
-                const uint32_t tt = stage_tt(c);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + C_W, desc_k(tt, C * 128, kk), desc_mn64(tb + L::TR, kk), ID_W, kk > 0);
-                umma_commit(&ctl->w_done);
-            }
-            ok = mbar_wait(&ctl->w_done, (uint32_t)c & 1u);
-            // the W tile of chunk c-2 was read by PW(c-2)
-            if (c >= 2) ok = mbar_wait(&ctl->pw_done[pb], (uint32_t)((c - 2) >> 1) & 1u) && ok;
-            if (!ok) ctl->abort = 1;
-            tc_fence_after_sync();
-            {   // W and (gamma_C / gamma) W -> bf16, rows tr, columns 16 hf..
-                // (KDA: Kc carries Gamma_C / Gamma, and dS reads W itself)
-                float w[16], wg[16];
-                tmem_ld16x2_16<16>(tq + C_W, w);
-                tmem_wait_ld();
-                store_half64(L::TWS + (uint32_t)pb * 4096u, tr, w);
-                if (!KDA) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) wg[j] = w[j] * gct_r;
-                    store_half64(L::TWGS, tr, wg);
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            mbar_arrive(&ctl->wready[pb]);   // the score group may issue PW(c)
-            bar_named(2, 128);
-            if (leader) {   // dS = K^T diag(gamma_C / gamma) W, K = tokens
-                tc_fence_after_sync();
-                // GDN: K^T (gamma_C/gamma W); KDA: Kc^T W
-                const uint32_t kb = KDA ? tb + L::STG_KC + (uint32_t)s * 16384u : stage_qk(c) + 64 * 128;
-                const uint32_t kacs = KDA ? (uint32_t)(C * 128) : QK_ACS;
-                const uint32_t wb = KDA ? tb + L::TWS + (uint32_t)pb * 4096u : tb + L::TWGS;
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + C_DS, desc_mn128(kb, kacs, kk), desc_mn64(wb, kk), ID_DS, kk > 0);
-                umma_commit(&ctl->ds_done);
-                umma_commit(&ctl->empty[s]);
-            }
-            if (!mbar_wait(&ctl->ds_done, (uint32_t)c & 1u)) ctl->abort = 1;
-            tc_fence_after_sync();
-            {   // S <- gamma_C S + dS, then its bf16 copy for chunk c+1
-                float ds[DVT];
-                tmem_ld32(tq + C_DS, ds);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < DVT; ++j) S[j] = fmaf(gC, S[j], ds[j]);
-                store_row64(tiles + L::TSS + (uint32_t)((c + 1) & 1) * 8192u, d, S);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before_sync();
-            bar_named(2, 128);
-            if (leader && c + 1 < nchunks) {
-                // the stage of c+1 landed, and the output epilogue of c-1 is done with
-                // the [X2 ; KS] accumulator that [Q ; K] S of c+1 overwrites
-                bool w1 = mbar_wait(&ctl->full[(c + 1) % NSTG], (uint32_t)((c + 1) / NSTG) & 1u);
-                if (c >= 1) w1 = mbar_wait(&ctl->oA[(c + 1) & 1], (uint32_t)((c - 1) >> 1) & 1u) && w1;
-                if (!w1) ctl->abort = 1;
-                tc_fence_after_sync();
-                issue_xk(c + 1);
-            }
-        }
-        if (leader) {   // every MMA issued by either group has finished before TMEM is released
-            umma_commit(&ctl->drain);
-            (void)mbar_drain(&ctl->drain, 0u);
-        }
-        if (!ctl->abort && p.S_out) {
-            float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVT);
-#pragma unroll
-            for (int j = 0; j < DVT; j += 4)
-                *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-        }
-    }
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
-}
-
 namespace gdn {
 // Shared memory of gdn_main_kernel (byte offsets from a 1 KB aligned base).
 //   ring A, 2 stages: [Q ; -U] as two atom columns of 128 rows (Q rows 0-63 from
@@ -1044,11 +615,13 @@ namespace gdn {
 //     that are never read) and K that of dS = K^T diag(gamma_C / gamma) W;
 //   W (2 buffers) and diag(gamma_C / gamma) W, bf16 [64][32], and S0, bf16
 //     [128][32], all with the 64-byte swizzle.
+template <bool KDA>
 struct ML {
     static constexpr int NA = 2, NB = 3;
     static constexpr uint32_t A_BYTES = 2 * QK_ACS;
     static constexpr uint32_t B_Z = 0, B_T = 8192, B_P = 16384, B_K = 24576, B_V = 40960;
-    static constexpr uint32_t B_BYTES = 45056;
+    static constexpr uint32_t B_GC = 45056;                     // KDA: Gamma_C, fp32 [128]
+    static constexpr uint32_t B_BYTES = KDA ? 46080 : 45056;    // stages stay 1 KB aligned
     static constexpr uint32_t SA = 0;
     static constexpr uint32_t SB = SA + NA * A_BYTES;
     static constexpr uint32_t TWS = SB + NB * B_BYTES;
@@ -1063,14 +636,15 @@ constexpr uint32_t M_DS = 64;   // 32,     M=128 dS
 constexpr uint32_t M_PW = 96;   // 2 x 32, M=128 [P ; K0] W (rows 0-63)
 
 struct MCtl {
-    uint64_t fullA[ML::NA], emptyA[ML::NA], fullB[ML::NB], emptyB[ML::NB];
+    uint64_t fullA[2], emptyA[2], fullB[3], emptyB[3];
     uint64_t wready[2], pw_done[2], w0_done[2], xk_done, ds_done, drain;
     uint32_t tmem_base;
     int abort, stopS, stopL[2];
-    // per ring-B stage: b = log2 of the inclusive cumulative alpha, gamma = 2^b,
-    // 1/gamma and gamma_C / gamma (written by the producer)
-    float b2[ML::NB][64], gam[ML::NB][64], ginv[ML::NB][64], gct[ML::NB][64];
+    // the gated delta rule, per ring-B stage: b = log2 of the inclusive cumulative
+    // alpha, gamma = 2^b, 1/gamma and gamma_C / gamma (written by the producer)
+    float b2[3][64], gam[3][64], ginv[3][64], gct[3][64];
 };
+static_assert(ML<false>::NA == 2 && ML<false>::NB == 3, "MCtl's barrier arrays follow the rings");
 }  // namespace gdn
 
 // The gated delta rule's main pass (one CTA per (batch, head, 32-column value
@@ -1086,10 +660,17 @@ struct MCtl {
 //               the chunk after next: [0 ; T diag(beta)] V;
 //   warps 5-8   state group: W -> bf16 (and diag(gamma_C / gamma) W), dS, the
 //               state update, and [Q ; -U] S0 of the next chunk.
+// KDA = true: the KDA main pass on kda_prep_kernel's outputs (chunk_kda.cuh has
+// the algebra): maps.q and maps.kc cover its Qp = Q o Gamma and Kc = K o
+// Gamma_C / Gamma, and its items hold T diag(beta), P, -U = -T diag(beta)(K o
+// Gamma) and Gamma_C.  Then X2 = Qp S0 already carries the decay, dS = Kc^T W,
+// and the state row d decays by Gamma_C[d].
+template <bool KDA>
 __global__ void __launch_bounds__(gdn::NTHREADS, 1)
 gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const uint8_t *ws) {
     using namespace gdn;
-    using L = ML;
+    using L = ML<KDA>;
+    constexpr uint32_t ITEM = KDA ? kda::ITEM_BYTES : ITEM_BYTES;   // workspace bytes per chunk
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     MCtl *ctl = reinterpret_cast<MCtl *>(smem_raw);
     uint8_t *tiles = smem_raw + align1k((uint32_t)sizeof(MCtl) + (smem_u32(smem_raw) & 1023u)) -
@@ -1128,7 +709,7 @@ gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const ui
         ctl->abort = 0;
         fence_barrier_init();
         tma_prefetch_desc(&maps.q);
-        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(KDA ? &maps.kc : &maps.k);
         tma_prefetch_desc(&maps.v);
     }
     if (warp == 0) {
@@ -1172,11 +753,13 @@ gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const ui
             const int stop = (lane == 0) ? ctl->abort : 0;
             return __shfl_sync(0xffffffffu, stop, 0) == 0;
         };
-        if (nchunks > 0) fetch(0);
+        if (!KDA && nchunks > 0) fetch(0);
         int issuedA = 0, issuedB = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int tm = sq.t0 + c * C;   // tensor-map coordinate of the chunk's first token
-            const uint8_t *item = ws + (bh * ws_chunks + c) * (int64_t)ITEM_BYTES;
+            // KDA: the prep's Qp, Kc (one row block per sequence, even when packed)
+            const int tqk = KDA ? c * C : tm, bqk = KDA ? (int)b : sq.b0;
+            const uint8_t *item = ws + (bh * ws_chunks + c) * (int64_t)ITEM;
             const int a = c & 1, s = c % L::NB;
             if (!acquire(&ctl->emptyA[a], (uint32_t)((c >> 1) - 1) & 1u, c >= L::NA)) break;
             if (lane == 0) {
@@ -1184,7 +767,7 @@ gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const ui
                 mbar_arrive_expect_tx(&ctl->fullA[a], 2u * KA * C * 128u);
 #pragma unroll
                 for (int ka = 0; ka < KA; ++ka) {
-                    tma_load_4d(qa + ka * QK_ACS, &maps.q, &ctl->fullA[a], 64 * ka, (int)h, tm, sq.b0);
+                    tma_load_4d(qa + ka * QK_ACS, &maps.q, &ctl->fullA[a], 64 * ka, (int)h, tqk, bqk);
                     bulk_load(qa + ka * QK_ACS + 64 * 128, item + ITEM_U + ka * 8192, 8192, &ctl->fullA[a]);
                 }
             }
@@ -1192,21 +775,25 @@ gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const ui
             if (!acquire(&ctl->emptyB[s], (uint32_t)((c / L::NB) - 1) & 1u, c >= L::NB)) break;
             if (lane == 0) {
                 uint8_t *sb = tiles + stage_b(c);
-                mbar_expect_tx(&ctl->fullB[s], KA * C * 128u + C * DVT * 2u + 2u * TT_BYTES);
+                mbar_expect_tx(&ctl->fullB[s], KA * C * 128u + C * DVT * 2u + 2u * TT_BYTES + (KDA ? 512u : 0u));
 #pragma unroll
                 for (int ka = 0; ka < KA; ++ka)
-                    tma_load_4d(sb + L::B_K + ka * 8192, &maps.k, &ctl->fullB[s], 64 * ka, (int)h, tm, sq.b0);
+                    tma_load_4d(sb + L::B_K + ka * 8192, KDA ? &maps.kc : &maps.k, &ctl->fullB[s], 64 * ka, (int)h,
+                                tqk, bqk);
                 tma_load_4d(sb + L::B_V, &maps.v, &ctl->fullB[s], dvt * DVT, (int)h, tm, sq.b0);
                 bulk_load(sb + L::B_T, item + ITEM_T, TT_BYTES, &ctl->fullB[s]);
                 bulk_load(sb + L::B_P, item + ITEM_P, TT_BYTES, &ctl->fullB[s]);
+                if (KDA) bulk_load(sb + L::B_GC, item + kda::ITEM_GC, 512, &ctl->fullB[s]);
             }
-            // the chunk's decay factors: gamma = 2^b, gamma_C / gamma = 2^(b_63 - b)
-            (void)gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
-            const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
-            __syncwarp();
-            ctl->gct[s][2 * lane] = exp2f(blast - ctl->b2[s][2 * lane]);
-            ctl->gct[s][2 * lane + 1] = exp2f(blast - ctl->b2[s][2 * lane + 1]);
-            if (c + 1 < nchunks) fetch(c + 1);   // in flight while the next slots free up
+            if constexpr (!KDA) {
+                // the chunk's decay factors: gamma = 2^b, gamma_C / gamma = 2^(b_63 - b)
+                (void)gate_scan(al, nullptr, ctl->b2[s], ctl->gam[s], ctl->ginv[s], nullptr, lane);
+                const float blast = __shfl_sync(0xffffffffu, ctl->b2[s][2 * lane + 1], 31);
+                __syncwarp();
+                ctl->gct[s][2 * lane] = exp2f(blast - ctl->b2[s][2 * lane]);
+                ctl->gct[s][2 * lane + 1] = exp2f(blast - ctl->b2[s][2 * lane + 1]);
+                if (c + 1 < nchunks) fetch(c + 1);   // in flight while the next slots free up
+            }
             mbar_arrive(&ctl->fullB[s]);
             issuedB = c + 1;
         }
@@ -1244,7 +831,8 @@ gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const ui
             const int64_t tj = (int64_t)j * C;
             const int nvalid = (int)min((int64_t)C, sq.len - tj);
             if (!mbar_wait(&ctl->wready[jb], (uint32_t)(j >> 1) & 1u)) ctl->abort = 1;
-            const float gam_o = ctl->gam[sj][ro & 63];   // read before the stage can be refilled
+            // read before the stage can be refilled (KDA: X2 = Qp S0 already decays)
+            const float gam_o = KDA ? 1.f : ctl->gam[sj][ro & 63];
             bar_named(1, 128);
             if (leader) {
                 // stage j landed long ago (the state group has its W); the wait makes the
@@ -1344,30 +932,36 @@ gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const ui
             ok = mbar_wait(&ctl->xk_done, (uint32_t)c & 1u) && ok;
             if (!ok) ctl->abort = 1;
             tc_fence_after_sync();
-            const float gC = ctl->gam[s][C - 1];   // read before the stage can be refilled
-            if (quad >= 2) {   // W row t -> bf16 W (for PW) and diag(gamma_C / gamma) W (for dS)
+            // decay of state row d over the chunk, read before the stage can be refilled
+            const float gC = KDA ? reinterpret_cast<const float *>(tiles + stage_b(c) + L::B_GC)[d]
+                                 : ctl->gam[s][C - 1];
+            if (quad >= 2) {   // W row t -> bf16 W (for PW) and diag(gamma_C / gamma) W (for dS;
+                               // KDA: Kc carries Gamma_C / Gamma and dS reads W itself)
                 const int t = d - 64;
                 // PW of chunk c-2 has read W buffer pb
                 if (c >= 2 && !mbar_wait(&ctl->pw_done[pb], (uint32_t)((c - 2) >> 1) & 1u)) ctl->abort = 1;
                 float w[32];
                 tmem_ld32(tq + M_XW + 32u * pb, w);
-                const float g = ctl->gct[s][t];
+                const float g = KDA ? 1.f : ctl->gct[s][t];
                 tmem_wait_ld();
                 store_row64(tiles + L::TWS + (uint32_t)pb * 4096u, t, w);
+                if (!KDA) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) w[j] *= g;
-                store_row64(tiles + L::TWGS, t, w);
+                    for (int j = 0; j < 32; ++j) w[j] *= g;
+                    store_row64(tiles + L::TWGS, t, w);
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before_sync();
             mbar_arrive(&ctl->wready[pb]);   // the output group may issue PW(c)
             bar_named(2, 128);
-            if (leader) {   // dS = K^T diag(gamma_C / gamma) W, K = tokens
+            if (leader) {   // dS = K^T diag(gamma_C / gamma) W (KDA: Kc^T W), K = tokens
                 tc_fence_after_sync();
                 const uint32_t kb = tb + stage_b(c) + L::B_K;
+                const uint32_t wb = KDA ? tb + L::TWS + (uint32_t)pb * 4096u : tb + L::TWGS;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    umma_bf16(tmem + M_DS, desc_mn128(kb, C * 128, kk), desc_mn64(tb + L::TWGS, kk), ID_DS, kk > 0);
+                    umma_bf16(tmem + M_DS, desc_mn128(kb, C * 128, kk), desc_mn64(wb, kk), ID_DS, kk > 0);
                 umma_commit(&ctl->ds_done);
                 umma_commit(&ctl->emptyB[s]);
             }

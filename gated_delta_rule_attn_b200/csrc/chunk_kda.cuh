@@ -1,5 +1,5 @@
 // chunk_kda.cuh — KDA (per-key-channel retention with the delta rule), chunked
-// prefill: a parallel prep kernel here, then chunk_gdn_kernel<true>.
+// prefill: a parallel prep kernel here, then gdn_main_kernel<true> (chunk_gdn.cuh).
 //
 // Rule (page "状态空间与线性注意力", KDA：逐通道遗忘与误差写入), per token:
 //   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,  o_t = S_t^T q_t,
@@ -31,10 +31,13 @@
 //
 // kda_prep_kernel, one (batch, head, chunk) item per CTA iteration (grid-stride,
 // 4 warps, 2 CTAs per SM), writes to the workspace:
-//   per item: the T image and the P image (bf16, 128-byte swizzled [64][64], the
-//   shared-memory operand layout of chunk_gdn_kernel) and Gamma_C (fp32 [128]);
-//   per token: Qp = q o Gamma, Kp = k o Gamma, Kc = k o Gamma_C / Gamma as bf16
-//   [B,Ls,H,128] tensors, which chunk_gdn_kernel<true> loads by TMA in place of q, k.
+//   per item: the images of T diag(beta), P and -U = -T diag(beta) (K o Gamma)
+//   (bf16, 128-byte swizzled, the shared-memory operand layout of
+//   gdn_main_kernel; U by one M=64, N=128 MMA) and Gamma_C (fp32 [128]);
+//   per token: Qp = q o Gamma and Kc = k o Gamma_C / Gamma as bf16 [B,Ls,H,128]
+//   tensors, which gdn_main_kernel<true> loads by TMA in place of q and k.
+// With W = T diag(beta) (V - (K o Gamma) S0) = T diag(beta) V - U S0 the main
+// pass runs the gated delta rule's chain unchanged.
 //   Dense layout: Ls = T.  Packed sequences: one row block per sequence,
 //   Ls = 64 ceil(max_seqlen / 64), so a sequence's tail chunk owns its padding
 //   rows, which are written as zeros (the next sequence's tokens never appear
@@ -51,12 +54,14 @@ namespace kda {
 constexpr int PREP_THREADS = 128;
 // (the per-chunk item layout, ITEM_*, is in chunk_gdn.cuh beside its reader)
 constexpr uint32_t QS_ACS = 128 * 128;         // [Qs ; Ks] atom column: 128 rows x 128 B
-constexpr uint32_t KR_ACS = 64 * 128;          // Kr_a atom column: 64 rows x 128 B
-constexpr uint32_t KR_BYTES = 2 * KR_ACS;
+// Kr_a holds the keys of sub-chunks 0..a: 16 (a + 1) rows, two atom columns
+__host__ __device__ constexpr uint32_t kr_acs(int a) { return 2048u * (uint32_t)(a + 1); }
+__host__ __device__ constexpr uint32_t kr_off(int a) { return 2048u * (uint32_t)(a * (a + 1)); }
 constexpr uint32_t P_QS = 0;                   // [Qs ; Ks], rows 32w..32w+15 = Qs of sub-chunk w,
                                                // rows 32w+16..32w+31 = Ks of sub-chunk w
-constexpr uint32_t P_KR = 2 * QS_ACS;          // Kr_a, a = 0..3
-constexpr uint32_t P_END = P_KR + 4 * KR_BYTES;
+constexpr uint32_t P_KR = 2 * QS_ACS;          // Kr_a, a = 0..3 (40 KB)
+constexpr uint32_t P_KP = P_KR + kr_off(4);    // K o Gamma, [64][128], two atom columns of 8 KB
+constexpr uint32_t P_END = P_KP + 16384;
 // A, then T (fp32 [64][AF_LD]), and the merge scratch reuse [Qs ; Ks] once the
 // MMAs that read it are done
 constexpr uint32_t P_AF = P_QS;
@@ -69,14 +74,14 @@ constexpr float kDown = 5.421010862427522e-20f;        // 2^-64
 }  // namespace kda
 
 struct KCtl {
-    uint64_t mma, drain;
+    uint64_t mma, mma_u, drain;
     uint32_t tmem_base;
     int abort, stop;
     // per sub-chunk and key channel: the product of alpha over its tokens up to
     // and including the middle one (D) and over the tokens after it (U)
     alignas(16) float D[4][128];
     alignas(16) float U[4][128];
-    float beta[64];
+    alignas(16) float beta[64];   // read as float4
 };
 
 struct KdaPrepParams {
@@ -86,7 +91,7 @@ struct KdaPrepParams {
     const __nv_bfloat16 *q, *k;       // [B,T,H,128] (packed: [1,T,H,128])
     const float *alpha, *beta;        // [B,T,H,128], [B,T,H] (packed: [1,T,H,*])
     uint8_t *items;                   // [B*H*nchunks][ITEM_BYTES]
-    __nv_bfloat16 *qp, *kp, *kc;      // [B,Ls,H,128]
+    __nv_bfloat16 *qp, *kc;           // [B,Ls,H,128]
     const int64_t *cu_seqlens;        // packed sequences, or nullptr (dense)
     int64_t max_seqlen;               // = T for the dense layout
 };
@@ -132,6 +137,7 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
 
     if (tid == 0) {
         mbar_init(&ctl->mma, 1);
+        mbar_init(&ctl->mma_u, 1);
         mbar_init(&ctl->drain, 1);
         ctl->abort = 0;
         fence_barrier_init();
@@ -140,17 +146,11 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
         tmem_alloc(&ctl->tmem_base, 256);
         tc_fence_before_sync();
     }
-    // rows of Kr_a past sub-chunk a are never written: zero them once
-    for (int i = tid; i < (int)(4 * KR_BYTES / 16); i += PREP_THREADS) {
-        const uint32_t off = (uint32_t)i * 16u, a = off / KR_BYTES, row = (off % KR_ACS) / 128u;
-        if (row >= 16u * (a + 1u)) *reinterpret_cast<uint4 *>(tiles + P_KR + off) = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lanes
-    constexpr uint32_t ID_S = idesc_bf16(128, 64, false, false);
+    constexpr uint32_t ID_U = idesc_bf16(64, 128, false, true);
 
     int it = 0;   // items processed (one MMA commit each): the mbarrier phase
     for (int64_t w = blockIdx.x; w < items; w += gridDim.x) {
@@ -259,18 +259,18 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
             const float4 G = g[j], Hf = rcp4(G);
             const float4 down = make_float4(kDown, kDown, kDown, kDown);
             const float4 Gd = mul4(G, down), Hd = mul4(Hf, down);
+            const float4 Gg = mul4(Gd, gm);   // Gamma_t
             st4_sw128(qs, QS_ACS, 32 * sc + j, d0, mul4(qf, G));
             st4_sw128(qs, QS_ACS, 32 * sc + 16 + j, d0, mul4(kf, G));
-            st4_sw128(tiles + P_KR + sc * KR_BYTES, KR_ACS, 16 * sc + j, d0, mul4(kf, Hf));
+            st4_sw128(tiles + P_KR + kr_off(sc), kr_acs(sc), 16 * sc + j, d0, mul4(kf, Hf));
 #pragma unroll
             for (int a = 0; a < 4; ++a)
-                if (a > sc) st4_sw128(tiles + P_KR + a * KR_BYTES, KR_ACS, 16 * sc + j, d0, mul4(kf, mul4(Hd, mk[a])));
+                if (a > sc) st4_sw128(tiles + P_KR + kr_off(a), kr_acs(a), 16 * sc + j, d0, mul4(kf, mul4(Hd, mk[a])));
+            st4_sw128(tiles + P_KP, 8192u, 16 * sc + j, d0, mul4(kf, Gg));   // 0 past T (k is)
             if (t < wlen) {
                 const int64_t row = ((b * p.Ls + t) * p.H + h) * DK + d0;
-                const float4 Gg = mul4(Gd, gm);   // Gamma_t
                 const bool in = t < sq.len;
                 *reinterpret_cast<uint2 *>(p.qp + row) = in ? f32_to_bf16x4(mul4(qf, Gg)) : make_uint2(0u, 0u);
-                *reinterpret_cast<uint2 *>(p.kp + row) = in ? f32_to_bf16x4(mul4(kf, Gg)) : make_uint2(0u, 0u);
                 *reinterpret_cast<uint2 *>(p.kc + row) =   // Gamma_C / Gamma_t
                     in ? f32_to_bf16x4(mul4(kf, mul4(Hd, cm))) : make_uint2(0u, 0u);
             }
@@ -280,7 +280,8 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
         tc_fence_before_sync();
         bar_named(1, 128);
 
-        // (4) four MMAs: rows of [Qs ; Ks] against Kr_a, into TMEM columns 64a
+        // (4) four MMAs: rows of [Qs ; Ks] against Kr_a (N = 16 (a + 1) keys), into
+        // TMEM columns 64a (columns past 16 (a + 1) are masked on readout)
         if (tid == 0) {
             tc_fence_after_sync();
 #pragma unroll
@@ -288,11 +289,11 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk)
                     umma_bf16(tmem + 64u * a, desc_k(tb + P_QS, QS_ACS, kk),
-                              desc_k(tb + P_KR + a * KR_BYTES, KR_ACS, kk), ID_S, kk > 0);
+                              desc_k(tb + P_KR + kr_off(a), kr_acs(a), kk), idesc_bf16(128, 16 * (a + 1), false, false),
+                              kk > 0);
             umma_commit(&ctl->mma);
         }
         if (!mbar_wait(&ctl->mma, (uint32_t)it & 1u)) ctl->abort = 1;
-        ++it;
         tc_fence_after_sync();
 
         // (5) lane l < 16: P row of token 16w + l; lane l >= 16: A row of token 16w + l - 16.
@@ -341,21 +342,63 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
         tc_fence_before_sync();
         bar_named(1, 128);
         gdn::invert_unit_lower64(AF, TMP, tid, lane, 1, 2);
-        {   // T -> the item's T image (128-byte swizzled [64][64] bf16)
+        {   // T diag(beta) -> the item's image (128-byte swizzled [64][64] bf16), and the
+            // same image over AF (once every thread has read its part of T) as the
+            // A operand of U = T diag(beta) (K o Gamma)
             const int t = tid >> 1, hh = tid & 1;
-            const float *Trow = AF + t * gdn::AF_LD + 32 * hh;
+            const float4 *Trow = reinterpret_cast<const float4 *>(AF + t * gdn::AF_LD + 32 * hh);
+            const float4 *be4 = reinterpret_cast<const float4 *>(ctl->beta + 32 * hh);
             uint8_t *dst = item + ITEM_T;
+            uint4 img[4];
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
-                uint4 u;
-                uint32_t *pu = &u.x;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pu[e] = pack_bf16x2(Trow[8 * cc + 2 * e], Trow[8 * cc + 2 * e + 1]);
+                const float4 t0 = Trow[2 * cc], t1 = Trow[2 * cc + 1], b0 = be4[2 * cc], b1 = be4[2 * cc + 1];
+                img[cc] = make_uint4(pack_bf16x2(t0.x * b0.x, t0.y * b0.y), pack_bf16x2(t0.z * b0.z, t0.w * b0.w),
+                                     pack_bf16x2(t1.x * b1.x, t1.y * b1.y), pack_bf16x2(t1.z * b1.z, t1.w * b1.w));
                 const int chunk = 4 * hh + cc;
-                *reinterpret_cast<uint4 *>(dst + (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4)) = u;
+                *reinterpret_cast<uint4 *>(dst + (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4)) = img[cc];
+            }
+            bar_named(1, 128);   // every read of T is done
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                const int chunk = 4 * hh + cc;
+                *reinterpret_cast<uint4 *>(tiles + P_AF + (uint32_t)t * 128u + (uint32_t)(((chunk ^ t) & 7) << 4)) =
+                    img[cc];
             }
         }
-        bar_named(1, 128);   // AF aliases [Qs ; Ks], which the next item rewrites
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        bar_named(1, 128);
+        if (tid == 0) {   // U: M=64 tokens, N=128 key channels, K=64 tokens
+            tc_fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk)
+                umma_bf16(tmem, desc_k(tb + P_AF, C * 128, kk), desc_mn128(tb + P_KP, 8192u, kk), ID_U, kk > 0);
+            umma_commit(&ctl->mma_u);
+        }
+        if (!mbar_wait(&ctl->mma_u, (uint32_t)it & 1u)) ctl->abort = 1;
+        ++it;
+        tc_fence_after_sync();
+        {   // -U -> the item: row tr = 16 warp + (lane & 15) of the M=64 accumulator,
+            // key channels 64 hf .. 64 hf + 63 = block hf of the image
+            const int tr = 16 * warp + (lane & 15), hf = lane >> 4;
+            float x[64];
+            tmem_ld16x2_32<64>(tw, *reinterpret_cast<float(*)[32]>(x));
+            tmem_ld16x2_32<64>(tw + 32u, *reinterpret_cast<float(*)[32]>(x + 32));
+            tmem_wait_ld();
+            uint8_t *dst = item + ITEM_U + (uint32_t)hf * 8192u + (uint32_t)tr * 128u;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                uint4 u;
+                u.x = pack_bf16x2(-x[8 * cc + 0], -x[8 * cc + 1]);
+                u.y = pack_bf16x2(-x[8 * cc + 2], -x[8 * cc + 3]);
+                u.z = pack_bf16x2(-x[8 * cc + 4], -x[8 * cc + 5]);
+                u.w = pack_bf16x2(-x[8 * cc + 6], -x[8 * cc + 7]);
+                *reinterpret_cast<uint4 *>(dst + (uint32_t)(((cc ^ tr) & 7) << 4)) = u;
+            }
+        }
+        tc_fence_before_sync();
+        bar_named(1, 128);   // AF aliases [Qs ; Ks], which the next item rewrites; TMEM too
     }
     // every MMA has finished before TMEM is released (a long wait even after a
     // timeout ended the loop)

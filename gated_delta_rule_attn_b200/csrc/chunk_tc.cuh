@@ -244,7 +244,7 @@ inline int resident_per_sm(const void *kernel, int threads, int dyn_smem, int tm
 // (Ls = T dense; 64 ceil(max_seqlen / 64) for packed sequences, one row block
 // per sequence).
 struct KdaWorkspace {
-    size_t items, qp, kp, kc, total;
+    size_t items, qp, kc, total;
 };
 inline KdaWorkspace kda_workspace(int64_t B, int64_t T, int64_t H) {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -252,8 +252,7 @@ inline KdaWorkspace kda_workspace(int64_t B, int64_t T, int64_t H) {
     w.items = 0;
     const size_t tensor = up((size_t)(B * T * H) * ck::DK * 2);
     w.qp = up((size_t)(B * H * ((T + ck::C - 1) / ck::C)) * ck::kda::ITEM_BYTES);
-    w.kp = w.qp + tensor;
-    w.kc = w.kp + tensor;
+    w.kc = w.qp + tensor;
     w.total = w.kc + tensor;
     return w;
 }
@@ -389,12 +388,9 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         kp.alpha = p.g; kp.beta = p.beta;
         kp.items = w8 + kw.items;
         kp.qp = reinterpret_cast<__nv_bfloat16 *>(w8 + kw.qp);
-        kp.kp = reinterpret_cast<__nv_bfloat16 *>(w8 + kw.kp);
         kp.kc = reinterpret_cast<__nv_bfloat16 *>(w8 + kw.kc);
         Maps mk = m;
         if (!make_map_4d(&mk.q, kp.qp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, Ls, p.H, DK, 64, C,
-                         CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !make_map_4d(&mk.k, kp.kp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, Ls, p.H, DK, 64, C,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
             !make_map_4d(&mk.kc, kp.kc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.B, Ls, p.H, DK, 64, C,
                          CU_TENSOR_MAP_SWIZZLE_128B)) {
@@ -407,10 +403,10 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         const int per_sm = resident_per_sm((const void *)kda_prep_kernel, kda::PREP_THREADS, psmem, 256);
         const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
         if (e == cudaSuccess) kda_prep_kernel<<<pgrid, kda::PREP_THREADS, psmem, st>>>(kp);
-        const int smem = (int)((sizeof(gdn::GCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::GL<true>::TEND;
-        if (e == cudaSuccess) e = allow_smem((const void *)chunk_gdn_kernel<true>, smem);
+        const int smem = (int)((sizeof(gdn::MCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::ML<true>::TEND;
+        if (e == cudaSuccess) e = allow_smem((const void *)gdn_main_kernel<true>, smem);
         if (e == cudaSuccess)
-            chunk_gdn_kernel<true><<<grid, gdn::NTHREADS, smem, st>>>(mk, pq, w8 + kw.items);
+            gdn_main_kernel<true><<<grid, gdn::NTHREADS, smem, st>>>(mk, pq, w8 + kw.items);
     } else if (rule == kRuleGDN) {
         const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv, packed, Lmax);
         if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
@@ -433,10 +429,10 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
             resident_per_sm((const void *)gdn_prep_kernel, gdn::PREP_THREADS, psmem, (int)gdn::PREP_TMEM_COLS);
         const unsigned pgrid = (unsigned)std::min<int64_t>(items, (int64_t)sm_count() * per_sm);
         if (e == cudaSuccess && items > 0) gdn_prep_kernel<<<pgrid, gdn::PREP_THREADS, psmem, st>>>(m.q, m.k, pp);
-        const int smem = (int)((sizeof(gdn::MCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::ML::TEND;
-        if (e == cudaSuccess) e = allow_smem((const void *)gdn_main_kernel, smem);
+        const int smem = (int)((sizeof(gdn::MCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::ML<false>::TEND;
+        if (e == cudaSuccess) e = allow_smem((const void *)gdn_main_kernel<false>, smem);
         if (e == cudaSuccess)
-            gdn_main_kernel<<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));
+            gdn_main_kernel<false><<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));
     } else {
         // packed sequences walk each sequence in one pass (no segments)
         const SegPlan sp = packed ? SegPlan{1, 1, (int)((Lmax + C - 1) / C)} : seg_plan(rule, p.B, p.T, p.H, p.dv);

@@ -124,10 +124,11 @@ typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
  *          piece's state contribution and its normaliser sum or gate product).
  *          Chunked GLA also keeps one 4-byte flag per (batch, head) there (a
  *          sequence to recompute, see la_rule), so its workspace is never 0.
- *          Chunked KDA keeps 16.5 KB per (batch, head, chunk) (the T and P
- *          operand images and the chunk's retention product) plus three bf16
- *          [B,Ls,H,128] tensors: q and k scaled by the cumulative retention, and
- *          k scaled by the retention from the token to its chunk's end (Ls = T;
+ *          Chunked KDA keeps 32.5 KB per (batch, head, chunk) (the operand
+ *          images of T diag(beta), P and -T diag(beta) (K o Gamma), and the
+ *          chunk's retention product) plus two bf16 [B,Ls,H,128] tensors: q
+ *          scaled by the cumulative retention, and k scaled by the retention
+ *          from the token to its chunk's end (Ls = T;
  *          with packed sequences Ls = 64 ceil(max_seqlen / 64), one row block
  *          per sequence).
  *          Calls that share

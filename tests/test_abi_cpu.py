@@ -117,10 +117,11 @@ def test_null_args_and_workspace_query(L):
 
 
 def test_kda_workspace_query():
-    """Chunked KDA (bf16, dk = 128, dense): 16.5 KB per (batch, head, 64-token
-    chunk) for the T image, the P image and the chunk's retention product, then
-    three bf16 [B,T,H,128] tensors (q and k times the cumulative retention, k
-    times the retention to the chunk's end), each at a 256-byte aligned offset.
+    """Chunked KDA (bf16, dk = 128, dense): 32.5 KB per (batch, head, 64-token
+    chunk) for the images of T diag(beta), P and -U and the chunk's retention
+    product, then two bf16 [B,T,H,128] tensors (q times the cumulative
+    retention, k times the retention to the chunk's end), each at a 256-byte
+    aligned offset.
     fp32 KDA runs on the recurrent kernel and needs none.  Queried through the
     binding, which reads shapes only (CPU tensors)."""
     import torch
@@ -130,9 +131,9 @@ def test_kda_workspace_query():
     g = torch.ones(B, T, H, 128)
     beta = torch.zeros(B, T, H)
     up = lambda x: (x + 255) // 256 * 256
-    items = up(B * H * 3 * (16384 + 512))
+    items = up(B * H * 3 * (32768 + 512))
     tensor = up(B * T * H * 128 * 2)
-    assert la.fwd_workspace_size("kda", q, q, v, g, beta) == items + 3 * tensor
+    assert la.fwd_workspace_size("kda", q, q, v, g, beta) == items + 2 * tensor
     assert la.fwd_workspace_size("kda", q.float(), q.float(), v.float(), g, beta) == 0
 
 
