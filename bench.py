@@ -479,7 +479,7 @@ def run_variants(torch, la, workloads, K, hbm_peak, seed):
     res["lightning_norm_prefill"]["norm_pass_ms"] = round(dn, 4)
     res["lightning_norm_prefill"]["norm_pass_gbs"] = round(nb / (dn / 1e3) / 1e9, 1) if dn > 0 else None
     # KDA (per-channel retention): chunked prefill (kda_prep_kernel +
-    # chunk_gdn_kernel<true>) at the benchmark shape and one decode step
+    # gdn_main_kernel<true>) at the benchmark shape and one decode step
     # (recurrent kernel) on the [256,16,128,128] fp32 state
     p = workloads.make_problem("kda", 2, 8192, 16, 128, 128, seed=seed)
     a = [t.cuda() for t in (p.q, p.k, p.v, p.g, p.beta)]
@@ -491,7 +491,7 @@ def run_variants(torch, la, workloads, K, hbm_peak, seed):
     w = prefill_bytes("gla", 2, 8192, 16, 128, 128) + 2 * 8192 * 16 * 4   # gla's bytes + beta
     res["kda_prefill"] = {"ms": round(ms, 4), "tokens_per_s": round(2 * 8192 / (ms / 1e3)),
                           "gbs": round(w / (ms / 1e3) / 1e9, 1), "hbm_frac": round(w / (ms / 1e3) / 1e9 / hbm_peak, 4),
-                          "kernel": "chunked: kda_prep_kernel + chunk_gdn_kernel<true>", "timed_calls": Kk}
+                          "kernel": "chunked: kda_prep_kernel + gdn_main_kernel<true>", "timed_calls": Kk}
     del a, o, S
     Sd = workloads.decode_state(seed=seed).cuda()
     pd = workloads.make_problem("kda", 256, 1, 16, 128, 128, seed=seed)

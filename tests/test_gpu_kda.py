@@ -2,7 +2,7 @@
 "状态空间与线性注意力", KDA：逐通道遗忘与误差写入) against the fp64 oracle.
 
 bf16 prefill with dk = 128 runs chunked on the tensor cores (kda_prep_kernel,
-then chunk_gdn_kernel<true>): ragged lengths that span several 64-token chunks
+then gdn_main_kernel<true>): ragged lengths that span several 64-token chunks
 and 16-token sub-chunks, every value width, zero and nonzero initial states, a
 split with the state carried across it, the benchmark shape on a sample of
 heads, the host-buffer entry point and the retention-range report.  fp32,
