@@ -434,18 +434,32 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
 
     constexpr uint32_t ID_QK = idesc_bf16(128, 64, false, false);
     constexpr uint32_t ID_U = idesc_bf16(64, 128, false, true);
+    // packed sequences: items are enumerated up to the longest sequence, and the
+    // chunks past a shorter sequence's end are skipped (nothing reads them).  The
+    // next item of this CTA is the first of its stride with a chunk to do; every
+    // thread computes it the same way.
+    auto next_item = [&](int64_t w) {
+        if (p.cu_seqlens)
+            for (; w < items; w += gridDim.x) {
+                const ItemPos ip = item_pos(w);
+                const SeqSpan sq = seq_span(p.cu_seqlens, ip.b, p.T, p.max_seqlen, false);
+                if ((int64_t)ip.c * C < sq.len) break;
+            }
+        return w;
+    };
     int it = 0;
-    if (warp == 2 && (int64_t)blockIdx.x < items) {
+    const int64_t w0 = next_item(blockIdx.x);
+    if (warp == 2 && w0 < items) {
         if (lane == 0) {
-            load_half(blockIdx.x, 0);
-            load_half(blockIdx.x, 1);
+            load_half(w0, 0);
+            load_half(w0, 1);
         }
-        fetch_gates(blockIdx.x);
+        fetch_gates(w0);
     }
     // copies in flight (thread 64's view)
-    bool q_pending = (int64_t)blockIdx.x < items, k_pending = q_pending;
+    bool q_pending = w0 < items, k_pending = q_pending;
     const uint32_t kb = tb + P_K;   // the K rows (atom column 0)
-    for (int64_t w = blockIdx.x; w < items; w += gridDim.x, ++it) {
+    for (int64_t w = w0, wn = next_item(w0 + gridDim.x); w < items; w = wn, wn = next_item(wn + gridDim.x), ++it) {
         if (warp == 2) {   // this item's gates (fetched one item ahead) into shared memory
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -473,12 +487,12 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
         if (!mbar_wait(&ctl->mma, (uint32_t)it & 1u)) ctl->abort = 1;
         tc_fence_after_sync();
         // Q is free: start the next item's Q and gates
-        if (warp == 2 && w + gridDim.x < items) {
+        if (warp == 2 && wn < items) {
             if (lane == 0 && !ctl->abort) {
-                load_half(w + gridDim.x, 0);
+                load_half(wn, 0);
                 q_pending = true;
             }
-            fetch_gates(w + gridDim.x);
+            fetch_gates(wn);
         }
         {   // row r = tid of the M=128 accumulator: warps 0-1 the P row of token r
             // (inclusive mask, to the item's P image), warps 2-3 the A row of token
@@ -563,8 +577,8 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
         if (!mbar_wait(&ctl->mma_u, (uint32_t)it & 1u)) ctl->abort = 1;
         tc_fence_after_sync();
         // K is free: the next item's K
-        if (tid == 64 && w + gridDim.x < items && !ctl->abort) {
-            load_half(w + gridDim.x, 1);
+        if (tid == 64 && wn < items && !ctl->abort) {
+            load_half(wn, 1);
             k_pending = true;
         }
         {   // -U -> the item: row tr = 16 warp + (lane & 15) of the M=64 accumulator,
