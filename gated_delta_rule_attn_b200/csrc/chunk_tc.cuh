@@ -239,8 +239,8 @@ inline int resident_per_sm(const void *kernel, int threads, int dyn_smem, int tm
     return std::max(n, 1);
 }
 
-// KDA workspace: the per-chunk items (T image, P image, Gamma_C), then the
-// Qp, Kp and Kc tensors [B,Ls,H,128] bf16, each at a 256-byte aligned offset
+// KDA workspace: the per-chunk items (T diag(beta), P and -U images, Gamma_C),
+// then the Qp and Kc tensors [B,Ls,H,128] bf16, each at a 256-byte aligned offset
 // (Ls = T dense; 64 ceil(max_seqlen / 64) for packed sequences, one row block
 // per sequence).
 struct KdaWorkspace {
@@ -268,7 +268,7 @@ inline size_t chunk_agg_bytes(int rule, int64_t B, int64_t T, int64_t H, int64_t
 inline size_t gla_flag_bytes(int64_t B, int64_t H) { return ((size_t)(B * H) * 4 + 255) & ~(size_t)255; }
 
 // Device workspace the chunked path needs: the gated delta rule keeps the
-// per-chunk T = (I + A)^-1 and P operand images (16 KB per (batch, head, chunk)); KDA
+// per-chunk operand images of T diag(beta), P and -U (32 KB per (batch, head, chunk)); KDA
 // its prep kernel's items and scaled q/k tensors; sequence-parallel ELU+1 and GLA the range
 // summaries of their first pass; GLA its per-sequence range flags.  `packed`: the
 // sequences are packed on one token axis with lengths up to max_seqlen (no
