@@ -87,7 +87,7 @@ struct KCtl {
 struct KdaPrepParams {
     int64_t B, T, H;
     int nchunks;                      // chunks per (sequence, head): ceil(max_seqlen / 64)
-    int64_t Ls;                       // token extent of qp, kp, kc: T, or 64 nchunks when packed
+    int64_t Ls;                       // token extent of qp, kc: T, or 64 nchunks when packed
     const __nv_bfloat16 *q, *k;       // [B,T,H,128] (packed: [1,T,H,128])
     const float *alpha, *beta;        // [B,T,H,128], [B,T,H] (packed: [1,T,H,*])
     uint8_t *items;                   // [B*H*nchunks][ITEM_BYTES]
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
         bar_named(1, 128);
         if (ctl->stop) break;
         if (t0 >= sq.len) continue;   // past this packed sequence's last chunk (uniform over the CTA)
-        // rows of qp, kp, kc this item writes: the sequence's tokens, plus (packed)
+        // rows of qp, kc this item writes: the sequence's tokens, plus (packed)
         // the padding rows of its tail chunk, as zeros
         const int64_t wlen = p.cu_seqlens ? p.Ls : sq.len;
 

@@ -22,8 +22,8 @@
 //   Gated delta rule (page "线性注意力与 SSM", GDN box): gamma_t = prod alpha,
 //     Gamma_ti = gamma_t / gamma_i (computed as exp2 of log2 differences <= 0),
 //     A = diag(beta) (K K^T o Gamma o strict-lower), T = (I + A)^-1,
-//     U = T diag(beta) V,  W_k = T diag(beta gamma) K,   (state independent)
-//     W = U - W_k S0,  O = diag(gamma) Q S0 + P W,  P = (Q K^T) o Gamma o M,
+//     U = T diag(beta gamma) K,                          (state independent)
+//     W = T diag(beta) V - U S0,  O = diag(gamma) Q S0 + P W,  P = (Q K^T) o Gamma o M,
 //     S <- gamma_C S0 + K^T diag(gamma_C / gamma) W.
 //   This is the WY / UT form of the delta rule's intra-chunk dependence (named
 //   on page "线性注意力速览" for DeltaNet and page "状态空间与线性注意力" for

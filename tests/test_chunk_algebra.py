@@ -271,11 +271,12 @@ def test_elu_segments_fold_to_the_recurrence():
 
 def gdn_one_mma_chain(q, k, v, alpha, beta, S0):
     """The gated delta rule with the state-dependent work of a chunk reduced to
-    products with S0 whose other factors are precomputable per chunk:
-      U = T diag(beta) V,  W_k = T diag(beta gamma) K,  (W = U - W_k S0)
-      G = K^T diag(gamma_C/gamma) W_k,  D = K^T diag(gamma_C/gamma) U,
+    products with S0 whose other factors are precomputable per chunk (U as in the
+    kernels, V_T the value part):
+      V_T = T diag(beta) V,  U = T diag(beta gamma) K,  (W = V_T - U S0)
+      G = K^T diag(gamma_C/gamma) U,  D = K^T diag(gamma_C/gamma) V_T,
       S <- gamma_C S0 + D - G S0,
-      O = (diag(gamma) Q - P W_k) S0 + P U,  P = (Q K^T) o Gamma o M."""
+      O = (diag(gamma) Q - P U) S0 + P V_T,  P = (Q K^T) o Gamma o M."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     o = np.zeros((B, T, H, dv))
@@ -291,13 +292,13 @@ def gdn_one_mma_chain(q, k, v, alpha, beta, S0):
                 gam = np.cumprod(al)
                 Gam = np.tril(gam[:, None] / gam[None, :])
                 Tm = np.linalg.inv(np.eye(C) + be[:, None] * np.tril(K @ K.T * Gam, -1))
-                U = Tm @ (be[:, None] * V)
-                Wk = Tm @ ((be * gam)[:, None] * K)
+                VT = Tm @ (be[:, None] * V)
+                U = Tm @ ((be * gam)[:, None] * K)
                 Kd = (gam[-1] / gam)[:, None] * K
-                G, D = Kd.T @ Wk, Kd.T @ U
+                G, D = Kd.T @ U, Kd.T @ VT
                 P = Q @ K.T * Gam
-                Qe = gam[:, None] * Q - P @ Wk
-                O = Qe @ S + P @ U
+                Qe = gam[:, None] * Q - P @ U
+                O = Qe @ S + P @ VT
                 S = gam[-1] * S + D - G @ S
                 o[b, c0:c0 + n, h] = O[:n]
             S_out[b, h] = S
