@@ -315,6 +315,64 @@ def test_gdn_one_mma_chain_form_equals_recurrence(T):
     assert _rel(o, ro) < 1e-12 and _rel(S, rS) < 1e-12
 
 
+def gdn_w_carried(q, k, v, alpha, beta, S0, rnd=None, f32=None):
+    """The gated delta rule with the recurrence carried through W instead of S:
+    S_{c+1} = gamma_C S_c + K_c^T diag(gamma_C/gamma) W_c inside W_{c+1} gives
+      W_{c+1} = T diag(beta) V_{c+1} - gamma_C U_{c+1} S_c - L_c W_c,
+      L_c = U_{c+1} K_c^T diag(gamma_C/gamma)_c   (U = T diag(beta gamma) K),
+    so that a chunk's W needs the previous chunk's W and the state one chunk
+    older; O_c = diag(gamma) Q_c S_c + P_c W_c as before.  With `rnd`/`f32` the
+    operands are rounded where a tensor-core kernel of this form reads them."""
+    R = rnd or (lambda x: x)
+    F = f32 or (lambda x: x)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    S_out = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            pre = []
+            for c0 in range(0, T, C):
+                n = min(C, T - c0)
+                Q, K, V = (_chunk(x, b, h, c0, n, 0.0, x.shape[-1]) for x in (q, k, v))
+                al = _chunk(alpha[..., None], b, h, c0, n, 1.0, 1)[:, 0]
+                be = _chunk(beta[..., None], b, h, c0, n, 0.0, 1)[:, 0]
+                gam = F(np.cumprod(al))
+                Gam = np.tril(gam[:, None] / gam[None, :])
+                Tm = F(np.linalg.inv(np.eye(C) + be[:, None] * np.tril(F(K @ K.T) * Gam, -1)))
+                pre.append(dict(n=n, c0=c0, Q=R(Q), K=R(K), gam=gam, Gam=Gam,
+                                negU=R(-F(R(Tm * (be * gam)[None, :]) @ R(K))),
+                                TV=R(F(R(Tm * be[None, :]) @ R(V)))))
+            S = np.zeros((dk, dv)) if S0 is None else S0[b, h].copy()
+            Sb = R(S)
+            W = F(pre[0]["TV"] + F(pre[0]["negU"] @ Sb))
+            for c, P_ in enumerate(pre):
+                Q, K, gam = P_["Q"], P_["K"], P_["gam"]
+                gC, gct = gam[-1], gam[-1] / gam
+                Wb = R(W)
+                O = F(gam[:, None] * F(Q @ Sb) + F(R(F(Q @ K.T) * P_["Gam"]) @ Wb))
+                o[b, P_["c0"]:P_["c0"] + P_["n"], h] = R(O)[:P_["n"]]
+                dS = F(K.T @ R(Wb * gct[:, None]))
+                if c + 1 < len(pre):
+                    nU = pre[c + 1]["negU"]
+                    negL = R(F(nU @ K.T) * gct[None, :])
+                    W = F(pre[c + 1]["TV"] + gC * F(nU @ Sb) + F(negL @ Wb))
+                S = F(gC * S + dS)
+                Sb = R(S)
+            S_out[b, h] = S
+    return o, S_out
+
+
+@pytest.mark.parametrize("T", [1, 37, 130])
+def test_gdn_w_carried_form_equals_recurrence(T):
+    """The W-carried chain (built on the GPU and measured, not kept) is exact:
+    a dropped gamma_C or a missing L term changes every chunk after the first."""
+    p = workloads.make_problem("gdn", 2, T, 2, 16, 8, seed=T + 9, init_state="normal")
+    ro, rS, _ = oracle.fwd(p)
+    o, S = gdn_w_carried(*(_f64(x) for x in (p.q, p.k, p.v, p.g, p.beta, p.S0)))
+    assert _rel(o, ro) < 1e-12 and _rel(S, rS) < 1e-12
+
+
 # ---------------------------------------------------------------------------
 # Rounding model: bf16 wherever a tensor-core operand is read, fp32 for the
 # accumulators and the carried state (the precision of the kernels), for the
@@ -368,15 +426,18 @@ def gdn_rounded(q, k, v, alpha, beta, one_mma):
 
 @pytest.mark.parametrize("alpha", ["sigmoid3", "ones"])
 def test_gdn_chain_forms_meet_the_bf16_bound_under_the_rounding_model(alpha):
-    """Both chain forms stay well inside the bf16 bound (2e-2) at d = 128 over 16
-    chunks: the current one (the GPU measures 4.4-5.4e-3 on this workload) and
-    the one-MMA form, whose bf16 G multiplies the state every chunk."""
+    """The chain forms stay well inside the bf16 bound (2e-2) at d = 128 over 16
+    chunks: the current one (the GPU measures 4.4-5.4e-3 on this workload), the
+    one-MMA form, whose bf16 G multiplies the state every chunk, and the
+    W-carried form, whose bf16 L multiplies W every chunk."""
     p = workloads.make_problem("gdn", 1, 1024, 1, 128, 128, seed=4, gdn_alpha=alpha)
     ro, rS, _ = oracle.fwd(p)
     args = [_f64(x) for x in (p.q, p.k, p.v, p.g, p.beta)]
     for one_mma in (False, True):
         o, S = gdn_rounded(*args, one_mma)
         assert _rel(o, ro) < 1e-2 and _rel(S, rS) < 1e-2, (one_mma, _rel(o, ro), _rel(S, rS))
+    o, S = gdn_w_carried(*args, None, rnd=_bf, f32=_f32)   # the W-carried chain
+    assert _rel(o, ro) < 1e-2 and _rel(S, rS) < 1e-2, ("w-carried", _rel(o, ro), _rel(S, rS))
 
 
 def test_kda_benchmark_workload_is_inside_the_chunked_domain():
