@@ -105,6 +105,9 @@ chunk_agg_kernel(const __grid_constant__ Maps maps, const AggParams p) {
     }
     __syncthreads();
     tc_fence_after_sync();
+    // the main pass, launched as a programmatic dependent, may be scheduled now: its
+    // CTAs wait for this grid's completion before they read the summaries or flags
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = ctl->tmem_base;
 
     if (warp < 8) {

@@ -391,6 +391,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap mapq, const __grid_constant_
     }
     __syncthreads();
     tc_fence_after_sync();
+    // the main pass, launched as a programmatic dependent, may be scheduled now: it
+    // waits for this grid's completion before it reads anything written here
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tq = tmem + ((uint32_t)(32 * warp) << 16);
 
@@ -747,6 +750,10 @@ gdn_main_kernel(const __grid_constant__ Maps maps, const ChunkParams p, const ui
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
+        // launched as a programmatic dependent of the prep kernel: its items (and,
+        // for KDA, Qp and Kc) are complete and visible once this returns; nothing
+        // else in this kernel reads them but through the producer's copies
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         float al[2] = {1.f, 1.f};   // the alphas of the chunk to be issued next
         auto fetch = [&](int c) {
 #pragma unroll

@@ -443,7 +443,11 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
             }
             if (!kGLA && p.z0) z = p.z0[bh * DK + d];
             // sequence-parallel pass: fold the state through the token ranges of the
-            // earlier segments, in order (ELU+1: S += dS, z += dz; GLA: S <- D o S + dS)
+            // earlier segments, in order (ELU+1: S += dS, z += dz; GLA: S <- D o S + dS).
+            // This kernel is then a programmatic dependent of the summary pass: the
+            // summaries (and its range flags, read at the end) are complete and visible
+            // once the wait returns.  The first segment needs neither.
+            if (seg > 0) asm volatile("griddepcontrol.wait;" ::: "memory");
             const int64_t blk = (int64_t)DK * p.dv + DK;
             for (int i = 0; i < seg * p.nparts; ++i) {
                 const float *a = p.agg + (bh * (p.nseg - 1) * p.nparts + i) * blk;
@@ -521,9 +525,10 @@ chunk_ge_kernel(const __grid_constant__ Maps maps, const ChunkParams p) {
         // a sequence flagged here or, for the earlier segments, by the summary
         // pass keeps S_out untouched (S0 may alias it): the recurrent kernel
         // recomputes it from S0
-        const bool flagged = kGLA && (*reinterpret_cast<volatile int *>(&ctl->seqfail) != 0 ||
-                                      (p.seq_flags && p.seq_flags[bh] == p.call_id));
-        if (!ctl->abort && seg == p.nseg - 1 && !flagged) {
+        const bool last = seg == p.nseg - 1;
+        const bool flagged = kGLA && last && (*reinterpret_cast<volatile int *>(&ctl->seqfail) != 0 ||
+                                              (p.seq_flags && p.seq_flags[bh] == p.call_id));
+        if (!ctl->abort && last && !flagged) {
             if (p.S_out) {
                 float *dst = p.S_out + ((bh * DK + d) * p.dv + dvt * DVS);
 #pragma unroll

@@ -148,6 +148,9 @@ __global__ void __launch_bounds__(kda::PREP_THREADS, 2) kda_prep_kernel(const Kd
     }
     __syncthreads();
     tc_fence_after_sync();
+    // the main pass, launched as a programmatic dependent, may be scheduled now: it
+    // waits for this grid's completion before it reads anything written here
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = ctl->tmem_base;
     const uint32_t tw = tmem + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lanes
     constexpr uint32_t ID_U = idesc_bf16(64, 128, false, true);

@@ -48,6 +48,7 @@
 #include <algorithm>
 #include <atomic>
 #include <string>
+#include <utility>
 
 #include "device.cuh"
 #include "recurrent.cuh"
@@ -282,7 +283,28 @@ inline size_t chunk_workspace_bytes(int rule, int64_t B, int64_t T, int64_t H, i
     return chunk_agg_bytes(rule, B, T, H, dv, packed) + (rule == kRuleGLA ? gla_flag_bytes(B, H) : 0);
 }
 
-// GLA / ELU: one CTA per (batch, head, 32-column value slab).
+// Launch `kern` as a programmatic dependent of the kernel before it in `st`
+// (when `dependent`): it may be scheduled once every CTA of that kernel has
+// signalled, and it waits (griddepcontrol.wait) before reading that kernel's
+// results.
+template <typename... Params, typename... Args>
+cudaError_t launch_maybe_dependent(void (*kern)(Params...), unsigned grid, unsigned block, int smem,
+                                   cudaStream_t st, bool dependent, Args &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = dependent ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// GLA / ELU: one CTA per (batch, head, value slab, segment); a programmatic
+// dependent of the summary pass when there is one.
 template <int RULE, int DVS>
 cudaError_t launch_ge(const ck::Maps &m, const ChunkParams &p, cudaStream_t st) {
     using L = ck::GE<RULE, DVS>;
@@ -290,7 +312,8 @@ cudaError_t launch_ge(const ck::Maps &m, const ChunkParams &p, cudaStream_t st) 
     cudaError_t e = allow_smem((const void *)ck::chunk_ge_kernel<RULE, DVS>, smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)(p.B * p.H * (p.dv / DVS) * p.nseg);
-    ck::chunk_ge_kernel<RULE, DVS><<<grid, L::NTHREADS, smem, st>>>(m, p);
+    e = launch_maybe_dependent(ck::chunk_ge_kernel<RULE, DVS>, grid, (unsigned)L::NTHREADS, smem, st, p.nseg > 1, m, p);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -406,7 +429,8 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         const int smem = (int)((sizeof(gdn::MCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::ML<true>::TEND;
         if (e == cudaSuccess) e = allow_smem((const void *)gdn_main_kernel<true>, smem);
         if (e == cudaSuccess)
-            gdn_main_kernel<true><<<grid, gdn::NTHREADS, smem, st>>>(mk, pq, w8 + kw.items);
+            e = launch_maybe_dependent(gdn_main_kernel<true>, grid, (unsigned)gdn::NTHREADS, smem, st, true, mk, pq,
+                                       (const uint8_t *)(w8 + kw.items));
     } else if (rule == kRuleGDN) {
         const size_t need = chunk_workspace_bytes(rule, p.B, p.T, p.H, p.dv, packed, Lmax);
         if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15u)) {
@@ -432,7 +456,8 @@ inline int launch_chunk_tc(int rule, const ChunkParams &p, void *ws, size_t ws_b
         const int smem = (int)((sizeof(gdn::MCtl) + 1023) / 1024 * 1024) + 1024 + (int)gdn::ML<false>::TEND;
         if (e == cudaSuccess) e = allow_smem((const void *)gdn_main_kernel<false>, smem);
         if (e == cudaSuccess)
-            gdn_main_kernel<false><<<grid, gdn::NTHREADS, smem, st>>>(m, pq, static_cast<const uint8_t *>(ws));
+            e = launch_maybe_dependent(gdn_main_kernel<false>, grid, (unsigned)gdn::NTHREADS, smem, st, items > 0, m,
+                                       pq, static_cast<const uint8_t *>(ws));
     } else {
         // packed sequences walk each sequence in one pass (no segments)
         const SegPlan sp = packed ? SegPlan{1, 1, (int)((Lmax + C - 1) / C)} : seg_plan(rule, p.B, p.T, p.H, p.dv);
