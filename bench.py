@@ -99,27 +99,44 @@ def load_peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+# The csrc files behind each leg's kernels and their launches: a leg's DRAM
+# traffic record stays valid while these files are unchanged.
+LEG_SOURCES = {
+    "gla_prefill": ["device.cuh", "chunk_tc.cuh", "chunk_ge.cuh", "chunk_agg.cuh", "recurrent.cuh", "la.cu"],
+    "elu_prefill": ["device.cuh", "chunk_tc.cuh", "chunk_ge.cuh", "chunk_agg.cuh", "la.cu"],
+    "gdn_prefill": ["device.cuh", "chunk_tc.cuh", "chunk_gdn.cuh", "la.cu"],
+    "gla_decode": ["device.cuh", "recurrent.cuh", "la.cu"],
+    "gdn_decode": ["device.cuh", "recurrent.cuh", "la.cu"],
+    "kda_prefill": ["device.cuh", "chunk_tc.cuh", "chunk_gdn.cuh", "chunk_kda.cuh", "la.cu"],
+}
+
+
+def kernel_source_hash(files=None) -> str:
+    """sha256 (first 16 hex digits) over the named csrc files, or all of them."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_attn_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def load_traffic():
-    """DRAM bytes per launch from a committed ncu capture, valid only while the
-    kernel sources are unchanged since the capture."""
+    """DRAM bytes per launch of each leg from a committed ncu capture; a leg's
+    figure is valid only while the sources of its kernels are unchanged since
+    the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except Exception:
         return {}
-    if d.get("source_hash") != kernel_source_hash():
-        return {}
-    return d.get("bytes_per_launch", {})
+    out = {}
+    for leg, rec in d.get("legs", {}).items():
+        files = LEG_SOURCES.get(leg)
+        if files is not None and rec.get("source_hash") == kernel_source_hash(files):
+            out[leg] = rec.get("bytes_per_launch")
+    return out
 
 
 class ClockSampler:

@@ -31,3 +31,25 @@ def test_macs_per_token_head():
 def test_reference_arm_sample_runs():
     dt, tokens = bench.oracle_sample(16)
     assert tokens == 32 and dt > 0
+
+
+def test_traffic_record_is_valid_per_leg(tmp_path, monkeypatch):
+    """A leg's committed DRAM traffic stays valid while the csrc files behind its
+    kernels are unchanged; editing one file voids exactly the legs that list it."""
+    import json
+    csrc = tmp_path / "gated_delta_rule_attn_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    files = sorted({f for fs in bench.LEG_SOURCES.values() for f in fs})
+    for f in files:
+        (csrc / f).write_text(f"// {f}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    legs = {leg: {"bytes_per_launch": 1000 + i, "source_hash": bench.kernel_source_hash(fs)}
+            for i, (leg, fs) in enumerate(bench.LEG_SOURCES.items())}
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"legs": legs}))
+    assert set(bench.load_traffic()) == set(bench.LEG_SOURCES)
+    (csrc / "chunk_ge.cuh").write_text("// edited\n")
+    valid = bench.load_traffic()
+    for leg, fs in bench.LEG_SOURCES.items():
+        assert (leg in valid) == ("chunk_ge.cuh" not in fs), leg
+    assert valid["gdn_prefill"] == legs["gdn_prefill"]["bytes_per_launch"]
