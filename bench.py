@@ -642,7 +642,43 @@ def cpu_baseline(budget_s: float = 15.0):
     return {"value": round(tokens / dt, 1), "unit": "tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": f"fp64 C oracle (OpenMP over heads): GLA + gated-delta prefill of the d=128 "
-                      f"T=8192 workloads, 16 heads, {what}; {dt:.1f} s"}
+                      f"T=8192 workloads, 16 heads, {what}; {dt:.1f} s",
+            "host": host_cpu(), "elu_fp32_small_ms": oracle_elu_small_ms()}
+
+
+def host_cpu():
+    """The host the oracle ran on: cores this process may use, the CPU model
+    and the oracle's OpenMP threads."""
+    import oracle
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count()
+    return {"affinity_cores": cores, "cpu_model": model, "omp_threads": oracle.num_threads()}
+
+
+def oracle_elu_small_ms(reps: int = 5):
+    """Median time of the oracle on the fp32 ELU+1 workload (B=1 H=1 T=256
+    d=32): one sequence, so one thread whatever the OpenMP setting."""
+    import oracle
+    import workloads
+    p = workloads.elu_fp32_small(seed=0)
+    ts = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        oracle.elu_fwd(p.q, p.k, p.v, p.S0, p.z0, eps=p.eps)
+        ts.append(time.perf_counter() - t0)
+    ts.sort()
+    return round(1e3 * ts[len(ts) // 2], 3)
 
 
 def run_reference(args):
@@ -689,7 +725,7 @@ def _reference_line(args, world):
                       "global_batch": 2, "seq_len": 8192, "parallelism": "CPU threads"},
            "impl": "reference",
            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores,
-                            "kind": "oracle", "sample": sample},
+                            "kind": "oracle", "sample": sample, "host": host_cpu()},
            "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)

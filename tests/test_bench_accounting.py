@@ -53,3 +53,12 @@ def test_traffic_record_is_valid_per_leg(tmp_path, monkeypatch):
     for leg, fs in bench.LEG_SOURCES.items():
         assert (leg in valid) == ("chunk_ge.cuh" not in fs), leg
     assert valid["gdn_prefill"] == legs["gdn_prefill"]["bytes_per_launch"]
+
+
+def test_cpu_baseline_records_its_host():
+    """The oracle baseline says where it ran: the cores this process may use, the
+    CPU model and the OpenMP threads, and the single-sequence fp32 time."""
+    h = bench.host_cpu()
+    assert h["affinity_cores"] >= 1 and h["omp_threads"] >= 1
+    assert "cpu_model" in h
+    assert bench.oracle_elu_small_ms(reps=1) > 0
