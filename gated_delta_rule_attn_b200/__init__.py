@@ -164,13 +164,16 @@ def make_fwd_args(rule, q, k, v, g=None, beta=None, S0=None, z0=None, eps=1e-6,
 _WORKSPACES = {}
 
 
-def _workspace(device, stream_handle: int, nbytes: int):
+def _workspace(device, stream, nbytes: int):
     """Scratch for la_fwd, cached per (device, stream): calls on one stream are
-    ordered, so they can share it."""
-    key = (device.index, stream_handle)
+    ordered, so they can share it.  It is allocated with that stream current, so
+    that when a larger one replaces it, the allocator reuses the old block only
+    for work ordered after the kernels that used it."""
+    key = (device.index, stream.cuda_stream)
     ws = _WORKSPACES.get(key)
     if ws is None or ws.numel() < nbytes:
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        with torch.cuda.stream(stream):
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         _WORKSPACES[key] = ws
     return ws
 
@@ -202,11 +205,12 @@ def fwd(rule: str, q, k, v, g=None, beta=None, S0=None, z0=None, eps: float = 1e
         z_out = torch.empty(NS, H, dk, dtype=torch.float32, device=q.device)
     a = make_fwd_args(rule, q, k, v, g, beta, S0, z0, eps, o, S_out, z_out, cu_seqlens, max_seqlen,
                       out_norm, norm_w, norm_eps)
-    sh = _stream_handle(stream)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    sh = _stream_handle(st)
     n = ctypes.c_size_t()
     _check(lib().la_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
     if n.value:
-        ws = workspace if workspace is not None else _workspace(q.device, sh.value or 0, n.value)
+        ws = workspace if workspace is not None else _workspace(q.device, st, n.value)
         a.workspace, a.workspace_bytes = ws.data_ptr(), ws.numel()
     _check(lib().la_fwd(ctypes.byref(a), sh))
     return o, S_out, z_out
