@@ -52,3 +52,16 @@ def test_oracle_never_reaches_the_package():
         assert "gated_delta_rule_attn_b200" not in _imported_modules(f), f
     for f in _files(ORACLE, (".c", ".h", ".cpp")):
         assert not any("csrc" in i or i.endswith(".cuh") or i == "la.h" for i in _includes(f)), f
+
+
+def test_package_fails_loudly_without_its_library(monkeypatch, tmp_path):
+    """No CPU fallback: with the CUDA library missing, the first call into the
+    package raises instead of computing anything."""
+    import pytest
+    import gated_delta_rule_attn_b200 as la
+    monkeypatch.setattr(la, "_lib", None)
+    monkeypatch.setattr(la, "LIB_PATH", str(tmp_path / "libla_b200.so"))
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        la.lib()
+    with pytest.raises(ImportError):
+        la.abi_version()
